@@ -1,0 +1,461 @@
+#!/usr/bin/env python
+"""Benchmark of the weight-quantized matmul hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+A *step* is one pass over every matmul of the workload (default: the Llama-7B-shaped
+W4A16 decode GEMVs, M in {1,4,16} x (N,K) in {(4096,4096),(11008,4096),(4096,11008)}),
+each on its own copy of the packed weights: every case rotates through enough copies
+that its copies together exceed 4x the 126 MB L2, so each launch streams its weights
+from HBM.  Weights are quantized once on the GPU (offline step, untimed).
+
+Timing: CUDA graphs of whole steps, replayed on one stream between CUDA events, after W
+warm-up steps, with a barrier + torch.cuda.synchronize() on both sides; the max over ranks
+is reported.  ``value`` = algorithmic bytes of all ranks / time (GB/s).  ``e2e`` repeats
+the measurement through the same C-ABI calls with pinned HOST activations and outputs:
+every step copies A host->device and C device->host inside the timed region.
+
+Algorithmic bytes per launch: packed weights N*K*b/8 + scales (+ zeros) N*G*2 (each) +
+activations M*K*bytes(A) (+ 4M for INT8 scales) + output M*N*2.
+
+``--impl reference`` times the CPU oracle (plain C, float64) on a bounded sample of the
+same workload on the host cores; it is a deliberately slow baseline, not a target.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import glob
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+import wq_synth
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+L2_BYTES = 126 * 1024 * 1024
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+
+
+# ------------------------------------------------------------------ workload arithmetic
+def alg_bytes(c: wq_synth.Case) -> int:
+    bits = 2 if c.quant == "tern2" else 4
+    w = c.N * c.K * bits // 8
+    if bits == 4:
+        G = c.K // c.group_size
+        w += c.N * G * 2 * (2 if c.quant == "asym4" else 1)
+    else:
+        w += 4
+    a = c.M * c.K * (1 if c.mode == "a8" else 2) + (4 * c.M if c.mode == "a8" else 0)
+    return w + a + c.M * c.N * 2
+
+
+def flops(c: wq_synth.Case) -> int:
+    return 2 * c.M * c.N * c.K
+
+
+def launches_per_call(c: wq_synth.Case) -> int:
+    return (c.M + 63) // 64
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        d = json.load(open(path))
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": FALLBACK_HBM_GBS, "bf16_tflops": FALLBACK_BF16_TFLOPS,
+                "bf16_tflops_sustained": FALLBACK_BF16_TFLOPS, "source": "fallback"}
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for p in sorted(glob.glob(os.path.join(ROOT, "gemv_wq_quantize_b200", "csrc", "*"))):
+        h.update(open(p, "rb").read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload: str):
+    """DRAM bytes per launch from the committed ncu summary, if it matches the current kernels."""
+    path = os.path.join(ROOT, "profiles", f"skinny_kernel_{workload}.md")
+    if not os.path.exists(path):
+        return None
+    src, traffic = None, None
+    for line in open(path):
+        if line.startswith("source_sha:"):
+            src = line.split(":", 1)[1].strip()
+        if line.startswith("dram_bytes_per_launch:"):
+            traffic = float(line.split(":", 1)[1].strip())
+    return traffic if (src == kernel_source_hash() and traffic) else None
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML while the timed region runs."""
+
+    REASONS = {"hw_slowdown": 0x8, "hw_thermal_slowdown": 0x40, "sw_thermal_slowdown": 0x20,
+               "sw_power_cap": 0x4, "hw_power_brake_slowdown": 0x80}
+
+    def __init__(self, device):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = self._handle(pynvml, device)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self.nv = None
+
+    @staticmethod
+    def _handle(nv, device):
+        props = torch.cuda.get_device_properties(device)
+        uuid = getattr(props, "uuid", None)
+        if uuid is not None:
+            try:
+                return nv.nvmlDeviceGetHandleByUUID("GPU-" + str(uuid))
+            except Exception:
+                pass
+        bus = getattr(props, "pci_bus_id", None)
+        if bus is not None:
+            dom = getattr(props, "pci_domain_id", 0)
+            dev = getattr(props, "pci_device_id", 0)
+            try:
+                return nv.nvmlDeviceGetHandleByPciBusId(f"{dom:08x}:{bus:02x}:{dev:02x}.0")
+            except Exception:
+                pass
+        return nv.nvmlDeviceGetHandleByIndex(0)
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                r = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for k, bit in self.REASONS.items():
+                    if r & bit:
+                        self.reasons.add(k)
+            except Exception:
+                break
+            time.sleep(0.002)
+
+    def __enter__(self):
+        if self.nv:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self.nv:
+            self.t.join()
+
+    def report(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons), "samples": 0}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# ------------------------------------------------------------------ our arm
+class Prepared:
+    """Quantized weight copies, activations and outputs of one case on the device."""
+
+    def __init__(self, c: wq_synth.Case, device, seed_base: int = 0):
+        import gemv_wq_quantize_b200 as wq
+        self.c = c
+        self.qc = wq.QuantConfig(bits=2) if c.quant == "tern2" else \
+            wq.QuantConfig(bits=4, group_size=c.group_size, symmetric=(c.quant == "sym4"))
+        W = wq_synth.weights(c.N, c.K, seed=seed_base).to(device)
+        Wq, s, z = wq.quantize_pack(W, self.qc)
+        del W
+        self.bytes = alg_bytes(c)
+        copies = max(2, math.ceil(4 * L2_BYTES / self.bytes))
+        self.weights = [(Wq, s, z)] + [(Wq.clone(), s.clone(), None if z is None else z.clone())
+                                        for _ in range(copies - 1)]
+        A = wq_synth.activations(c.M, c.K, seed=seed_base + 1, dtype=c.a_dtype, outlier_frac=c.outlier_frac)
+        self.A = A.to(device)
+        self.A_host = A.pin_memory()
+        if c.mode == "a8":
+            self.Aq, self.a_scale = wq.act_quant_int8(self.A)
+        self.C = torch.empty(c.M, c.N, dtype=torch.float16 if c.mode == "a8" else c.a_dtype, device=device)
+        self.C_host = torch.empty(self.C.shape, dtype=self.C.dtype).pin_memory()
+        self.ws = wq.make_workspace(wq.workspace_size(c.M, c.N, c.K, self.qc), device)
+        self.i = 0
+
+    def launch(self, e2e: bool = False):
+        import gemv_wq_quantize_b200 as wq
+        Wq, s, z = self.weights[self.i % len(self.weights)]
+        self.i += 1
+        c = self.c
+        if e2e:
+            self.A.copy_(self.A_host, non_blocking=True)
+        if c.mode == "a16":
+            wq.w4a16_gemm(self.A, Wq, s, z, c.N, c.K, self.qc, out=self.C, workspace=self.ws)
+        else:
+            if e2e:  # the INT8 path starts from the fp16 activations: quantize them too
+                wq.act_quant_int8(self.A, out_q=self.Aq, out_scale=self.a_scale)
+            wq.w4a8_gemm(self.Aq, self.a_scale, Wq, s, z, c.N, c.K, self.qc, out=self.C, workspace=self.ws)
+        if e2e:
+            self.C_host.copy_(self.C, non_blocking=True)
+
+
+def capture(preps, nsteps: int, e2e: bool):
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for _ in range(nsteps):
+            for p in preps:
+                p.launch(e2e)
+    return g
+
+
+def timed_replays(preps, steps: int, warmup: int, e2e: bool, dist_on: bool, sampler=None):
+    """Runs `warmup` untimed steps, then exactly `steps` timed steps; returns seconds (max over ranks)."""
+    chunk = max(1, min(steps, 200))
+    g_chunk = capture(preps, chunk, e2e)
+    rem = steps % chunk
+    g_rem = capture(preps, rem, e2e) if rem else None
+    stream = torch.cuda.current_stream()
+    # warm-up
+    done = 0
+    while done < warmup:
+        n = min(chunk, warmup - done)
+        if n == chunk:
+            g_chunk.replay()
+        else:
+            for p in preps:
+                p.launch(e2e)
+        done += n
+    torch.cuda.synchronize()
+    if dist_on:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ctx = sampler if sampler is not None else _Null()
+    with ctx:
+        t0.record(stream)
+        for _ in range(steps // chunk):
+            g_chunk.replay()
+        if g_rem is not None:
+            g_rem.replay()
+        t1.record(stream)
+        torch.cuda.synchronize()
+    if dist_on:
+        torch.distributed.barrier()
+    sec = t0.elapsed_time(t1) / 1e3
+    if dist_on:
+        t = torch.tensor([sec], device="cuda")
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        sec = float(t.item())
+    del g_chunk, g_rem
+    return sec
+
+
+class _Null:
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *a):
+        pass
+
+
+def per_case_breakdown(preps, reps: int = 200):
+    """Per-case microseconds (graph of `reps` launches of that case alone, events around it)."""
+    out = []
+    pk = peaks()
+    for p in preps:
+        g = capture([p], reps, False)
+        g.replay()
+        torch.cuda.synchronize()
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0.record()
+        g.replay()
+        t1.record()
+        torch.cuda.synchronize()
+        us = t0.elapsed_time(t1) * 1e3 / reps
+        gbs = p.bytes / (us * 1e-6) / 1e9
+        tf = flops(p.c) / (us * 1e-6) / 1e12
+        peak_tc = pk["bf16_tflops"] * (2.0 if p.c.mode == "a8" else 1.0)
+        t_roof = max(p.bytes / (pk["hbm_gbs"] * 1e9), flops(p.c) / (peak_tc * 1e12))
+        out.append({"case": p.c.name, "us": round(us, 3), "GB/s": round(gbs, 1), "TFLOP/s": round(tf, 2),
+                    "hbm_frac": round(gbs / pk["hbm_gbs"], 4), "roofline_frac": round(t_roof / (us * 1e-6), 4)})
+        del g
+    return out
+
+
+def run_ours(args, rank, world, local_rank, dist_on):
+    import gemv_wq_quantize_b200 as wq
+    from gemv_wq_quantize_b200 import build
+    build.build(quiet=True)
+    wq.load_library()
+    device = torch.device("cuda", local_rank)
+    torch.cuda.set_device(device)
+    wl = wq_synth.WORKLOADS[args.workload]
+    preps = [Prepared(c, device, seed_base=0) for c in wl.cases]
+    for p in preps:          # first calls configure the kernels outside any capture
+        p.launch(False)
+        p.launch(True)
+    torch.cuda.synchronize()
+    sampler = ClockSampler(device)
+    sec = timed_replays(preps, args.steps, args.warmup, False, dist_on, sampler)
+    sec_e2e = timed_replays(preps, args.steps, args.warmup, True, dist_on)
+    assert wq.device_error() == 0, "a kernel gave up a bounded wait"
+    step_bytes = sum(p.bytes for p in preps)
+    step_flops = sum(flops(p.c) for p in preps)
+    launches = sum(launches_per_call(p.c) for p in preps)
+    total_bytes = step_bytes * args.steps * world
+    value = total_bytes / sec / 1e9
+    e2e_value = total_bytes / sec_e2e / 1e9
+    pk = peaks()
+    avg_launch_s = sec / (args.steps * launches)
+    achieved = (step_bytes / launches) / avg_launch_s / 1e9
+    tensor_bound = args.workload == "prefill-llama7b"
+    result = {
+        "metric": "W4 GEMV GB/s & GEMM TFLOP/s at 1 B200; fraction of HBM / tensor roofline",
+        "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(sec / args.steps * 1e3, 6), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f16" if not tensor_bound else "bf16", "weight_dtype": "int4" if
+        "tern" not in args.workload else "int2",
+        "data": "synthetic (seeded N(0,0.02) weights, N(0,1) activations, 1% outlier channels x20)",
+        "config": {"workload": wl.name, "description": wl.description,
+                   "cases": [p.c.name for p in preps],
+                   "l2": "inputs larger than L2: each case rotates over >= 4x126MB of weight copies",
+                   "timing": "CUDA graphs of whole steps, CUDA events on the launch stream, max over ranks"},
+        "e2e": {"value": round(e2e_value, 2), "unit": "GB/s",
+                "h2d_bytes_per_step": sum(p.A.numel() * p.A.element_size() for p in preps),
+                "d2h_bytes_per_step": sum(p.C.numel() * p.C.element_size() for p in preps)},
+        "gpu_launches": args.steps * (launches + 0),
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": pk["hbm_gbs"], "unit": "GB/s",
+                     "frac": round(achieved / pk["hbm_gbs"], 4), "traffic": recorded_traffic(args.workload),
+                     "peak_source": pk["source"]},
+        "tflops": round(step_flops * args.steps * world / sec / 1e12, 3),
+        "clocks": sampler.report(),
+    }
+    if not args.no_breakdown:
+        result["cases"] = per_case_breakdown(preps)
+    return result
+
+
+# ------------------------------------------------------------------ oracle timing
+def oracle_sample(wl, budget_s: float, threads: int):
+    """Runs the CPU oracle on a bounded sample of every case (a subset of output columns,
+    all tokens) and returns (algorithmic bytes covered, seconds, description)."""
+    import oracle
+    oracle.build()
+    prepared = []
+    for c in wl.cases:
+        W = wq_synth.weights(c.N, c.K, seed=0).numpy()
+        A = wq_synth.activations(c.M, c.K, seed=1, dtype=c.a_dtype, outlier_frac=c.outlier_frac)
+        Abits = A.contiguous().view(torch.int16).numpy().view(np.uint16)
+        if c.quant == "tern2":
+            Wq, s = oracle.quantize_ternary(W)
+            z, bits, sym = None, 2, True
+        else:
+            Wq, s, z = oracle.quantize_int4(W, c.group_size, c.quant == "sym4")
+            bits, sym = 4, c.quant == "sym4"
+        prepared.append((c, Abits, Wq, s, z, bits, sym))
+
+    def run(frac):
+        t = 0.0
+        covered = 0.0
+        for c, Abits, Wq, s, z, bits, sym in prepared:
+            n_cnt = max(1, int(round(c.N * frac)))
+            ni = np.arange(n_cnt) * (c.N // n_cnt)
+            t0 = time.perf_counter()
+            if c.mode == "a16":
+                adt = oracle.F16 if c.a_dtype == torch.float16 else oracle.BF16
+                oracle.gemm_a16(Abits, adt, Wq, c.N, c.K, bits, sym, c.group_size, s, z, n_idx=ni, threads=threads)
+            else:
+                Aq, asc = oracle.act_quant_int8(Abits, oracle.F16)
+                oracle.gemm_a8(Aq, asc, Wq, c.N, c.K, bits, sym, c.group_size, s, z, n_idx=ni, threads=threads)
+            t += time.perf_counter() - t0
+            covered += alg_bytes(c) * n_cnt / c.N
+        return covered, t
+
+    frac = 1.0 / 512
+    covered, t = run(frac)
+    if t < budget_s / 4:
+        frac = min(1.0, frac * budget_s / max(t, 1e-3) / 2)
+        covered, t = run(frac)
+    desc = f"oracle on {frac:.4%} of the output columns of every case (all tokens), {threads} threads"
+    return covered, t, desc
+
+
+def run_reference(args):
+    wl = wq_synth.WORKLOADS[args.workload]
+    threads = os.cpu_count() or 1
+    budget = max(2.0, min(20.0, 60.0 / max(1, args.steps + args.warmup)))
+    for _ in range(args.warmup):
+        oracle_sample(wl, budget / 4, threads)
+    covered = secs = 0.0
+    desc = ""
+    for _ in range(args.steps):
+        cb, s, desc = oracle_sample(wl, budget, threads)
+        covered += cb
+        secs += s
+    v = covered / secs / 1e9
+    return {"metric": "W4 GEMV GB/s & GEMM TFLOP/s at 1 B200; fraction of HBM / tensor roofline",
+            "value": round(v, 6), "unit": "GB/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(secs / max(1, args.steps) * 1e3, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+            "config": {"workload": wl.name, "description": wl.description},
+            "cpu_baseline": {"value": round(v, 6), "unit": "GB/s", "cores": threads, "kind": "oracle",
+                             "sample": desc},
+            "e2e": {"value": round(v, 6), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+# ------------------------------------------------------------------ main
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20000)
+    ap.add_argument("--warmup", type=int, default=200)
+    ap.add_argument("--workload", default="decode-llama7b", choices=sorted(wq_synth.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-breakdown", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=10.0, help="seconds of oracle work for cpu_baseline")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args)), flush=True)
+        return
+
+    dist_on = world > 1
+    if dist_on:
+        import datetime
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local_rank))
+    result = run_ours(args, rank, world, local_rank, dist_on)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        wl = wq_synth.WORKLOADS[args.workload]
+        threads = os.cpu_count() or 1
+        covered, secs, desc = oracle_sample(wl, args.cpu_budget, threads)
+        result["cpu_baseline"] = {"value": round(covered / secs / 1e9, 6), "unit": "GB/s", "cores": threads,
+                                  "kind": "oracle", "sample": desc}
+    if dist_on:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,180 @@
+// wq_api.cu -- C ABI of libwq: argument validation, dispatch of the matmul entry
+// points, workspace sizing, error reporting, device properties and TMA descriptors.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "wq_host.h"
+
+namespace wq {
+
+wq_status skinny_gemm(int WB, int AM, const void *A, const float *a_scale, const uint8_t *Wq, const void *scales,
+                      const void *zeros, const void *bias, void *C, int32_t *acc_out, int64_t M, int64_t N, int64_t K,
+                      const wq_qconfig &c, void *ws, size_t ws_bytes, cudaStream_t st);
+size_t skinny_workspace_size(int WB, int AM, int64_t M, int64_t N, int64_t K);
+int skinny_read_error();
+
+namespace {
+thread_local char g_last_error[512] = "";
+}
+
+wq_status fail(wq_status s, const char *fmt, ...)
+{
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_last_error, sizeof g_last_error, fmt, ap);
+    va_end(ap);
+    return s;
+}
+
+wq_status check_launch(const char *what)
+{
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return fail(WQ_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+    return WQ_OK;
+}
+
+const DeviceInfo &device_info()
+{
+    static std::mutex mu;
+    static std::vector<DeviceInfo> cache;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    std::lock_guard<std::mutex> lock(mu);
+    if (int(cache.size()) <= dev) cache.resize(dev + 1);
+    DeviceInfo &d = cache[dev];
+    if (d.device != dev) {
+        d.device = dev;
+        cudaDeviceGetAttribute(&d.sm_count, cudaDevAttrMultiProcessorCount, dev);
+        cudaDeviceGetAttribute(&d.max_smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+        if (d.sm_count <= 0) d.sm_count = 1;
+        if (d.max_smem_optin <= 0) d.max_smem_optin = 48 * 1024;
+    }
+    return d;
+}
+
+namespace {
+using EncodeFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                              const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                              CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeFn encode_fn()
+{
+    static EncodeFn fn = [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q{};
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) !=
+                cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            p = nullptr;
+        return reinterpret_cast<EncodeFn>(p);
+    }();
+    return fn;
+}
+}  // namespace
+
+wq_status encode_tmap_2d(CUtensorMap *map, CUtensorMapDataType dt, const void *base, uint64_t dim0, uint64_t dim1,
+                         uint64_t stride1_bytes, uint32_t box0, uint32_t box1)
+{
+    EncodeFn fn = encode_fn();
+    if (!fn) return fail(WQ_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+    cuuint64_t dims[2] = {dim0, dim1};
+    cuuint64_t strides[1] = {stride1_bytes};
+    cuuint32_t box[2] = {box0, box1};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(map, dt, 2, const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(WQ_ERR_INVALID_ARG, "cuTensorMapEncodeTiled failed (%d)", int(r));
+    return WQ_OK;
+}
+
+int read_device_errors() { return skinny_read_error(); }
+
+namespace {
+
+wq_status check_weights(const uint8_t *Wq, const void *scales, const void *zeros, int64_t M, int64_t N, int64_t K,
+                        const wq_qconfig &c)
+{
+    if (M <= 0 || N <= 0 || K <= 0) return fail(WQ_ERR_INVALID_ARG, "M, N and K must be positive");
+    if (M > 0x7fffffff || N > 0x7fffffff || K > 0x7fffffff) return fail(WQ_ERR_INVALID_ARG, "sizes exceed int32");
+    if (!Wq || !scales) return fail(WQ_ERR_INVALID_ARG, "Wq and scales must be non-null");
+    if (!aligned16(Wq) || !aligned16(scales) || (zeros && !aligned16(zeros)))
+        return fail(WQ_ERR_ALIGNMENT, "Wq, scales and zeros must be 16-byte aligned");
+    if (c.bits == 4) {
+        if (K % 128) return fail(WQ_ERR_INVALID_ARG, "INT4 needs K %% 128 == 0");
+        if (c.group_size <= 0 || K % c.group_size) return fail(WQ_ERR_INVALID_ARG, "K %% group_size != 0");
+        if (c.group_size % 128) return fail(WQ_ERR_UNSUPPORTED, "group_size must be a multiple of 128");
+        if (!c.symmetric && !zeros) return fail(WQ_ERR_INVALID_ARG, "asymmetric INT4 needs zeros");
+    } else if (c.bits == 2) {
+        if (!c.ternary) return fail(WQ_ERR_UNSUPPORTED, "INT2 weights must be ternary");
+        if (K % 64) return fail(WQ_ERR_INVALID_ARG, "INT2 needs K %% 64 == 0");
+    } else {
+        return fail(WQ_ERR_INVALID_ARG, "bits must be 4 or 2");
+    }
+    return WQ_OK;
+}
+
+}  // namespace
+}  // namespace wq
+
+using namespace wq;
+
+extern "C" const char *wq_status_string(wq_status s)
+{
+    switch (s) {
+    case WQ_OK: return "ok";
+    case WQ_ERR_INVALID_ARG: return "invalid argument";
+    case WQ_ERR_ALIGNMENT: return "misaligned pointer";
+    case WQ_ERR_UNSUPPORTED: return "unsupported configuration";
+    case WQ_ERR_CUDA: return "CUDA error";
+    case WQ_ERR_WORKSPACE: return "workspace too small";
+    }
+    return "unknown status";
+}
+
+extern "C" const char *wq_last_error(void) { return g_last_error; }
+
+// Reads and clears the device-side error word (a bounded wait that gave up).
+// Synchronous; for tests and diagnostics.
+extern "C" int wq_device_error(void) { return read_device_errors(); }
+
+extern "C" size_t wq_workspace_size(int64_t M, int64_t N, int64_t K, wq_qconfig c)
+{
+    if (M <= 0 || N <= 0 || K <= 0 || (c.bits != 4 && c.bits != 2)) return 0;
+    // the INT8 path has the smaller activation blocks; size for the larger of the two
+    return std::max(skinny_workspace_size(c.bits, 0, M, N, K), skinny_workspace_size(c.bits, 2, M, N, K));
+}
+
+extern "C" wq_status w4a16_gemm(const void *A, wq_dtype a_dt, const uint8_t *Wq, const void *scales,
+                                const void *zeros, const void *bias, void *C, int64_t M, int64_t N, int64_t K,
+                                wq_qconfig c, void *workspace, size_t ws_bytes, cudaStream_t stream)
+{
+    wq_status rc = check_weights(Wq, scales, zeros, M, N, K, c);
+    if (rc != WQ_OK) return rc;
+    if (a_dt != WQ_F16 && a_dt != WQ_BF16) return fail(WQ_ERR_INVALID_ARG, "a_dt must be WQ_F16 or WQ_BF16");
+    if (!A || !C) return fail(WQ_ERR_INVALID_ARG, "A and C must be non-null");
+    if (!aligned16(A) || !aligned16(C) || (bias && !aligned16(bias)) || (workspace && !aligned16(workspace)))
+        return fail(WQ_ERR_ALIGNMENT, "A, C, bias and workspace must be 16-byte aligned");
+    return skinny_gemm(c.bits, a_dt == WQ_F16 ? 0 : 1, A, nullptr, Wq, scales, c.bits == 4 && !c.symmetric ? zeros : nullptr,
+                       bias, C, nullptr, M, N, K, c, workspace, ws_bytes, stream);
+}
+
+extern "C" wq_status w4a8_gemm(const int8_t *Aq, const float *a_scale, const uint8_t *Wq, const void *scales,
+                               const void *zeros, const void *bias, void *C, int32_t *acc_out, int64_t M, int64_t N,
+                               int64_t K, wq_qconfig c, void *workspace, size_t ws_bytes, cudaStream_t stream)
+{
+    wq_status rc = check_weights(Wq, scales, zeros, M, N, K, c);
+    if (rc != WQ_OK) return rc;
+    if (!Aq || !a_scale || !C) return fail(WQ_ERR_INVALID_ARG, "Aq, a_scale and C must be non-null");
+    if (!aligned16(Aq) || !aligned16(C) || (bias && !aligned16(bias)) || (workspace && !aligned16(workspace)))
+        return fail(WQ_ERR_ALIGNMENT, "Aq, C, bias and workspace must be 16-byte aligned");
+    if (acc_out && c.bits == 4 && c.group_size != 128)
+        return fail(WQ_ERR_UNSUPPORTED, "acc_out needs group_size == 128");
+    return skinny_gemm(c.bits, 2, Aq, a_scale, Wq, scales, c.bits == 4 && !c.symmetric ? zeros : nullptr, bias, C,
+                       acc_out, M, N, K, c, workspace, ws_bytes, stream);
+}

@@ -1,0 +1,36 @@
+// wq_host.h -- host-side helpers shared by the libwq translation units:
+// status reporting, argument checks, device properties and TMA descriptors.
+#pragma once
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <cstdarg>
+#include <cstdio>
+
+#include "../../include/wq.h"
+
+namespace wq {
+
+// Records a one-line reason for the calling thread and returns the status.
+wq_status fail(wq_status s, const char *fmt, ...);
+wq_status check_launch(const char *what);
+
+inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+struct DeviceInfo {
+    int device = -1;
+    int sm_count = 0;
+    int max_smem_optin = 0;  // bytes of shared memory a block may opt in to
+};
+// Properties of the current device (cached per device).
+const DeviceInfo &device_info();
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no libcuda link).
+wq_status encode_tmap_2d(CUtensorMap *map, CUtensorMapDataType dt, const void *base, uint64_t dim0,
+                         uint64_t dim1, uint64_t stride1_bytes, uint32_t box0, uint32_t box1);
+
+// Reads (and clears) the device error words of all kernels with bounded waits.
+int read_device_errors();
+
+}  // namespace wq

@@ -1,0 +1,374 @@
+// wq_quant.cu -- weight quantization / packing, unpacking and per-token INT8
+// activation quantization for sm_100a.
+//
+// Sources: "Accelerating LLM inference with CUDA Graph and INT4 quantization"
+// (cnblogs), part 1: step 1 (absmax scale, round, clip, two INT4 per byte) and
+// step 2 (q = round(a / a_scale)); "BitBLAS practical guide: mixed-precision
+// compute in vLLM" (mlqm): "Advanced features 2" (group_size 128, scales,
+// "original" zero points) and the BitNet-b1.58 ternary weights of "Real-world case".
+//
+// Every decision that turns a float into an integer code is taken in binary32
+// with IEEE division (__fdiv_rn) and round-half-to-even (rintf), and the scale is
+// rounded to binary16 (RNE) before it is used, so the codes are bit-exact with
+// any other implementation of the same readings.
+#include <cuda_fp16.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include <algorithm>
+
+#include "wq_host.h"
+
+namespace wq {
+namespace {
+
+template <typename T>
+__device__ __forceinline__ float to_f(T v);
+template <>
+__device__ __forceinline__ float to_f<float>(float v) { return v; }
+template <>
+__device__ __forceinline__ float to_f<__half>(__half v) { return __half2float(v); }
+template <>
+__device__ __forceinline__ float to_f<__nv_bfloat16>(__nv_bfloat16 v) { return __bfloat162float(v); }
+
+// Four consecutive elements (the pointer is aligned to four elements).
+template <typename T>
+__device__ __forceinline__ void load4(const T *p, float (&v)[4])
+{
+#pragma unroll
+    for (int i = 0; i < 4; ++i) v[i] = to_f(p[i]);
+}
+template <>
+__device__ __forceinline__ void load4<float>(const float *p, float (&v)[4])
+{
+    float4 x = __ldg(reinterpret_cast<const float4 *>(p));
+    v[0] = x.x; v[1] = x.y; v[2] = x.z; v[3] = x.w;
+}
+
+__device__ __forceinline__ float clampf(float v, float lo, float hi) { return fminf(fmaxf(v, lo), hi); }
+
+__device__ __forceinline__ float warp_max(float v)
+{
+#pragma unroll
+    for (int o = 16; o; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    return v;
+}
+__device__ __forceinline__ float warp_min(float v)
+{
+#pragma unroll
+    for (int o = 16; o; o >>= 1) v = fminf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    return v;
+}
+
+// One warp per (row n, group g).  Lane l handles elements c*128 + 4l .. +3 of the
+// group for each 128-chunk c, and writes their four nibbles as two bytes.
+template <typename T, bool kSym>
+__global__ void __launch_bounds__(256) quant_int4_kernel(const T *__restrict__ W, int64_t N, int64_t K, int gs,
+                                                         uint8_t *__restrict__ Wq, __half *__restrict__ scales,
+                                                         __half *__restrict__ zeros)
+{
+    const int64_t G = K / gs;
+    const int64_t warp = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+    const int lane = threadIdx.x & 31;
+    if (warp >= N * G) return;
+    const int64_t n = warp / G, g = warp % G;
+    const T *w = W + n * K + g * gs;
+    const int chunks = gs / 128;
+
+    float amax = 0.f, mn = 0.f, mx = 0.f;
+    for (int c = 0; c < chunks; ++c) {
+        float v[4];
+        load4(w + c * 128 + 4 * lane, v);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            amax = fmaxf(amax, fabsf(v[i]));
+            mn = fminf(mn, v[i]);
+            mx = fmaxf(mx, v[i]);
+        }
+    }
+    float s, z = 0.f;
+    __half sh;
+    if (kSym) {
+        amax = warp_max(amax);
+        sh = __float2half_rn(__fdiv_rn(amax, 7.0f));
+        s = __half2float(sh);
+    } else {
+        mn = warp_min(mn);   // the range always contains 0
+        mx = warp_max(mx);
+        sh = __float2half_rn(__fdiv_rn(__fsub_rn(mx, mn), 15.0f));
+        s = __half2float(sh);
+        if (s != 0.f) z = clampf(rintf(__fdiv_rn(-mn, s)), 0.f, 15.f);
+    }
+    if (lane == 0) {
+        scales[n * G + g] = sh;
+        if (!kSym) zeros[n * G + g] = __float2half_rn(z);
+    }
+    for (int c = 0; c < chunks; ++c) {
+        float v[4];
+        load4(w + c * 128 + 4 * lane, v);
+        uint32_t packed = 0;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            float q = 0.f;
+            if (s != 0.f) {
+                if (kSym) q = clampf(rintf(__fdiv_rn(v[i], s)), -7.f, 7.f);
+                else q = clampf(__fadd_rn(rintf(__fdiv_rn(v[i], s)), z), 0.f, 15.f);
+            }
+            uint32_t field = kSym ? uint32_t(int(q) + 8) : uint32_t(int(q));
+            packed |= field << (4 * i);
+        }
+        uint8_t *dst = Wq + n * (K / 2) + (g * gs + c * 128 + 4 * lane) / 2;
+        *reinterpret_cast<uint16_t *>(dst) = uint16_t(packed);
+    }
+}
+
+// ---- ternary: exact mean |w| via per-exponent integer bins ----------------
+// |w| = m * 2^(E-149) with integer m < 2^24 and E = max(biased exponent, 1) - 1,
+// so sum|w| = (sum_E bins[E] * 2^E) * 2^-149 exactly, where bins[E] sums the m's.
+constexpr int kBins = 256;
+
+template <typename T>
+__global__ void __launch_bounds__(256) abs_bins_kernel(const T *__restrict__ W, int64_t count,
+                                                       unsigned long long *__restrict__ gbins)
+{
+    __shared__ unsigned long long bins[kBins];
+    for (int i = threadIdx.x; i < kBins; i += blockDim.x) bins[i] = 0;
+    __syncthreads();
+    const int64_t stride = int64_t(gridDim.x) * blockDim.x;
+    for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i - threadIdx.x < count; i += stride) {
+        const bool live = i < count;
+        uint32_t u = live ? __float_as_uint(to_f(W[i])) : 0u;
+        uint32_t be = (u >> 23) & 0xffu, frac = u & 0x7fffffu;
+        uint32_t m = be ? (frac | 0x800000u) : frac;
+        int E = (be ? int(be) : 1) - 1;
+        // lanes that share an exponent add their mantissas once
+        const unsigned act = __activemask();
+        unsigned same = __match_any_sync(act, E);
+        unsigned sum = __reduce_add_sync(same, m);  // at most 32 * 2^24 < 2^32
+        if ((threadIdx.x & 31) == __ffs(same) - 1 && sum) atomicAdd(&bins[E], (unsigned long long)sum);
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < kBins; i += blockDim.x)
+        if (bins[i]) atomicAdd(&gbins[i], bins[i]);
+}
+
+// One thread: the exact integer sum, rounded once to binary64 (ties to even),
+// divided by the count in binary64, rounded to binary32.  Clears the bins.
+__global__ void ternary_scale_kernel(unsigned long long *__restrict__ gbins, int64_t count, float *__restrict__ scale)
+{
+    if (threadIdx.x != 0 || blockIdx.x != 0) return;
+    unsigned long long limb[12] = {0};
+    for (int e = 0; e < kBins; ++e) {
+        unsigned long long v = gbins[e];
+        gbins[e] = 0;
+        if (!v) continue;
+        unsigned __int128 x = (unsigned __int128)v << (e & 31);
+        int j = e >> 5;
+        limb[j] += (uint32_t)x;
+        limb[j + 1] += (uint32_t)(x >> 32);
+        limb[j + 2] += (uint32_t)(x >> 64);
+    }
+    for (int j = 0; j < 11; ++j) {
+        limb[j + 1] += limb[j] >> 32;
+        limb[j] &= 0xffffffffull;
+    }
+    int top = -1;
+    for (int j = 11; j >= 0 && top < 0; --j)
+        if (limb[j]) top = 32 * j + 63 - __clzll(limb[j]);
+    double sum;
+    if (top < 0) {
+        sum = 0.0;
+    } else {
+        auto bit = [&](int p) -> unsigned long long { return p < 0 ? 0ull : (limb[p >> 5] >> (p & 31)) & 1ull; };
+        int lo = top - 52;
+        unsigned long long mant = 0;
+        for (int p = top; p >= (lo > 0 ? lo : 0); --p) mant = (mant << 1) | bit(p);
+        if (lo <= 0) {
+            sum = scalbn((double)mant, -149);
+        } else {
+            unsigned long long rb = bit(lo - 1), sticky = 0;
+            for (int p = lo - 2; p >= 0 && !sticky; --p) sticky |= bit(p);
+            if (rb && (sticky || (mant & 1))) ++mant;
+            sum = scalbn((double)mant, lo - 149);
+        }
+    }
+    scale[0] = __double2float_rn(__ddiv_rn(sum, (double)count));
+}
+
+// 16 consecutive elements per thread -> 4 bytes of 2-bit codes.
+template <typename T>
+__global__ void __launch_bounds__(256) pack_ternary_kernel(const T *__restrict__ W, int64_t count,
+                                                           const float *__restrict__ scale, uint8_t *__restrict__ Wq)
+{
+    const int64_t t = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (t * 16 >= count) return;
+    const float s = *scale;
+    uint32_t word = 0;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+        float v[4];
+        load4(W + t * 16 + 4 * c, v);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            float q = s != 0.f ? clampf(rintf(__fdiv_rn(v[i], s)), -1.f, 1.f) : 0.f;
+            word |= (uint32_t(int(q)) & 3u) << (2 * (4 * c + i));
+        }
+    }
+    reinterpret_cast<uint32_t *>(Wq)[t] = word;
+}
+
+__global__ void __launch_bounds__(256) unpack_kernel(const uint8_t *__restrict__ Wq, int64_t nbytes, int bits, int sym,
+                                                     int8_t *__restrict__ q)
+{
+    const int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (i >= nbytes) return;
+    const uint32_t b = Wq[i];
+    if (bits == 4) {
+        int lo = b & 15, hi = b >> 4;
+        q[2 * i] = int8_t(sym ? lo - 8 : lo);
+        q[2 * i + 1] = int8_t(sym ? hi - 8 : hi);
+    } else {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            int f = (b >> (2 * j)) & 3;
+            q[4 * i + j] = int8_t(f >= 2 ? f - 4 : f);
+        }
+    }
+}
+
+// One block per token row: absmax, a_scale = absmax / 127, codes.  8 elements per access.
+template <typename T>
+__global__ void __launch_bounds__(256) act_quant_kernel(const T *__restrict__ A, int64_t K, int8_t *__restrict__ Aq,
+                                                        float *__restrict__ a_scale)
+{
+    const int64_t m = blockIdx.x;
+    const T *a = A + m * K;
+    const int64_t K8 = K / 8;
+    float amax = 0.f;
+    for (int64_t j = threadIdx.x; j < K8; j += blockDim.x) {
+        uint4 raw = __ldg(reinterpret_cast<const uint4 *>(a) + j);
+        const T *e = reinterpret_cast<const T *>(&raw);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(to_f(e[i])));
+    }
+    __shared__ float red[32];
+    amax = warp_max(amax);
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = amax;
+    __syncthreads();
+    if (threadIdx.x < 32) {
+        float v = threadIdx.x < (blockDim.x >> 5) ? red[threadIdx.x] : 0.f;
+        v = warp_max(v);
+        if (threadIdx.x == 0) red[0] = v;
+    }
+    __syncthreads();
+    const float sc = __fdiv_rn(red[0], 127.0f);
+    if (threadIdx.x == 0) a_scale[m] = sc;
+    for (int64_t j = threadIdx.x; j < K8; j += blockDim.x) {
+        uint4 raw = __ldg(reinterpret_cast<const uint4 *>(a) + j);
+        const T *e = reinterpret_cast<const T *>(&raw);
+        uint32_t w[2] = {0, 0};
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            float q = sc != 0.f ? clampf(rintf(__fdiv_rn(to_f(e[i]), sc)), -127.f, 127.f) : 0.f;
+            w[i / 4] |= (uint32_t(int(q)) & 0xffu) << (8 * (i % 4));
+        }
+        reinterpret_cast<uint2 *>(Aq + m * K)[j] = make_uint2(w[0], w[1]);
+    }
+}
+
+int blocks_for(int64_t threads, int per_block = 256) { return int((threads + per_block - 1) / per_block); }
+
+template <typename T>
+wq_status quantize_typed(const T *W, int64_t N, int64_t K, wq_qconfig c, uint8_t *Wq, void *scales, void *zeros,
+                         void *ws, size_t ws_bytes, cudaStream_t st)
+{
+    if (c.bits == 4) {
+        const int64_t G = K / c.group_size;
+        const int64_t warps = N * G;
+        const int grid = blocks_for(warps * 32);
+        if (c.symmetric)
+            quant_int4_kernel<T, true><<<grid, 256, 0, st>>>(W, N, K, c.group_size, Wq,
+                                                             static_cast<__half *>(scales), nullptr);
+        else
+            quant_int4_kernel<T, false><<<grid, 256, 0, st>>>(W, N, K, c.group_size, Wq,
+                                                              static_cast<__half *>(scales),
+                                                              static_cast<__half *>(zeros));
+        return check_launch("quant_int4_kernel");
+    }
+    // ternary
+    auto *bins = static_cast<unsigned long long *>(ws);
+    if (!bins || ws_bytes < kBins * sizeof(unsigned long long))
+        return fail(WQ_ERR_WORKSPACE, "ternary quantization needs %zu bytes of workspace",
+                    size_t(kBins * sizeof(unsigned long long)));
+    const int64_t count = N * K;
+    if (cudaMemsetAsync(bins, 0, kBins * sizeof(unsigned long long), st) != cudaSuccess)
+        return check_launch("cudaMemsetAsync(bins)");
+    const int grid = int(std::min<int64_t>(4 * device_info().sm_count, blocks_for(count)));
+    abs_bins_kernel<T><<<grid, 256, 0, st>>>(W, count, bins);
+    ternary_scale_kernel<<<1, 32, 0, st>>>(bins, count, static_cast<float *>(scales));
+    pack_ternary_kernel<T><<<blocks_for(count / 16), 256, 0, st>>>(W, count, static_cast<const float *>(scales), Wq);
+    return check_launch("ternary quantization kernels");
+}
+
+}  // namespace
+}  // namespace wq
+
+using namespace wq;
+
+extern "C" size_t wq_quantize_workspace_size(int64_t, int64_t, wq_qconfig c)
+{
+    return c.bits == 2 ? kBins * sizeof(unsigned long long) : 0;
+}
+
+extern "C" wq_status wq_quantize_pack(const void *W, wq_dtype w_dt, int64_t N, int64_t K, wq_qconfig c, uint8_t *Wq,
+                                      void *scales, void *zeros, void *workspace, size_t ws_bytes,
+                                      cudaStream_t stream)
+{
+    if (N <= 0 || K <= 0) return fail(WQ_ERR_INVALID_ARG, "N and K must be positive");
+    if (!W || !Wq || !scales) return fail(WQ_ERR_INVALID_ARG, "W, Wq and scales must be non-null");
+    if (w_dt != WQ_F32 && w_dt != WQ_F16 && w_dt != WQ_BF16)
+        return fail(WQ_ERR_INVALID_ARG, "w_dt must be WQ_F32, WQ_F16 or WQ_BF16");
+    if (!aligned16(W) || !aligned16(Wq) || (zeros && !aligned16(zeros)) || !aligned16(scales))
+        return fail(WQ_ERR_ALIGNMENT, "device pointers must be 16-byte aligned");
+    if (c.bits == 4) {
+        if (c.group_size <= 0 || K % c.group_size) return fail(WQ_ERR_INVALID_ARG, "K %% group_size != 0");
+        if (c.group_size % 128) return fail(WQ_ERR_UNSUPPORTED, "group_size must be a multiple of 128");
+        if (!c.symmetric && !zeros) return fail(WQ_ERR_INVALID_ARG, "asymmetric INT4 needs a zeros buffer");
+    } else if (c.bits == 2) {
+        if (!c.ternary) return fail(WQ_ERR_UNSUPPORTED, "INT2 weights are produced by the ternary quantizer only");
+        if (K % 64) return fail(WQ_ERR_INVALID_ARG, "INT2 needs K %% 64 == 0");
+    } else {
+        return fail(WQ_ERR_INVALID_ARG, "bits must be 4 or 2");
+    }
+    switch (w_dt) {
+    case WQ_F32: return quantize_typed(static_cast<const float *>(W), N, K, c, Wq, scales, zeros, workspace, ws_bytes, stream);
+    case WQ_F16: return quantize_typed(static_cast<const __half *>(W), N, K, c, Wq, scales, zeros, workspace, ws_bytes, stream);
+    default: return quantize_typed(static_cast<const __nv_bfloat16 *>(W), N, K, c, Wq, scales, zeros, workspace, ws_bytes, stream);
+    }
+}
+
+extern "C" wq_status wq_unpack(const uint8_t *Wq, int64_t N, int64_t K, wq_qconfig c, int8_t *q, cudaStream_t stream)
+{
+    if (N <= 0 || K <= 0 || !Wq || !q) return fail(WQ_ERR_INVALID_ARG, "bad sizes or null pointer");
+    if (c.bits != 4 && c.bits != 2) return fail(WQ_ERR_INVALID_ARG, "bits must be 4 or 2");
+    if (K % (8 / c.bits)) return fail(WQ_ERR_INVALID_ARG, "K must fill whole bytes");
+    const int64_t nbytes = N * K * c.bits / 8;
+    unpack_kernel<<<blocks_for(nbytes), 256, 0, stream>>>(Wq, nbytes, c.bits, c.bits == 4 ? c.symmetric : 1, q);
+    return check_launch("unpack_kernel");
+}
+
+extern "C" wq_status act_quant_int8(const void *A, wq_dtype a_dt, int64_t M, int64_t K, int8_t *Aq, float *a_scale,
+                                    cudaStream_t stream)
+{
+    if (M <= 0 || K <= 0 || !A || !Aq || !a_scale) return fail(WQ_ERR_INVALID_ARG, "bad sizes or null pointer");
+    if (a_dt != WQ_F16 && a_dt != WQ_BF16) return fail(WQ_ERR_INVALID_ARG, "a_dt must be WQ_F16 or WQ_BF16");
+    if (K % 8) return fail(WQ_ERR_INVALID_ARG, "K %% 8 != 0");
+    if (!aligned16(A) || !aligned16(Aq)) return fail(WQ_ERR_ALIGNMENT, "A and Aq must be 16-byte aligned");
+    if (M > 0x7fffffff) return fail(WQ_ERR_INVALID_ARG, "M too large");
+    if (a_dt == WQ_F16)
+        act_quant_kernel<__half><<<unsigned(M), 256, 0, stream>>>(static_cast<const __half *>(A), K, Aq, a_scale);
+    else
+        act_quant_kernel<__nv_bfloat16><<<unsigned(M), 256, 0, stream>>>(static_cast<const __nv_bfloat16 *>(A), K, Aq,
+                                                                         a_scale);
+    return check_launch("act_quant_kernel");
+}

@@ -1,0 +1,158 @@
+/*
+ * wq.h -- C ABI of libwq: INT4 / INT2 weight-quantized matmul on NVIDIA B200 (sm_100a).
+ *
+ * The operation (statement of the problem in "BitBLAS practical guide: mixed-precision
+ * compute in vLLM" (mlqm), section "What is BitBLAS"):
+ *
+ *     C[M,N] = A[M,K] x dequant(Wq[N,K])^T          (layout "nt": A and W both K-contiguous,
+ *                                                    section "Advanced features 1")
+ *
+ * with packed low-bit weights Wq, per-group scales and optional zero points
+ * (section "Advanced features 2, weight group quantization": group_size 128, with_scaling,
+ * with_zeros, zeros_mode "original"), in two activation paths:
+ *
+ *   W4A16  FP16 / BF16 activations; weights dequantized in registers; FP32 accumulation.
+ *   W4A8   per-token INT8 activations ("Accelerating LLM inference with CUDA Graph and INT4
+ *          quantization" (cnblogs), part 1, step 2); exact INT32 accumulation of integer
+ *          dot products (step 3, the DP4A definition c += a0*b0 + ... + a3*b3); then the
+ *          float dequantization by weight_scale x activation_scale and an optional bias
+ *          (steps 3-4).
+ *
+ * and the same two paths for ternary / INT2 weights with one scale per tensor
+ * (BitBLAS guide, "Core advantages 2" FP16xINT2 and INT8xINT2, "Real-world case"
+ * BitNet-b1.58).
+ *
+ * Data formats (fixed):
+ *   - all matrices row-major; A [M,K], W [N,K], C [M,N];
+ *   - INT4: byte j of a row holds element 2j in bits 0..3 and element 2j+1 in bits 4..7;
+ *     symmetric weights store q + 8 (q in [-7,7]); asymmetric weights store q in [0,15]
+ *     and dequantize as (q - z) * s;
+ *   - INT2 (ternary): element 4j+i in bits 2i..2i+1 of byte j, 2-bit two's complement;
+ *   - scales / zeros: binary16 [N, K/group_size] row-major (INT4); one binary32 (INT2).
+ *
+ * Quantization readings (the pages print an INT8 range inside the INT4 passage):
+ *   symmetric  s = fp16(absmax/7), q = clip(rint(w/s), -7, 7);
+ *   asymmetric s = fp16((max(w,0) - min(w,0))/15), z = clip(rint(-min/s), 0, 15),
+ *              q = clip(rint(w/s) + z, 0, 15);
+ *   ternary    s = mean|w| (exact sum rounded once to binary64, / count, -> binary32),
+ *              q = clip(rint(w/s), -1, 1);
+ *   activations a_scale[m] = absmax_k|A[m,k]| / 127 (binary32), Aq = clip(rint(A/a_scale), -127, 127).
+ * rint is round-half-to-even; divisions are IEEE binary32 divisions; the stored binary16 scale
+ * is the one used to quantize.  Scale 0 gives code 0.
+ *
+ * Conventions for every entry point:
+ *   - Pointers named W, A, Aq, a_scale, Wq, scales, zeros, bias, C, acc_out, q, workspace are
+ *     DEVICE pointers owned by the caller; the library never allocates, frees or keeps them.
+ *   - Every call is asynchronous on `stream` (0 = legacy default stream): it validates its
+ *     arguments on the host, enqueues its kernels and returns.  No call synchronizes.
+ *   - Argument errors return before anything is enqueued: WQ_ERR_INVALID_ARG (bad sizes,
+ *     null required pointer, unsupported combination of flags), WQ_ERR_ALIGNMENT (a device
+ *     pointer not 16-byte aligned), WQ_ERR_UNSUPPORTED (a valid request this build does not
+ *     implement, e.g. a group size that is not a multiple of 128).  A failed launch returns
+ *     WQ_ERR_CUDA.  wq_last_error() gives a one-line reason for the calling thread.
+ *   - Nothing traps on the device.
+ */
+#ifndef WQ_H
+#define WQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    WQ_OK = 0,
+    WQ_ERR_INVALID_ARG = 1,
+    WQ_ERR_ALIGNMENT = 2,
+    WQ_ERR_UNSUPPORTED = 3,
+    WQ_ERR_CUDA = 4,
+    WQ_ERR_WORKSPACE = 5
+} wq_status;
+
+typedef enum { WQ_F32 = 0, WQ_F16 = 1, WQ_BF16 = 2, WQ_I8 = 3, WQ_I32 = 4 } wq_dtype;
+
+typedef struct {
+    int32_t bits;        /* 4 (INT4) or 2 (INT2 / ternary)                                    */
+    int32_t group_size;  /* INT4: elements of K per scale, a multiple of 128 dividing K;     */
+                         /*       K itself means one scale per output channel.              */
+                         /* INT2: ignored (one scale per tensor).                          */
+    int32_t symmetric;   /* INT4: 1 = symmetric (q + 8 stored, no zeros), 0 = zero points.  */
+    int32_t ternary;     /* INT2: must be 1 (codes -1, 0, 1 from the ternary quantizer).    */
+} wq_qconfig;
+
+/* Weight quantization and packing ("Accelerating LLM inference with CUDA Graph and INT4
+ * quantization", part 1, step 1; BitBLAS guide, "Advanced features 2").
+ *   W       [N,K] device, dtype w_dt in {WQ_F32, WQ_F16, WQ_BF16}.
+ *   Wq      [N, K*bits/8] bytes, device, written.
+ *   scales  INT4: binary16 [N, K/group_size]; INT2: one binary32. Written.
+ *   zeros   INT4 asymmetric: binary16 [N, K/group_size] (integers 0..15), written; else NULL.
+ *   workspace / ws_bytes: scratch for the INT2 per-tensor mean (wq_quantize_workspace_size
+ *   bytes); unused for INT4 (may be NULL).
+ * Requires K % group_size == 0 (INT4) or K % 64 == 0 (INT2), N >= 1, K >= 1.
+ * Bit-exact with the CPU reference of the same readings. */
+wq_status wq_quantize_pack(const void *W, wq_dtype w_dt, int64_t N, int64_t K, wq_qconfig c,
+                           uint8_t *Wq, void *scales, void *zeros,
+                           void *workspace, size_t ws_bytes, cudaStream_t stream);
+size_t wq_quantize_workspace_size(int64_t N, int64_t K, wq_qconfig c);
+
+/* Inverse of the packing: signed codes q [N,K] int8 (symmetric INT4: nibble - 8; asymmetric
+ * INT4: nibble; INT2: two's complement).  For tests and debugging ("Accelerating LLM
+ * inference...", part 1, step 3: unpack each byte into two INT4 values). */
+wq_status wq_unpack(const uint8_t *Wq, int64_t N, int64_t K, wq_qconfig c, int8_t *q,
+                    cudaStream_t stream);
+
+/* Per-token dynamic INT8 activation quantization ("Accelerating LLM inference...", part 1,
+ * step 2).  A [M,K] binary16 or bfloat16 (a_dt); Aq [M,K] int8 and a_scale [M] binary32
+ * written.  K % 8 == 0.  Bit-exact with the CPU reference. */
+wq_status act_quant_int8(const void *A, wq_dtype a_dt, int64_t M, int64_t K,
+                         int8_t *Aq, float *a_scale, cudaStream_t stream);
+
+/* W4A16 (and W2A16):  C[m,n] = sum_k A[m,k] * (q[n,k] - z[n,g]) * s[n,g]  (+ bias[n]),
+ * accumulated in binary32 and rounded once to a_dt.
+ *   A      [M,K] a_dt in {WQ_F16, WQ_BF16};  C [M,N] a_dt;  bias [N] a_dt or NULL.
+ *   Wq, scales, zeros as written by wq_quantize_pack (zeros NULL unless asymmetric INT4).
+ *   workspace: device scratch of at least wq_workspace_size(M,N,K,c) bytes, ZERO-FILLED
+ *   before its first use; every call returns it to all-zero when its kernels finish.  A
+ *   workspace that is NULL or too small is allowed: the call then uses a launch plan that
+ *   needs none (possibly slower).  Calls that share one workspace must not overlap.
+ * Requires K % 128 == 0 for INT4 (K % 64 == 0 for INT2), M, N >= 1. */
+wq_status w4a16_gemm(const void *A, wq_dtype a_dt, const uint8_t *Wq, const void *scales,
+                     const void *zeros, const void *bias, void *C,
+                     int64_t M, int64_t N, int64_t K, wq_qconfig c,
+                     void *workspace, size_t ws_bytes, cudaStream_t stream);
+
+/* W4A8 (and W2A8):
+ *   acc_g[m,n] = sum_{k in group g} Aq[m,k] * (q[n,k] - z[n,g])        exact INT32
+ *   C[m,n]     = fp16( a_scale[m] * sum_g s[n,g] * acc_g[m,n]  (+ bias[n]) )
+ * INT2 weights have a single group spanning K and a single binary32 scale.
+ *   Aq [M,K] int8, a_scale [M] binary32 (from act_quant_int8); C [M,N] binary16;
+ *   bias [N] binary16 or NULL; zeros (asymmetric INT4) must hold integers.
+ *   acc_out: NULL, or int32 [M, N, G] receiving every acc_g (G = K/128 for INT4, which
+ *   then requires group_size == 128; G = 1 for INT2), bit-exact with the CPU reference.
+ *   workspace: as for w4a16_gemm. */
+wq_status w4a8_gemm(const int8_t *Aq, const float *a_scale, const uint8_t *Wq, const void *scales,
+                    const void *zeros, const void *bias, void *C, int32_t *acc_out,
+                    int64_t M, int64_t N, int64_t K, wq_qconfig c,
+                    void *workspace, size_t ws_bytes, cudaStream_t stream);
+
+/* Bytes of workspace that lets w4a16_gemm / w4a8_gemm use their split-K plans on the
+ * current device. */
+size_t wq_workspace_size(int64_t M, int64_t N, int64_t K, wq_qconfig c);
+
+const char *wq_status_string(wq_status s);
+
+/* Reads and clears the library's device-side error word.  Non-zero (1) means that a
+ * kernel gave up a bounded wait on one of its own barriers (about 2 s) and returned
+ * early, so its outputs are not valid.  Synchronous (device-to-host copy of one word);
+ * for tests and diagnostics. */
+int wq_device_error(void);
+/* One-line reason for the last non-OK status returned on the calling thread. */
+const char *wq_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* WQ_H */

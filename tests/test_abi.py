@@ -1,0 +1,105 @@
+"""The C ABI library loads on a machine without a GPU, exports every entry point
+declared in include/wq.h, and rejects bad arguments on the host before touching the
+device (no kernel is launched by these tests)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import gemv_wq_quantize_b200 as wq
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "wq.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?\w+\s*\*?\s*(\w+)\s*\(", text, flags=re.M)) - {"if"})
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from gemv_wq_quantize_b200 import build
+    build.build(quiet=True)
+    return wq.load_library()
+
+
+def test_header_declares_the_five_entry_points():
+    names = declared_functions()
+    for n in ("wq_quantize_pack", "wq_unpack", "act_quant_int8", "w4a16_gemm", "w4a8_gemm"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    names = declared_functions()
+    assert len(names) >= 9
+    for n in names:
+        assert hasattr(lib, n), n
+        assert ctypes.cast(getattr(lib, n), ctypes.c_void_p).value
+
+
+def test_status_strings(lib):
+    for s in range(6):
+        assert lib.wq_status_string(s)
+
+
+FAKE = ctypes.c_void_p(0x10000)        # aligned, never dereferenced: validation fails first
+FAKE_MIS = ctypes.c_void_p(0x10008)    # 8-byte aligned only
+
+
+def _qc(bits=4, gs=128, sym=1):
+    return wq.QConfig(bits, gs, sym, int(bits == 2))
+
+
+@pytest.mark.parametrize("M,N,K,qc,code", [
+    (0, 128, 128, _qc(), wq.WQ_ERR_INVALID_ARG),
+    (1, 0, 128, _qc(), wq.WQ_ERR_INVALID_ARG),
+    (1, 128, 100, _qc(), wq.WQ_ERR_INVALID_ARG),           # K % 128
+    (1, 128, 384, _qc(gs=256), wq.WQ_ERR_INVALID_ARG),     # K % group_size
+    (1, 128, 256, _qc(gs=64), wq.WQ_ERR_INVALID_ARG),      # K % 128 ok, group 64 -> K%g ok but unsupported
+    (1, 128, 256, _qc(bits=3), wq.WQ_ERR_INVALID_ARG),
+    (1, 128, 96, _qc(bits=2), wq.WQ_ERR_INVALID_ARG),      # INT2 K % 64
+    (1, 128, 256, _qc(sym=0), wq.WQ_ERR_INVALID_ARG),      # asymmetric without zeros
+])
+def test_w4a16_rejects_bad_arguments(lib, M, N, K, qc, code):
+    rc = lib.w4a16_gemm(FAKE, wq.WQ_F16, FAKE, FAKE, None, None, FAKE, M, N, K, qc, None, 0, None)
+    if qc.group_size == 64 and qc.bits == 4:
+        assert rc == wq.WQ_ERR_UNSUPPORTED
+    else:
+        assert rc == code
+    assert lib.wq_last_error()
+
+
+def test_alignment_and_null_checks(lib):
+    qc = _qc()
+    assert lib.w4a16_gemm(FAKE, wq.WQ_F16, FAKE_MIS, FAKE, None, None, FAKE, 1, 128, 128, qc, None, 0, None) \
+        == wq.WQ_ERR_ALIGNMENT
+    assert lib.w4a16_gemm(None, wq.WQ_F16, FAKE, FAKE, None, None, FAKE, 1, 128, 128, qc, None, 0, None) \
+        == wq.WQ_ERR_INVALID_ARG
+    assert lib.w4a16_gemm(FAKE, wq.WQ_I8, FAKE, FAKE, None, None, FAKE, 1, 128, 128, qc, None, 0, None) \
+        == wq.WQ_ERR_INVALID_ARG
+    assert lib.w4a8_gemm(FAKE, None, FAKE, FAKE, None, None, FAKE, None, 1, 128, 128, qc, None, 0, None) \
+        == wq.WQ_ERR_INVALID_ARG
+    assert lib.w4a8_gemm(FAKE, FAKE, FAKE, FAKE, None, None, FAKE, FAKE, 1, 128, 256, _qc(gs=256), None, 0,
+                         None) == wq.WQ_ERR_UNSUPPORTED      # acc_out needs 128-groups
+    assert lib.act_quant_int8(FAKE, wq.WQ_F16, 1, 100, FAKE, FAKE, None) == wq.WQ_ERR_INVALID_ARG
+    assert lib.act_quant_int8(FAKE_MIS, wq.WQ_F16, 1, 128, FAKE, FAKE, None) == wq.WQ_ERR_ALIGNMENT
+    assert lib.wq_quantize_pack(FAKE, wq.WQ_I8, 4, 128, qc, FAKE, FAKE, None, None, 0, None) \
+        == wq.WQ_ERR_INVALID_ARG
+    # ternary quantization needs its scratch for the exact mean
+    assert lib.wq_quantize_pack(FAKE, wq.WQ_F32, 4, 128, _qc(bits=2, sym=1), FAKE, FAKE, None, None, 0, None) \
+        == wq.WQ_ERR_WORKSPACE
+    assert lib.wq_unpack(FAKE, 4, 7, qc, FAKE, None) == wq.WQ_ERR_INVALID_ARG
+
+
+def test_quantize_workspace_size(lib):
+    assert lib.wq_quantize_workspace_size(4, 128, _qc()) == 0
+    assert lib.wq_quantize_workspace_size(4, 128, _qc(bits=2)) >= 2048
+
+
+def test_binding_refuses_cpu_tensors(lib):
+    import torch
+    with pytest.raises(ValueError):
+        wq.act_quant_int8(torch.zeros(2, 128, dtype=torch.float16))

@@ -1,0 +1,282 @@
+"""GPU parity: the CUDA path (through the C ABI) against the CPU oracle, on the same
+seeded inputs.
+
+* quantization, packing, unpacking, activation quantization and the W4A8 INT32
+  group sums: bit-exact;
+* matmul outputs: relative Frobenius error ||C_gpu - C_ref||_F / ||C_ref||_F <= 1e-3,
+  computed in float64 over the output-dtype values (the bound stated for the FP paths).
+
+Small cases run the oracle on every output and cover several 128-row tiles, ragged
+N / M / K tails, bias, zero groups and both launch plans (with and without split-K
+workspace); full-size cases (the Llama-7B / BitNet-3B shapes) compare sampled outputs.
+"""
+import numpy as np
+import pytest
+import torch
+
+import gemv_wq_quantize_b200 as wq
+import oracle
+import wq_synth
+
+pytestmark = pytest.mark.gpu
+
+TOL = 1e-3
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from gemv_wq_quantize_b200 import build
+    build.build(quiet=True)
+    wq.load_library()
+    oracle.build()
+    yield
+    torch.cuda.synchronize()
+    assert wq.device_error() == 0
+
+
+def bits_np(t: torch.Tensor) -> np.ndarray:
+    return t.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+def out_f64(bits: np.ndarray, dtype) -> np.ndarray:
+    if dtype == torch.bfloat16:
+        return oracle.bf16_bits_to_f64(bits)
+    return bits.view(np.float16).astype(np.float64)
+
+
+def rel_fro(gpu_bits, ref_bits, dtype) -> float:
+    g, r = out_f64(gpu_bits, dtype), out_f64(ref_bits, dtype)
+    den = np.linalg.norm(r)
+    return float(np.linalg.norm(g - r) / den) if den > 0 else float(np.linalg.norm(g))
+
+
+def qc_of(quant, gs=128):
+    if quant == "tern2":
+        return wq.QuantConfig(bits=2)
+    return wq.QuantConfig(bits=4, group_size=gs, symmetric=(quant == "sym4"))
+
+
+def quantize_both(W_cpu, qc):
+    """GPU quantization, asserted bit-exact against the oracle's; returns the GPU tensors."""
+    Wq, s, z = wq.quantize_pack(W_cpu.cuda(), qc)
+    torch.cuda.synchronize()
+    if qc.bits == 2:
+        oWq, os_ = oracle.quantize_ternary(W_cpu.numpy())
+        assert np.array_equal(Wq.cpu().numpy(), oWq)
+        assert np.array_equal(s.cpu().numpy().view(np.uint32), os_.view(np.uint32))
+        return Wq, s, None, (oWq, os_, None)
+    oWq, os_, oz = oracle.quantize_int4(W_cpu.numpy(), qc.group_size, qc.symmetric)
+    assert np.array_equal(Wq.cpu().numpy(), oWq)
+    assert np.array_equal(bits_np(s), os_)
+    if not qc.symmetric:
+        assert np.array_equal(bits_np(z), oz)
+    return Wq, s, z, (oWq, os_, oz)
+
+
+def workspace(M, N, K, qc):
+    return wq.make_workspace(wq.workspace_size(M, N, K, qc))
+
+
+# ------------------------------------------------------------------ quantizers
+@pytest.mark.parametrize("quant", ["sym4", "asym4", "tern2"])
+@pytest.mark.parametrize("N,K", [(1, 128), (37, 256), (300, 1024), (64, 8640 if False else 640)])
+def test_quantize_pack_bit_exact(quant, N, K):
+    W = wq_synth.weights(N, K, seed=100 + N)
+    W[0, :128] = 0.0                       # a degenerate (all-zero) group
+    if N > 2:
+        W[1, 128:256] = 0.37                # one-sided group
+    quantize_both(W, qc_of(quant))
+
+
+@pytest.mark.parametrize("dtype", [torch.float16, torch.bfloat16])
+def test_quantize_from_half_inputs(dtype):
+    W = wq_synth.weights(96, 512, seed=7).to(dtype)
+    for quant in ("sym4", "asym4"):
+        qc = qc_of(quant)
+        Wq, s, z = wq.quantize_pack(W.cuda(), qc)
+        oWq, os_, oz = oracle.quantize_int4(W.float().numpy(), 128, qc.symmetric)
+        assert np.array_equal(Wq.cpu().numpy(), oWq) and np.array_equal(bits_np(s), os_)
+
+
+def test_quantize_group_per_channel():
+    W = wq_synth.weights(40, 512, seed=8)
+    quantize_both(W, wq.QuantConfig(bits=4, group_size=512, symmetric=False))
+
+
+@pytest.mark.parametrize("quant", ["sym4", "asym4", "tern2"])
+def test_unpack_bit_exact(quant):
+    qc = qc_of(quant)
+    N, K = 50, 512
+    Wq = wq_synth.uniform_bytes((N, K * qc.bits // 8), seed=9)
+    q = wq.unpack(Wq.cuda(), N, K, qc)
+    assert np.array_equal(q.cpu().numpy(), oracle.unpack(Wq.numpy(), N, K, qc.bits, qc.symmetric))
+
+
+@pytest.mark.parametrize("dtype", [torch.float16, torch.bfloat16])
+@pytest.mark.parametrize("M,K", [(1, 128), (7, 4096), (16, 11008), (3, 8)])
+def test_act_quant_bit_exact(dtype, M, K):
+    A = wq_synth.activations(M, K, seed=11, dtype=dtype, outlier_frac=0.01)
+    if M > 2:
+        A[2] = 0
+    Aq, sc = wq.act_quant_int8(A.cuda())
+    oAq, osc = oracle.act_quant_int8(bits_np(A), oracle.F16 if dtype == torch.float16 else oracle.BF16)
+    assert np.array_equal(Aq.cpu().numpy(), oAq)
+    assert np.array_equal(sc.cpu().numpy().view(np.uint32), osc.view(np.uint32))
+
+
+# ------------------------------------------------------------------ W4A16 / W2A16
+SMALL = [(1, 256, 512), (3, 200, 384), (8, 128, 128), (13, 1000, 1024), (16, 384, 256), (33, 130, 640),
+         (64, 256, 384), (100, 136, 256)]
+
+
+def run_a16(M, N, K, quant, dtype, use_ws=True, bias=False, seed=0, outliers=0.0):
+    qc = qc_of(quant)
+    W = wq_synth.weights(N, K, seed=seed)
+    A = wq_synth.activations(M, K, seed=seed + 1, dtype=dtype, outlier_frac=outliers)
+    b = wq_synth.activations(1, N, seed=seed + 2, dtype=dtype)[0] if bias else None
+    Wq, s, z, (oWq, os_, oz) = quantize_both(W, qc)
+    ws = workspace(M, N, K, qc) if use_ws else None
+    C = wq.w4a16_gemm(A.cuda(), Wq, s, z, N, K, qc, bias=None if b is None else b.cuda(), workspace=ws)
+    torch.cuda.synchronize()
+    return C, A, b, qc, (oWq, os_, oz)
+
+
+@pytest.mark.parametrize("quant", ["sym4", "asym4", "tern2"])
+@pytest.mark.parametrize("dtype", [torch.float16, torch.bfloat16])
+@pytest.mark.parametrize("M,N,K", SMALL)
+def test_a16_small_all_outputs(quant, dtype, M, N, K):
+    if quant == "tern2":
+        K = max(64, K // 64 * 64)
+    C, A, _, qc, (oWq, os_, oz) = run_a16(M, N, K, quant, dtype, seed=M + N)
+    adt = oracle.F16 if dtype == torch.float16 else oracle.BF16
+    _, ref = oracle.gemm_a16(bits_np(A), adt, oWq, N, K, qc.bits, qc.symmetric, qc.group_size, os_, oz)
+    err = rel_fro(bits_np(C), ref, dtype)
+    assert err <= TOL, err
+
+
+@pytest.mark.parametrize("use_ws", [True, False])
+def test_a16_plans_agree_with_oracle(use_ws):
+    M, N, K = 4, 1024, 2048
+    C, A, _, qc, (oWq, os_, oz) = run_a16(M, N, K, "asym4", torch.float16, use_ws=use_ws, outliers=0.01)
+    _, ref = oracle.gemm_a16(bits_np(A), oracle.F16, oWq, N, K, 4, False, 128, os_, oz)
+    assert rel_fro(bits_np(C), ref, torch.float16) <= TOL
+
+
+def test_a16_bias_and_ragged_tail():
+    M, N, K = 5, 333, 1152
+    for quant in ("asym4", "tern2"):
+        KK = K if quant != "tern2" else 1088
+        C, A, b, qc, (oWq, os_, oz) = run_a16(M, N, KK, quant, torch.float16, bias=True)
+        _, ref = oracle.gemm_a16(bits_np(A), oracle.F16, oWq, N, KK, qc.bits, qc.symmetric, 128, os_, oz, bits_np(b))
+        assert rel_fro(bits_np(C), ref, torch.float16) <= TOL
+
+
+def test_a16_deterministic():
+    M, N, K = 16, 4096, 4096
+    qc = qc_of("asym4")
+    W = wq_synth.weights(N, K)
+    A = wq_synth.activations(M, K, outlier_frac=0.01).cuda()
+    Wq, s, z = wq.quantize_pack(W.cuda(), qc)
+    ws = workspace(M, N, K, qc)
+    C1 = wq.w4a16_gemm(A, Wq, s, z, N, K, qc, workspace=ws)
+    C2 = wq.w4a16_gemm(A, Wq, s, z, N, K, qc, workspace=ws)
+    assert torch.equal(C1, C2)
+    assert int(ws.count_nonzero()) == 0          # the workspace is left all-zero
+
+
+def test_a16_identity_closed_form():
+    # A = I: C = dequant(W)^T, exact when the scales are powers of two
+    K = N = 256
+    rng = np.random.default_rng(3)
+    q = rng.integers(0, 16, (N, K))
+    z = rng.integers(0, 16, (N, K // 128)).astype(np.float16)
+    s = np.ldexp(1.0, rng.integers(-8, -2, (N, K // 128))).astype(np.float16)
+    Wq = torch.from_numpy(oracle.pack(q.astype(np.uint8), 4)).cuda()
+    st, zt = torch.from_numpy(s).cuda(), torch.from_numpy(z).cuda()
+    qc = wq.QuantConfig(4, 128, False)
+    C = wq.w4a16_gemm(torch.eye(K, dtype=torch.float16).cuda(), Wq, st, zt, N, K, qc,
+                      workspace=workspace(K, N, K, qc))
+    w = (q - np.repeat(z.astype(np.float64), 128, 1)) * np.repeat(s.astype(np.float64), 128, 1)
+    assert np.array_equal(C.cpu().numpy().astype(np.float64), w.T)
+
+
+# ------------------------------------------------------------------ W4A8 / W2A8
+def run_a8(M, N, K, quant, seed=0, bias=False, use_ws=True, want_acc=True):
+    qc = qc_of(quant)
+    W = wq_synth.weights(N, K, seed=seed)
+    A = wq_synth.activations(M, K, seed=seed + 1, outlier_frac=0.01)
+    b = wq_synth.activations(1, N, seed=seed + 2)[0] if bias else None
+    Wq, s, z, (oWq, os_, oz) = quantize_both(W, qc)
+    Aq, asc = wq.act_quant_int8(A.cuda())
+    G = 1 if qc.bits == 2 else K // 128
+    acc = torch.zeros(M, N, G, dtype=torch.int32, device="cuda") if want_acc else None
+    ws = workspace(M, N, K, qc) if use_ws else None
+    C = wq.w4a8_gemm(Aq, asc, Wq, s, z, N, K, qc, bias=None if b is None else b.cuda(), acc_out=acc, workspace=ws)
+    torch.cuda.synchronize()
+    oAq, oasc = oracle.act_quant_int8(bits_np(A), oracle.F16)
+    assert np.array_equal(Aq.cpu().numpy(), oAq)
+    return C, acc, qc, (oAq, oasc, oWq, os_, oz), b
+
+
+@pytest.mark.parametrize("quant", ["sym4", "asym4", "tern2"])
+@pytest.mark.parametrize("M,N,K", SMALL)
+def test_a8_small_bit_exact_sums(quant, M, N, K):
+    if quant == "tern2":
+        K = max(64, K // 64 * 64)
+    C, acc, qc, (oAq, oasc, oWq, os_, oz), _ = run_a8(M, N, K, quant, seed=M * 7 + N)
+    _, ref, oacc = oracle.gemm_a8(oAq, oasc, oWq, N, K, qc.bits, qc.symmetric, 128, os_, oz, want_acc=True)
+    assert np.array_equal(acc.cpu().numpy(), oacc)
+    err = rel_fro(bits_np(C), ref, torch.float16)
+    assert err <= TOL, err
+
+
+@pytest.mark.parametrize("use_ws", [True, False])
+def test_a8_bias_and_plans(use_ws):
+    M, N, K = 16, 520, 1024
+    C, acc, qc, (oAq, oasc, oWq, os_, oz), b = run_a8(M, N, K, "sym4", bias=True, use_ws=use_ws)
+    _, ref, oacc = oracle.gemm_a8(oAq, oasc, oWq, N, K, 4, True, 128, os_, None, bits_np(b), want_acc=True)
+    assert np.array_equal(acc.cpu().numpy(), oacc)
+    assert rel_fro(bits_np(C), ref, torch.float16) <= TOL
+
+
+# ------------------------------------------------------------------ full-size workloads
+def sample_idx(n, k, seed):
+    rng = np.random.default_rng(seed)
+    return np.unique(np.concatenate([[0, n - 1], rng.choice(n, size=min(n, k), replace=False)]))
+
+
+FULL = [c for w in ("gemv-small", "decode-llama7b", "w4a8", "bitnet3b") for c in wq_synth.WORKLOADS[w].cases]
+FULL += list(wq_synth.WORKLOADS["prefill-llama7b"].cases)
+
+
+@pytest.mark.parametrize("case", FULL, ids=lambda c: c.name)
+def test_full_size_sampled(case):
+    M, N, K = case.M, case.N, case.K
+    qc = qc_of(case.quant)
+    W = wq_synth.weights(N, K, seed=0)
+    A = wq_synth.activations(M, K, seed=1, dtype=case.a_dtype, outlier_frac=case.outlier_frac)
+    Wq, s, z, (oWq, os_, oz) = quantize_both(W, qc)
+    ws = workspace(M, N, K, qc)
+    ni = sample_idx(N, 192, 5)
+    mi = sample_idx(M, 24, 6)
+    if case.mode == "a16":
+        C = wq.w4a16_gemm(A.cuda(), Wq, s, z, N, K, qc, workspace=ws)
+        adt = oracle.F16 if case.a_dtype == torch.float16 else oracle.BF16
+        _, ref = oracle.gemm_a16(bits_np(A), adt, oWq, N, K, qc.bits, qc.symmetric, 128, os_, oz,
+                                 m_idx=mi, n_idx=ni)
+        got = bits_np(C)[np.ix_(mi, ni)]
+        assert rel_fro(got, ref, case.a_dtype) <= TOL
+    else:
+        Aq, asc = wq.act_quant_int8(A.cuda())
+        G = 1 if qc.bits == 2 else K // 128
+        acc = torch.zeros(M, N, G, dtype=torch.int32, device="cuda")
+        C = wq.w4a8_gemm(Aq, asc, Wq, s, z, N, K, qc, acc_out=acc, workspace=ws)
+        oAq, oasc = oracle.act_quant_int8(bits_np(A), oracle.F16)
+        assert np.array_equal(Aq.cpu().numpy(), oAq)
+        _, ref, oacc = oracle.gemm_a8(oAq, oasc, oWq, N, K, qc.bits, qc.symmetric, 128, os_, oz,
+                                      m_idx=mi, n_idx=ni, want_acc=True)
+        assert np.array_equal(acc.cpu().numpy()[np.ix_(mi, ni)], oacc)
+        assert rel_fro(bits_np(C)[np.ix_(mi, ni)], ref, torch.float16) <= TOL
+    torch.cuda.synchronize()
