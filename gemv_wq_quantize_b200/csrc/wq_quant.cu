@@ -97,7 +97,7 @@ __global__ void __launch_bounds__(256) quant_int4_kernel(const T *__restrict__ W
         mx = warp_max(mx);
         sh = __float2half_rn(__fdiv_rn(__fsub_rn(mx, mn), 15.0f));
         s = __half2float(sh);
-        if (s != 0.f) z = clampf(rintf(__fdiv_rn(-mn, s)), 0.f, 15.f);
+        if (s != 0.f) z = __fadd_rn(clampf(rintf(__fdiv_rn(-mn, s)), 0.f, 15.f), 0.f);  // -0 -> +0
     }
     if (lane == 0) {
         scales[n * G + g] = sh;

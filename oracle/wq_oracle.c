@@ -249,7 +249,8 @@ int orc_quant_int4_asym(const float *W, int64_t N, int64_t K, int64_t gs, uint8_
             uint16_t sh = orc_f64_to_f16((double)s32);
             float s = (float)orc_f16_to_f64(sh);
             float z = 0.0f;
-            if (s != 0.0f) z = clampf(rintf(-mn / s), 0.0f, 15.0f);
+            /* + 0.0f: a zero point is an integer in [0,15]; -0 (from -mn when mn == 0) becomes +0 */
+            if (s != 0.0f) z = clampf(rintf(-mn / s), 0.0f, 15.0f) + 0.0f;
             scales[n * G + g] = sh;
             zeros[n * G + g] = orc_f64_to_f16((double)z);
             for (int64_t i = 0; i < gs; ++i) {

@@ -256,8 +256,9 @@ def test_degenerate_groups():
     assert s[0, 0] == 0 and s[0, 1] == 0 and np.all(Wq[0] == 0x88)
     Wq, s, z = oracle.quantize_int4(W, 128, False)
     assert s[0, 0] == 0 and z[0, 0] == 0 and np.all(Wq[0] == 0)
-    # one-sided group: min widened to 0, so the zero point is 0
-    assert f16_val(z[1, 1]) == 0 and np.all(Wq[1, 64:] == 0xFF)
+    # one-sided group: min widened to 0, so the zero point is +0 (an integer, never -0)
+    assert z[1, 1] == 0x0000 and np.all(Wq[1, 64:] == 0xFF)
+    assert not np.any(z == 0x8000)
 
 
 def test_ternary_scale_and_codes():
