@@ -120,7 +120,7 @@ def workspace_size(M: int, N: int, K: int, qc: QuantConfig) -> int:
 
 
 def make_workspace(nbytes: int, device=None) -> torch.Tensor:
-    """Zero-filled device scratch (the matmuls keep it all-zero between calls)."""
+    """Zero-filled device scratch for the split-K plans (reusable across calls without clearing)."""
     return torch.zeros(max(int(nbytes), 16), dtype=torch.uint8, device=device or "cuda")
 
 

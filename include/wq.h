@@ -115,9 +115,11 @@ wq_status act_quant_int8(const void *A, wq_dtype a_dt, int64_t M, int64_t K,
  *   A      [M,K] a_dt in {WQ_F16, WQ_BF16};  C [M,N] a_dt;  bias [N] a_dt or NULL.
  *   Wq, scales, zeros as written by wq_quantize_pack (zeros NULL unless asymmetric INT4).
  *   workspace: device scratch of at least wq_workspace_size(M,N,K,c) bytes, ZERO-FILLED
- *   before its first use; every call returns it to all-zero when its kernels finish.  A
- *   workspace that is NULL or too small is allowed: the call then uses a launch plan that
- *   needs none (possibly slower).  Calls that share one workspace must not overlap.
+ *   once before its first use.  It holds split-K partial sums (overwritten by every call)
+ *   and arrival counters that every call leaves at zero again, so it can be reused by
+ *   later calls of any shape without clearing.  A workspace that is NULL or too small is
+ *   allowed: the call then uses a launch plan that needs none (possibly slower).  Calls
+ *   that share one workspace must not overlap on the GPU.
  * Requires K % 128 == 0 for INT4 (K % 64 == 0 for INT2), M, N >= 1. */
 wq_status w4a16_gemm(const void *A, wq_dtype a_dt, const uint8_t *Wq, const void *scales,
                      const void *zeros, const void *bias, void *C,
