@@ -19,6 +19,10 @@ wq_status skinny_gemm(int WB, int AM, const void *A, const float *a_scale, const
                       const wq_qconfig &c, void *ws, size_t ws_bytes, cudaStream_t st);
 size_t skinny_workspace_size(int WB, int AM, int64_t M, int64_t N, int64_t K);
 int skinny_read_error();
+wq_status gemv_small_m(int WB, int AM, const void *A, const float *a_scale, const uint8_t *Wq, const void *scales,
+                       const void *zeros, const void *bias, void *C, int32_t *acc_out, int64_t M, int64_t N,
+                       int64_t K, const wq_qconfig &c, cudaStream_t st);
+int gemv_read_error();
 
 namespace {
 thread_local char g_last_error[512] = "";
@@ -93,7 +97,25 @@ wq_status encode_tmap_2d(CUtensorMap *map, CUtensorMapDataType dt, const void *b
     return WQ_OK;
 }
 
-int read_device_errors() { return skinny_read_error(); }
+int read_device_errors()
+{
+    const int a = skinny_read_error(), b = gemv_read_error();
+    return a ? a : b;
+}
+
+namespace {
+// Few tokens go to the weight-streaming GEMV; more tokens to the tiled path.
+wq_status dispatch(int WB, int AM, const void *A, const float *a_scale, const uint8_t *Wq, const void *scales,
+                   const void *zeros, const void *bias, void *C, int32_t *acc_out, int64_t M, int64_t N, int64_t K,
+                   const wq_qconfig &c, void *ws, size_t ws_bytes, cudaStream_t st)
+{
+    if (M <= 16) {
+        wq_status rc = gemv_small_m(WB, AM, A, a_scale, Wq, scales, zeros, bias, C, acc_out, M, N, K, c, st);
+        if (rc != WQ_ERR_UNSUPPORTED) return rc;
+    }
+    return skinny_gemm(WB, AM, A, a_scale, Wq, scales, zeros, bias, C, acc_out, M, N, K, c, ws, ws_bytes, st);
+}
+}  // namespace
 
 namespace {
 
@@ -147,6 +169,7 @@ extern "C" size_t wq_workspace_size(int64_t M, int64_t N, int64_t K, wq_qconfig 
 {
     if (M <= 0 || N <= 0 || K <= 0 || (c.bits != 4 && c.bits != 2)) return 0;
     // the INT8 path has the smaller activation blocks; size for the larger of the two
+    if (M <= 16) return 0;  // the few-token kernel needs no workspace
     return std::max(skinny_workspace_size(c.bits, 0, M, N, K), skinny_workspace_size(c.bits, 2, M, N, K));
 }
 
@@ -160,7 +183,7 @@ extern "C" wq_status w4a16_gemm(const void *A, wq_dtype a_dt, const uint8_t *Wq,
     if (!A || !C) return fail(WQ_ERR_INVALID_ARG, "A and C must be non-null");
     if (!aligned16(A) || !aligned16(C) || (bias && !aligned16(bias)) || (workspace && !aligned16(workspace)))
         return fail(WQ_ERR_ALIGNMENT, "A, C, bias and workspace must be 16-byte aligned");
-    return skinny_gemm(c.bits, a_dt == WQ_F16 ? 0 : 1, A, nullptr, Wq, scales, c.bits == 4 && !c.symmetric ? zeros : nullptr,
+    return dispatch(c.bits, a_dt == WQ_F16 ? 0 : 1, A, nullptr, Wq, scales, c.bits == 4 && !c.symmetric ? zeros : nullptr,
                        bias, C, nullptr, M, N, K, c, workspace, ws_bytes, stream);
 }
 
@@ -175,6 +198,6 @@ extern "C" wq_status w4a8_gemm(const int8_t *Aq, const float *a_scale, const uin
         return fail(WQ_ERR_ALIGNMENT, "Aq, C, bias and workspace must be 16-byte aligned");
     if (acc_out && c.bits == 4 && c.group_size != 128)
         return fail(WQ_ERR_UNSUPPORTED, "acc_out needs group_size == 128");
-    return skinny_gemm(c.bits, 2, Aq, a_scale, Wq, scales, c.bits == 4 && !c.symmetric ? zeros : nullptr, bias, C,
+    return dispatch(c.bits, 2, Aq, a_scale, Wq, scales, c.bits == 4 && !c.symmetric ? zeros : nullptr, bias, C,
                        acc_out, M, N, K, c, workspace, ws_bytes, stream);
 }

@@ -164,6 +164,16 @@ def test_a16_plans_agree_with_oracle(use_ws):
     assert rel_fro(bits_np(C), ref, torch.float16) <= TOL
 
 
+@pytest.mark.parametrize("M,N,K,quant", [(1, 24000, 256, "asym4"), (16, 16000, 256, "sym4"), (4, 24000, 320, "tern2"),
+                                          (9, 2368, 8960, "asym4")])
+def test_a16_many_tiles_per_cta(M, N, K, quant):
+    # more 16-row tiles per CTA than fit in registers at once (several tile groups), long K
+    C, A, _, qc, (oWq, os_, oz) = run_a16(M, N, K, quant, torch.float16, seed=5)
+    ni = np.unique(np.concatenate([np.arange(0, N, 37), [N - 1]]))
+    _, ref = oracle.gemm_a16(bits_np(A), oracle.F16, oWq, N, K, qc.bits, qc.symmetric, 128, os_, oz, n_idx=ni)
+    assert rel_fro(bits_np(C)[:, ni], ref, torch.float16) <= TOL
+
+
 def test_a16_bias_and_ragged_tail():
     M, N, K = 5, 333, 1152
     for quant in ("asym4", "tern2"):
