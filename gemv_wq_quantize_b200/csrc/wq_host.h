@@ -8,7 +8,7 @@
 #include <cstdarg>
 #include <cstdio>
 
-#include "../../include/wq.h"
+#include "wq.h"
 
 namespace wq {
 
