@@ -27,7 +27,7 @@ WQ_OK, WQ_ERR_INVALID_ARG, WQ_ERR_ALIGNMENT, WQ_ERR_UNSUPPORTED, WQ_ERR_CUDA, WQ
 WQ_F32, WQ_F16, WQ_BF16, WQ_I8, WQ_I32 = range(5)
 
 EXPORTED = ("wq_quantize_pack", "wq_quantize_workspace_size", "wq_unpack", "act_quant_int8", "w4a16_gemm",
-            "w4a8_gemm", "wq_workspace_size", "wq_status_string", "wq_last_error")
+            "w4a16_gemm_noalloc", "w4a8_gemm", "wq_workspace_size", "wq_status_string", "wq_last_error")
 
 
 class WqError(RuntimeError):
@@ -75,6 +75,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.act_quant_int8.restype = st
     lib.w4a16_gemm.argtypes = [vp, st, vp, vp, vp, vp, vp, i64, i64, i64, QConfig, vp, sz, vp]
     lib.w4a16_gemm.restype = st
+    lib.w4a16_gemm_noalloc.argtypes = [vp, st, vp, vp, vp, vp, vp, i64, i64, i64, QConfig, vp]
+    lib.w4a16_gemm_noalloc.restype = st
     lib.w4a8_gemm.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, QConfig, vp, sz, vp]
     lib.w4a8_gemm.restype = st
     lib.wq_workspace_size.argtypes = [i64, i64, i64, QConfig]
@@ -180,6 +182,25 @@ def w4a16_gemm(A, Wq, scales, zeros, N: int, K: int, qc: QuantConfig, bias=None,
     rc = load_library().w4a16_gemm(_ptr(A), _DT[A.dtype], _ptr(Wq), _ptr(scales), _ptr(zeros), _ptr(bias), _ptr(C),
                                    M, N, K, qc.c(), _ptr(workspace), wsb, _stream(stream))
     _check(rc, "w4a16_gemm")
+    return C
+
+
+def w4a16_gemm_noalloc(A, Wq, scales, zeros, N: int, K: int, qc: QuantConfig, bias=None, out=None,
+                       stream=None) -> torch.Tensor:
+    """w4a16_gemm with the library's static device scratch instead of a workspace.
+
+    The C entry point allocates nothing; pass ``out`` so that this wrapper does not
+    allocate the result either.  The first call on a device sets the scratch up and
+    waits for the device (do it before any stream capture); calls that overlap on the
+    GPU share the scratch and must be serialised by the caller.
+    """
+    for t, n in ((A, "A"), (Wq, "Wq"), (scales, "scales"), (zeros, "zeros"), (bias, "bias"), (out, "out")):
+        _dev(t, n)
+    M = A.shape[0]
+    C = out if out is not None else torch.empty(M, N, dtype=A.dtype, device=A.device)
+    rc = load_library().w4a16_gemm_noalloc(_ptr(A), _DT[A.dtype], _ptr(Wq), _ptr(scales), _ptr(zeros), _ptr(bias),
+                                           _ptr(C), M, N, K, qc.c(), _stream(stream))
+    _check(rc, "w4a16_gemm_noalloc")
     return C
 
 

@@ -144,6 +144,28 @@ wq_status w4a8_gemm(const int8_t *Aq, const float *a_scale, const uint8_t *Wq, c
  * current device. */
 size_t wq_workspace_size(int64_t M, int64_t N, int64_t K, wq_qconfig c);
 
+/* Capacity of the static scratch that w4a16_gemm_noalloc uses (one array per device). */
+#define WQ_NOALLOC_SCRATCH_BYTES ((size_t)16 << 20)
+
+/* w4a16_gemm without a workspace argument, and without allocating anything.
+ * (A library convenience: the quantised-matmul method itself has no counterpart of it.)
+ * For callers that cannot provide a workspace: a plain C host loop that owns no device
+ * allocator, or a plug-in inside a runtime that hands out no scratch.  Allocating for
+ * them is no way out, because cudaFree synchronises the device and a per-shape workspace
+ * would be reallocated whenever a larger shape arrives.
+ *   Arguments, layouts, results and errors as for w4a16_gemm (bit-identical output).
+ *   Scratch: a static device array of WQ_NOALLOC_SCRATCH_BYTES per device, inside
+ *   libwq.  The FIRST call on a device looks up its address (cudaGetSymbolAddress, with
+ *   that device current), clears it and waits for the device: make that first call
+ *   before any stream capture.  Later calls allocate, clear and wait for nothing.
+ *   A shape with wq_workspace_size(M,N,K,c) > WQ_NOALLOC_SCRATCH_BYTES is refused with
+ *   WQ_ERR_WORKSPACE (see wq_last_error) before anything runs.
+ *   Calls that overlap on the GPU (several streams or host threads on one device) share
+ *   the one array and race: the caller must serialise them. */
+wq_status w4a16_gemm_noalloc(const void *A, wq_dtype a_dt, const uint8_t *Wq, const void *scales,
+                             const void *zeros, const void *bias, void *C,
+                             int64_t M, int64_t N, int64_t K, wq_qconfig c, cudaStream_t stream);
+
 const char *wq_status_string(wq_status s);
 
 /* Reads and clears the library's device-side error word.  Non-zero (1) means that a
