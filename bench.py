@@ -254,11 +254,23 @@ def timed_replays(preps, steps: int, warmup: int, e2e: bool, dist_on: bool, samp
         torch.distributed.barrier()
     sec = t0.elapsed_time(t1) / 1e3
     if dist_on:
-        t = torch.tensor([sec], device="cuda")
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        sec = float(t.item())
+        sec = max_over_ranks(sec, torch.device("cuda", torch.cuda.current_device()))
     del g_chunk, g_rem
     return sec
+
+
+def max_over_ranks(sec: float, device=None) -> float:
+    """The slowest rank's duration (every rank gets it); the local value without a process group."""
+    if not (torch.distributed.is_available() and torch.distributed.is_initialized()):
+        return sec
+    t = torch.tensor([sec], dtype=torch.float64, device=device if device is not None else "cpu")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(units_per_step_per_rank: float, steps: int, world: int, sec: float) -> float:
+    """Units processed by all ranks together per second of the slowest rank (weak scaling)."""
+    return units_per_step_per_rank * steps * world / sec
 
 
 class _Null:
@@ -313,9 +325,8 @@ def run_ours(args, rank, world, local_rank, dist_on):
     step_bytes = sum(p.bytes for p in preps)
     step_flops = sum(flops(p.c) for p in preps)
     launches = sum(launches_per_call(p.c) for p in preps)
-    total_bytes = step_bytes * args.steps * world
-    value = total_bytes / sec / 1e9
-    e2e_value = total_bytes / sec_e2e / 1e9
+    value = whole_job_rate(step_bytes, args.steps, world, sec) / 1e9
+    e2e_value = whole_job_rate(step_bytes, args.steps, world, sec_e2e) / 1e9
     pk = peaks()
     avg_launch_s = sec / (args.steps * launches)
     achieved = (step_bytes / launches) / avg_launch_s / 1e9

@@ -1,0 +1,70 @@
+"""Multi-rank logic of the benchmark on CPU: two `gloo` ranks.
+
+The path shards by output rows with no data-path exchange (weak-scaling replicas); what
+ranks share is the timing protocol: the reported time is the slowest rank's, and the
+throughput counts the work of all ranks.  The reference arm runs on rank 0 alone.
+"""
+import os
+import socket
+import subprocess
+import sys
+
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port() -> int:
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank, world, port, q):
+    import datetime
+    sys.path.insert(0, ROOT)
+    import bench
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=30))
+    try:
+        local = 0.5 + rank          # rank 1 is the slow one
+        slowest = bench.max_over_ranks(local)
+        rate = bench.whole_job_rate(1000.0, 10, world, slowest)
+        q.put((rank, slowest, rate))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_max_over_ranks_and_whole_job_rate_two_gloo_ranks():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=120)
+    assert all(p.exitcode == 0 for p in procs)
+    got = sorted(q.get(timeout=5) for _ in range(2))
+    for rank, slowest, rate in got:
+        assert slowest == 1.5                       # every rank sees the slowest rank's time
+        assert rate == pytest.approx(1000.0 * 10 * 2 / 1.5)
+
+
+def test_helpers_without_a_process_group():
+    sys.path.insert(0, ROOT)
+    import bench
+    assert not dist.is_initialized()
+    assert bench.max_over_ranks(0.25) == 0.25
+    assert bench.whole_job_rate(8.0, 4, 1, 2.0) == 16.0
+
+
+def test_reference_arm_runs_on_rank_zero_only():
+    env = dict(os.environ, RANK="1", WORLD_SIZE="2", LOCAL_RANK="1")
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--gpus", "2",
+                        "--steps", "1", "--warmup", "3"], env=env, capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0
+    assert r.stdout.strip() == ""
