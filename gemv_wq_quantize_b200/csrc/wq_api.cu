@@ -97,6 +97,27 @@ wq_status encode_tmap_2d(CUtensorMap *map, CUtensorMapDataType dt, const void *b
     return WQ_OK;
 }
 
+wq_status encode_tmap(CUtensorMap *map, CUtensorMapDataType dt, int rank, const void *base, const uint64_t *dims,
+                      const uint64_t *strides_bytes, const uint32_t *box, bool swizzle128)
+{
+    EncodeFn fn = encode_fn();
+    if (!fn) return fail(WQ_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+    if (rank < 1 || rank > 3) return fail(WQ_ERR_INVALID_ARG, "tensor map rank %d", rank);
+    cuuint64_t d[3] = {}, st[2] = {};
+    cuuint32_t b[3] = {}, estr[3] = {1, 1, 1};
+    for (int i = 0; i < rank; ++i) {
+        d[i] = dims[i];
+        b[i] = box[i];
+    }
+    for (int i = 0; i + 1 < rank; ++i) st[i] = strides_bytes[i];
+    CUresult r = fn(map, dt, cuuint32_t(rank), const_cast<void *>(base), d, st, b, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(WQ_ERR_INVALID_ARG, "cuTensorMapEncodeTiled (rank %d) failed (%d)", rank, int(r));
+    return WQ_OK;
+}
+
 int read_device_errors()
 {
     const int a = skinny_read_error(), b = gemv_read_error();

@@ -85,6 +85,22 @@ __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, i
         : "memory");
 }
 
+// 3D tiled TMA load (x as for tma_load_2d).
+__device__ __forceinline__ void tma_load_3d(void *dst, const CUtensorMap *map, int32_t x, int32_t y, int32_t z,
+                                            uint64_t *bar)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
+        : "memory");
+}
+
+// Shared-memory offset of byte `lin` of a box written by TMA with CU_TENSOR_MAP_SWIZZLE_128B
+// into a 1024-byte aligned buffer: the 16-byte chunk index (bits 4-6) is XORed with the
+// 128-byte line index modulo 8 (bits 7-9).
+__device__ __forceinline__ uint32_t swz128(uint32_t lin) { return lin ^ ((lin >> 3) & 0x70u); }
+
 // 1D bulk copy global -> shared (both addresses and the size multiples of 16 bytes).
 __device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t bytes, uint64_t *bar)
 {
@@ -211,6 +227,13 @@ __device__ __forceinline__ uint4 lds128(const void *p)
     asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
                  : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
                  : "r"(smem_u32(p)));
+    return v;
+}
+
+__device__ __forceinline__ uint2 lds64(const void *p)
+{
+    uint2 v;
+    asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(smem_u32(p)));
     return v;
 }
 

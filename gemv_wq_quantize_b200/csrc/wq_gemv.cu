@@ -5,24 +5,27 @@
 // INT32 group sums and the (a_scale x w_scale) epilogue (W4A8: "Accelerating LLM inference
 // with CUDA Graph and INT4 quantization", part 1, steps 3-4).
 //
-// The kernel is HBM-bound and short (a few microseconds); it is built to have every SM's
-// share of the packed weights in flight early and to keep the tensor pipe fed:
+// The kernel is HBM-bound and lasts a few microseconds, so it is built to put each SM's
+// whole share of the packed weights in flight at once and to spend few instructions per
+// byte once it arrives:
 //  * Rows are cut into 16-row tiles; CTA c (one per SM) owns tiles [cT/P, (c+1)T/P) and all
-//    of K, so no CTA needs another's result.
-//  * K is walked in chunks of 8 units (a unit = 64 packed bytes of a row: 128 k of INT4,
-//    256 k of INT2).  A producer warp issues, per chunk, two 2D TMA boxes of 16 rows x 256 B
-//    per tile into an S-stage ring (256-byte rows: narrower TMA rows stream markedly slower,
-//    and each TMA instruction costs tens of nanoseconds to issue).  The weight boxes of the
-//    first S chunks are issued before griddepcontrol.wait, so with programmatic dependent
-//    launch they stream while the previous kernel finishes; only the activations wait.
+//    of K, so no CTA needs another's result.  K is walked in chunks of KC units (a unit =
+//    64 packed bytes of a row: 128 k of INT4, 256 k of INT2).
+//  * One TMA box per tile and chunk brings 16 rows x KC units (a 3D box over unit pairs;
+//    a 2D box per unit pair when rows are not a whole number of pairs), written with the
+//    128-byte swizzle so that the warps' 16-byte reads of 8 rows hit 8 different bank
+//    groups.  The boxes of the first S chunks are issued, spread over the warps, before
+//    griddepcontrol.wait: with programmatic dependent launch they stream while the previous
+//    kernel in the stream finishes.  When all chunks fit in shared memory nothing else is
+//    issued; otherwise the last warp to finish a stage refills it.
 //  * The activations are staged once for all of K (one bulk copy per token row) when they
-//    fit, else per chunk by TMA.  The CTA's scale / zero rows (contiguous in the [N, K/g]
-//    layout) arrive with one bulk copy each and are turned into an fp32 table.
-//  * Sixteen consumer warps: warp w takes unit w % 8 of every chunk and half (w / 8) of its
-//    k-steps, for all of the CTA's tiles, two tiles at a time.  It builds its mma.sync B
-//    fragments once per chunk and reuses them for every tile; weights are unpacked with LOP3
-//    into exact integers q - z and multiplied on the tensor cores (two tiles x two k-step
-//    chains in flight); each unit's fp32 / int32 sum is folded with its group scale.
+//    fit, else per chunk by a swizzled 3D TMA box.  The CTA's scales / zero points become a
+//    group-major fp32 table.
+//  * 16 warps; warp w takes unit w % KC of every chunk and, for 9..16 tokens, every other
+//    tile.  It builds the unit's mma.sync B fragments (activations in the k order of the
+//    nibble unpack) once and uses them for all its tiles: weights are unpacked with LOP3
+//    into the exact integers q - z, multiplied on the tensor cores, and each unit's fp32 /
+//    int32 sum is folded with its group scale.
 //  * The warps' partial sums are added in a fixed order through shared memory
 //    (deterministic) and the epilogue writes C.
 #include <cuda_bf16.h>
@@ -42,30 +45,30 @@ static __device__ int g_gemv_error;
 
 namespace {
 
-constexpr int kCW = 16;                    // consumer warps
-constexpr int kThreads = (kCW + 1) * 32;   // + producer warp
-constexpr int kKC = 8;                     // units per chunk
+constexpr int kCW = 16;  // warps
+constexpr int kThreads = kCW * 32;
 constexpr int kTileRows = 16;
-constexpr int kUnitBytes = 64;
-constexpr int kWBoxBytes = 256;                      // weight box row: 4 units
-constexpr int kUPB = kWBoxBytes / kUnitBytes;        // units per weight box
-constexpr int kWBox = kTileRows * kWBoxBytes;        // 4 KB
-constexpr int kTileChunk = kKC * kTileRows * kUnitBytes;  // one tile's part of a chunk: 8 KB
-constexpr int kABoxElems = 256;                      // activation box row: 256 elements
-constexpr int kAPadBytes = 16;                       // activation row padding (bank spread)
-
-// tiles whose sums live in registers at once (even: tiles go through the MMA in pairs)
-__host__ __device__ constexpr int tg_max(int NT) { return NT == 1 ? 6 : 2; }
+constexpr int kPairBytes = 128;                   // two units of a row: one swizzle line
+constexpr int kPairBox = kTileRows * kPairBytes;  // 2 KB
+__host__ __device__ constexpr int wpu_of(int NT) { return NT == 1 ? 1 : 2; }  // warps sharing a unit
+__host__ __device__ constexpr int kc_of(int NT) { return kCW / wpu_of(NT); }  // units per chunk
+__host__ __device__ constexpr int tm_of(int NT) { return NT == 1 ? 6 : 3; }   // tiles per warp and pass
+__host__ __device__ constexpr int ntl_of(int NT) { return NT == 1 ? 2 : 1; }  // tiles per MMA batch
 
 struct GemvParams {
     const void *A;
     int M, N, K, G, gs, sym;
-    int KB, T, P, nch, TG, S;
-    int a_whole;     // 1: all of K staged once; 0: per chunk by TMA
-    int a_pitch_b;   // bytes between token rows of the staged activations
-    int abox_bytes;  // chunked activations: bytes of one TMA box (M x 256 elements)
-    int wpart_bytes, stage_bytes;
-    int sc_smem, sc_rows_cap;
+    int KB, T, P;
+    int nch, TPP, S;         // chunks per pass, tiles per pass, ring stages
+    int w3d;                 // 1: one 3D box per tile and chunk; 0: one 2D box per unit pair
+    int wtile_bytes;         // one tile's weights of a chunk: KC x 1 KB
+    int wpart_bytes;         // TPP tiles
+    int stage_bytes;         // weights + chunked activations
+    int a_whole, a_pitch_b;  // whole activations: bytes between token rows
+    int abox_bytes, MB;      // chunked activations: bytes per stage, token rows of the box
+    int rows_cap;            // CTA rows covered by the scale table
+    int tab_rs;              // table row stride (float2 entries, odd: spreads the banks)
+    int abuf_off, scst_off, stab_off, red_off, bar_off;
     const uint16_t *scales16;
     const float *scale32;
     const uint16_t *zeros;
@@ -97,13 +100,6 @@ __device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity)
     }
 }
 
-__device__ __forceinline__ uint2 lds64(const void *p)
-{
-    uint2 v;
-    asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(smem_u32(p)));
-    return v;
-}
-
 template <int AM>
 __device__ __forceinline__ void store_out(void *C, long long idx, float v)
 {
@@ -132,181 +128,192 @@ __device__ __forceinline__ float finish(const GemvParams &p, float total_f, int 
     return v + bias_at<AM>(p.bias, n);
 }
 
-// ACC: also add every INT32 group sum into p.acc_out (W4A8 debugging output; zeroed by the
-// host first, the two halves of a unit arrive from two warps).
+// ACC: also store every INT32 group sum into p.acc_out (W4A8 with group_size 128).
 template <int WB, int AM, int NT, bool ACC>
 __global__ void __launch_bounds__(kThreads, 1)
     gemv_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_a,
                 const GemvParams p)
 {
-    constexpr int MP = NT * 8;
     constexpr int KU = kunit_of(WB);
-    constexpr int QH = qh_of(WB, AM);
-    constexpr int kTGMax = tg_max(NT);
+    constexpr int QN = qn_of(WB, AM);
     constexpr int ES = (AM == A_I8) ? 1 : 2;
-    constexpr int UPA = kABoxElems / KU;  // units per activation box
+    constexpr int AU = KU * ES;  // activation bytes of one unit and token
+    constexpr int WPU = wpu_of(NT), KC = kc_of(NT), TM = tm_of(NT), NTL = ntl_of(NT);
     using Tot = typename std::conditional<AM == A_I8 && WB == 2, int, float>::type;
 
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int S = p.S;
     uint8_t *ring = smem;
-    uint8_t *abuf = ring + size_t(S) * p.stage_bytes;  // whole activations (a_whole)
-    const size_t abuf_bytes = p.a_whole ? ((size_t(p.M) * p.a_pitch_b + 127) & ~size_t(127)) : 0;
-    float2 *stab = reinterpret_cast<float2 *>(abuf + abuf_bytes);
-    uint16_t *sc = reinterpret_cast<uint16_t *>(stab + size_t(p.sc_rows_cap) * p.G);
-    uint16_t *zc = sc + size_t(p.sc_rows_cap) * p.G;
-    float *red = reinterpret_cast<float *>(
-        (reinterpret_cast<uintptr_t>(zc + size_t(p.sc_rows_cap) * p.G) + 15) & ~uintptr_t(15));
-    uint64_t *bars = reinterpret_cast<uint64_t *>(red + size_t(kCW) * p.TG * kTileRows * MP);
-    uint64_t *full = bars, *empty = bars + S, *scbar = bars + 2 * S, *abar = scbar + 1, *cbar = scbar + 2;
+    uint8_t *abuf = smem + p.abuf_off;
+    uint16_t *sc_st = reinterpret_cast<uint16_t *>(smem + p.scst_off);  // [rows][G] fp16 scales
+    uint16_t *zc_st = sc_st + size_t(p.rows_cap) * p.G;                 // then zero points
+    float2 *stab = reinterpret_cast<float2 *>(smem + p.stab_off);       // [G][tab_rs] {scale, zero}
+    float *red = reinterpret_cast<float *>(smem + p.red_off);
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + p.bar_off);
+    uint64_t *abar = full + S, *cbar = full + S + 1, *scbar = full + S + 2;
+    unsigned *cnt = reinterpret_cast<unsigned *>(full + S + 3);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int c = blockIdx.x;
     const int t0 = int((long long)c * p.T / p.P), t1 = int((long long)(c + 1) * p.T / p.P);
     const int ntc = t1 - t0;
-    const int ngrp = (ntc + p.TG - 1) / p.TG;
-    const int total_it = ngrp * p.nch;
-    const int r0 = t0 * kTileRows, r1 = min(t1 * kTileRows, p.N);
+    const int npass = (ntc + p.TPP - 1) / p.TPP;
+    const int total_it = npass * p.nch;
+    const int r0 = t0 * kTileRows;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&empty[s], kCW);
+            cnt[s] = 0;
         }
-        mbar_init(scbar, 1);
         mbar_init(abar, 1);
-        mbar_init(cbar, kCW * 32);
+        mbar_init(cbar, kThreads);
+        mbar_init(scbar, 1);
         fence_barrier_init();
     }
     __syncthreads();
     grid_dep_launch();  // the next kernel in the stream may start launching as SMs free up
 
-    if (warp == kCW) {
-        // ------------------------------------------------------------ producer warp
-        if (lane == 0) {
+    // ---- stage `it` of the ring: weights of the pass's tiles (and the expected bytes of all)
+    auto issue_w = [&](int it) {
+        const int s = it % S;
+        const int pass = it / p.nch, ch = it % p.nch;
+        const int tp0 = t0 + pass * p.TPP;
+        const int ntp = min(p.TPP, ntc - pass * p.TPP);
+        const int pair0 = ch * KC / 2;
+        const int npair = min(KC / 2, (p.KB + 1) / 2 - pair0);
+        uint8_t *st = ring + size_t(s) * p.stage_bytes;
+        const uint32_t wbytes = p.w3d ? uint32_t(ntp * p.wtile_bytes) : uint32_t(ntp * npair * kPairBox);
+        mbar_arrive_expect_tx(&full[s], wbytes + (p.a_whole ? 0u : uint32_t(p.abox_bytes)));
+        for (int i = 0; i < ntp; ++i) {
+            uint8_t *dst = st + size_t(i) * p.wtile_bytes;
+            if (p.w3d) {
+                tma_load_3d(dst, &tmap_w, 0, (tp0 + i) * kTileRows, pair0, &full[s]);
+            } else {
+                for (int q = 0; q < npair; ++q)
+                    tma_load_2d(dst + q * kPairBox, &tmap_w, (pair0 + q) * kPairBytes, (tp0 + i) * kTileRows,
+                                &full[s]);
+            }
+        }
+    };
+    auto issue_a = [&](int it) {  // chunked activations (after the grid dependency)
+        const int s = it % S, ch = it % p.nch;
+        tma_load_3d(ring + size_t(s) * p.stage_bytes + p.wpart_bytes, &tmap_a, 0, 0, ch * KC * AU / 128, &full[s]);
+    };
+
+    // the CTA's scale / zero rows are contiguous in [N, G]: one bulk copy each (a ragged
+    // tail of < 16 bytes is read directly below)
+    const int nrows = min(ntc * kTileRows, p.N - r0);
+    const uint32_t sc_bytes = (WB == 4) ? uint32_t(nrows) * p.G * 2u : 0u;
+    const uint32_t sc16 = sc_bytes & ~15u;
+    const int pro = min(S, total_it);
+    if (lane == 0) {
+        if (warp == 0) {
             tma_prefetch_desc(&tmap_w);
             if (!p.a_whole) tma_prefetch_desc(&tmap_a);
-        }
-        // scale / zero rows of this CTA: contiguous, 16-byte aligned at the start
-        const uint32_t sc_bytes = (WB == 4 && p.sc_smem) ? uint32_t(r1 - r0) * p.G * 2 : 0u;
-        const uint32_t sc16 = sc_bytes & ~15u;
-        if constexpr (WB == 4) {
-            for (uint32_t e = (sc16 >> 1) + uint32_t(lane); e < (sc_bytes >> 1); e += 32u) {  // ragged tail
-                sc[e] = p.scales16[(size_t)r0 * p.G + e];
-                if (!p.sym) zc[e] = p.zeros[(size_t)r0 * p.G + e];
-            }
-        }
-        __syncwarp();
-        if (lane == 0) {
-            mbar_arrive_expect_tx(scbar, sc16 * (p.sym ? 1 : 2));
-            if (sc16) {
-                bulk_load(sc, p.scales16 + (size_t)r0 * p.G, sc16, scbar);
-                if (!p.sym) bulk_load(zc, p.zeros + (size_t)r0 * p.G, sc16, scbar);
-            }
-        }
-
-        auto issue = [&](int it, bool weights, bool acts) {
-            const int s = it % S;
-            const int grp = it / p.nch, ch = it % p.nch;
-            const int ntg = min(p.TG, ntc - grp * p.TG);
-            const int kb0 = ch * kKC, nkb = min(kKC, p.KB - kb0);
-            const int nwb = (nkb + kUPB - 1) / kUPB, nab = p.a_whole ? 0 : (nkb + UPA - 1) / UPA;
-            uint8_t *st = ring + size_t(s) * p.stage_bytes;
-            if (weights) {
-                if (lane == 0) mbar_arrive_expect_tx(&full[s], uint32_t(ntg * nwb * kWBox + nab * p.abox_bytes));
-                __syncwarp();
-                for (int idx = lane; idx < ntg * nwb; idx += 32) {
-                    const int i = idx / nwb, b = idx % nwb;
-                    tma_load_2d(st + i * kTileChunk + b * kWBox, &tmap_w, (kb0 + b * kUPB) * kUnitBytes,
-                                (t0 + grp * p.TG + i) * kTileRows, &full[s]);
+            if constexpr (WB == 4) {
+                mbar_arrive_expect_tx(scbar, sc16 * (p.sym ? 1u : 2u));
+                if (sc16) {
+                    bulk_load(sc_st, p.scales16 + (size_t)r0 * p.G, sc16, scbar);
+                    if (!p.sym) bulk_load(zc_st, p.zeros + (size_t)r0 * p.G, sc16, scbar);
                 }
             }
-            if (acts)
-                for (int b = lane; b < nab; b += 32)
-                    tma_load_2d(st + p.wpart_bytes + b * p.abox_bytes, &tmap_a, (kb0 + b * UPA) * KU, 0, &full[s]);
-        };
-        const int pro = min(S, total_it);
-        for (int it = 0; it < pro; ++it) issue(it, true, false);
-        grid_dep_wait();  // activations may be produced by the previous kernel
-        if (p.a_whole) {
-            if (lane == 0) {
-                // all of K, one bulk copy per token row; zeros past K up to the last unit
-                const int kpad = p.KB * KU;
-                for (int m = 0; m < p.M; ++m)
-                    for (int k = p.K; k < kpad; ++k) {
-                        if constexpr (ES == 1) abuf[(size_t)m * p.a_pitch_b + k] = 0;
-                        else reinterpret_cast<uint16_t *>(abuf + (size_t)m * p.a_pitch_b)[k] = 0;
-                    }
-                const uint32_t bytes = uint32_t(p.K) * ES;
-                mbar_arrive_expect_tx(abar, bytes * p.M);
-                for (int m = 0; m < p.M; ++m)
-                    bulk_load(abuf + (size_t)m * p.a_pitch_b, static_cast<const uint8_t *>(p.A) + (size_t)m * bytes,
-                              bytes, abar);
-            }
-        } else {
-            for (int it = 0; it < pro; ++it) issue(it, false, true);
         }
-        int it = pro;
-        for (; it < total_it; ++it) {
-            if (!wait_bar(&empty[it % S], ((it / S) - 1) & 1)) break;
-            issue(it, true, true);
-        }
-        for (int k = max(0, it - S); k < it; ++k) wait_bar(&full[k % S], (k / S) & 1);
-        if (p.a_whole) wait_bar(abar, 0);
-        return;
+        for (int it = warp; it < pro; it += kCW) issue_w(it);
     }
 
-    // ---------------------------------------------------------------- consumer warps
-    const int g = lane >> 2, t = lane & 3;
-    const int us = warp & (kKC - 1), hf = warp >> 3;  // unit slot in the chunk, k-step half
+    // ---- scale / zero table of the CTA's rows, group-major: {scale, zero point as integer bits}
+    if constexpr (WB == 4) {
+        wait_bar(scbar, 0);  // on expiry the error is recorded; carry on to the next barrier
+        const int nent = ntc * kTileRows * p.G;
+        const int nsm = int(sc16 >> 1);
+        for (int e = threadIdx.x; e < nent; e += kThreads) {
+            const int rl = e / p.G, gi = e - rl * p.G;
+            float sv = 0.f;
+            uint32_t zv = 8;
+            if (rl < nrows) {
+                const uint16_t sb = e < nsm ? sc_st[e] : p.scales16[(size_t)r0 * p.G + e];
+                sv = __half2float(__ushort_as_half(sb));
+                if (!p.sym) {
+                    const uint16_t zb = e < nsm ? zc_st[e] : p.zeros[(size_t)r0 * p.G + e];
+                    zv = uint32_t(__half2float(__ushort_as_half(zb))) & 15u;
+                }
+            }
+            stab[(size_t)gi * p.tab_rs + rl] = make_float2(sv, __uint_as_float(zv));
+        }
+    }
+
+    grid_dep_wait();  // activations, a_scale and bias may be written by the previous kernel
+    if (lane == 0 && !p.a_whole)
+        for (int it = warp; it < pro; it += kCW) issue_a(it);
+    if (p.a_whole && threadIdx.x == 0) {
+        // all of K, one bulk copy per token row; zeros past K up to the last unit
+        const int kpad = p.KB * KU;
+        for (int m = 0; m < p.M; ++m)
+            for (int k = p.K; k < kpad; ++k) {
+                if constexpr (ES == 1) abuf[(size_t)m * p.a_pitch_b + k] = 0;
+                else reinterpret_cast<uint16_t *>(abuf + (size_t)m * p.a_pitch_b)[k] = 0;
+            }
+        const uint32_t bytes = uint32_t(p.K) * ES;
+        mbar_arrive_expect_tx(abar, bytes * p.M);
+        for (int m = 0; m < p.M; ++m)
+            bulk_load(abuf + (size_t)m * p.a_pitch_b, static_cast<const uint8_t *>(p.A) + (size_t)m * bytes, bytes,
+                      abar);
+    }
+    __syncthreads();  // table (and activation padding) visible; no early exit before this point
+    if (p.a_whole && !wait_bar(abar, 0)) return;
+
     uint32_t cphase = 0;
-    auto csync = [&]() -> bool {  // bounded barrier of the consumer warps
+    auto csync = [&]() -> bool {  // bounded barrier of all threads
         mbar_arrive(cbar);
         const bool ok = wait_bar(cbar, cphase & 1);
         ++cphase;
         return ok;
     };
-    if (!wait_bar(scbar, 0)) return;
-    if constexpr (WB == 4) {
-        if (p.sc_smem) {
-            const int nent = (r1 - r0) * p.G;
-            for (int e = threadIdx.x; e < nent; e += kCW * 32)
-                stab[e] = make_float2(__half2float(__ushort_as_half(sc[e])),
-                                      p.sym ? 8.f : __half2float(__ushort_as_half(zc[e])));
-        }
-    }
-    if (!csync()) return;
-    grid_dep_wait();  // a_scale and bias may come from the previous kernel
-    if (p.a_whole && !wait_bar(abar, 0)) return;
 
-    // this lane's bytes inside a tile's 8 KB chunk part: box us/4, bytes (us%4)*64 + 16t + 8hf
-    const int woff = (us / kUPB) * kWBox + (us % kUPB) * kUnitBytes + 16 * t + 8 * hf;
+    const int g = lane >> 2, t = lane & 3;
+    const int us = warp % KC, hf = warp / KC;
+    // this lane's 16 bytes of rows g and g+8 of a tile, unit slot us ([pair][16 rows][128 B], swizzled)
+    const uint32_t lin_lo = uint32_t(((us >> 1) * kTileRows + g) * kPairBytes + (us & 1) * 64 + 16 * t);
+    const uint32_t off_lo = swz128(lin_lo), off_hi = swz128(lin_lo + 8 * kPairBytes);
 
-    for (int grp = 0; grp < ngrp; ++grp) {
-        const int ntg = min(p.TG, ntc - grp * p.TG);
-        Tot tot[kTGMax][NT][4];
+    int it = 0;
+    for (int pass = 0; pass < npass; ++pass) {
+        const int ntp = min(p.TPP, ntc - pass * p.TPP);
+        const int nmine = max(0, (ntp - hf + WPU - 1) / WPU);  // tiles hf, hf + WPU, ...
+        Tot tot[TM][NT][4];
 #pragma unroll
-        for (int i = 0; i < kTGMax; ++i)
+        for (int i = 0; i < TM; ++i)
 #pragma unroll
             for (int j = 0; j < NT; ++j)
 #pragma unroll
                 for (int e = 0; e < 4; ++e) tot[i][j][e] = Tot(0);
 
-        for (int ch = 0; ch < p.nch; ++ch) {
-            const int it = grp * p.nch + ch;
+        for (int ch = 0; ch < p.nch; ++ch, ++it) {
             const int s = it % S;
             if (!wait_bar(&full[s], (it / S) & 1)) return;
             const uint8_t *st = ring + size_t(s) * p.stage_bytes;
-            const int kb = ch * kKC + us;
-            if (kb < p.KB) {
-                const uint8_t *ablk = p.a_whole ? abuf + (size_t)kb * KU * ES
-                                                : st + p.wpart_bytes + (us / UPA) * p.abox_bytes + (us % UPA) * KU * ES;
-                const int pitch = p.a_whole ? p.a_pitch_b : kABoxElems * ES;
-                uint4 bf[NT][QH];
+            const int kb = ch * KC + us;
+            if (kb < p.KB && nmine > 0) {
+                uint4 bf[NT][QN];
                 int asum[NT];
+                if (p.a_whole) {
+                    const uint8_t *ablk = abuf + (size_t)kb * AU;
+                    const int pitch = p.a_pitch_b;
+                    auto addr = [=](int m, int o) { return ablk + m * pitch + o; };
 #pragma unroll
-                for (int j = 0; j < NT; ++j) build_bfrag_half<WB, AM>(ablk, pitch, p.M, j, lane, hf, bf[j], asum[j]);
+                    for (int j = 0; j < NT; ++j) build_bfrag<WB, AM>(addr, p.M, j, lane, bf[j], asum[j]);
+                } else {
+                    const uint8_t *abase = st + p.wpart_bytes;
+                    const int MB = p.MB;
+                    auto addr = [=](int m, int o) {
+                        const uint32_t x = uint32_t(us * AU + o);
+                        return abase + swz128(((x >> 7) * MB + m) * 128u + (x & 127u));
+                    };
+#pragma unroll
+                    for (int j = 0; j < NT; ++j) build_bfrag<WB, AM>(addr, p.M, j, lane, bf[j], asum[j]);
+                }
                 int sA[NT][2];
                 if constexpr (AM == A_I8) {
 #pragma unroll
@@ -319,56 +326,45 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                 }
                 const int gi = (WB == 4) ? (kb * KU) / p.gs : 0;
+                const float2 *srow = stab + (size_t)gi * p.tab_rs + pass * p.TPP * kTileRows + g;
 #pragma unroll
-                for (int ip = 0; ip < kTGMax / 2; ++ip) {
-                    if (2 * ip >= ntg) break;
-                    uint2 wa[2], wb[2];
-                    float s_lo[2], s_hi[2];
-                    uint32_t zl[2], zh[2];
+                for (int jp = 0; jp < TM; jp += NTL) {
+                    if (jp >= nmine) break;
+                    uint4 wa[NTL], wb[NTL];
+                    float s_lo[NTL], s_hi[NTL];
+                    uint32_t zl[NTL], zh[NTL];
 #pragma unroll
-                    for (int l = 0; l < 2; ++l) {
-                        const int i = 2 * ip + l;  // tile i >= ntg: stale data, result discarded
-                        const uint8_t *wt = st + i * kTileChunk + woff;
-                        wa[l] = lds64(wt + g * kWBoxBytes);
-                        wb[l] = lds64(wt + (g + 8) * kWBoxBytes);
+                    for (int l = 0; l < NTL; ++l) {
+                        const int j = min(jp + l, nmine - 1);  // a missing partner repeats a tile, unused
+                        const int i = hf + WPU * j;
+                        const uint8_t *wt = st + i * p.wtile_bytes;
+                        wa[l] = lds128(wt + off_lo);
+                        wb[l] = lds128(wt + off_hi);
                         s_lo[l] = s_hi[l] = 0.f;
                         zl[l] = zh[l] = 8;
                         if constexpr (WB == 4) {
-                            const int rl = (grp * p.TG + i) * kTileRows + g;  // row within the CTA
-                            if (p.sc_smem) {
-                                // rows past the CTA's end read stale table entries: never stored
-                                const float2 v_lo = stab[rl * p.G + gi];
-                                const float2 v_hi = stab[(rl + 8) * p.G + gi];
-                                s_lo[l] = v_lo.x;
-                                s_hi[l] = v_hi.x;
-                                zl[l] = uint32_t(v_lo.y) & 15u;
-                                zh[l] = uint32_t(v_hi.y) & 15u;
-                            } else {
-                                const int n_lo = r0 + rl, n_hi = n_lo + 8;
-                                if (n_lo < p.N) {
-                                    s_lo[l] = __half2float(__ushort_as_half(p.scales16[(size_t)n_lo * p.G + gi]));
-                                    if (!p.sym) zl[l] = uint32_t(__half2float(__ushort_as_half(p.zeros[(size_t)n_lo * p.G + gi])));
-                                }
-                                if (n_hi < p.N) {
-                                    s_hi[l] = __half2float(__ushort_as_half(p.scales16[(size_t)n_hi * p.G + gi]));
-                                    if (!p.sym) zh[l] = uint32_t(__half2float(__ushort_as_half(p.zeros[(size_t)n_hi * p.G + gi])));
-                                }
-                            }
+                            const float2 v_lo = srow[i * kTileRows];
+                            const float2 v_hi = srow[i * kTileRows + 8];
+                            s_lo[l] = v_lo.x;
+                            s_hi[l] = v_hi.x;
+                            zl[l] = __float_as_uint(v_lo.y);
+                            zh[l] = __float_as_uint(v_hi.y);
                         }
                     }
-                    acc_t<AM> ua[2][2][NT][4];
+                    acc_t<AM> ua[2][NTL][NT][4];
 #pragma unroll
                     for (int a = 0; a < 2; ++a)
 #pragma unroll
-                        for (int l = 0; l < 2; ++l)
+                        for (int l = 0; l < NTL; ++l)
 #pragma unroll
                             for (int j = 0; j < NT; ++j)
 #pragma unroll
                                 for (int e = 0; e < 4; ++e) ua[a][l][j][e] = acc_t<AM>(0);
-                    unit_mma_half<WB, AM, NT, 2>(wa, wb, bf, zl, zh, ua);
+                    unit_mma<WB, AM, NT, NTL>(wa, wb, bf, zl, zh, ua);
 #pragma unroll
-                    for (int l = 0; l < 2; ++l) {
-                        const int i = 2 * ip + l;
+                    for (int l = 0; l < NTL; ++l) {
+                        if (jp + l >= nmine) break;
+                        const int i = hf + WPU * (jp + l);
 #pragma unroll
                         for (int j = 0; j < NT; ++j)
 #pragma unroll
@@ -376,59 +372,71 @@ __global__ void __launch_bounds__(kThreads, 1)
                                 const acc_t<AM> v = ua[0][l][j][e] + ua[1][l][j][e];
                                 const float sc_e = (e < 2) ? s_lo[l] : s_hi[l];
                                 if constexpr (AM == A_I8 && WB == 2) {
-                                    tot[i][j][e] += v - 2 * sA[j][e & 1];
+                                    tot[jp + l][j][e] += v - 2 * sA[j][e & 1];
                                 } else if constexpr (AM == A_I8) {
                                     const int corr = v - int((e < 2) ? zl[l] : zh[l]) * sA[j][e & 1];
                                     if constexpr (ACC) {
-                                        const int n = r0 + (grp * p.TG + i) * kTileRows + g + ((e & 2) ? 8 : 0);
+                                        const int n = r0 + (pass * p.TPP + i) * kTileRows + g + ((e & 2) ? 8 : 0);
                                         const int m = j * 8 + 2 * t + (e & 1);
-                                        if (i < ntg && n < p.N && m < p.M)
-                                            atomicAdd(&p.acc_out[((long long)m * p.N + n) * p.G + kb], corr);
+                                        if (n < p.N && m < p.M) p.acc_out[((long long)m * p.N + n) * p.G + kb] = corr;
                                     }
-                                    tot[i][j][e] = fmaf(sc_e, float(corr), tot[i][j][e]);
+                                    tot[jp + l][j][e] = fmaf(sc_e, float(corr), tot[jp + l][j][e]);
                                 } else if constexpr (WB == 2) {
-                                    tot[i][j][e] += v;
+                                    tot[jp + l][j][e] += v;
                                 } else {
-                                    tot[i][j][e] = fmaf(sc_e, v, tot[i][j][e]);
+                                    tot[jp + l][j][e] = fmaf(sc_e, v, tot[jp + l][j][e]);
                                 }
                             }
                     }
                 }
             }
+            // stage consumed: the last of the 16 warps refills it with chunk it + S
             __syncwarp();
-            if (lane == 0) mbar_arrive(&empty[s]);
-        }
-
-        // ---- add the 16 warps' partial sums (fixed order) and write C ----
-#pragma unroll
-        for (int i = 0; i < kTGMax; ++i) {
-            if (i >= ntg) break;
-#pragma unroll
-            for (int j = 0; j < NT; ++j) {
-                float v[4];
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    if constexpr (AM == A_I8 && WB == 2) v[e] = __int_as_float(tot[i][j][e]);
-                    else v[e] = tot[i][j][e];
+            if (lane == 0) {
+                __threadfence_block();
+                if ((atomicAdd(&cnt[s], 1u) + 1u) % kCW == 0u) {
+                    __threadfence_block();
+                    fence_proxy_async();
+                    if (it + S < total_it) {
+                        issue_w(it + S);
+                        if (!p.a_whole) issue_a(it + S);
+                    }
                 }
-                const int m = j * 8 + 2 * t;
-                float *base = red + ((size_t)(warp * p.TG + i) * kTileRows) * MP;
-                *reinterpret_cast<float2 *>(base + g * MP + m) = make_float2(v[0], v[1]);
-                *reinterpret_cast<float2 *>(base + (g + 8) * MP + m) = make_float2(v[2], v[3]);
             }
         }
+
+        // ---- the pass's partial sums: red[tile][unit slot][row][token], then a fixed-order sum
+        if (!csync()) return;  // every warp is past the pass's last chunk
+#pragma unroll
+        for (int jj = 0; jj < TM; ++jj) {
+            if (jj >= nmine) break;
+            const int i = hf + WPU * jj;
+#pragma unroll
+            for (int j = 0; j < NT; ++j)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int m = j * 8 + 2 * t + (e & 1);
+                    const int r = g + ((e & 2) ? 8 : 0);
+                    if (m < p.M) {
+                        float v;
+                        if constexpr (AM == A_I8 && WB == 2) v = __int_as_float(tot[jj][j][e]);
+                        else v = tot[jj][j][e];
+                        red[((size_t)(m * p.TPP + i) * KC + us) * kTileRows + r] = v;
+                    }
+                }
+        }
         if (!csync()) return;
-        const int rows = ntg * kTileRows;
-        for (int e = threadIdx.x; e < rows * MP; e += kCW * 32) {
-            const int m = e / rows, rr = e % rows;
+        const int rows = ntp * kTileRows;
+        for (int e = threadIdx.x; e < rows * p.M; e += kThreads) {
+            const int m = e / rows, rr = e - m * rows;
             const int i = rr / kTileRows, r = rr % kTileRows;
-            const int n = r0 + (grp * p.TG + i) * kTileRows + r;
-            if (n >= p.N || m >= p.M) continue;
+            const int n = r0 + (pass * p.TPP + i) * kTileRows + r;
+            if (n >= p.N) continue;
             float sf = 0.f;
             int si = 0;
 #pragma unroll
-            for (int w = 0; w < kCW; ++w) {
-                const float v = red[((size_t)(w * p.TG + i) * kTileRows + r) * MP + m];
+            for (int u = 0; u < KC; ++u) {
+                const float v = red[((size_t)(m * p.TPP + i) * KC + u) * kTileRows + r];
                 sf += v;
                 si += __float_as_int(v);
             }
@@ -436,71 +444,88 @@ __global__ void __launch_bounds__(kThreads, 1)
             if constexpr (AM == A_I8 && WB == 2)
                 if (p.acc_out) p.acc_out[(long long)m * p.N + n] = si;
         }
-        if (grp + 1 < ngrp && !csync()) return;  // red is reused by the next group
+        if (pass + 1 < npass && !csync()) return;  // red is reused by the next pass
     }
 }
 
 // ---------------------------------------------------------------- host side
 struct Plan {
-    int NT = 1, MP = 8, KU = 128, KB = 0, T = 0, P = 0, nch = 0, TG = 1, S = 2;
-    int a_whole = 0, a_pitch_b = 0, abox = 0, wpart = 0, stage = 0, sc_smem = 0, sc_rows_cap = 0;
+    int NT = 1, KC = 16, KU = 128, KB = 0, T = 0, P = 0, nch = 0, TPP = 1, S = 1;
+    int w3d = 0, wtile = 0, wpart = 0, stage = 0;
+    int a_whole = 0, a_pitch_b = 0, abox = 0, MB = 8, rows_cap = 0, tab_rs = 1;
+    int abuf_off = 0, scst_off = 0, stab_off = 0, red_off = 0, bar_off = 0;
     size_t smem = 0;
     bool ok = false;
 };
+
+size_t up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 Plan make_plan(int64_t M, int64_t N, int64_t K, int WB, int AM, int G, const DeviceInfo &dev)
 {
     Plan pl;
     pl.NT = M <= 8 ? 1 : 2;
-    pl.MP = pl.NT * 8;
+    if (WB == 2 && AM != A_I8 && pl.NT == 2) return pl;  // B fragments would not fit in registers
+    pl.KC = kc_of(pl.NT);
     pl.KU = kunit_of(WB);
     pl.KB = int((K + pl.KU - 1) / pl.KU);
     pl.T = int((N + kTileRows - 1) / kTileRows);
     pl.P = std::min(dev.sm_count, pl.T);
-    pl.nch = (pl.KB + kKC - 1) / kKC;
-    const int tiles_max = (pl.T + pl.P - 1) / pl.P;
+    const int ntc_max = (pl.T + pl.P - 1) / pl.P;
+    pl.TPP = std::min(ntc_max, tm_of(pl.NT) * wpu_of(pl.NT));
+    const int npass = (ntc_max + pl.TPP - 1) / pl.TPP;
+    pl.nch = (pl.KB + pl.KC - 1) / pl.KC;
+    const long long total = (long long)npass * pl.nch;
     const int es = AM == A_I8 ? 1 : 2;
-    pl.sc_rows_cap = tiles_max * kTileRows;
-    const size_t sc_bytes = (WB == 4) ? size_t(pl.sc_rows_cap) * G * (8 + 2 + 2) : 0;
-    pl.sc_smem = (WB == 4 && sc_bytes <= 48 * 1024) ? 1 : 0;
-    if (!pl.sc_smem) pl.sc_rows_cap = 0;
-    const size_t sc_area = pl.sc_smem ? sc_bytes : 0;
-    pl.TG = std::min(tg_max(pl.NT), tiles_max);
-    const int tg_alloc = pl.TG + (pl.TG & 1);  // pairs: the odd tile's partner is read but unused
-    pl.wpart = tg_alloc * kTileChunk;
-    const size_t red = size_t(kCW) * pl.TG * kTileRows * pl.MP * 4;
-    const size_t fixed = 1024 + sc_area + 16 + red + 8 * (2 * 8 + 3) + 16;
-    const size_t budget = size_t(dev.max_smem_optin);
-    const int ngrp = (tiles_max + pl.TG - 1) / pl.TG;
-    const long long total = (long long)ngrp * pl.nch;
+    const int au = pl.KU * es;
+    const int64_t row_bytes = K * WB / 8;
+    pl.w3d = (row_bytes % kPairBytes) == 0 ? 1 : 0;
+    pl.wtile = pl.KC * kTileRows * 64;
+    pl.wpart = pl.TPP * pl.wtile;
+    pl.rows_cap = ntc_max * kTileRows;
+    pl.tab_rs = pl.rows_cap | 1;
+    const size_t scst = (WB == 4) ? up(size_t(pl.rows_cap) * G * 2 * 2, 16) : 0;
+    const size_t table = (WB == 4) ? up(size_t(pl.tab_rs) * G * 8, 16) : 0;
+    const size_t red = up(size_t(pl.TPP) * pl.KC * kTileRows * M * 4, 16);
+    const size_t tail = scst + table + red + 8 * 19 + 4 * 16 + 64;  // + barriers (S <= 16), counters
+    const size_t budget = size_t(dev.max_smem_optin) - 1024;  // 1 KB for the alignment of the base
     auto stages_for = [&](size_t stage, size_t extra) -> long long {
-        if (budget <= fixed + extra) return 0;
-        return std::min<long long>({8, total, (long long)((budget - fixed - extra) / stage)});
+        if (budget <= tail + extra) return 0;
+        return std::min<long long>({16, total, (long long)((budget - tail - extra) / stage)});
     };
-    // whole activations: one copy for all of K; otherwise per chunk by TMA
-    const int a_pitch_whole = pl.KB * pl.KU * es + kAPadBytes;
-    const size_t abuf = (size_t(M) * a_pitch_whole + 127) & ~size_t(127);
+    const int a_pitch_whole = pl.KB * au + 16;  // padded rows spread the token rows over the banks
+    const size_t abuf = up(size_t(M) * a_pitch_whole, 128);
     const long long s_whole = stages_for(pl.wpart, abuf);
-    const int abox = int(M) * kABoxElems * es;
-    const int apart = (kKC * pl.KU / kABoxElems) * abox;
-    const size_t stage_chunked = (size_t(pl.wpart + apart) + 1023) & ~size_t(1023);
-    const long long s_chunked = stages_for(stage_chunked, 0);
-    const long long want = std::min<long long>(4, total);
+    pl.MB = int(up(size_t(M), 8));
+    const int abox = pl.MB * pl.KC * au;
+    const bool chunk_ok = (K * es) % 128 == 0;
+    const long long s_chunked = chunk_ok ? stages_for(size_t(pl.wpart) + abox, 0) : 0;
+    const long long want = std::min<long long>(2, total);
     if (s_whole >= want || (s_whole >= 1 && s_whole >= s_chunked)) {
         pl.a_whole = 1;
         pl.a_pitch_b = a_pitch_whole;
         pl.stage = pl.wpart;
         pl.S = int(s_whole);
-        pl.smem = fixed + abuf + size_t(pl.S) * pl.stage;
-    } else {
+    } else if (s_chunked >= 1) {
         pl.a_whole = 0;
-        pl.a_pitch_b = kABoxElems * es;
         pl.abox = abox;
-        pl.stage = int(stage_chunked);
+        pl.stage = pl.wpart + abox;
         pl.S = int(s_chunked);
-        pl.smem = fixed + size_t(pl.S) * pl.stage;
+    } else {
+        return pl;
     }
-    pl.ok = pl.S >= 1 && pl.smem <= budget;
+    size_t off = size_t(pl.S) * pl.stage;
+    pl.abuf_off = int(off);
+    off += pl.a_whole ? abuf : 0;
+    pl.scst_off = int(off);
+    off += scst;
+    pl.stab_off = int(off);
+    off += table;
+    pl.red_off = int(off);
+    off += red;
+    pl.bar_off = int(up(off, 8));
+    off = pl.bar_off + size_t(8) * (pl.S + 3) + size_t(4) * pl.S;
+    pl.smem = up(off, 16) + 1024;
+    pl.ok = pl.smem <= size_t(dev.max_smem_optin);
     return pl;
 }
 
@@ -538,19 +563,37 @@ wq_status gemv_small_m(int WB, int AM, const void *A, const float *a_scale, cons
 {
     const DeviceInfo &dev = device_info();
     const int G = WB == 4 ? int(K / c.group_size) : 1;
-    const Plan pl = make_plan(M, N, K, WB, AM, G, dev);
-    if (!pl.ok) return fail(WQ_ERR_UNSUPPORTED, "no shared-memory plan for M=%lld K=%lld", (long long)M, (long long)K);
+    Plan pl = make_plan(M, N, K, WB, AM, G, dev);
+    if (!pl.ok) return fail(WQ_ERR_UNSUPPORTED, "no few-token plan for M=%lld K=%lld", (long long)M, (long long)K);
     CUtensorMap tw, ta;
     const uint64_t row_bytes = uint64_t(K) * WB / 8;
-    wq_status rc = encode_tmap_2d(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, Wq, row_bytes, uint64_t(N), row_bytes,
-                                  kWBoxBytes, kTileRows);
+    wq_status rc = WQ_ERR_UNSUPPORTED;
+    if (pl.w3d) {
+        // (128-byte unit pair, row, pair): one box = 16 rows x KC units
+        const uint64_t dims[3] = {uint64_t(kPairBytes), uint64_t(N), row_bytes / kPairBytes};
+        const uint64_t strides[2] = {row_bytes, uint64_t(kPairBytes)};
+        const uint32_t box[3] = {uint32_t(kPairBytes), uint32_t(kTileRows), uint32_t(pl.KC / 2)};
+        rc = encode_tmap(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, Wq, dims, strides, box, true);
+        if (rc != WQ_OK) pl.w3d = 0;  // same shared-memory layout from one 2D box per unit pair
+    }
+    if (!pl.w3d) {
+        const uint64_t dims[2] = {row_bytes, uint64_t(N)};
+        const uint64_t strides[1] = {row_bytes};
+        const uint32_t box[2] = {uint32_t(kPairBytes), uint32_t(kTileRows)};
+        rc = encode_tmap(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, Wq, dims, strides, box, true);
+    }
     if (rc != WQ_OK) return rc;
-    const int esize = AM == A_I8 ? 1 : 2;
+    const int es = AM == A_I8 ? 1 : 2;
     ta = tw;  // unused when the activations are staged whole
     if (!pl.a_whole) {
-        rc = encode_tmap_2d(&ta, AM == A_I8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_UINT16, A,
-                            uint64_t(K), uint64_t(M), uint64_t(K) * esize, uint32_t(kABoxElems), uint32_t(M));
-        if (rc != WQ_OK) return rc;
+        // (128 bytes, token, 128-byte block of K): one box = MB tokens x KC units
+        const uint64_t kbytes = uint64_t(K) * es;
+        const uint64_t dims[3] = {uint64_t(128 / es), uint64_t(M), kbytes / 128};
+        const uint64_t strides[2] = {kbytes, 128};
+        const uint32_t box[3] = {uint32_t(128 / es), uint32_t(pl.MB), uint32_t(pl.KC * pl.KU * es / 128)};
+        rc = encode_tmap(&ta, es == 1 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_UINT16, 3, A, dims,
+                         strides, box, true);
+        if (rc != WQ_OK) return fail(WQ_ERR_UNSUPPORTED, "few-token plan: activation tensor map (%s)", wq_last_error());
     }
     GemvParams p{};
     p.A = A;
@@ -564,15 +607,23 @@ wq_status gemv_small_m(int WB, int AM, const void *A, const float *a_scale, cons
     p.T = pl.T;
     p.P = pl.P;
     p.nch = pl.nch;
-    p.TG = pl.TG;
+    p.TPP = pl.TPP;
     p.S = pl.S;
+    p.w3d = pl.w3d;
+    p.wtile_bytes = pl.wtile;
+    p.wpart_bytes = pl.wpart;
+    p.stage_bytes = pl.stage;
     p.a_whole = pl.a_whole;
     p.a_pitch_b = pl.a_pitch_b;
     p.abox_bytes = pl.abox;
-    p.wpart_bytes = pl.wpart;
-    p.stage_bytes = pl.stage;
-    p.sc_smem = pl.sc_smem;
-    p.sc_rows_cap = pl.sc_rows_cap;
+    p.MB = pl.MB;
+    p.rows_cap = pl.rows_cap;
+    p.tab_rs = pl.tab_rs;
+    p.abuf_off = pl.abuf_off;
+    p.scst_off = pl.scst_off;
+    p.stab_off = pl.stab_off;
+    p.red_off = pl.red_off;
+    p.bar_off = pl.bar_off;
     p.scales16 = static_cast<const uint16_t *>(scales);
     p.scale32 = static_cast<const float *>(scales);
     p.zeros = static_cast<const uint16_t *>(zeros);
@@ -580,21 +631,16 @@ wq_status gemv_small_m(int WB, int AM, const void *A, const float *a_scale, cons
     p.a_scale = a_scale;
     p.C = C;
     p.acc_out = acc_out;
-    const int NT = pl.NT;
-#define WQ_LAUNCH(wb, am) return NT == 1 ? launch<wb, am, 1>(pl, tw, ta, p, st) : launch<wb, am, 2>(pl, tw, ta, p, st)
-    if (WB == 4 && AM == A_F16) WQ_LAUNCH(4, A_F16);
-    if (WB == 4 && AM == A_BF16) WQ_LAUNCH(4, A_BF16);
-    if (WB == 4 && acc_out) {
-        // each group sum arrives in two halves from two warps: start from zero
-        if (cudaMemsetAsync(acc_out, 0, size_t(M) * N * G * sizeof(int32_t), st) != cudaSuccess)
-            return check_launch("cudaMemsetAsync(acc_out)");
-        return NT == 1 ? launch<4, A_I8, 1, true>(pl, tw, ta, p, st) : launch<4, A_I8, 2, true>(pl, tw, ta, p, st);
-    }
-    if (WB == 4) WQ_LAUNCH(4, A_I8);
-    if (AM == A_F16) WQ_LAUNCH(2, A_F16);
-    if (AM == A_BF16) WQ_LAUNCH(2, A_BF16);
-    WQ_LAUNCH(2, A_I8);
-#undef WQ_LAUNCH
+    const bool one = pl.NT == 1;
+    if (WB == 4 && AM == A_F16) return one ? launch<4, A_F16, 1>(pl, tw, ta, p, st) : launch<4, A_F16, 2>(pl, tw, ta, p, st);
+    if (WB == 4 && AM == A_BF16)
+        return one ? launch<4, A_BF16, 1>(pl, tw, ta, p, st) : launch<4, A_BF16, 2>(pl, tw, ta, p, st);
+    if (WB == 4 && acc_out)
+        return one ? launch<4, A_I8, 1, true>(pl, tw, ta, p, st) : launch<4, A_I8, 2, true>(pl, tw, ta, p, st);
+    if (WB == 4) return one ? launch<4, A_I8, 1>(pl, tw, ta, p, st) : launch<4, A_I8, 2>(pl, tw, ta, p, st);
+    if (AM == A_F16) return launch<2, A_F16, 1>(pl, tw, ta, p, st);
+    if (AM == A_BF16) return launch<2, A_BF16, 1>(pl, tw, ta, p, st);
+    return one ? launch<2, A_I8, 1>(pl, tw, ta, p, st) : launch<2, A_I8, 2>(pl, tw, ta, p, st);
 }
 
 int gemv_read_error()
