@@ -23,6 +23,9 @@ wq_status gemv_small_m(int WB, int AM, const void *A, const float *a_scale, cons
                        const void *zeros, const void *bias, void *C, int32_t *acc_out, int64_t M, int64_t N,
                        int64_t K, const wq_qconfig &c, cudaStream_t st);
 int gemv_read_error();
+wq_status tc_gemm(int WB, int AM, const void *A, const uint8_t *Wq, const void *scales, const void *zeros,
+                  const void *bias, void *C, int64_t M, int64_t N, int64_t K, const wq_qconfig &c, cudaStream_t st);
+int tc_read_error();
 
 namespace {
 thread_local char g_last_error[512] = "";
@@ -98,7 +101,7 @@ wq_status encode_tmap_2d(CUtensorMap *map, CUtensorMapDataType dt, const void *b
 }
 
 wq_status encode_tmap(CUtensorMap *map, CUtensorMapDataType dt, int rank, const void *base, const uint64_t *dims,
-                      const uint64_t *strides_bytes, const uint32_t *box, bool swizzle128)
+                      const uint64_t *strides_bytes, const uint32_t *box, int swizzle_bytes)
 {
     EncodeFn fn = encode_fn();
     if (!fn) return fail(WQ_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
@@ -112,7 +115,9 @@ wq_status encode_tmap(CUtensorMap *map, CUtensorMapDataType dt, int rank, const 
     for (int i = 0; i + 1 < rank; ++i) st[i] = strides_bytes[i];
     CUresult r = fn(map, dt, cuuint32_t(rank), const_cast<void *>(base), d, st, b, estr,
                     CU_TENSOR_MAP_INTERLEAVE_NONE,
-                    swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                    swizzle_bytes == 128  ? CU_TENSOR_MAP_SWIZZLE_128B
+                    : swizzle_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                          : CU_TENSOR_MAP_SWIZZLE_NONE,
                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return fail(WQ_ERR_INVALID_ARG, "cuTensorMapEncodeTiled (rank %d) failed (%d)", rank, int(r));
     return WQ_OK;
@@ -120,18 +125,22 @@ wq_status encode_tmap(CUtensorMap *map, CUtensorMapDataType dt, int rank, const 
 
 int read_device_errors()
 {
-    const int a = skinny_read_error(), b = gemv_read_error();
-    return a ? a : b;
+    const int a = skinny_read_error(), b = gemv_read_error(), t = tc_read_error();
+    return a ? a : (b ? b : t);
 }
 
 namespace {
-// Few tokens go to the weight-streaming GEMV; more tokens to the tiled path.
+// Few tokens go to the weight-streaming GEMV; more tokens to the tcgen05 GEMM (INT4 weights,
+// FP activations) or else to the tiled mma.sync path.
 wq_status dispatch(int WB, int AM, const void *A, const float *a_scale, const uint8_t *Wq, const void *scales,
                    const void *zeros, const void *bias, void *C, int32_t *acc_out, int64_t M, int64_t N, int64_t K,
                    const wq_qconfig &c, void *ws, size_t ws_bytes, cudaStream_t st)
 {
     if (M <= 16) {
         wq_status rc = gemv_small_m(WB, AM, A, a_scale, Wq, scales, zeros, bias, C, acc_out, M, N, K, c, st);
+        if (rc != WQ_ERR_UNSUPPORTED) return rc;
+    } else if (AM != 2 && !acc_out) {
+        wq_status rc = tc_gemm(WB, AM, A, Wq, scales, zeros, bias, C, M, N, K, c, st);
         if (rc != WQ_ERR_UNSUPPORTED) return rc;
     }
     return skinny_gemm(WB, AM, A, a_scale, Wq, scales, zeros, bias, C, acc_out, M, N, K, c, ws, ws_bytes, st);

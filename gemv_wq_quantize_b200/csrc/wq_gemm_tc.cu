@@ -1,0 +1,474 @@
+// wq_gemm_tc.cu -- many-token W4A16 matmul on the 5th-generation tensor cores (tcgen05).
+//
+// C[M,N] = A[M,K] x dequant(Wq[N,K])^T with FP16 / BF16 activations and INT4 weights
+// (group scales, optional zero points): "BitBLAS practical guide", "What is BitBLAS" and
+// "Weight group quantization"; fp32 accumulation, one rounding to the output dtype.
+//
+// At prefill sizes the product is tensor-bound.  The weights are the MMA's A operand
+// (M = 128 weight rows) and live in Tensor Memory; the activations are the B operand
+// (N = 128 tokens), brought into shared memory by TMA with the 128-byte swizzle that the
+// MMA's K-major descriptor expects.  Per block of 128 k:
+//  * a producer warp TMAs the block's activations (32 KB) and packed weights (8 KB) into
+//    an S-stage ring;
+//  * eight math warps unpack the packed weights of their own row (thread = weight row,
+//    warp pairs split the 128 k) into the exact integers q - z as f16 / bf16 pairs in
+//    natural k order, and store them to a TMEM A-buffer (tcgen05.st);
+//  * one thread issues 8 MMAs of 128 x 128 x 16 into a TMEM accumulator of that block
+//    alone, and commits to mbarriers;
+//  * the math warps read the block's accumulator back (tcgen05.ld) and add it, times the
+//    row's group scale, into fp32 totals held in registers (each thread: one weight row x
+//    64 tokens).  A-buffers and accumulators are double-buffered, so unpacking, MMA and
+//    folding of consecutive blocks overlap.
+// The products are exact (|q - z| <= 15 times an f16 / bf16 activation); the only
+// rounding besides fp32 accumulation is the final conversion.  Persistent CTAs walk the
+// (weight tile, token tile) grid token-tile fastest so that concurrent CTAs share weight
+// tiles in L2.  Every wait is bounded; on expiry the CTA records an error, stops, waits
+// for what it has in flight and frees its Tensor Memory.
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <stdint.h>
+
+#include <algorithm>
+
+#include "wq_device.cuh"
+#include "wq_host.h"
+#include "wq_tc.cuh"
+
+namespace wq {
+
+static __device__ int g_tc_error;
+
+namespace {
+
+constexpr int kBW = 128;  // weight rows per tile: MMA M
+constexpr int kBT = 128;  // tokens per tile: MMA N
+constexpr int kKB = 128;  // k per block
+constexpr int kMathWarps = 8;
+constexpr int kThreads = (2 + kMathWarps) * 32;  // warp 0 TMA, warp 1 MMA + TMEM, warps 2..9 math
+constexpr int kActBox = kBT * 128;               // one 64-k box of activations: 128 rows x 128 B
+constexpr int kActBytes = 2 * kActBox;           // 32 KB
+constexpr int kWBytes = kBW * kKB / 2;           // 8 KB of packed weights
+constexpr int kStageBytes = kActBytes + kWBytes;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kAcol = 0;    // 2 x 64 columns: unpacked weights of a block (A operand)
+constexpr uint32_t kDcol = 128;  // 2 x 128 columns: the block's accumulators
+
+struct TcParams {
+    int M, N, K, G, gs, sym;
+    int nkb;     // K / 128
+    int TT, NT;  // token tiles, tiles
+    int S;       // ring stages
+    int scst_off, tab_off, bar_off;
+    int tab_rs;  // table row stride (entries; odd)
+    const uint16_t *scales16;
+    const uint16_t *zeros;
+    const void *bias;
+    void *C;
+};
+
+__device__ __forceinline__ uint64_t globaltimer()
+{
+    uint64_t t;
+    asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+    return t;
+}
+
+// Bounded wait (~2 s); on expiry, or once another warp has given up, returns false.
+__device__ __forceinline__ bool tc_wait(uint64_t *bar, uint32_t parity, volatile int *abort)
+{
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = globaltimer();
+    for (;;) {
+        for (int i = 0; i < 32; ++i)
+            if (mbar_try_wait(bar, parity)) return true;
+        if (*abort) return false;
+        if (globaltimer() - t0 > 2000000000ull) {
+            atomicCAS(&g_tc_error, kErrNone, kErrWaitTimeout);
+            *abort = 1;
+            return false;
+        }
+    }
+}
+
+
+template <bool BF16>
+__device__ __forceinline__ void store_out(void *C, long long idx, float v)
+{
+    if constexpr (BF16) static_cast<__nv_bfloat16 *>(C)[idx] = __float2bfloat16_rn(v);
+    else static_cast<__half *>(C)[idx] = __float2half_rn(v);
+}
+
+// Unpacks one 32-bit word (8 nibbles, k0 in the low nibble) into 4 pairs (k0,k1) .. (k6,k7)
+// of magic + nibble (f16: 1024 + q, bf16: 128 + q), then adds zc = -(magic + z): exact q - z.
+template <bool BF16>
+__device__ __forceinline__ void unpack_word(uint32_t w, uint32_t zc, uint32_t *o)
+{
+    const uint32_t magic = BF16 ? 0x43434343u : 0x64646464u;
+    const uint32_t lo = w & 0x0F0F0F0Fu;         // k0 k2 k4 k6
+    const uint32_t hi = (w >> 4) & 0x0F0F0F0Fu;  // k1 k3 k5 k7
+    const uint32_t p0 = prmt(lo, hi, 0x5140);    // k0 k1 k2 k3
+    const uint32_t p1 = prmt(lo, hi, 0x7362);    // k4 k5 k6 k7
+    uint32_t x[4] = {prmt(p0, magic, 0x4140), prmt(p0, magic, 0x4342), prmt(p1, magic, 0x4140),
+                     prmt(p1, magic, 0x4342)};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) o[i] = BF16 ? bf2_fma(x[i], 0x3F803F80u, zc) : h2_add(x[i], zc);
+}
+
+template <bool BF16>
+__global__ void __launch_bounds__(kThreads, 1)
+    tc_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_w,
+                   const TcParams p)
+{
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int S = p.S;
+    uint8_t *ring = smem;  // S x (activations 32 KB | packed weights 8 KB)
+    uint16_t *scst = reinterpret_cast<uint16_t *>(smem + p.scst_off);  // 2 x (scales, zeros) [128][G]
+    uint32_t *tab = reinterpret_cast<uint32_t *>(smem + p.tab_off);    // [G][tab_rs]: scale bits | z << 16
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + p.bar_off);
+    uint64_t *full = bars, *empty = bars + S;
+    uint64_t *afull = bars + 2 * S, *afree = afull + 2, *dfull = afull + 4, *dfree = afull + 6;
+    uint64_t *scbar = afull + 8, *fin = afull + 10, *mbar = afull + 11;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(afull + 12);
+    volatile int *abort = reinterpret_cast<volatile int *>(tmem_slot + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const size_t stab_elems = size_t(kBW) * p.G;  // one staging buffer (scales or zeros)
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < S; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], kMathWarps + 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&afull[b], kMathWarps);
+            mbar_init(&afree[b], 1);
+            mbar_init(&dfull[b], 1);
+            mbar_init(&dfree[b], kMathWarps);
+            mbar_init(&scbar[b], 1);
+        }
+        mbar_init(fin, 1);
+        mbar_init(mbar, kMathWarps * 32);
+        *abort = 0;
+        fence_barrier_init();
+    }
+    if (warp == 1) {
+        tc::tmem_alloc(tmem_slot, kTmemCols);
+        tc::tmem_relinquish();
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tbase = *tmem_slot;
+    grid_dep_launch();
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            tma_prefetch_desc(&tmap_a);
+            tma_prefetch_desc(&tmap_w);
+            grid_dep_wait();  // activations may be written by the previous kernel
+            uint32_t step = 0;
+            int tl = 0;
+            for (int t = blockIdx.x; t < p.NT && !*abort; t += gridDim.x, ++tl) {
+                const int n0 = (t / p.TT) * kBW, m0 = (t % p.TT) * kBT;
+                // the tile's scale / zero rows: contiguous in [N, G]
+                const int nrows = min(kBW, p.N - n0);
+                const uint32_t bytes16 = (uint32_t(nrows) * p.G * 2u) & ~15u;
+                uint16_t *sc = scst + size_t(tl & 1) * 2 * stab_elems;
+                mbar_arrive_expect_tx(&scbar[tl & 1], bytes16 * (p.sym ? 1u : 2u));
+                if (bytes16) {
+                    bulk_load(sc, p.scales16 + (size_t)n0 * p.G, bytes16, &scbar[tl & 1]);
+                    if (!p.sym) bulk_load(sc + stab_elems, p.zeros + (size_t)n0 * p.G, bytes16, &scbar[tl & 1]);
+                }
+                for (int kb = 0; kb < p.nkb; ++kb, ++step) {
+                    const int s = int(step % uint32_t(S));
+                    if (!tc_wait(&empty[s], ((step / S) & 1) ^ 1, abort)) break;
+                    uint8_t *st = ring + size_t(s) * kStageBytes;
+                    mbar_arrive_expect_tx(&full[s], kStageBytes);
+                    tma_load_2d(st, &tmap_a, kb * kKB, m0, &full[s]);
+                    tma_load_2d(st + kActBox, &tmap_a, kb * kKB + 64, m0, &full[s]);
+                    tma_load_2d(st + kActBytes, &tmap_w, kb * (kKB / 2), n0, &full[s]);
+                }
+            }
+            // nothing may land in shared memory after the CTA exits: wait for the last stages
+            for (uint32_t k = step > uint32_t(S) ? step - S : 0; k < step; ++k)
+                tc_wait(&full[k % S], (k / S) & 1, abort);
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            const uint32_t idesc = tc::idesc_f16(BF16, kBW, kBT);
+            uint32_t step = 0;
+            bool issued = false;
+            for (int t = blockIdx.x; t < p.NT && !*abort; t += gridDim.x) {
+                for (int kb = 0; kb < p.nkb; ++kb, ++step) {
+                    const int s = int(step % uint32_t(S));
+                    const uint32_t ab = step & 1, ph = (step >> 1) & 1;
+                    if (!tc_wait(&full[s], (step / S) & 1, abort)) break;
+                    if (!tc_wait(&afull[ab], ph, abort)) break;
+                    if (!tc_wait(&dfree[ab], ph ^ 1, abort)) break;
+                    tc::fence_after_sync();
+                    const uint32_t act = smem_u32(ring + size_t(s) * kStageBytes);
+#pragma unroll
+                    for (int kk = 0; kk < kKB / 16; ++kk) {
+                        const uint64_t bdesc = tc::sdesc_sw128(act + (kk >> 2) * kActBox + (kk & 3) * 32);
+                        tc::mma_f16_ts(tbase + kDcol + ab * kBT, tbase + kAcol + ab * 64 + kk * 8, bdesc, idesc,
+                                       kk > 0 ? 1u : 0u);
+                    }
+                    tc::commit(&dfull[ab]);
+                    tc::commit(&empty[s]);
+                    tc::commit(&afree[ab]);
+                    issued = true;
+                }
+            }
+            if (issued) {  // all MMAs complete before the Tensor Memory is freed
+                tc::commit(fin);
+                tc_wait(fin, 0, abort);
+            }
+        }
+    } else {
+        // ------------------------------------------------------------ math warps
+        const int q = warp & 3;             // TMEM lane quadrant of this warp
+        const int kh = (warp - 2) >> 2;     // k half (unpack) / token half (fold)
+        const int r = q * 32 + lane;        // weight row within the tile
+        const uint32_t tlane = tbase + (uint32_t(q * 32) << 16);
+        const uint32_t magic_z = BF16 ? 0xC300u : 0xE400u;  // -(magic + z) = magic_z | z
+        uint32_t step = 0, mphase = 0;
+        auto math_sync = [&]() -> bool {  // bounded barrier of the math warps
+            mbar_arrive(mbar);
+            const bool ok = tc_wait(mbar, mphase & 1, abort);
+            ++mphase;
+            return ok;
+        };
+        grid_dep_wait();  // C and bias belong to this kernel only once the previous one is done
+        int tl = 0;
+        for (int t = blockIdx.x; t < p.NT && !*abort; t += gridDim.x, ++tl) {
+            const int n0 = (t / p.TT) * kBW, m0 = (t % p.TT) * kBT;
+            const int nrows = min(kBW, p.N - n0);
+            // ---- scale / zero table of the tile: [g][row] = fp16 scale bits | z << 16
+            if (!tc_wait(&scbar[tl & 1], (tl >> 1) & 1, abort)) break;
+            if (!math_sync()) break;  // everyone is done with the previous tile's table
+            {
+                const uint16_t *sc = scst + size_t(tl & 1) * 2 * stab_elems;
+                const int n16 = int(((uint32_t(nrows) * p.G * 2u) & ~15u) >> 1);
+                for (int e = threadIdx.x - 64; e < kBW * p.G; e += kMathWarps * 32) {
+                    const int rl = e / p.G, gi = e - rl * p.G;
+                    uint32_t v = 0;
+                    if (rl < nrows) {
+                        const uint16_t sb = e < n16 ? sc[e] : p.scales16[(size_t)n0 * p.G + e];
+                        uint32_t z = 8;
+                        if (!p.sym) {
+                            const uint16_t zb = e < n16 ? sc[stab_elems + e] : p.zeros[(size_t)n0 * p.G + e];
+                            z = uint32_t(__half2float(__ushort_as_half(zb))) & 15u;
+                        }
+                        v = uint32_t(sb) | (z << 16);
+                    }
+                    tab[(size_t)gi * p.tab_rs + rl] = v;
+                }
+            }
+            if (!math_sync()) break;
+
+            float tot[64];
+#pragma unroll
+            for (int j = 0; j < 64; ++j) tot[j] = 0.f;
+            float s_prev = 0.f;
+            // fold the accumulator of step `fs` (its block scale `sv`) into the totals
+            auto fold = [&](uint32_t fs, float sv) -> bool {
+                const uint32_t db = fs & 1;
+                if (!tc_wait(&dfull[db], (fs >> 1) & 1, abort)) return false;
+                tc::fence_after_sync();
+                uint32_t d0[32], d1[32];
+                tc::ld_32x32b_x32(tlane + kDcol + db * kBT + kh * 64, d0);
+                tc::ld_32x32b_x32(tlane + kDcol + db * kBT + kh * 64 + 32, d1);
+                tc::wait_ld();
+                tc::fence_before_sync();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&dfree[db]);
+#pragma unroll
+                for (int j = 0; j < 32; ++j) {
+                    tot[j] = fmaf(sv, __uint_as_float(d0[j]), tot[j]);
+                    tot[32 + j] = fmaf(sv, __uint_as_float(d1[j]), tot[32 + j]);
+                }
+                return true;
+            };
+
+            bool ok = true;
+            for (int kb = 0; kb < p.nkb && ok; ++kb, ++step) {
+                const int s = int(step % uint32_t(S));
+                const uint32_t ab = step & 1, ph = (step >> 1) & 1;
+                if (!tc_wait(&full[s], (step / S) & 1, abort)) { ok = false; break; }
+                // this row's 32 packed bytes of the k half (64-byte rows, 64-byte swizzle)
+                const uint8_t *wrow = ring + size_t(s) * kStageBytes + kActBytes + r * 64;
+                const uint32_t sw = uint32_t((r >> 1) & 3);
+                const uint4 w0 = lds128(wrow + (((2 * kh) ^ sw) << 4));
+                const uint4 w1 = lds128(wrow + (((2 * kh + 1) ^ sw) << 4));
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&empty[s]);
+                const uint32_t tv = tab[(size_t)((kb * kKB) / p.gs) * p.tab_rs + r];
+                const uint32_t zc1 = magic_z | (tv >> 16);
+                const uint32_t zc = zc1 | (zc1 << 16);
+                uint32_t v[32];
+                unpack_word<BF16>(w0.x, zc, v + 0);
+                unpack_word<BF16>(w0.y, zc, v + 4);
+                unpack_word<BF16>(w0.z, zc, v + 8);
+                unpack_word<BF16>(w0.w, zc, v + 12);
+                unpack_word<BF16>(w1.x, zc, v + 16);
+                unpack_word<BF16>(w1.y, zc, v + 20);
+                unpack_word<BF16>(w1.z, zc, v + 24);
+                unpack_word<BF16>(w1.w, zc, v + 28);
+                if (!tc_wait(&afree[ab], ph ^ 1, abort)) { ok = false; break; }
+                tc::fence_after_sync();
+                tc::st_32x32b_x32(tlane + kAcol + ab * 64 + kh * 32, v);
+                tc::wait_st();
+                tc::fence_before_sync();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&afull[ab]);
+                if (kb > 0 && !fold(step - 1, s_prev)) { ok = false; break; }
+                s_prev = __half2float(__ushort_as_half(uint16_t(tv & 0xFFFFu)));
+            }
+            if (!ok || !fold(step - 1, s_prev)) break;
+
+            // ---- epilogue: C[m][n] = total (+ bias[n]), one weight row x 64 tokens per thread
+            const int n = n0 + r;
+            if (n < p.N) {
+                float b = 0.f;
+                if (p.bias) {
+                    if constexpr (BF16) b = __bfloat162float(static_cast<const __nv_bfloat16 *>(p.bias)[n]);
+                    else b = __half2float(static_cast<const __half *>(p.bias)[n]);
+                }
+                const int mb = m0 + kh * 64;
+#pragma unroll
+                for (int j = 0; j < 64; ++j)
+                    if (mb + j < p.M) store_out<BF16>(p.C, (long long)(mb + j) * p.N + n, tot[j] + b);
+            }
+        }
+    }
+
+    // every role has stopped, and its copies and MMAs have completed: free the Tensor Memory
+    __syncwarp();
+    tc::fence_before_sync();
+    __syncthreads();
+    if (warp == 1) {
+        tc::fence_after_sync();
+        tc::tmem_dealloc(tbase, kTmemCols);
+    }
+}
+
+struct TcPlan {
+    int S = 0, scst_off = 0, tab_off = 0, bar_off = 0, tab_rs = 1;
+    size_t smem = 0;
+    bool ok = false;
+};
+
+TcPlan make_plan(int64_t K, int G, const DeviceInfo &dev)
+{
+    TcPlan pl;
+    const int nkb = int(K / kKB);
+    const size_t scst = (size_t(2) * 2 * kBW * G * 2 + 15) & ~size_t(15);
+    pl.tab_rs = kBW + 1;
+    const size_t tab = (size_t(G) * pl.tab_rs * 4 + 15) & ~size_t(15);
+    const size_t bars = 8 * (2 * 8 + 12) + 16;
+    const size_t budget = size_t(dev.max_smem_optin) - 1024;
+    if (budget <= scst + tab + bars) return pl;
+    const long long s = std::min<long long>({4, nkb, (long long)((budget - scst - tab - bars) / kStageBytes)});
+    if (s < 2) return pl;
+    pl.S = int(s);
+    size_t off = size_t(pl.S) * kStageBytes;
+    pl.scst_off = int(off);
+    off += scst;
+    pl.tab_off = int(off);
+    off += tab;
+    pl.bar_off = int((off + 7) & ~size_t(7));
+    off = pl.bar_off + size_t(8) * (2 * pl.S + 12) + 8;
+    pl.smem = ((off + 15) & ~size_t(15)) + 1024;
+    pl.ok = pl.smem <= size_t(dev.max_smem_optin);
+    return pl;
+}
+
+template <bool BF16>
+wq_status launch(const TcPlan &pl, const CUtensorMap &ta, const CUtensorMap &tw, const TcParams &p, int grid,
+                 cudaStream_t st)
+{
+    auto kern = tc_gemm_kernel<BF16>;
+    static size_t configured = 0;
+    if (pl.smem > configured) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(pl.smem)) != cudaSuccess)
+            return check_launch("cudaFuncSetAttribute(tc_gemm)");
+        configured = pl.smem;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = pl.smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, kern, ta, tw, p);
+    if (e != cudaSuccess) return fail(WQ_ERR_CUDA, "tc_gemm_kernel launch: %s", cudaGetErrorString(e));
+    return check_launch("tc_gemm_kernel");
+}
+
+}  // namespace
+
+// Many-token W4A16 path (INT4, FP16 / BF16 activations).  WQ_ERR_UNSUPPORTED when the
+// configuration has no plan here (the caller then uses the tiled mma.sync path).
+wq_status tc_gemm(int WB, int AM, const void *A, const uint8_t *Wq, const void *scales, const void *zeros,
+                  const void *bias, void *C, int64_t M, int64_t N, int64_t K, const wq_qconfig &c, cudaStream_t st)
+{
+    if (WB != 4 || (AM != 0 && AM != 1)) return fail(WQ_ERR_UNSUPPORTED, "tc_gemm: INT4 weights, FP activations");
+    if (K % kKB || c.group_size % kKB) return fail(WQ_ERR_UNSUPPORTED, "tc_gemm: K and group_size multiples of 128");
+    const DeviceInfo &dev = device_info();
+    const int G = int(K / c.group_size);
+    const TcPlan pl = make_plan(K, G, dev);
+    if (!pl.ok) return fail(WQ_ERR_UNSUPPORTED, "tc_gemm: no shared-memory plan for K=%lld", (long long)K);
+    CUtensorMap ta, tw;
+    {
+        const uint64_t dims[2] = {uint64_t(K), uint64_t(M)};
+        const uint64_t strides[1] = {uint64_t(K) * 2};
+        const uint32_t box[2] = {64, uint32_t(kBT)};
+        wq_status rc = encode_tmap(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, A, dims, strides, box, 128);
+        if (rc != WQ_OK) return rc;
+    }
+    {
+        const uint64_t dims[2] = {uint64_t(K / 2), uint64_t(N)};
+        const uint64_t strides[1] = {uint64_t(K / 2)};
+        const uint32_t box[2] = {uint32_t(kKB / 2), uint32_t(kBW)};
+        wq_status rc = encode_tmap(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, Wq, dims, strides, box, 64);
+        if (rc != WQ_OK) return rc;
+    }
+    TcParams p{};
+    p.M = int(M);
+    p.N = int(N);
+    p.K = int(K);
+    p.G = G;
+    p.gs = c.group_size;
+    p.sym = c.symmetric;
+    p.nkb = int(K / kKB);
+    p.TT = int((M + kBT - 1) / kBT);
+    p.NT = p.TT * int((N + kBW - 1) / kBW);
+    p.S = pl.S;
+    p.scst_off = pl.scst_off;
+    p.tab_off = pl.tab_off;
+    p.bar_off = pl.bar_off;
+    p.tab_rs = pl.tab_rs;
+    p.scales16 = static_cast<const uint16_t *>(scales);
+    p.zeros = static_cast<const uint16_t *>(zeros);
+    p.bias = bias;
+    p.C = C;
+    const int grid = std::min(dev.sm_count, p.NT);
+    return AM == 1 ? launch<true>(pl, ta, tw, p, grid, st) : launch<false>(pl, ta, tw, p, grid, st);
+}
+
+int tc_read_error()
+{
+    int v = 0, zero = 0;
+    cudaMemcpyFromSymbol(&v, g_tc_error, sizeof v);
+    cudaMemcpyToSymbol(g_tc_error, &zero, sizeof zero);
+    return v;
+}
+
+}  // namespace wq

@@ -573,14 +573,14 @@ wq_status gemv_small_m(int WB, int AM, const void *A, const float *a_scale, cons
         const uint64_t dims[3] = {uint64_t(kPairBytes), uint64_t(N), row_bytes / kPairBytes};
         const uint64_t strides[2] = {row_bytes, uint64_t(kPairBytes)};
         const uint32_t box[3] = {uint32_t(kPairBytes), uint32_t(kTileRows), uint32_t(pl.KC / 2)};
-        rc = encode_tmap(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, Wq, dims, strides, box, true);
+        rc = encode_tmap(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, Wq, dims, strides, box, 128);
         if (rc != WQ_OK) pl.w3d = 0;  // same shared-memory layout from one 2D box per unit pair
     }
     if (!pl.w3d) {
         const uint64_t dims[2] = {row_bytes, uint64_t(N)};
         const uint64_t strides[1] = {row_bytes};
         const uint32_t box[2] = {uint32_t(kPairBytes), uint32_t(kTileRows)};
-        rc = encode_tmap(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, Wq, dims, strides, box, true);
+        rc = encode_tmap(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, Wq, dims, strides, box, 128);
     }
     if (rc != WQ_OK) return rc;
     const int es = AM == A_I8 ? 1 : 2;
@@ -592,7 +592,7 @@ wq_status gemv_small_m(int WB, int AM, const void *A, const float *a_scale, cons
         const uint64_t strides[2] = {kbytes, 128};
         const uint32_t box[3] = {uint32_t(128 / es), uint32_t(pl.MB), uint32_t(pl.KC * pl.KU * es / 128)};
         rc = encode_tmap(&ta, es == 1 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_UINT16, 3, A, dims,
-                         strides, box, true);
+                         strides, box, 128);
         if (rc != WQ_OK) return fail(WQ_ERR_UNSUPPORTED, "few-token plan: activation tensor map (%s)", wq_last_error());
     }
     GemvParams p{};

@@ -31,9 +31,9 @@ wq_status encode_tmap_2d(CUtensorMap *map, CUtensorMapDataType dt, const void *b
                          uint64_t dim1, uint64_t stride1_bytes, uint32_t box0, uint32_t box1);
 
 // Tiled tensor map of rank 2 or 3: dims[0] innermost (elements), strides_bytes[r-1] for
-// dims 1..r-1, box[] in elements, optional 128-byte swizzle.
+// dims 1..r-1, box[] in elements, swizzle_bytes 0 (none), 64 or 128.
 wq_status encode_tmap(CUtensorMap *map, CUtensorMapDataType dt, int rank, const void *base, const uint64_t *dims,
-                      const uint64_t *strides_bytes, const uint32_t *box, bool swizzle128);
+                      const uint64_t *strides_bytes, const uint32_t *box, int swizzle_bytes);
 
 // Reads (and clears) the device error words of all kernels with bounded waits.
 int read_device_errors();
