@@ -86,17 +86,20 @@ def kernel_source_hash() -> str:
 
 
 def recorded_traffic(workload: str):
-    """DRAM bytes per launch from the committed ncu summary, if it matches the current kernels."""
-    path = os.path.join(ROOT, "profiles", f"skinny_kernel_{workload}.md")
-    if not os.path.exists(path):
-        return None
-    src, traffic = None, None
-    for line in open(path):
-        if line.startswith("source_sha:"):
-            src = line.split(":", 1)[1].strip()
-        if line.startswith("dram_bytes_per_launch:"):
-            traffic = float(line.split(":", 1)[1].strip())
-    return traffic if (src == kernel_source_hash() and traffic) else None
+    """DRAM bytes per launch of the workload's dominant kernel, from the committed ncu summary
+    (profiles/<kernel>_<workload>.md), if it was taken of the current kernel sources."""
+    for path in sorted(glob.glob(os.path.join(ROOT, "profiles", f"*_{workload}.md"))):
+        fields = {}
+        for line in open(path):
+            if ":" in line and not line.startswith((" ", "#", "|")):
+                k, v = line.split(":", 1)
+                fields[k.strip()] = v.strip()
+        if fields.get("dominant") == "yes" and fields.get("source_sha") == kernel_source_hash():
+            try:
+                return float(fields["dram_bytes_per_launch"])
+            except (KeyError, ValueError):
+                return None
+    return None
 
 
 # ------------------------------------------------------------------ clocks
@@ -171,7 +174,7 @@ class ClockSampler:
 class Prepared:
     """Quantized weight copies, activations and outputs of one case on the device."""
 
-    def __init__(self, c: wq_synth.Case, device, seed_base: int = 0):
+    def __init__(self, c: wq_synth.Case, device, seed_base: int = 0, copies: int = 0):
         import gemv_wq_quantize_b200 as wq
         self.c = c
         self.qc = wq.QuantConfig(bits=2) if c.quant == "tern2" else \
@@ -180,7 +183,7 @@ class Prepared:
         Wq, s, z = wq.quantize_pack(W, self.qc)
         del W
         self.bytes = alg_bytes(c)
-        copies = max(2, math.ceil(4 * L2_BYTES / self.bytes))
+        copies = copies or max(2, math.ceil(4 * L2_BYTES / self.bytes))
         self.weights = [(Wq, s, z)] + [(Wq.clone(), s.clone(), None if z is None else z.clone())
                                         for _ in range(copies - 1)]
         A = wq_synth.activations(c.M, c.K, seed=seed_base + 1, dtype=c.a_dtype, outlier_frac=c.outlier_frac)
@@ -425,6 +428,24 @@ def run_reference(args):
             "e2e": {"value": round(v, 6), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
+def run_profile(args):
+    """One plain launch per case (one weight copy each; ncu flushes the caches itself)."""
+    import gemv_wq_quantize_b200 as wq
+    from gemv_wq_quantize_b200 import build
+    build.build(quiet=True)
+    wq.load_library()
+    device = torch.device("cuda", 0)
+    wl = wq_synth.WORKLOADS[args.workload]
+    preps = [Prepared(c, device, seed_base=0, copies=1) for c in wl.cases]
+    torch.cuda.synchronize()
+    for p in preps:
+        p.launch(False)
+    torch.cuda.synchronize()
+    assert wq.device_error() == 0, "a kernel gave up a bounded wait"
+    print(json.dumps({"profile": wl.name, "cases": [p.c.name for p in preps],
+                      "source_sha": kernel_source_hash()}), flush=True)
+
+
 # ------------------------------------------------------------------ main
 def main():
     ap = argparse.ArgumentParser()
@@ -436,6 +457,8 @@ def main():
     ap.add_argument("--no-breakdown", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=10.0, help="seconds of oracle work for cpu_baseline")
+    ap.add_argument("--profile", action="store_true",
+                    help="launch each case of the workload once, untimed (the command an ncu capture wraps)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -443,6 +466,9 @@ def main():
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
 
+    if args.profile:
+        run_profile(args)
+        return
     if args.impl == "reference":
         if rank == 0:
             print(json.dumps(run_reference(args)), flush=True)

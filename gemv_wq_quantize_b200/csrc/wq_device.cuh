@@ -9,10 +9,10 @@
 
 namespace wq {
 
-// Upper bound on polls of one mbarrier wait (each poll suspends in hardware for a
-// short while): a wait that exceeds it records an error and gives up instead of
-// spinning forever.
-constexpr uint32_t kMaxPolls = 1u << 24;
+// Upper bound on polls of one mbarrier wait in mbar_wait (each poll suspends for at most
+// kSuspendNs): a wait that exceeds it records an error and gives up instead of spinning
+// forever.
+constexpr uint32_t kMaxPolls = 256;
 
 // Error codes recorded in the per-translation-unit device error word.
 enum : int { kErrNone = 0, kErrWaitTimeout = 1 };
@@ -50,12 +50,30 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t by
                  : "memory");
 }
 
+// The waiting thread is suspended until the phase completes or kSuspendNs pass, so that
+// waiting warps take no issue slots from working ones.
+constexpr uint32_t kSuspendNs = 10000000u;
+
 __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity)
 {
     uint32_t ok;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(kSuspendNs)
+        : "memory");
+    return ok != 0;
+}
+
+// Non-blocking check whether the phase with the given parity has completed.
+__device__ __forceinline__ bool mbar_test_wait(uint64_t *bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(ok)
         : "r"(smem_u32(bar)), "r"(parity)

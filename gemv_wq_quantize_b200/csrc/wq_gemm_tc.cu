@@ -43,15 +43,18 @@ namespace {
 constexpr int kBW = 128;  // weight rows per tile: MMA M
 constexpr int kBT = 128;  // tokens per tile: MMA N
 constexpr int kKB = 128;  // k per block
-constexpr int kMathWarps = 8;
-constexpr int kThreads = (2 + kMathWarps) * 32;  // warp 0 TMA, warp 1 MMA + TMEM, warps 2..9 math
+constexpr int kDeqWarps = 8;   // unpack weights into TMEM (two per TMEM lane quadrant: k halves)
+constexpr int kFoldWarps = 8;  // fold block accumulators into the totals, write C
+constexpr int kThreads = (2 + kDeqWarps + kFoldWarps) * 32;  // + warp 0 TMA, warp 1 MMA / TMEM
 constexpr int kActBox = kBT * 128;               // one 64-k box of activations: 128 rows x 128 B
 constexpr int kActBytes = 2 * kActBox;           // 32 KB
 constexpr int kWBytes = kBW * kKB / 2;           // 8 KB of packed weights
 constexpr int kStageBytes = kActBytes + kWBytes;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kAcol = 0;    // 2 x 64 columns: unpacked weights of a block (A operand)
-constexpr uint32_t kDcol = 128;  // 2 x 128 columns: the block's accumulators
+constexpr int kNA = 4;          // TMEM A-buffers: unpacked weights of a block, 64 columns each
+constexpr int kND = 2;          // TMEM accumulators of a block, 128 columns each
+constexpr uint32_t kAcol = 0;
+constexpr uint32_t kDcol = kNA * 64;
 
 struct TcParams {
     int M, N, K, G, gs, sym;
@@ -76,10 +79,10 @@ __device__ __forceinline__ uint64_t globaltimer()
 // Bounded wait (~2 s); on expiry, or once another warp has given up, returns false.
 __device__ __forceinline__ bool tc_wait(uint64_t *bar, uint32_t parity, volatile int *abort)
 {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_test_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer();
     for (;;) {
-        for (int i = 0; i < 32; ++i)
+        for (int i = 0; i < 4; ++i)
             if (mbar_try_wait(bar, parity)) return true;
         if (*abort) return false;
         if (globaltimer() - t0 > 2000000000ull) {
@@ -121,34 +124,36 @@ __global__ void __launch_bounds__(kThreads, 1)
 {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    const int S = p.S;
-    uint8_t *ring = smem;  // S x (activations 32 KB | packed weights 8 KB)
+    uint8_t *ring = smem;  // kNA x (activations 32 KB | packed weights 8 KB)
     uint16_t *scst = reinterpret_cast<uint16_t *>(smem + p.scst_off);  // 2 x (scales, zeros) [128][G]
-    uint32_t *tab = reinterpret_cast<uint32_t *>(smem + p.tab_off);    // [G][tab_rs]: scale bits | z << 16
+    uint32_t *tabs = reinterpret_cast<uint32_t *>(smem + p.tab_off);   // 2 x [G][tab_rs]: scale | z << 16
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + p.bar_off);
-    uint64_t *full = bars, *empty = bars + S;
-    uint64_t *afull = bars + 2 * S, *afree = afull + 2, *dfull = afull + 4, *dfree = afull + 6;
-    uint64_t *scbar = afull + 8, *fin = afull + 10, *mbar = afull + 11;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(afull + 12);
+    // rel[s]: the MMAs of the step in stage s have completed: stage s and A-buffer s are free
+    // and accumulator step % kND holds the block's sums
+    uint64_t *full = bars, *rel = bars + kNA;
+    uint64_t *afull = bars + 2 * kNA, *dfree = afull + kNA;
+    uint64_t *scbar = dfree + kND, *tready = scbar + 2, *tdone = tready + 2, *fin = tdone + 2, *mbar = fin + 1;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(mbar + 1);
     volatile int *abort = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const size_t stab_elems = size_t(kBW) * p.G;  // one staging buffer (scales or zeros)
+    const size_t stab_elems = size_t(kBW) * p.G;          // one staging buffer (scales or zeros)
+    const size_t tab_elems = size_t(p.G) * p.tab_rs;      // one table
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < S; ++s) {
-            mbar_init(&full[s], 1);
-            mbar_init(&empty[s], kMathWarps + 1);
+        for (int b = 0; b < kNA; ++b) {
+            mbar_init(&full[b], 1);
+            mbar_init(&rel[b], 1);
+            mbar_init(&afull[b], kDeqWarps);
         }
+        for (int b = 0; b < kND; ++b) mbar_init(&dfree[b], kFoldWarps);
         for (int b = 0; b < 2; ++b) {
-            mbar_init(&afull[b], kMathWarps);
-            mbar_init(&afree[b], 1);
-            mbar_init(&dfull[b], 1);
-            mbar_init(&dfree[b], kMathWarps);
             mbar_init(&scbar[b], 1);
+            mbar_init(&tready[b], 1);
+            mbar_init(&tdone[b], kFoldWarps);
         }
         mbar_init(fin, 1);
-        mbar_init(mbar, kMathWarps * 32);
+        mbar_init(mbar, kDeqWarps * 32);
         *abort = 0;
         fence_barrier_init();
     }
@@ -182,8 +187,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (!p.sym) bulk_load(sc + stab_elems, p.zeros + (size_t)n0 * p.G, bytes16, &scbar[tl & 1]);
                 }
                 for (int kb = 0; kb < p.nkb; ++kb, ++step) {
-                    const int s = int(step % uint32_t(S));
-                    if (!tc_wait(&empty[s], ((step / S) & 1) ^ 1, abort)) break;
+                    const int s = int(step % kNA);
+                    if (!tc_wait(&rel[s], ((step / kNA) & 1) ^ 1, abort)) break;
                     uint8_t *st = ring + size_t(s) * kStageBytes;
                     mbar_arrive_expect_tx(&full[s], kStageBytes);
                     tma_load_2d(st, &tmap_a, kb * kKB, m0, &full[s]);
@@ -192,33 +197,32 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
             // nothing may land in shared memory after the CTA exits: wait for the last stages
-            for (uint32_t k = step > uint32_t(S) ? step - S : 0; k < step; ++k)
-                tc_wait(&full[k % S], (k / S) & 1, abort);
+            for (uint32_t k = step > uint32_t(kNA) ? step - kNA : 0; k < step; ++k)
+                tc_wait(&full[k % kNA], (k / kNA) & 1, abort);
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
             const uint32_t idesc = tc::idesc_f16(BF16, kBW, kBT);
+            uint64_t desc0[kNA];  // descriptor of each stage's activations (k step 0)
+#pragma unroll
+            for (int b = 0; b < kNA; ++b) desc0[b] = tc::sdesc_sw128(smem_u32(ring + size_t(b) * kStageBytes));
             uint32_t step = 0;
             bool issued = false;
             for (int t = blockIdx.x; t < p.NT && !*abort; t += gridDim.x) {
                 for (int kb = 0; kb < p.nkb; ++kb, ++step) {
-                    const int s = int(step % uint32_t(S));
-                    const uint32_t ab = step & 1, ph = (step >> 1) & 1;
-                    if (!tc_wait(&full[s], (step / S) & 1, abort)) break;
-                    if (!tc_wait(&afull[ab], ph, abort)) break;
-                    if (!tc_wait(&dfree[ab], ph ^ 1, abort)) break;
+                    const uint32_t s = step % kNA, db = step % kND;
+                    // afull: the unpacking warps have seen the stage's data and stored the weights
+                    if (!tc_wait(&afull[s], (step / kNA) & 1, abort)) break;
+                    if (!tc_wait(&dfree[db], ((step / kND) & 1) ^ 1, abort)) break;
                     tc::fence_after_sync();
-                    const uint32_t act = smem_u32(ring + size_t(s) * kStageBytes);
+                    const uint64_t d0 = s == 0 ? desc0[0] : s == 1 ? desc0[1] : s == 2 ? desc0[2] : desc0[3];
+                    const uint32_t dcol = tbase + kDcol + db * kBT, acol = tbase + kAcol + s * 64;
 #pragma unroll
-                    for (int kk = 0; kk < kKB / 16; ++kk) {
-                        const uint64_t bdesc = tc::sdesc_sw128(act + (kk >> 2) * kActBox + (kk & 3) * 32);
-                        tc::mma_f16_ts(tbase + kDcol + ab * kBT, tbase + kAcol + ab * 64 + kk * 8, bdesc, idesc,
-                                       kk > 0 ? 1u : 0u);
-                    }
-                    tc::commit(&dfull[ab]);
-                    tc::commit(&empty[s]);
-                    tc::commit(&afree[ab]);
+                    for (int kk = 0; kk < kKB / 16; ++kk)
+                        tc::mma_f16_ts(dcol, acol + kk * 8, d0 + uint64_t(((kk >> 2) * kActBox + (kk & 3) * 32) >> 4),
+                                       idesc, kk > 0 ? 1u : 0u);
+                    tc::commit(&rel[s]);
                     issued = true;
                 }
             }
@@ -227,32 +231,33 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tc_wait(fin, 0, abort);
             }
         }
-    } else {
-        // ------------------------------------------------------------ math warps
-        const int q = warp & 3;             // TMEM lane quadrant of this warp
-        const int kh = (warp - 2) >> 2;     // k half (unpack) / token half (fold)
-        const int r = q * 32 + lane;        // weight row within the tile
+    } else if (warp < 2 + kDeqWarps) {
+        // ------------------------------------------------------------ unpacking warps
+        const int q = warp & 3;          // TMEM lane quadrant of this warp
+        const int kh = (warp - 2) >> 2;  // k half of the block
+        const int r = q * 32 + lane;     // weight row within the tile
         const uint32_t tlane = tbase + (uint32_t(q * 32) << 16);
         const uint32_t magic_z = BF16 ? 0xC300u : 0xE400u;  // -(magic + z) = magic_z | z
         uint32_t step = 0, mphase = 0;
-        auto math_sync = [&]() -> bool {  // bounded barrier of the math warps
+        auto deq_sync = [&]() -> bool {  // bounded barrier of the unpacking warps
             mbar_arrive(mbar);
             const bool ok = tc_wait(mbar, mphase & 1, abort);
             ++mphase;
             return ok;
         };
-        grid_dep_wait();  // C and bias belong to this kernel only once the previous one is done
         int tl = 0;
         for (int t = blockIdx.x; t < p.NT && !*abort; t += gridDim.x, ++tl) {
-            const int n0 = (t / p.TT) * kBW, m0 = (t % p.TT) * kBT;
+            const int n0 = (t / p.TT) * kBW;
             const int nrows = min(kBW, p.N - n0);
+            uint32_t *tab = tabs + size_t(tl & 1) * tab_elems;
             // ---- scale / zero table of the tile: [g][row] = fp16 scale bits | z << 16
             if (!tc_wait(&scbar[tl & 1], (tl >> 1) & 1, abort)) break;
-            if (!math_sync()) break;  // everyone is done with the previous tile's table
+            if (tl >= 2 && !tc_wait(&tdone[tl & 1], ((tl - 2) >> 1) & 1, abort)) break;  // tile tl-2 folded
+            if (!deq_sync()) break;
             {
                 const uint16_t *sc = scst + size_t(tl & 1) * 2 * stab_elems;
                 const int n16 = int(((uint32_t(nrows) * p.G * 2u) & ~15u) >> 1);
-                for (int e = threadIdx.x - 64; e < kBW * p.G; e += kMathWarps * 32) {
+                for (int e = threadIdx.x - 64; e < kBW * p.G; e += kDeqWarps * 32) {
                     const int rl = e / p.G, gi = e - rl * p.G;
                     uint32_t v = 0;
                     if (rl < nrows) {
@@ -267,67 +272,80 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tab[(size_t)gi * p.tab_rs + rl] = v;
                 }
             }
-            if (!math_sync()) break;
+            if (!deq_sync()) break;
+            if (threadIdx.x == 64) mbar_arrive(&tready[tl & 1]);
 
-            float tot[64];
-#pragma unroll
-            for (int j = 0; j < 64; ++j) tot[j] = 0.f;
-            float s_prev = 0.f;
-            // fold the accumulator of step `fs` (its block scale `sv`) into the totals
-            auto fold = [&](uint32_t fs, float sv) -> bool {
-                const uint32_t db = fs & 1;
-                if (!tc_wait(&dfull[db], (fs >> 1) & 1, abort)) return false;
-                tc::fence_after_sync();
-                uint32_t d0[32], d1[32];
-                tc::ld_32x32b_x32(tlane + kDcol + db * kBT + kh * 64, d0);
-                tc::ld_32x32b_x32(tlane + kDcol + db * kBT + kh * 64 + 32, d1);
-                tc::wait_ld();
-                tc::fence_before_sync();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&dfree[db]);
-#pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    tot[j] = fmaf(sv, __uint_as_float(d0[j]), tot[j]);
-                    tot[32 + j] = fmaf(sv, __uint_as_float(d1[j]), tot[32 + j]);
-                }
-                return true;
-            };
-
-            bool ok = true;
-            for (int kb = 0; kb < p.nkb && ok; ++kb, ++step) {
-                const int s = int(step % uint32_t(S));
-                const uint32_t ab = step & 1, ph = (step >> 1) & 1;
-                if (!tc_wait(&full[s], (step / S) & 1, abort)) { ok = false; break; }
-                // this row's 32 packed bytes of the k half (64-byte rows, 64-byte swizzle)
+            for (int kb = 0; kb < p.nkb; ++kb, ++step) {
+                const uint32_t s = step % kNA;  // ring stage and TMEM A-buffer
+                // full also tells that the MMAs of step - kNA (stage and A-buffer s) have completed
+                if (!tc_wait(&full[s], (step / kNA) & 1, abort)) break;
+                // this row's 64 packed bytes (64-byte rows, 64-byte swizzle)
                 const uint8_t *wrow = ring + size_t(s) * kStageBytes + kActBytes + r * 64;
                 const uint32_t sw = uint32_t((r >> 1) & 3);
-                const uint4 w0 = lds128(wrow + (((2 * kh) ^ sw) << 4));
-                const uint4 w1 = lds128(wrow + (((2 * kh + 1) ^ sw) << 4));
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&empty[s]);
+                const uint4 w0 = lds128(wrow + ((uint32_t(2 * kh) ^ sw) << 4));
+                const uint4 w1 = lds128(wrow + ((uint32_t(2 * kh + 1) ^ sw) << 4));
                 const uint32_t tv = tab[(size_t)((kb * kKB) / p.gs) * p.tab_rs + r];
                 const uint32_t zc1 = magic_z | (tv >> 16);
                 const uint32_t zc = zc1 | (zc1 << 16);
-                uint32_t v[32];
-                unpack_word<BF16>(w0.x, zc, v + 0);
-                unpack_word<BF16>(w0.y, zc, v + 4);
-                unpack_word<BF16>(w0.z, zc, v + 8);
-                unpack_word<BF16>(w0.w, zc, v + 12);
-                unpack_word<BF16>(w1.x, zc, v + 16);
-                unpack_word<BF16>(w1.y, zc, v + 20);
-                unpack_word<BF16>(w1.z, zc, v + 24);
-                unpack_word<BF16>(w1.w, zc, v + 28);
-                if (!tc_wait(&afree[ab], ph ^ 1, abort)) { ok = false; break; }
                 tc::fence_after_sync();
-                tc::st_32x32b_x32(tlane + kAcol + ab * 64 + kh * 32, v);
+                {
+                    uint32_t v[32];
+                    unpack_word<BF16>(w0.x, zc, v + 0);
+                    unpack_word<BF16>(w0.y, zc, v + 4);
+                    unpack_word<BF16>(w0.z, zc, v + 8);
+                    unpack_word<BF16>(w0.w, zc, v + 12);
+                    unpack_word<BF16>(w1.x, zc, v + 16);
+                    unpack_word<BF16>(w1.y, zc, v + 20);
+                    unpack_word<BF16>(w1.z, zc, v + 24);
+                    unpack_word<BF16>(w1.w, zc, v + 28);
+                    tc::st_32x32b_x32(tlane + kAcol + s * 64 + kh * 32, v);
+                }
                 tc::wait_st();
                 tc::fence_before_sync();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&afull[ab]);
-                if (kb > 0 && !fold(step - 1, s_prev)) { ok = false; break; }
-                s_prev = __half2float(__ushort_as_half(uint16_t(tv & 0xFFFFu)));
+                if (lane == 0) mbar_arrive(&afull[s]);
             }
-            if (!ok || !fold(step - 1, s_prev)) break;
+        }
+    } else {
+        // ------------------------------------------------------------ folding warps
+        const int q = warp & 3;                       // TMEM lane quadrant of this warp
+        const int th = (warp - 2 - kDeqWarps) >> 2;   // token half of the tile
+        const int r = q * 32 + lane;                  // weight row within the tile
+        const uint32_t tlane = tbase + (uint32_t(q * 32) << 16);
+        grid_dep_wait();  // C and bias belong to this kernel only once the previous one is done
+        uint32_t step = 0;
+        int tl = 0;
+        for (int t = blockIdx.x; t < p.NT && !*abort; t += gridDim.x, ++tl) {
+            const int n0 = (t / p.TT) * kBW, m0 = (t % p.TT) * kBT;
+            const uint32_t *tab = tabs + size_t(tl & 1) * tab_elems;
+            if (!tc_wait(&tready[tl & 1], (tl >> 1) & 1, abort)) break;
+            float tot[64];
+#pragma unroll
+            for (int j = 0; j < 64; ++j) tot[j] = 0.f;
+            bool ok = true;
+            for (int kb = 0; kb < p.nkb; ++kb, ++step) {
+                const uint32_t db = step % kND, s = step % kNA;
+                const uint32_t tv = tab[(size_t)((kb * kKB) / p.gs) * p.tab_rs + r];
+                const float sv = __half2float(__ushort_as_half(uint16_t(tv & 0xFFFFu)));
+                if (!tc_wait(&rel[s], (step / kNA) & 1, abort)) { ok = false; break; }
+                tc::fence_after_sync();
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    uint32_t d[16];
+                    tc::ld_32x32b_x16(tlane + kDcol + db * kBT + th * 64 + c * 16, d);
+                    tc::wait_ld();
+                    if (c == 3) {
+                        tc::fence_before_sync();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&dfree[db]);
+                    }
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) tot[c * 16 + j] = fmaf(sv, __uint_as_float(d[j]), tot[c * 16 + j]);
+                }
+            }
+            if (!ok) break;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&tdone[tl & 1]);
 
             // ---- epilogue: C[m][n] = total (+ bias[n]), one weight row x 64 tokens per thread
             const int n = n0 + r;
@@ -337,7 +355,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if constexpr (BF16) b = __bfloat162float(static_cast<const __nv_bfloat16 *>(p.bias)[n]);
                     else b = __half2float(static_cast<const __half *>(p.bias)[n]);
                 }
-                const int mb = m0 + kh * 64;
+                const int mb = m0 + th * 64;
 #pragma unroll
                 for (int j = 0; j < 64; ++j)
                     if (mb + j < p.M) store_out<BF16>(p.C, (long long)(mb + j) * p.N + n, tot[j] + b);
@@ -367,20 +385,20 @@ TcPlan make_plan(int64_t K, int G, const DeviceInfo &dev)
     const int nkb = int(K / kKB);
     const size_t scst = (size_t(2) * 2 * kBW * G * 2 + 15) & ~size_t(15);
     pl.tab_rs = kBW + 1;
-    const size_t tab = (size_t(G) * pl.tab_rs * 4 + 15) & ~size_t(15);
-    const size_t bars = 8 * (2 * 8 + 12) + 16;
+    const size_t tab = (size_t(2) * G * pl.tab_rs * 4 + 15) & ~size_t(15);
+    const size_t bars = 8 * (2 * 8 + 20) + 16;
     const size_t budget = size_t(dev.max_smem_optin) - 1024;
     if (budget <= scst + tab + bars) return pl;
-    const long long s = std::min<long long>({4, nkb, (long long)((budget - scst - tab - bars) / kStageBytes)});
-    if (s < 2) return pl;
-    pl.S = int(s);
+    // the ring has one stage per TMEM A-buffer
+    if (nkb < kNA || (budget - scst - tab - bars) / kStageBytes < size_t(kNA)) return pl;
+    pl.S = kNA;
     size_t off = size_t(pl.S) * kStageBytes;
     pl.scst_off = int(off);
     off += scst;
     pl.tab_off = int(off);
     off += tab;
     pl.bar_off = int((off + 7) & ~size_t(7));
-    off = pl.bar_off + size_t(8) * (2 * pl.S + 12) + 8;
+    off = pl.bar_off + size_t(8) * (3 * kNA + 2 * kND + 11) + 8;
     pl.smem = ((off + 15) & ~size_t(15)) + 1024;
     pl.ok = pl.smem <= size_t(dev.max_smem_optin);
     return pl;

@@ -88,10 +88,10 @@ __device__ __forceinline__ uint64_t globaltimer()
 // Bounded wait (~2 s of wall clock); records an error and returns false on expiry.
 __device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity)
 {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_test_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer();
     for (;;) {
-        for (int i = 0; i < 64; ++i)
+        for (int i = 0; i < 4; ++i)
             if (mbar_try_wait(bar, parity)) return true;
         if (globaltimer() - t0 > 2000000000ull) {
             atomicCAS(&g_gemv_error, kErrNone, kErrWaitTimeout);
