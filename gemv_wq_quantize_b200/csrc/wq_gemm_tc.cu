@@ -153,7 +153,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&tdone[b], kFoldWarps);
         }
         mbar_init(fin, 1);
-        mbar_init(mbar, kDeqWarps * 32);
+        mbar_init(mbar, kDeqWarps);
         *abort = 0;
         fence_barrier_init();
     }
@@ -239,8 +239,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t tlane = tbase + (uint32_t(q * 32) << 16);
         const uint32_t magic_z = BF16 ? 0xC300u : 0xE400u;  // -(magic + z) = magic_z | z
         uint32_t step = 0, mphase = 0;
-        auto deq_sync = [&]() -> bool {  // bounded barrier of the unpacking warps
-            mbar_arrive(mbar);
+        auto deq_sync = [&]() -> bool {  // bounded barrier of the unpacking warps (one arrival per warp)
+            __syncwarp();
+            if (lane == 0) mbar_arrive(mbar);
             const bool ok = tc_wait(mbar, mphase & 1, abort);
             ++mphase;
             return ok;

@@ -168,7 +168,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             cnt[s] = 0;
         }
         mbar_init(abar, 1);
-        mbar_init(cbar, kThreads);
+        mbar_init(cbar, kCW);
         mbar_init(scbar, 1);
         fence_barrier_init();
     }
@@ -265,8 +265,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (p.a_whole && !wait_bar(abar, 0)) return;
 
     uint32_t cphase = 0;
-    auto csync = [&]() -> bool {  // bounded barrier of all threads
-        mbar_arrive(cbar);
+    auto csync = [&]() -> bool {  // bounded barrier of all threads (one arrival per warp)
+        __syncwarp();
+        if (lane == 0) mbar_arrive(cbar);
         const bool ok = wait_bar(cbar, cphase & 1);
         ++cphase;
         return ok;
