@@ -23,8 +23,9 @@ wq_status gemv_small_m(int WB, int AM, const void *A, const float *a_scale, cons
                        const void *zeros, const void *bias, void *C, int32_t *acc_out, int64_t M, int64_t N,
                        int64_t K, const wq_qconfig &c, cudaStream_t st);
 int gemv_read_error();
-wq_status tc_gemm(int WB, int AM, const void *A, const uint8_t *Wq, const void *scales, const void *zeros,
-                  const void *bias, void *C, int64_t M, int64_t N, int64_t K, const wq_qconfig &c, cudaStream_t st);
+wq_status tc_gemm(int WB, int AM, const void *A, const float *a_scale, const uint8_t *Wq, const void *scales,
+                  const void *zeros, const void *bias, void *C, int64_t M, int64_t N, int64_t K,
+                  const wq_qconfig &c, cudaStream_t st);
 int tc_read_error();
 
 namespace {
@@ -130,8 +131,8 @@ int read_device_errors()
 }
 
 namespace {
-// Few tokens go to the weight-streaming GEMV; more tokens to the tcgen05 GEMM (INT4 weights,
-// FP activations) or else to the tiled mma.sync path.
+// Few tokens go to the weight-streaming GEMV; more tokens to the tcgen05 GEMM, or else (the
+// INT32 group-sum output, shapes without a plan there) to the tiled mma.sync path.
 wq_status dispatch(int WB, int AM, const void *A, const float *a_scale, const uint8_t *Wq, const void *scales,
                    const void *zeros, const void *bias, void *C, int32_t *acc_out, int64_t M, int64_t N, int64_t K,
                    const wq_qconfig &c, void *ws, size_t ws_bytes, cudaStream_t st)
@@ -139,8 +140,8 @@ wq_status dispatch(int WB, int AM, const void *A, const float *a_scale, const ui
     if (M <= 16) {
         wq_status rc = gemv_small_m(WB, AM, A, a_scale, Wq, scales, zeros, bias, C, acc_out, M, N, K, c, st);
         if (rc != WQ_ERR_UNSUPPORTED) return rc;
-    } else if (AM != 2 && !acc_out) {
-        wq_status rc = tc_gemm(WB, AM, A, Wq, scales, zeros, bias, C, M, N, K, c, st);
+    } else if (!acc_out) {
+        wq_status rc = tc_gemm(WB, AM, A, a_scale, Wq, scales, zeros, bias, C, M, N, K, c, st);
         if (rc != WQ_ERR_UNSUPPORTED) return rc;
     }
     return skinny_gemm(WB, AM, A, a_scale, Wq, scales, zeros, bias, C, acc_out, M, N, K, c, ws, ws_bytes, st);

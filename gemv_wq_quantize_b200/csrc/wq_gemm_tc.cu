@@ -1,29 +1,35 @@
-// wq_gemm_tc.cu -- many-token W4A16 matmul on the 5th-generation tensor cores (tcgen05).
+// wq_gemm_tc.cu -- many-token weight-quantized matmul on the 5th-generation tensor cores
+// (tcgen05), for INT4 (group scales, optional zero points) and ternary INT2 weights.
 //
-// C[M,N] = A[M,K] x dequant(Wq[N,K])^T with FP16 / BF16 activations and INT4 weights
-// (group scales, optional zero points): "BitBLAS practical guide", "What is BitBLAS" and
-// "Weight group quantization"; fp32 accumulation, one rounding to the output dtype.
+// C[M,N] = A[M,K] x dequant(Wq[N,K])^T: "BitBLAS practical guide", "What is BitBLAS",
+// "Weight group quantization" and the FP16 x INT4 / INT2 and INT8 x INT4 / INT2 rows of its
+// data-type table.  FP16 / BF16 activations use kind::f16 MMAs with fp32 accumulation;
+// per-token INT8 activations ("Accelerating LLM inference with CUDA Graph and INT4
+// quantization", part 1, steps 2-4) use kind::i8 MMAs whose int32 group sums are exact,
+// followed by the (a_scale x w_scale) epilogue.
 //
-// At prefill sizes the product is tensor-bound.  The weights are the MMA's A operand
+// At these sizes the product is tensor-bound.  The weights are the MMA's A operand
 // (M = 128 weight rows) and live in Tensor Memory; the activations are the B operand
 // (N = 128 tokens), brought into shared memory by TMA with the 128-byte swizzle that the
 // MMA's K-major descriptor expects.  Per block of 128 k:
-//  * a producer warp TMAs the block's activations (32 KB) and packed weights (8 KB) into
-//    an S-stage ring;
-//  * eight math warps unpack the packed weights of their own row (thread = weight row,
-//    warp pairs split the 128 k) into the exact integers q - z as f16 / bf16 pairs in
-//    natural k order, and store them to a TMEM A-buffer (tcgen05.st);
-//  * one thread issues 8 MMAs of 128 x 128 x 16 into a TMEM accumulator of that block
-//    alone, and commits to mbarriers;
-//  * the math warps read the block's accumulator back (tcgen05.ld) and add it, times the
+//  * a producer warp TMAs the block's activations and packed weights into a 4-stage ring;
+//  * eight unpacking warps turn the packed weights of their own row (thread = weight row,
+//    warp pairs split the 128 k) into exact integers in natural k order -- q - z (INT4) or
+//    the ternary value (INT2), as f16 / bf16 pairs, or as signed bytes for INT8
+//    activations -- and store them to the stage's TMEM A-buffer (tcgen05.st);
+//  * one thread issues the block's MMAs (8 of k 16, or 4 of k 32 for INT8) into a TMEM
+//    accumulator of that block alone, and one tcgen05.commit frees the stage, its A-buffer
+//    and announces the accumulator;
+//  * eight folding warps read the accumulator back (tcgen05.ld) and add it, times the
 //    row's group scale, into fp32 totals held in registers (each thread: one weight row x
-//    64 tokens).  A-buffers and accumulators are double-buffered, so unpacking, MMA and
-//    folding of consecutive blocks overlap.
-// The products are exact (|q - z| <= 15 times an f16 / bf16 activation); the only
-// rounding besides fp32 accumulation is the final conversion.  Persistent CTAs walk the
-// (weight tile, token tile) grid token-tile fastest so that concurrent CTAs share weight
-// tiles in L2.  Every wait is bounded; on expiry the CTA records an error, stops, waits
-// for what it has in flight and frees its Tensor Memory.
+//    64 tokens), then write C.
+// Four A-buffers and two accumulators let unpacking run ahead of the MMAs and folding
+// trail them.  The products are exact (|q - z| <= 15 times an f16 / bf16 / int8
+// activation); the only rounding besides fp32 accumulation (int32 for INT8) is the
+// final conversion.  Persistent CTAs walk the (weight tile, token tile) grid token-tile
+// fastest so that concurrent CTAs share weight tiles in L2.  Every wait is bounded; on
+// expiry the CTA records an error, stops, waits for what it has in flight and frees its
+// Tensor Memory.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <stdint.h>
@@ -46,10 +52,10 @@ constexpr int kKB = 128;  // k per block
 constexpr int kDeqWarps = 8;   // unpack weights into TMEM (two per TMEM lane quadrant: k halves)
 constexpr int kFoldWarps = 8;  // fold block accumulators into the totals, write C
 constexpr int kThreads = (2 + kDeqWarps + kFoldWarps) * 32;  // + warp 0 TMA, warp 1 MMA / TMEM
-constexpr int kActBox = kBT * 128;               // one 64-k box of activations: 128 rows x 128 B
-constexpr int kActBytes = 2 * kActBox;           // 32 KB
-constexpr int kWBytes = kBW * kKB / 2;           // 8 KB of packed weights
-constexpr int kStageBytes = kActBytes + kWBytes;
+constexpr int kActBox = kBT * 128;  // one box of activations: 128 rows x 128 B (64 k FP, 128 k INT8)
+__host__ __device__ constexpr int act_bytes(int AM) { return AM == 2 ? kActBox : 2 * kActBox; }
+__host__ __device__ constexpr int w_bytes(int WB) { return kBW * kKB * WB / 8; }  // 8 KB / 4 KB packed
+__host__ __device__ constexpr int stage_bytes(int WB, int AM) { return act_bytes(AM) + w_bytes(WB); }
 constexpr uint32_t kTmemCols = 512;
 constexpr int kNA = 4;          // TMEM A-buffers: unpacked weights of a block, 64 columns each
 constexpr int kND = 2;          // TMEM accumulators of a block, 128 columns each
@@ -58,6 +64,8 @@ constexpr uint32_t kDcol = kNA * 64;
 
 struct TcParams {
     int M, N, K, G, gs, sym;
+    const float *a_scale;  // INT8 activations: per-token scale
+    const float *scale32;  // INT2 weights: per-tensor scale
     int nkb;     // K / 128
     int TT, NT;  // token tiles, tiles
     int S;       // ring stages
@@ -101,6 +109,51 @@ __device__ __forceinline__ void store_out(void *C, long long idx, float v)
     else static_cast<__half *>(C)[idx] = __float2half_rn(v);
 }
 
+// INT4, INT8 activations: one word (8 nibbles) -> 8 signed bytes q - z in natural k order.
+// zc = (0x80 - z) in every byte: q + 128 - z stays in 113 .. 143, no carries; ^0x80 makes it
+// the two's complement byte of q - z.
+__device__ __forceinline__ void unpack_word_s8(uint32_t w, uint32_t zc, uint32_t *o)
+{
+    const uint32_t lo = w & 0x0F0F0F0Fu, hi = (w >> 4) & 0x0F0F0F0Fu;
+    o[0] = (prmt(lo, hi, 0x5140) + zc) ^ 0x80808080u;  // k0 k1 k2 k3
+    o[1] = (prmt(lo, hi, 0x7362) + zc) ^ 0x80808080u;  // k4 .. k7
+}
+
+// Ternary INT2 (two's complement code, element 4j+i in bits 2i of byte j): with c = code ^ 2
+// in 0..3 the value is c - 2.  FP: one word (16 codes) -> 8 pairs (k0,k1) .. (k14,k15): the
+// nibble of a pair is placed in both halves, masked to (c_even, 4 c_odd), offset by the magic
+// number (f16 1024, bf16 128) and mapped exactly to (c - 2) by one fma with (1, 1/4).
+template <bool BF16>
+__device__ __forceinline__ void unpack2_word(uint32_t w, uint32_t *o)
+{
+    const uint32_t y = w ^ 0xAAAAAAAAu;
+    const uint32_t lo = y & 0x0F0F0F0Fu, hi = (y >> 4) & 0x0F0F0F0Fu;  // pairs 0,2,4,6 / 1,3,5,7
+    const uint32_t magic = BF16 ? 0x43004300u : 0x64006400u;
+    const uint32_t mul = BF16 ? 0x3E803F80u : 0x34003C00u;  // (1, 1/4)
+    const uint32_t add = BF16 ? 0xC208C302u : 0xDC08E402u;  // (-(magic + 2), -(magic / 4 + 2))
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+        const uint32_t b = uint32_t(q >> 1);
+        const uint32_t x = prmt((q & 1) ? hi : lo, 0u, b | (4u << 4) | (b << 8) | (4u << 12));
+        const uint32_t v = and_or(x, 0x000C0003u, magic);
+        o[q] = BF16 ? bf2_fma(v, mul, add) : h2_fma(v, mul, add);
+    }
+}
+
+// Ternary INT2, INT8 activations: one word -> 16 signed bytes c - 2 in natural k order.
+__device__ __forceinline__ void unpack2_word_s8(uint32_t w, uint32_t *o)
+{
+    const uint32_t y = w ^ 0xAAAAAAAAu;
+    const uint32_t t0 = y & 0x03030303u, t1 = (y >> 2) & 0x03030303u;  // k0 k4 k8 k12 / k1 k5 ..
+    const uint32_t t2 = (y >> 4) & 0x03030303u, t3 = (y >> 6) & 0x03030303u;
+    const uint32_t u0 = prmt(t0, t1, 0x5140), u1 = prmt(t2, t3, 0x5140);  // k0 k1 k4 k5 / k2 k3 k6 k7
+    const uint32_t u2 = prmt(t0, t1, 0x7362), u3 = prmt(t2, t3, 0x7362);  // k8 k9 k12 k13 / ..
+    o[0] = (prmt(u0, u1, 0x5410) + 0x7E7E7E7Eu) ^ 0x80808080u;
+    o[1] = (prmt(u0, u1, 0x7632) + 0x7E7E7E7Eu) ^ 0x80808080u;
+    o[2] = (prmt(u2, u3, 0x5410) + 0x7E7E7E7Eu) ^ 0x80808080u;
+    o[3] = (prmt(u2, u3, 0x7632) + 0x7E7E7E7Eu) ^ 0x80808080u;
+}
+
 // Unpacks one 32-bit word (8 nibbles, k0 in the low nibble) into 4 pairs (k0,k1) .. (k6,k7)
 // of magic + nibble (f16: 1024 + q, bf16: 128 + q), then adds zc = -(magic + z): exact q - z.
 template <bool BF16>
@@ -117,14 +170,16 @@ __device__ __forceinline__ void unpack_word(uint32_t w, uint32_t zc, uint32_t *o
     for (int i = 0; i < 4; ++i) o[i] = BF16 ? bf2_fma(x[i], 0x3F803F80u, zc) : h2_add(x[i], zc);
 }
 
-template <bool BF16>
+template <int WB, int AM>
 __global__ void __launch_bounds__(kThreads, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_w,
                    const TcParams p)
 {
+    constexpr bool BF16 = AM == 1, I8 = AM == 2;
+    constexpr int kActBytes = act_bytes(AM), kStageBytes = stage_bytes(WB, AM);
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t *ring = smem;  // kNA x (activations 32 KB | packed weights 8 KB)
+    uint8_t *ring = smem;  // kNA x (activations | packed weights)
     uint16_t *scst = reinterpret_cast<uint16_t *>(smem + p.scst_off);  // 2 x (scales, zeros) [128][G]
     uint32_t *tabs = reinterpret_cast<uint32_t *>(smem + p.tab_off);   // 2 x [G][tab_rs]: scale | z << 16
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + p.bar_off);
@@ -177,14 +232,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             int tl = 0;
             for (int t = blockIdx.x; t < p.NT && !*abort; t += gridDim.x, ++tl) {
                 const int n0 = (t / p.TT) * kBW, m0 = (t % p.TT) * kBT;
-                // the tile's scale / zero rows: contiguous in [N, G]
-                const int nrows = min(kBW, p.N - n0);
-                const uint32_t bytes16 = (uint32_t(nrows) * p.G * 2u) & ~15u;
-                uint16_t *sc = scst + size_t(tl & 1) * 2 * stab_elems;
-                mbar_arrive_expect_tx(&scbar[tl & 1], bytes16 * (p.sym ? 1u : 2u));
-                if (bytes16) {
-                    bulk_load(sc, p.scales16 + (size_t)n0 * p.G, bytes16, &scbar[tl & 1]);
-                    if (!p.sym) bulk_load(sc + stab_elems, p.zeros + (size_t)n0 * p.G, bytes16, &scbar[tl & 1]);
+                if constexpr (WB == 4) {
+                    // the tile's scale / zero rows: contiguous in [N, G]
+                    const int nrows = min(kBW, p.N - n0);
+                    const uint32_t bytes16 = (uint32_t(nrows) * p.G * 2u) & ~15u;
+                    uint16_t *sc = scst + size_t(tl & 1) * 2 * stab_elems;
+                    mbar_arrive_expect_tx(&scbar[tl & 1], bytes16 * (p.sym ? 1u : 2u));
+                    if (bytes16) {
+                        bulk_load(sc, p.scales16 + (size_t)n0 * p.G, bytes16, &scbar[tl & 1]);
+                        if (!p.sym) bulk_load(sc + stab_elems, p.zeros + (size_t)n0 * p.G, bytes16, &scbar[tl & 1]);
+                    }
                 }
                 for (int kb = 0; kb < p.nkb; ++kb, ++step) {
                     const int s = int(step % kNA);
@@ -192,8 +249,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     uint8_t *st = ring + size_t(s) * kStageBytes;
                     mbar_arrive_expect_tx(&full[s], kStageBytes);
                     tma_load_2d(st, &tmap_a, kb * kKB, m0, &full[s]);
-                    tma_load_2d(st + kActBox, &tmap_a, kb * kKB + 64, m0, &full[s]);
-                    tma_load_2d(st + kActBytes, &tmap_w, kb * (kKB / 2), n0, &full[s]);
+                    if constexpr (!I8) tma_load_2d(st + kActBox, &tmap_a, kb * kKB + 64, m0, &full[s]);
+                    tma_load_2d(st + kActBytes, &tmap_w, kb * (kKB * WB / 8), n0, &full[s]);
                 }
             }
             // nothing may land in shared memory after the CTA exits: wait for the last stages
@@ -203,7 +260,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
-            const uint32_t idesc = tc::idesc_f16(BF16, kBW, kBT);
+            const uint32_t idesc = I8 ? tc::idesc_i8(kBW, kBT) : tc::idesc_f16(BF16, kBW, kBT);
             uint64_t desc0[kNA];  // descriptor of each stage's activations (k step 0)
 #pragma unroll
             for (int b = 0; b < kNA; ++b) desc0[b] = tc::sdesc_sw128(smem_u32(ring + size_t(b) * kStageBytes));
@@ -218,10 +275,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tc::fence_after_sync();
                     const uint64_t d0 = s == 0 ? desc0[0] : s == 1 ? desc0[1] : s == 2 ? desc0[2] : desc0[3];
                     const uint32_t dcol = tbase + kDcol + db * kBT, acol = tbase + kAcol + s * 64;
+                    if constexpr (I8) {
 #pragma unroll
-                    for (int kk = 0; kk < kKB / 16; ++kk)
-                        tc::mma_f16_ts(dcol, acol + kk * 8, d0 + uint64_t(((kk >> 2) * kActBox + (kk & 3) * 32) >> 4),
-                                       idesc, kk > 0 ? 1u : 0u);
+                        for (int kk = 0; kk < kKB / 32; ++kk)  // k 32: 32 bytes per step
+                            tc::mma_i8_ts(dcol, acol + kk * 8, d0 + uint64_t((kk * 32) >> 4), idesc, kk > 0 ? 1u : 0u);
+                    } else {
+#pragma unroll
+                        for (int kk = 0; kk < kKB / 16; ++kk)  // k 16: 32 bytes per step
+                            tc::mma_f16_ts(dcol, acol + kk * 8,
+                                           d0 + uint64_t(((kk >> 2) * kActBox + (kk & 3) * 32) >> 4), idesc,
+                                           kk > 0 ? 1u : 0u);
+                    }
                     tc::commit(&rel[s]);
                     issued = true;
                 }
@@ -251,7 +315,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int n0 = (t / p.TT) * kBW;
             const int nrows = min(kBW, p.N - n0);
             uint32_t *tab = tabs + size_t(tl & 1) * tab_elems;
-            // ---- scale / zero table of the tile: [g][row] = fp16 scale bits | z << 16
+            // ---- scale / zero table of the tile (INT4): [g][row] = fp16 scale bits | z << 16
+            if constexpr (WB == 4) {
             if (!tc_wait(&scbar[tl & 1], (tl >> 1) & 1, abort)) break;
             if (tl >= 2 && !tc_wait(&tdone[tl & 1], ((tl - 2) >> 1) & 1, abort)) break;  // tile tl-2 folded
             if (!deq_sync()) break;
@@ -275,31 +340,66 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             if (!deq_sync()) break;
             if (threadIdx.x == 64) mbar_arrive(&tready[tl & 1]);
+            }
 
             for (int kb = 0; kb < p.nkb; ++kb, ++step) {
                 const uint32_t s = step % kNA;  // ring stage and TMEM A-buffer
                 // full also tells that the MMAs of step - kNA (stage and A-buffer s) have completed
                 if (!tc_wait(&full[s], (step / kNA) & 1, abort)) break;
-                // this row's 64 packed bytes (64-byte rows, 64-byte swizzle)
-                const uint8_t *wrow = ring + size_t(s) * kStageBytes + kActBytes + r * 64;
-                const uint32_t sw = uint32_t((r >> 1) & 3);
-                const uint4 w0 = lds128(wrow + ((uint32_t(2 * kh) ^ sw) << 4));
-                const uint4 w1 = lds128(wrow + ((uint32_t(2 * kh + 1) ^ sw) << 4));
-                const uint32_t tv = tab[(size_t)((kb * kKB) / p.gs) * p.tab_rs + r];
-                const uint32_t zc1 = magic_z | (tv >> 16);
-                const uint32_t zc = zc1 | (zc1 << 16);
-                tc::fence_after_sync();
-                {
-                    uint32_t v[32];
-                    unpack_word<BF16>(w0.x, zc, v + 0);
-                    unpack_word<BF16>(w0.y, zc, v + 4);
-                    unpack_word<BF16>(w0.z, zc, v + 8);
-                    unpack_word<BF16>(w0.w, zc, v + 12);
-                    unpack_word<BF16>(w1.x, zc, v + 16);
-                    unpack_word<BF16>(w1.y, zc, v + 20);
-                    unpack_word<BF16>(w1.z, zc, v + 24);
-                    unpack_word<BF16>(w1.w, zc, v + 28);
-                    tc::st_32x32b_x32(tlane + kAcol + s * 64 + kh * 32, v);
+                const uint8_t *wst = ring + size_t(s) * kStageBytes + kActBytes;
+                if constexpr (WB == 4) {
+                    // this row's 32 packed bytes of the k half (64-byte rows, 64-byte swizzle)
+                    const uint8_t *wrow = wst + r * 64;
+                    const uint32_t sw = uint32_t((r >> 1) & 3);
+                    const uint4 w0 = lds128(wrow + ((uint32_t(2 * kh) ^ sw) << 4));
+                    const uint4 w1 = lds128(wrow + ((uint32_t(2 * kh + 1) ^ sw) << 4));
+                    const uint32_t z = tab[(size_t)((kb * kKB) / p.gs) * p.tab_rs + r] >> 16;
+                    tc::fence_after_sync();
+                    if constexpr (I8) {
+                        const uint32_t zc = (0x80u - z) * 0x01010101u;
+                        uint32_t v[16];
+                        unpack_word_s8(w0.x, zc, v + 0);
+                        unpack_word_s8(w0.y, zc, v + 2);
+                        unpack_word_s8(w0.z, zc, v + 4);
+                        unpack_word_s8(w0.w, zc, v + 6);
+                        unpack_word_s8(w1.x, zc, v + 8);
+                        unpack_word_s8(w1.y, zc, v + 10);
+                        unpack_word_s8(w1.z, zc, v + 12);
+                        unpack_word_s8(w1.w, zc, v + 14);
+                        tc::st_32x32b_x16(tlane + kAcol + s * 64 + kh * 16, v);
+                    } else {
+                        const uint32_t zc1 = magic_z | z;
+                        const uint32_t zc = zc1 | (zc1 << 16);
+                        uint32_t v[32];
+                        unpack_word<BF16>(w0.x, zc, v + 0);
+                        unpack_word<BF16>(w0.y, zc, v + 4);
+                        unpack_word<BF16>(w0.z, zc, v + 8);
+                        unpack_word<BF16>(w0.w, zc, v + 12);
+                        unpack_word<BF16>(w1.x, zc, v + 16);
+                        unpack_word<BF16>(w1.y, zc, v + 20);
+                        unpack_word<BF16>(w1.z, zc, v + 24);
+                        unpack_word<BF16>(w1.w, zc, v + 28);
+                        tc::st_32x32b_x32(tlane + kAcol + s * 64 + kh * 32, v);
+                    }
+                } else {
+                    // this row's 16 packed bytes of the k half (32-byte rows, not swizzled)
+                    const uint4 w = lds128(wst + r * 32 + kh * 16);
+                    tc::fence_after_sync();
+                    if constexpr (I8) {
+                        uint32_t v[16];
+                        unpack2_word_s8(w.x, v + 0);
+                        unpack2_word_s8(w.y, v + 4);
+                        unpack2_word_s8(w.z, v + 8);
+                        unpack2_word_s8(w.w, v + 12);
+                        tc::st_32x32b_x16(tlane + kAcol + s * 64 + kh * 16, v);
+                    } else {
+                        uint32_t v[32];
+                        unpack2_word<BF16>(w.x, v + 0);
+                        unpack2_word<BF16>(w.y, v + 8);
+                        unpack2_word<BF16>(w.z, v + 16);
+                        unpack2_word<BF16>(w.w, v + 24);
+                        tc::st_32x32b_x32(tlane + kAcol + s * 64 + kh * 32, v);
+                    }
                 }
                 tc::wait_st();
                 tc::fence_before_sync();
@@ -319,15 +419,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int t = blockIdx.x; t < p.NT && !*abort; t += gridDim.x, ++tl) {
             const int n0 = (t / p.TT) * kBW, m0 = (t % p.TT) * kBT;
             const uint32_t *tab = tabs + size_t(tl & 1) * tab_elems;
-            if (!tc_wait(&tready[tl & 1], (tl >> 1) & 1, abort)) break;
+            if constexpr (WB == 4)
+                if (!tc_wait(&tready[tl & 1], (tl >> 1) & 1, abort)) break;
             float tot[64];
 #pragma unroll
             for (int j = 0; j < 64; ++j) tot[j] = 0.f;
             bool ok = true;
             for (int kb = 0; kb < p.nkb; ++kb, ++step) {
                 const uint32_t db = step % kND, s = step % kNA;
-                const uint32_t tv = tab[(size_t)((kb * kKB) / p.gs) * p.tab_rs + r];
-                const float sv = __half2float(__ushort_as_half(uint16_t(tv & 0xFFFFu)));
+                float sv = 1.f;  // INT2: the per-tensor scale is applied at the end
+                if constexpr (WB == 4)
+                    sv = __half2float(__ushort_as_half(uint16_t(tab[(size_t)((kb * kKB) / p.gs) * p.tab_rs + r])));
                 if (!tc_wait(&rel[s], (step / kNA) & 1, abort)) { ok = false; break; }
                 tc::fence_after_sync();
 #pragma unroll
@@ -341,12 +443,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                         if (lane == 0) mbar_arrive(&dfree[db]);
                     }
 #pragma unroll
-                    for (int j = 0; j < 16; ++j) tot[c * 16 + j] = fmaf(sv, __uint_as_float(d[j]), tot[c * 16 + j]);
+                    for (int j = 0; j < 16; ++j) {
+                        // INT8: exact int32 block sums (< 2^24 in magnitude, exact in fp32)
+                        const float dv = I8 ? float(int(d[j])) : __uint_as_float(d[j]);
+                        tot[c * 16 + j] = fmaf(sv, dv, tot[c * 16 + j]);
+                    }
                 }
             }
             if (!ok) break;
             __syncwarp();
-            if (lane == 0) mbar_arrive(&tdone[tl & 1]);
+            if constexpr (WB == 4)
+                if (lane == 0) mbar_arrive(&tdone[tl & 1]);
 
             // ---- epilogue: C[m][n] = total (+ bias[n]), one weight row x 64 tokens per thread
             const int n = n0 + r;
@@ -356,10 +463,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if constexpr (BF16) b = __bfloat162float(static_cast<const __nv_bfloat16 *>(p.bias)[n]);
                     else b = __half2float(static_cast<const __half *>(p.bias)[n]);
                 }
+                const float ws = (WB == 2) ? p.scale32[0] : 1.f;
                 const int mb = m0 + th * 64;
 #pragma unroll
-                for (int j = 0; j < 64; ++j)
-                    if (mb + j < p.M) store_out<BF16>(p.C, (long long)(mb + j) * p.N + n, tot[j] + b);
+                for (int j = 0; j < 64; ++j) {
+                    if (mb + j >= p.M) continue;
+                    float v;
+                    if constexpr (I8) v = p.a_scale[mb + j] * (WB == 2 ? ws * tot[j] : tot[j]);
+                    else v = ws * tot[j];
+                    store_out<BF16>(p.C, (long long)(mb + j) * p.N + n, v + b);
+                }
             }
         }
     }
@@ -380,20 +493,20 @@ struct TcPlan {
     bool ok = false;
 };
 
-TcPlan make_plan(int64_t K, int G, const DeviceInfo &dev)
+// G: groups of the INT4 scale table (0 for INT2: one per-tensor scale, no table).
+TcPlan make_plan(int nkb, int G, int stage, const DeviceInfo &dev)
 {
     TcPlan pl;
-    const int nkb = int(K / kKB);
     const size_t scst = (size_t(2) * 2 * kBW * G * 2 + 15) & ~size_t(15);
     pl.tab_rs = kBW + 1;
     const size_t tab = (size_t(2) * G * pl.tab_rs * 4 + 15) & ~size_t(15);
-    const size_t bars = 8 * (2 * 8 + 20) + 16;
+    const size_t bars = 8 * (3 * kNA + 2 * kND + 11) + 16;
     const size_t budget = size_t(dev.max_smem_optin) - 1024;
-    if (budget <= scst + tab + bars) return pl;
     // the ring has one stage per TMEM A-buffer
-    if (nkb < kNA || (budget - scst - tab - bars) / kStageBytes < size_t(kNA)) return pl;
+    if (nkb < kNA || budget <= scst + tab + bars || (budget - scst - tab - bars) / size_t(stage) < size_t(kNA))
+        return pl;
     pl.S = kNA;
-    size_t off = size_t(pl.S) * kStageBytes;
+    size_t off = size_t(pl.S) * stage;
     pl.scst_off = int(off);
     off += scst;
     pl.tab_off = int(off);
@@ -405,11 +518,11 @@ TcPlan make_plan(int64_t K, int G, const DeviceInfo &dev)
     return pl;
 }
 
-template <bool BF16>
+template <int WB, int AM>
 wq_status launch(const TcPlan &pl, const CUtensorMap &ta, const CUtensorMap &tw, const TcParams &p, int grid,
                  cudaStream_t st)
 {
-    auto kern = tc_gemm_kernel<BF16>;
+    auto kern = tc_gemm_kernel<WB, AM>;
     static size_t configured = 0;
     if (pl.smem > configured) {
         if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(pl.smem)) != cudaSuccess)
@@ -433,30 +546,42 @@ wq_status launch(const TcPlan &pl, const CUtensorMap &ta, const CUtensorMap &tw,
 
 }  // namespace
 
-// Many-token W4A16 path (INT4, FP16 / BF16 activations).  WQ_ERR_UNSUPPORTED when the
-// configuration has no plan here (the caller then uses the tiled mma.sync path).
-wq_status tc_gemm(int WB, int AM, const void *A, const uint8_t *Wq, const void *scales, const void *zeros,
-                  const void *bias, void *C, int64_t M, int64_t N, int64_t K, const wq_qconfig &c, cudaStream_t st)
+// Many-token path on the tcgen05 tensor cores: INT4 (group size a multiple of 128) or ternary
+// INT2 weights, FP16 / BF16 (AM 0 / 1) or INT8 (AM 2, with a_scale) activations.
+// WQ_ERR_UNSUPPORTED when the configuration has no plan here (the caller then uses the
+// tiled mma.sync path).
+wq_status tc_gemm(int WB, int AM, const void *A, const float *a_scale, const uint8_t *Wq, const void *scales,
+                  const void *zeros, const void *bias, void *C, int64_t M, int64_t N, int64_t K,
+                  const wq_qconfig &c, cudaStream_t st)
 {
-    if (WB != 4 || (AM != 0 && AM != 1)) return fail(WQ_ERR_UNSUPPORTED, "tc_gemm: INT4 weights, FP activations");
-    if (K % kKB || c.group_size % kKB) return fail(WQ_ERR_UNSUPPORTED, "tc_gemm: K and group_size multiples of 128");
+    if (WB == 4 && (K % kKB || c.group_size % kKB))
+        return fail(WQ_ERR_UNSUPPORTED, "tc_gemm: INT4 needs K and group_size multiples of 128");
+    const int es = AM == 2 ? 1 : 2;
+    if ((K * es) % 16) return fail(WQ_ERR_UNSUPPORTED, "tc_gemm: activation rows must be 16-byte multiples");
     const DeviceInfo &dev = device_info();
-    const int G = int(K / c.group_size);
-    const TcPlan pl = make_plan(K, G, dev);
+    const int G = WB == 4 ? int(K / c.group_size) : 0;
+    const int nkb = int((K + kKB - 1) / kKB);
+    const int stage = WB == 4 ? (AM == 2 ? stage_bytes(4, 2) : stage_bytes(4, 0))
+                              : (AM == 2 ? stage_bytes(2, 2) : stage_bytes(2, 0));
+    const TcPlan pl = make_plan(nkb, G, stage, dev);
     if (!pl.ok) return fail(WQ_ERR_UNSUPPORTED, "tc_gemm: no shared-memory plan for K=%lld", (long long)K);
     CUtensorMap ta, tw;
     {
+        // activations [M][K]: one box = 128 tokens x 128 bytes (past K: zeros)
         const uint64_t dims[2] = {uint64_t(K), uint64_t(M)};
-        const uint64_t strides[1] = {uint64_t(K) * 2};
-        const uint32_t box[2] = {64, uint32_t(kBT)};
-        wq_status rc = encode_tmap(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, A, dims, strides, box, 128);
+        const uint64_t strides[1] = {uint64_t(K) * es};
+        const uint32_t box[2] = {uint32_t(128 / es), uint32_t(kBT)};
+        wq_status rc = encode_tmap(&ta, es == 1 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_UINT16, 2,
+                                   A, dims, strides, box, 128);
         if (rc != WQ_OK) return rc;
     }
     {
-        const uint64_t dims[2] = {uint64_t(K / 2), uint64_t(N)};
-        const uint64_t strides[1] = {uint64_t(K / 2)};
-        const uint32_t box[2] = {uint32_t(kKB / 2), uint32_t(kBW)};
-        wq_status rc = encode_tmap(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, Wq, dims, strides, box, 64);
+        // packed weights [N][K*WB/8]: one box = 128 rows x one block (64 B INT4 / 32 B INT2)
+        const uint64_t row_bytes = uint64_t(K) * WB / 8;
+        const uint64_t dims[2] = {row_bytes, uint64_t(N)};
+        const uint64_t strides[1] = {row_bytes};
+        const uint32_t box[2] = {uint32_t(kKB * WB / 8), uint32_t(kBW)};
+        wq_status rc = encode_tmap(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, Wq, dims, strides, box, WB == 4 ? 64 : 0);
         if (rc != WQ_OK) return rc;
     }
     TcParams p{};
@@ -464,9 +589,11 @@ wq_status tc_gemm(int WB, int AM, const void *A, const uint8_t *Wq, const void *
     p.N = int(N);
     p.K = int(K);
     p.G = G;
-    p.gs = c.group_size;
-    p.sym = c.symmetric;
-    p.nkb = int(K / kKB);
+    p.gs = WB == 4 ? c.group_size : int(K);
+    p.sym = WB == 4 ? c.symmetric : 1;
+    p.a_scale = a_scale;
+    p.scale32 = static_cast<const float *>(scales);
+    p.nkb = nkb;
     p.TT = int((M + kBT - 1) / kBT);
     p.NT = p.TT * int((N + kBW - 1) / kBW);
     p.S = pl.S;
@@ -479,7 +606,14 @@ wq_status tc_gemm(int WB, int AM, const void *A, const uint8_t *Wq, const void *
     p.bias = bias;
     p.C = C;
     const int grid = std::min(dev.sm_count, p.NT);
-    return AM == 1 ? launch<true>(pl, ta, tw, p, grid, st) : launch<false>(pl, ta, tw, p, grid, st);
+    if (WB == 4) {
+        if (AM == 0) return launch<4, 0>(pl, ta, tw, p, grid, st);
+        if (AM == 1) return launch<4, 1>(pl, ta, tw, p, grid, st);
+        return launch<4, 2>(pl, ta, tw, p, grid, st);
+    }
+    if (AM == 0) return launch<2, 0>(pl, ta, tw, p, grid, st);
+    if (AM == 1) return launch<2, 1>(pl, ta, tw, p, grid, st);
+    return launch<2, 2>(pl, ta, tw, p, grid, st);
 }
 
 int tc_read_error()

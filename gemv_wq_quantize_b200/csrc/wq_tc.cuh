@@ -58,6 +58,16 @@ __device__ __forceinline__ void ld_32x32b_x32(uint32_t taddr, uint32_t (&v)[32])
         : "memory");
 }
 
+__device__ __forceinline__ void st_32x32b_x16(uint32_t taddr, const uint32_t (&v)[16])
+{
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
+        "%14, %15, %16};" ::"r"(taddr),
+        "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]),
+        "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
+        : "memory");
+}
+
 __device__ __forceinline__ void ld_32x32b_x16(uint32_t taddr, uint32_t (&v)[16])
 {
     asm volatile(
@@ -80,6 +90,16 @@ __device__ __forceinline__ void mma_f16_ts(uint32_t d_taddr, uint32_t a_taddr, u
         : "memory");
 }
 
+__device__ __forceinline__ void mma_i8_ts(uint32_t d_taddr, uint32_t a_taddr, uint64_t b_desc, uint32_t idesc,
+                                          uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::i8 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_taddr),
+        "r"(a_taddr), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
 // The mbarrier receives one arrival once all tcgen05 operations this thread issued before
 // have completed.
 __device__ __forceinline__ void commit(uint64_t *bar)
@@ -95,6 +115,13 @@ __host__ __device__ constexpr uint32_t idesc_f16(bool bf16, int M, int N)
 {
     return (1u << 4) | (uint32_t(bf16) << 7) | (uint32_t(bf16) << 10) | (uint32_t(N >> 3) << 17) |
            (uint32_t(M >> 4) << 24);
+}
+
+// Instruction descriptor of kind::i8 with int32 accumulation (D format bits 4-5 = S32),
+// both operands signed 8-bit (A / B format bits 7-9 / 10-12 = 1) and K-major.
+__host__ __device__ constexpr uint32_t idesc_i8(int M, int N)
+{
+    return (2u << 4) | (1u << 7) | (1u << 10) | (uint32_t(N >> 3) << 17) | (uint32_t(M >> 4) << 24);
 }
 
 // Shared-memory matrix descriptor, K-major operand written with the 128-byte swizzle:
