@@ -25,7 +25,8 @@ wq_status gemv_small_m(int WB, int AM, const void *A, const float *a_scale, cons
 int gemv_read_error();
 wq_status tc_gemm(int WB, int AM, const void *A, const float *a_scale, const uint8_t *Wq, const void *scales,
                   const void *zeros, const void *bias, void *C, int64_t M, int64_t N, int64_t K,
-                  const wq_qconfig &c, cudaStream_t st);
+                  const wq_qconfig &c, void *ws, size_t ws_bytes, cudaStream_t st);
+size_t tc_workspace_size(int64_t M, int64_t N, int64_t K);
 int tc_read_error();
 
 namespace {
@@ -141,7 +142,7 @@ wq_status dispatch(int WB, int AM, const void *A, const float *a_scale, const ui
         wq_status rc = gemv_small_m(WB, AM, A, a_scale, Wq, scales, zeros, bias, C, acc_out, M, N, K, c, st);
         if (rc != WQ_ERR_UNSUPPORTED) return rc;
     } else if (!acc_out) {
-        wq_status rc = tc_gemm(WB, AM, A, a_scale, Wq, scales, zeros, bias, C, M, N, K, c, st);
+        wq_status rc = tc_gemm(WB, AM, A, a_scale, Wq, scales, zeros, bias, C, M, N, K, c, ws, ws_bytes, st);
         if (rc != WQ_ERR_UNSUPPORTED) return rc;
     }
     return skinny_gemm(WB, AM, A, a_scale, Wq, scales, zeros, bias, C, acc_out, M, N, K, c, ws, ws_bytes, st);
@@ -201,7 +202,8 @@ extern "C" size_t wq_workspace_size(int64_t M, int64_t N, int64_t K, wq_qconfig 
     if (M <= 0 || N <= 0 || K <= 0 || (c.bits != 4 && c.bits != 2)) return 0;
     // the INT8 path has the smaller activation blocks; size for the larger of the two
     if (M <= 16) return 0;  // the few-token kernel needs no workspace
-    return std::max(skinny_workspace_size(c.bits, 0, M, N, K), skinny_workspace_size(c.bits, 2, M, N, K));
+    return std::max({skinny_workspace_size(c.bits, 0, M, N, K), skinny_workspace_size(c.bits, 2, M, N, K),
+                     tc_workspace_size(M, N, K)});
 }
 
 extern "C" wq_status w4a16_gemm(const void *A, wq_dtype a_dt, const uint8_t *Wq, const void *scales,

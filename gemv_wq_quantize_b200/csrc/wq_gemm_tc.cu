@@ -66,7 +66,10 @@ struct TcParams {
     int M, N, K, G, gs, sym;
     const float *a_scale;  // INT8 activations: per-token scale
     const float *scale32;  // INT2 weights: per-tensor scale
-    int nkb;     // K / 128
+    int nkb;     // blocks of 128 k
+    int ks;      // K slices per tile (split-K when tiles are fewer than SMs)
+    float *ws_part;     // ks > 1: fp32 partial totals [tile][slice][128 rows][128 tokens]
+    unsigned *ws_cnt;   // ks > 1: per-tile arrival counters (left at zero)
     int TT, NT;  // token tiles, tiles
     int S;       // ring stages
     int scst_off, tab_off, bar_off;
@@ -188,8 +191,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint64_t *full = bars, *rel = bars + kNA;
     uint64_t *afull = bars + 2 * kNA, *dfree = afull + kNA;
     uint64_t *scbar = dfree + kND, *tready = scbar + 2, *tdone = tready + 2, *fin = tdone + 2, *mbar = fin + 1;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(mbar + 1);
+    uint64_t *fbar = mbar + 1;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(fbar + 1);
     volatile int *abort = reinterpret_cast<volatile int *>(tmem_slot + 1);
+    volatile int *last_flag = abort + 1;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const size_t stab_elems = size_t(kBW) * p.G;          // one staging buffer (scales or zeros)
@@ -209,6 +214,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         mbar_init(fin, 1);
         mbar_init(mbar, kDeqWarps);
+        mbar_init(fbar, kFoldWarps);
         *abort = 0;
         fence_barrier_init();
     }
@@ -227,13 +233,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) {
             tma_prefetch_desc(&tmap_a);
             tma_prefetch_desc(&tmap_w);
-            grid_dep_wait();  // activations may be written by the previous kernel
-            uint32_t step = 0;
-            int tl = 0;
-            for (int t = blockIdx.x; t < p.NT && !*abort; t += gridDim.x, ++tl) {
-                const int n0 = (t / p.TT) * kBW, m0 = (t % p.TT) * kBT;
+            auto issue_scales = [&](int n0, int tl) {  // the tile's scale / zero rows: contiguous in [N, G]
                 if constexpr (WB == 4) {
-                    // the tile's scale / zero rows: contiguous in [N, G]
                     const int nrows = min(kBW, p.N - n0);
                     const uint32_t bytes16 = (uint32_t(nrows) * p.G * 2u) & ~15u;
                     uint16_t *sc = scst + size_t(tl & 1) * 2 * stab_elems;
@@ -243,14 +244,41 @@ __global__ void __launch_bounds__(kThreads, 1)
                         if (!p.sym) bulk_load(sc + stab_elems, p.zeros + (size_t)n0 * p.G, bytes16, &scbar[tl & 1]);
                     }
                 }
-                for (int kb = 0; kb < p.nkb; ++kb, ++step) {
+            };
+            // Weights and scales do not depend on the previous kernel: the first task's scales and
+            // the packed weights of its first kNA blocks go out before griddepcontrol.wait.
+            int npre = 0;
+            if (blockIdx.x < p.NT * p.ks) {
+                const int tile = blockIdx.x / p.ks, sp = blockIdx.x - tile * p.ks;
+                const int kb0 = sp * p.nkb / p.ks, kb1 = (sp + 1) * p.nkb / p.ks;
+                const int n0 = (tile / p.TT) * kBW;
+                issue_scales(n0, 0);
+                npre = min(kNA, kb1 - kb0);
+                for (int i = 0; i < npre; ++i) {
+                    uint8_t *st = ring + size_t(i) * kStageBytes;
+                    mbar_arrive_expect_tx(&full[i], kStageBytes);
+                    tma_load_2d(st + kActBytes, &tmap_w, (kb0 + i) * (kKB * WB / 8), n0, &full[i]);
+                }
+            }
+            grid_dep_wait();  // activations may be written by the previous kernel
+            uint32_t step = 0;
+            int tl = 0;
+            for (int t = blockIdx.x; t < p.NT * p.ks && !*abort; t += gridDim.x, ++tl) {
+                const int tile = t / p.ks, sp = t - tile * p.ks;
+                const int kb0 = sp * p.nkb / p.ks, kb1 = (sp + 1) * p.nkb / p.ks;
+                const int n0 = (tile / p.TT) * kBW, m0 = (tile % p.TT) * kBT;
+                if (tl > 0) issue_scales(n0, tl);
+                for (int kb = kb0; kb < kb1; ++kb, ++step) {
                     const int s = int(step % kNA);
-                    if (!tc_wait(&rel[s], ((step / kNA) & 1) ^ 1, abort)) break;
                     uint8_t *st = ring + size_t(s) * kStageBytes;
-                    mbar_arrive_expect_tx(&full[s], kStageBytes);
+                    const bool pre = tl == 0 && kb - kb0 < npre;  // weights already on their way
+                    if (!pre) {
+                        if (!tc_wait(&rel[s], ((step / kNA) & 1) ^ 1, abort)) break;
+                        mbar_arrive_expect_tx(&full[s], kStageBytes);
+                        tma_load_2d(st + kActBytes, &tmap_w, kb * (kKB * WB / 8), n0, &full[s]);
+                    }
                     tma_load_2d(st, &tmap_a, kb * kKB, m0, &full[s]);
                     if constexpr (!I8) tma_load_2d(st + kActBox, &tmap_a, kb * kKB + 64, m0, &full[s]);
-                    tma_load_2d(st + kActBytes, &tmap_w, kb * (kKB * WB / 8), n0, &full[s]);
                 }
             }
             // nothing may land in shared memory after the CTA exits: wait for the last stages
@@ -266,8 +294,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int b = 0; b < kNA; ++b) desc0[b] = tc::sdesc_sw128(smem_u32(ring + size_t(b) * kStageBytes));
             uint32_t step = 0;
             bool issued = false;
-            for (int t = blockIdx.x; t < p.NT && !*abort; t += gridDim.x) {
-                for (int kb = 0; kb < p.nkb; ++kb, ++step) {
+            for (int t = blockIdx.x; t < p.NT * p.ks && !*abort; t += gridDim.x) {
+                const int tile = t / p.ks, sp = t - tile * p.ks;
+                const int nb = (sp + 1) * p.nkb / p.ks - sp * p.nkb / p.ks;
+                for (int kb = 0; kb < nb; ++kb, ++step) {
                     const uint32_t s = step % kNA, db = step % kND;
                     // afull: the unpacking warps have seen the stage's data and stored the weights
                     if (!tc_wait(&afull[s], (step / kNA) & 1, abort)) break;
@@ -311,8 +341,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             return ok;
         };
         int tl = 0;
-        for (int t = blockIdx.x; t < p.NT && !*abort; t += gridDim.x, ++tl) {
-            const int n0 = (t / p.TT) * kBW;
+        for (int t = blockIdx.x; t < p.NT * p.ks && !*abort; t += gridDim.x, ++tl) {
+            const int tile = t / p.ks, sp = t - tile * p.ks;
+            const int kb0 = sp * p.nkb / p.ks, kb1 = (sp + 1) * p.nkb / p.ks;
+            const int n0 = (tile / p.TT) * kBW;
             const int nrows = min(kBW, p.N - n0);
             uint32_t *tab = tabs + size_t(tl & 1) * tab_elems;
             // ---- scale / zero table of the tile (INT4): [g][row] = fp16 scale bits | z << 16
@@ -342,7 +374,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (threadIdx.x == 64) mbar_arrive(&tready[tl & 1]);
             }
 
-            for (int kb = 0; kb < p.nkb; ++kb, ++step) {
+            for (int kb = kb0; kb < kb1; ++kb, ++step) {
                 const uint32_t s = step % kNA;  // ring stage and TMEM A-buffer
                 // full also tells that the MMAs of step - kNA (stage and A-buffer s) have completed
                 if (!tc_wait(&full[s], (step / kNA) & 1, abort)) break;
@@ -416,8 +448,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         grid_dep_wait();  // C and bias belong to this kernel only once the previous one is done
         uint32_t step = 0;
         int tl = 0;
-        for (int t = blockIdx.x; t < p.NT && !*abort; t += gridDim.x, ++tl) {
-            const int n0 = (t / p.TT) * kBW, m0 = (t % p.TT) * kBT;
+        uint32_t fphase = 0;
+        auto fold_sync = [&]() -> bool {  // bounded barrier of the folding warps (one arrival per warp)
+            __syncwarp();
+            if (lane == 0) mbar_arrive(fbar);
+            const bool ok = tc_wait(fbar, fphase & 1, abort);
+            ++fphase;
+            return ok;
+        };
+        for (int t = blockIdx.x; t < p.NT * p.ks && !*abort; t += gridDim.x, ++tl) {
+            const int tile = t / p.ks, sp = t - tile * p.ks;
+            const int kb0 = sp * p.nkb / p.ks, kb1 = (sp + 1) * p.nkb / p.ks;
+            const int n0 = (tile / p.TT) * kBW, m0 = (tile % p.TT) * kBT;
             const uint32_t *tab = tabs + size_t(tl & 1) * tab_elems;
             if constexpr (WB == 4)
                 if (!tc_wait(&tready[tl & 1], (tl >> 1) & 1, abort)) break;
@@ -425,7 +467,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int j = 0; j < 64; ++j) tot[j] = 0.f;
             bool ok = true;
-            for (int kb = 0; kb < p.nkb; ++kb, ++step) {
+            for (int kb = kb0; kb < kb1; ++kb, ++step) {
                 const uint32_t db = step % kND, s = step % kNA;
                 float sv = 1.f;  // INT2: the per-tensor scale is applied at the end
                 if constexpr (WB == 4)
@@ -454,6 +496,38 @@ __global__ void __launch_bounds__(kThreads, 1)
             __syncwarp();
             if constexpr (WB == 4)
                 if (lane == 0) mbar_arrive(&tdone[tl & 1]);
+
+            if (p.ks > 1) {
+                // split K: publish this slice's totals; the last slice of the tile to arrive adds
+                // all slices in slice order (deterministic) and writes C
+                float *part = p.ws_part + ((size_t(tile) * p.ks + sp) * kBW + r) * kBT + th * 64;
+#pragma unroll
+                for (int j = 0; j < 64; j += 4)
+                    *reinterpret_cast<float4 *>(part + j) = make_float4(tot[j], tot[j + 1], tot[j + 2], tot[j + 3]);
+                __threadfence();
+                if (!fold_sync()) break;
+                if (threadIdx.x == 64 + kDeqWarps * 32) {
+                    const unsigned old = atomicAdd(&p.ws_cnt[tile], 1u);
+                    *last_flag = (old == unsigned(p.ks - 1)) ? 1 : 0;
+                    if (old == unsigned(p.ks - 1)) p.ws_cnt[tile] = 0u;  // left at zero for the next call
+                }
+                if (!fold_sync()) break;
+                if (!*last_flag) continue;
+                __threadfence();
+#pragma unroll
+                for (int j = 0; j < 64; ++j) tot[j] = 0.f;
+                for (int q2 = 0; q2 < p.ks; ++q2) {
+                    const float *pq = p.ws_part + ((size_t(tile) * p.ks + q2) * kBW + r) * kBT + th * 64;
+#pragma unroll
+                    for (int j = 0; j < 64; j += 4) {
+                        const float4 v4 = __ldcg(reinterpret_cast<const float4 *>(pq + j));
+                        tot[j] += v4.x;
+                        tot[j + 1] += v4.y;
+                        tot[j + 2] += v4.z;
+                        tot[j + 3] += v4.w;
+                    }
+                }
+            }
 
             // ---- epilogue: C[m][n] = total (+ bias[n]), one weight row x 64 tokens per thread
             const int n = n0 + r;
@@ -500,7 +574,7 @@ TcPlan make_plan(int nkb, int G, int stage, const DeviceInfo &dev)
     const size_t scst = (size_t(2) * 2 * kBW * G * 2 + 15) & ~size_t(15);
     pl.tab_rs = kBW + 1;
     const size_t tab = (size_t(2) * G * pl.tab_rs * 4 + 15) & ~size_t(15);
-    const size_t bars = 8 * (3 * kNA + 2 * kND + 11) + 16;
+    const size_t bars = 8 * (3 * kNA + 2 * kND + 12) + 16;
     const size_t budget = size_t(dev.max_smem_optin) - 1024;
     // the ring has one stage per TMEM A-buffer
     if (nkb < kNA || budget <= scst + tab + bars || (budget - scst - tab - bars) / size_t(stage) < size_t(kNA))
@@ -512,7 +586,7 @@ TcPlan make_plan(int nkb, int G, int stage, const DeviceInfo &dev)
     pl.tab_off = int(off);
     off += tab;
     pl.bar_off = int((off + 7) & ~size_t(7));
-    off = pl.bar_off + size_t(8) * (3 * kNA + 2 * kND + 11) + 8;
+    off = pl.bar_off + size_t(8) * (3 * kNA + 2 * kND + 12) + 16;
     pl.smem = ((off + 15) & ~size_t(15)) + 1024;
     pl.ok = pl.smem <= size_t(dev.max_smem_optin);
     return pl;
@@ -544,15 +618,40 @@ wq_status launch(const TcPlan &pl, const CUtensorMap &ta, const CUtensorMap &tw,
     return check_launch("tc_gemm_kernel");
 }
 
+// K slices per tile: when the tiles are fewer than the SMs, each tile's K range is cut
+// into slices (at least 4 blocks each) so that tiles x slices <= SMs.
+int choose_slices(int64_t M, int64_t N, int64_t K, int sm_count)
+{
+    const int64_t tiles = ((M + kBT - 1) / kBT) * ((N + kBW - 1) / kBW);
+    const int64_t nkb = (K + kKB - 1) / kKB;
+    if (tiles >= sm_count) return 1;
+    return int(std::max<int64_t>(1, std::min<int64_t>(sm_count / tiles, nkb / 4)));
+}
+
+size_t split_bytes(int64_t M, int64_t N, int ks)
+{
+    if (ks <= 1) return 0;
+    const int64_t tiles = ((M + kBT - 1) / kBT) * ((N + kBW - 1) / kBW);
+    return (size_t(tiles) * ks * kBW * kBT * 4 + size_t(tiles) * 4 + 255) & ~size_t(255);
+}
+
 }  // namespace
+
+// Workspace that lets the tcgen05 path split K when it has fewer tiles than SMs.
+size_t tc_workspace_size(int64_t M, int64_t N, int64_t K)
+{
+    return split_bytes(M, N, choose_slices(M, N, K, device_info().sm_count));
+}
 
 // Many-token path on the tcgen05 tensor cores: INT4 (group size a multiple of 128) or ternary
 // INT2 weights, FP16 / BF16 (AM 0 / 1) or INT8 (AM 2, with a_scale) activations.
 // WQ_ERR_UNSUPPORTED when the configuration has no plan here (the caller then uses the
 // tiled mma.sync path).
+// The workspace (zero-filled once, see the ABI) is used for split-K partial sums when it
+// is large enough; otherwise every tile covers all of K.
 wq_status tc_gemm(int WB, int AM, const void *A, const float *a_scale, const uint8_t *Wq, const void *scales,
                   const void *zeros, const void *bias, void *C, int64_t M, int64_t N, int64_t K,
-                  const wq_qconfig &c, cudaStream_t st)
+                  const wq_qconfig &c, void *ws, size_t ws_bytes, cudaStream_t st)
 {
     if (WB == 4 && (K % kKB || c.group_size % kKB))
         return fail(WQ_ERR_UNSUPPORTED, "tc_gemm: INT4 needs K and group_size multiples of 128");
@@ -596,6 +695,12 @@ wq_status tc_gemm(int WB, int AM, const void *A, const float *a_scale, const uin
     p.nkb = nkb;
     p.TT = int((M + kBT - 1) / kBT);
     p.NT = p.TT * int((N + kBW - 1) / kBW);
+    p.ks = choose_slices(M, N, K, dev.sm_count);
+    if (p.ks > 1 && (!ws || ws_bytes < split_bytes(M, N, p.ks))) p.ks = 1;
+    if (p.ks > 1) {
+        p.ws_part = static_cast<float *>(ws);
+        p.ws_cnt = reinterpret_cast<unsigned *>(static_cast<uint8_t *>(ws) + size_t(p.NT) * p.ks * kBW * kBT * 4);
+    }
     p.S = pl.S;
     p.scst_off = pl.scst_off;
     p.tab_off = pl.tab_off;
@@ -605,7 +710,7 @@ wq_status tc_gemm(int WB, int AM, const void *A, const float *a_scale, const uin
     p.zeros = static_cast<const uint16_t *>(zeros);
     p.bias = bias;
     p.C = C;
-    const int grid = std::min(dev.sm_count, p.NT);
+    const int grid = std::min(dev.sm_count, p.NT * p.ks);
     if (WB == 4) {
         if (AM == 0) return launch<4, 0>(pl, ta, tw, p, grid, st);
         if (AM == 1) return launch<4, 1>(pl, ta, tw, p, grid, st);
