@@ -628,11 +628,13 @@ int choose_slices(int64_t M, int64_t N, int64_t K, int sm_count)
     return int(std::max<int64_t>(1, std::min<int64_t>(sm_count / tiles, nkb / 4)));
 }
 
+// Partials of tiles x slices <= SMs (64 KB each) fill at most the shared scratch area;
+// the per-tile counters follow it.
 size_t split_bytes(int64_t M, int64_t N, int ks)
 {
     if (ks <= 1) return 0;
     const int64_t tiles = ((M + kBT - 1) / kBT) * ((N + kBW - 1) / kBW);
-    return (size_t(tiles) * ks * kBW * kBT * 4 + size_t(tiles) * 4 + 255) & ~size_t(255);
+    return (ws_scratch_bytes() + size_t(tiles) * 4 + 255) & ~size_t(255);
 }
 
 }  // namespace
@@ -699,7 +701,7 @@ wq_status tc_gemm(int WB, int AM, const void *A, const float *a_scale, const uin
     if (p.ks > 1 && (!ws || ws_bytes < split_bytes(M, N, p.ks))) p.ks = 1;
     if (p.ks > 1) {
         p.ws_part = static_cast<float *>(ws);
-        p.ws_cnt = reinterpret_cast<unsigned *>(static_cast<uint8_t *>(ws) + size_t(p.NT) * p.ks * kBW * kBT * 4);
+        p.ws_cnt = reinterpret_cast<unsigned *>(static_cast<uint8_t *>(ws) + ws_scratch_bytes());
     }
     p.S = pl.S;
     p.scst_off = pl.scst_off;

@@ -35,6 +35,12 @@ wq_status encode_tmap_2d(CUtensorMap *map, CUtensorMapDataType dt, const void *b
 wq_status encode_tmap(CUtensorMap *map, CUtensorMapDataType dt, int rank, const void *base, const uint64_t *dims,
                       const uint64_t *strides_bytes, const uint32_t *box, int swizzle_bytes);
 
+// Layout shared by every kernel that uses the caller's workspace, so that one workspace
+// can serve calls of any shape and kernel in turn: scratch partial sums in the first
+// ws_scratch_bytes() (64 KB per SM: the most any plan uses), then the self-resetting
+// arrival counters.  A counter slot is therefore never some other call's scratch.
+inline size_t ws_scratch_bytes() { return size_t(device_info().sm_count) * 65536; }
+
 // Reads (and clears) the device error words of all kernels with bounded waits.
 int read_device_errors();
 

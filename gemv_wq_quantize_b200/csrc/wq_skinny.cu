@@ -636,7 +636,9 @@ Plan make_plan(int64_t M, int64_t N, int64_t K, int WB, int AM, size_t ws_bytes,
     pl.ablk = pl.MP * pl.KU * esize;
     const int steps = steps_of(WB, AM);
     pl.frag = pl.NT * steps * 256 + (AM == A_I8 ? 256 : 0);
-    pl.ws_need = size_t(dev.sm_count) * 2 * kRows * pl.MP * sizeof(float) + size_t(pl.RG) * sizeof(unsigned);
+    // partials: sm_count CTAs x 2 x kRows x MP floats (<= 64 KB per SM); counters after the
+    // shared scratch area
+    pl.ws_need = ws_scratch_bytes() + size_t(pl.RG) * sizeof(unsigned);
     pl.ws_need = (pl.ws_need + 255) & ~size_t(255);
     pl.split = (ws_bytes >= pl.ws_need) ? 1 : 0;
     pl.P = int(std::min<long long>(dev.sm_count, pl.split ? pl.U : pl.RG));
@@ -720,9 +722,7 @@ wq_status skinny_gemm(int WB, int AM, const void *A, const float *a_scale, const
     p.C = C;
     p.acc_out = acc_out;
     p.ws_partial = pl.split ? static_cast<float *>(ws) : nullptr;
-    p.ws_counter = pl.split ? reinterpret_cast<unsigned *>(static_cast<uint8_t *>(ws) +
-                                                           size_t(dev.sm_count) * 2 * kRows * pl.MP * sizeof(float))
-                            : nullptr;
+    p.ws_counter = pl.split ? reinterpret_cast<unsigned *>(static_cast<uint8_t *>(ws) + ws_scratch_bytes()) : nullptr;
     for (int64_t m0 = 0; m0 < M; m0 += 64) {
         p.m0 = int(m0);
         p.M = int(std::min<int64_t>(64, M - m0));

@@ -244,6 +244,42 @@ def test_a8_small_bit_exact_sums(quant, M, N, K):
     assert err <= TOL, err
 
 
+@pytest.mark.parametrize("quant", ["sym4", "asym4", "tern2"])
+@pytest.mark.parametrize("M,N,K", SMALL + [(128, 384, 1024), (200, 136, 640)])
+def test_a8_small_without_group_sums(quant, M, N, K):
+    # without acc_out, more than 16 tokens run on the tcgen05 kernel (kind::i8)
+    if quant == "tern2":
+        K = max(64, K // 64 * 64)
+    C, _, qc, (oAq, oasc, oWq, os_, oz), _ = run_a8(M, N, K, quant, seed=M * 5 + N, want_acc=False)
+    _, ref, _ = oracle.gemm_a8(oAq, oasc, oWq, N, K, qc.bits, qc.symmetric, 128, os_, oz)
+    err = rel_fro(bits_np(C), ref, torch.float16)
+    assert err <= TOL, err
+
+
+@pytest.mark.parametrize("use_ws", [True, False])
+def test_a8_split_k_plans(use_ws):
+    # 128 tokens x 512 rows: 4 tiles, so K is split over CTAs when the workspace allows it
+    M, N, K = 128, 512, 2048
+    C, _, qc, (oAq, oasc, oWq, os_, oz), b = run_a8(M, N, K, "asym4", bias=True, use_ws=use_ws, want_acc=False)
+    _, ref, _ = oracle.gemm_a8(oAq, oasc, oWq, N, K, 4, False, 128, os_, oz, bits_np(b))
+    assert rel_fro(bits_np(C), ref, torch.float16) <= TOL
+
+
+@pytest.mark.parametrize("quant,dtype", [("asym4", torch.bfloat16), ("sym4", torch.float16),
+                                         ("tern2", torch.float16)])
+def test_a16_split_k_deterministic_and_matches_unsplit(quant, dtype):
+    # few tiles: with a workspace K is split over CTAs (slices added in a fixed order)
+    M, N, K = 128, 384, 4096
+    C1, A, _, qc, (oWq, os_, oz) = run_a16(M, N, K, quant, dtype, use_ws=True, seed=21)
+    C2, _, _, _, _ = run_a16(M, N, K, quant, dtype, use_ws=True, seed=21)
+    C0, _, _, _, _ = run_a16(M, N, K, quant, dtype, use_ws=False, seed=21)
+    assert torch.equal(C1, C2)
+    adt = oracle.F16 if dtype == torch.float16 else oracle.BF16
+    _, ref = oracle.gemm_a16(bits_np(A), adt, oWq, N, K, qc.bits, qc.symmetric, 128, os_, oz)
+    assert rel_fro(bits_np(C1), ref, dtype) <= TOL
+    assert rel_fro(bits_np(C0), ref, dtype) <= TOL
+
+
 @pytest.mark.parametrize("use_ws", [True, False])
 def test_a8_bias_and_plans(use_ws):
     M, N, K = 16, 520, 1024
@@ -291,4 +327,7 @@ def test_full_size_sampled(case):
                                       m_idx=mi, n_idx=ni, want_acc=True)
         assert np.array_equal(acc.cpu().numpy()[np.ix_(mi, ni)], oacc)
         assert rel_fro(bits_np(C)[np.ix_(mi, ni)], ref, torch.float16) <= TOL
+        # and without the group sums (the tcgen05 kernel when M > 16)
+        C2 = wq.w4a8_gemm(Aq, asc, Wq, s, z, N, K, qc, workspace=ws)
+        assert rel_fro(bits_np(C2)[np.ix_(mi, ni)], ref, torch.float16) <= TOL
     torch.cuda.synchronize()
