@@ -8,7 +8,7 @@
 // The kernel is HBM-bound and lasts a few microseconds, so it is built to put each SM's
 // whole share of the packed weights in flight at once and to spend few instructions per
 // byte once it arrives:
-//  * Rows are cut into 16-row tiles; CTA c (one per SM) owns tiles [cT/P, (c+1)T/P) and all
+//  * Rows are cut into 16-row tiles; CTA c (one per SM) owns a contiguous run of tiles and all
 //    of K, so no CTA needs another's result.  K is walked in chunks of KC units (a unit =
 //    64 packed bytes of a row: 128 k of INT4, 256 k of INT2).
 //  * One TMA box per tile and chunk brings 16 rows x KC units (a 3D box over unit pairs;
@@ -156,7 +156,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int c = blockIdx.x;
-    const int t0 = int((long long)c * p.T / p.P), t1 = int((long long)(c + 1) * p.T / p.P);
+    // tiles T = base * P + R: the first R CTAs take one more.  CTAs start in index order as the
+    // previous kernel's CTAs leave their SMs, so the late ones get the smaller share.
+    const int base = p.T / p.P, rem = p.T - base * p.P;
+    const int t0 = c * base + min(c, rem), t1 = t0 + base + (c < rem ? 1 : 0);
     const int ntc = t1 - t0;
     const int npass = (ntc + p.TPP - 1) / p.TPP;
     const int total_it = npass * p.nch;
