@@ -58,6 +58,7 @@ __host__ __device__ constexpr int ntl_of(int NT) { return NT == 1 ? 2 : 1; }  //
 struct GemvParams {
     const void *A;
     int M, N, K, G, gs, sym;
+    int upg;                 // units per scale group (INT4: group_size / 128)
     int KB, T, P;
     int nch, TPP, S;         // chunks per pass, tiles per pass, ring stages
     int w3d;                 // 1: one 3D box per tile and chunk; 0: one 2D box per unit pair
@@ -277,9 +278,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     };
 
     const int g = lane >> 2, t = lane & 3;
+    // MMA row g holds tile row gr (and g + 8 row gr + 8).  The lanes of a quarter-warp (g = 2q,
+    // 2q + 1) then read rows q and q + 4, whose 128-byte swizzle phases put their 64 bytes in
+    // opposite halves of the banks: one 128-bit load is 4 shared-memory wavefronts, not 8.
+    const int gr = (g >> 1) | ((g & 1) << 2);
     const int us = warp % KC, hf = warp / KC;
-    // this lane's 16 bytes of rows g and g+8 of a tile, unit slot us ([pair][16 rows][128 B], swizzled)
-    const uint32_t lin_lo = uint32_t(((us >> 1) * kTileRows + g) * kPairBytes + (us & 1) * 64 + 16 * t);
+    // this lane's 16 bytes of rows gr and gr+8 of a tile, unit slot us ([pair][16 rows][128 B], swizzled)
+    const uint32_t lin_lo = uint32_t(((us >> 1) * kTileRows + gr) * kPairBytes + (us & 1) * 64 + 16 * t);
     const uint32_t off_lo = swz128(lin_lo), off_hi = swz128(lin_lo + 8 * kPairBytes);
 
     int it = 0;
@@ -329,8 +334,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                         sA[j][1] = __shfl_sync(0xffffffffu, v, (2 * t + 1) * 4);
                     }
                 }
-                const int gi = (WB == 4) ? (kb * KU) / p.gs : 0;
-                const float2 *srow = stab + (size_t)gi * p.tab_rs + pass * p.TPP * kTileRows + g;
+                const int gi = (WB == 4) ? (p.upg == 1 ? kb : kb / p.upg) : 0;
+                const float2 *srow = stab + (size_t)gi * p.tab_rs + pass * p.TPP * kTileRows + gr;
 #pragma unroll
                 for (int jp = 0; jp < TM; jp += NTL) {
                     if (jp >= nmine) break;
@@ -380,7 +385,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                 } else if constexpr (AM == A_I8) {
                                     const int corr = v - int((e < 2) ? zl[l] : zh[l]) * sA[j][e & 1];
                                     if constexpr (ACC) {
-                                        const int n = r0 + (pass * p.TPP + i) * kTileRows + g + ((e & 2) ? 8 : 0);
+                                        const int n = r0 + (pass * p.TPP + i) * kTileRows + gr + ((e & 2) ? 8 : 0);
                                         const int m = j * 8 + 2 * t + (e & 1);
                                         if (n < p.N && m < p.M) p.acc_out[((long long)m * p.N + n) * p.G + kb] = corr;
                                     }
@@ -420,7 +425,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     const int m = j * 8 + 2 * t + (e & 1);
-                    const int r = g + ((e & 2) ? 8 : 0);
+                    const int r = gr + ((e & 2) ? 8 : 0);
                     if (m < p.M) {
                         float v;
                         if constexpr (AM == A_I8 && WB == 2) v = __int_as_float(tot[jj][j][e]);
@@ -606,6 +611,7 @@ wq_status gemv_small_m(int WB, int AM, const void *A, const float *a_scale, cons
     p.K = int(K);
     p.G = G;
     p.gs = WB == 4 ? c.group_size : int(K);
+    p.upg = WB == 4 ? c.group_size / kunit_of(WB) : 1;
     p.sym = WB == 4 ? c.symmetric : 1;
     p.KB = pl.KB;
     p.T = pl.T;
