@@ -166,19 +166,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int total_it = npass * p.nch;
     const int r0 = t0 * kTileRows;
 
-    if (threadIdx.x == 0) {
-        for (int s = 0; s < S; ++s) {
-            mbar_init(&full[s], 1);
-            cnt[s] = 0;
-        }
-        mbar_init(abar, 1);
-        mbar_init(cbar, kCW);
-        mbar_init(scbar, 1);
-        fence_barrier_init();
-    }
-    __syncthreads();
-    grid_dep_launch();  // the next kernel in the stream may start launching as SMs free up
-
     // ---- stage `it` of the ring: weights of the pass's tiles (and the expected bytes of all)
     auto issue_w = [&](int it) {
         const int s = it % S;
@@ -212,39 +199,54 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t sc_bytes = (WB == 4) ? uint32_t(nrows) * p.G * 2u : 0u;
     const uint32_t sc16 = sc_bytes & ~15u;
     const int pro = min(S, total_it);
-    if (lane == 0) {
-        if (warp == 0) {
-            tma_prefetch_desc(&tmap_w);
-            if (!p.a_whole) tma_prefetch_desc(&tmap_a);
-            if constexpr (WB == 4) {
-                mbar_arrive_expect_tx(scbar, sc16 * (p.sym ? 1u : 2u));
-                if (sc16) {
-                    bulk_load(sc_st, p.scales16 + (size_t)r0 * p.G, sc16, scbar);
-                    if (!p.sym) bulk_load(zc_st, p.zeros + (size_t)r0 * p.G, sc16, scbar);
-                }
+    // Thread 0 sets up the barriers and at once sends the first stage's weights, which are on
+    // the critical path, then the scales; the other stages follow after the block barrier.
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < S; ++s) {
+            mbar_init(&full[s], 1);
+            cnt[s] = 0;
+        }
+        mbar_init(abar, 1);
+        mbar_init(cbar, kCW);
+        mbar_init(scbar, 1);
+        fence_barrier_init();
+        tma_prefetch_desc(&tmap_w);
+        if (!p.a_whole) tma_prefetch_desc(&tmap_a);
+        issue_w(0);
+        if constexpr (WB == 4) {
+            mbar_arrive_expect_tx(scbar, sc16 * (p.sym ? 1u : 2u));
+            if (sc16) {
+                bulk_load(sc_st, p.scales16 + (size_t)r0 * p.G, sc16, scbar);
+                if (!p.sym) bulk_load(zc_st, p.zeros + (size_t)r0 * p.G, sc16, scbar);
             }
         }
-        for (int it = warp; it < pro; it += kCW) issue_w(it);
     }
+    __syncthreads();
+    grid_dep_launch();  // the next kernel in the stream may start launching as SMs free up
+    if (lane == 0)
+        for (int it = warp; it < pro; it += kCW)
+            if (it > 0) issue_w(it);
 
     // ---- scale / zero table of the CTA's rows, group-major: {scale, zero point as integer bits}
     if constexpr (WB == 4) {
         wait_bar(scbar, 0);  // on expiry the error is recorded; carry on to the next barrier
-        const int nent = ntc * kTileRows * p.G;
         const int nsm = int(sc16 >> 1);
-        for (int e = threadIdx.x; e < nent; e += kThreads) {
-            const int rl = e / p.G, gi = e - rl * p.G;
-            float sv = 0.f;
-            uint32_t zv = 8;
-            if (rl < nrows) {
-                const uint16_t sb = e < nsm ? sc_st[e] : p.scales16[(size_t)r0 * p.G + e];
-                sv = __half2float(__ushort_as_half(sb));
-                if (!p.sym) {
-                    const uint16_t zb = e < nsm ? zc_st[e] : p.zeros[(size_t)r0 * p.G + e];
-                    zv = uint32_t(__half2float(__ushort_as_half(zb))) & 15u;
+        const int nrow_t = ntc * kTileRows;  // a warp per row, its lanes over the groups
+        for (int rl = warp; rl < nrow_t; rl += kCW) {
+            for (int gi = lane; gi < p.G; gi += 32) {
+                const int e = rl * p.G + gi;
+                float sv = 0.f;
+                uint32_t zv = 8;
+                if (rl < nrows) {
+                    const uint16_t sb = e < nsm ? sc_st[e] : p.scales16[(size_t)r0 * p.G + e];
+                    sv = __half2float(__ushort_as_half(sb));
+                    if (!p.sym) {
+                        const uint16_t zb = e < nsm ? zc_st[e] : p.zeros[(size_t)r0 * p.G + e];
+                        zv = uint32_t(__half2float(__ushort_as_half(zb))) & 15u;
+                    }
                 }
+                stab[(size_t)gi * p.tab_rs + rl] = make_float2(sv, __uint_as_float(zv));
             }
-            stab[(size_t)gi * p.tab_rs + rl] = make_float2(sv, __uint_as_float(zv));
         }
     }
 
@@ -336,43 +338,41 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 const int gi = (WB == 4) ? (p.upg == 1 ? kb : kb / p.upg) : 0;
                 const float2 *srow = stab + (size_t)gi * p.tab_rs + pass * p.TPP * kTileRows + gr;
+                // a batch of B tiles (jp .. jp + B - 1); an odd last tile runs alone
+                auto batch = [&](int jp, auto nb) {
+                    constexpr int B = decltype(nb)::value;
+                    uint4 wa[B], wb[B];
+                    float s_lo[B], s_hi[B];
+                    uint32_t zl[B], zh[B];
 #pragma unroll
-                for (int jp = 0; jp < TM; jp += NTL) {
-                    if (jp >= nmine) break;
-                    uint4 wa[NTL], wb[NTL];
-                    float s_lo[NTL], s_hi[NTL];
-                    uint32_t zl[NTL], zh[NTL];
-#pragma unroll
-                    for (int l = 0; l < NTL; ++l) {
-                        const int j = min(jp + l, nmine - 1);  // a missing partner repeats a tile, unused
-                        const int i = hf + WPU * j;
+                    for (int l = 0; l < B; ++l) {
+                        const int i = hf + WPU * (jp + l);
                         const uint8_t *wt = st + i * p.wtile_bytes;
                         wa[l] = lds128(wt + off_lo);
                         wb[l] = lds128(wt + off_hi);
                         s_lo[l] = s_hi[l] = 0.f;
                         zl[l] = zh[l] = 8;
                         if constexpr (WB == 4) {
-                            const float2 v_lo = srow[i * kTileRows];
-                            const float2 v_hi = srow[i * kTileRows + 8];
-                            s_lo[l] = v_lo.x;
-                            s_hi[l] = v_hi.x;
-                            zl[l] = __float_as_uint(v_lo.y);
-                            zh[l] = __float_as_uint(v_hi.y);
+                            const uint2 v_lo = lds64(srow + i * kTileRows);
+                            const uint2 v_hi = lds64(srow + i * kTileRows + 8);
+                            s_lo[l] = __uint_as_float(v_lo.x);
+                            s_hi[l] = __uint_as_float(v_hi.x);
+                            zl[l] = v_lo.y;
+                            zh[l] = v_hi.y;
                         }
                     }
-                    acc_t<AM> ua[2][NTL][NT][4];
+                    acc_t<AM> ua[2][B][NT][4];
 #pragma unroll
                     for (int a = 0; a < 2; ++a)
 #pragma unroll
-                        for (int l = 0; l < NTL; ++l)
+                        for (int l = 0; l < B; ++l)
 #pragma unroll
                             for (int j = 0; j < NT; ++j)
 #pragma unroll
                                 for (int e = 0; e < 4; ++e) ua[a][l][j][e] = acc_t<AM>(0);
-                    unit_mma<WB, AM, NT, NTL>(wa, wb, bf, zl, zh, ua);
+                    unit_mma<WB, AM, NT, B>(wa, wb, bf, zl, zh, ua);
 #pragma unroll
-                    for (int l = 0; l < NTL; ++l) {
-                        if (jp + l >= nmine) break;
+                    for (int l = 0; l < B; ++l) {
                         const int i = hf + WPU * (jp + l);
 #pragma unroll
                         for (int j = 0; j < NT; ++j)
@@ -397,6 +397,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                                 }
                             }
                     }
+                };
+#pragma unroll
+                for (int jp = 0; jp < TM; jp += NTL) {
+                    if (jp >= nmine) break;
+                    if (NTL == 1 || jp + NTL <= nmine) batch(jp, std::integral_constant<int, NTL>{});
+                    else batch(jp, std::integral_constant<int, 1>{});
                 }
             }
             // stage consumed: the last of the 16 warps refills it with chunk it + S
