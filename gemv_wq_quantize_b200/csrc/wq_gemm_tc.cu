@@ -94,7 +94,7 @@ __device__ __forceinline__ bool tc_wait(uint64_t *bar, uint32_t parity, volatile
     const uint64_t t0 = globaltimer();
     for (;;) {
         for (int i = 0; i < 4; ++i)
-            if (mbar_try_wait(bar, parity)) return true;
+            if (mbar_try_wait_short(bar, parity)) return true;
         if (*abort) return false;
         if (globaltimer() - t0 > 2000000000ull) {
             atomicCAS(&g_tc_error, kErrNone, kErrWaitTimeout);

@@ -93,7 +93,7 @@ __device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity)
     const uint64_t t0 = globaltimer();
     for (;;) {
         for (int i = 0; i < 4; ++i)
-            if (mbar_try_wait(bar, parity)) return true;
+            if (mbar_try_wait_short(bar, parity)) return true;
         if (globaltimer() - t0 > 2000000000ull) {
             atomicCAS(&g_gemv_error, kErrNone, kErrWaitTimeout);
             return false;
