@@ -64,6 +64,7 @@ constexpr uint32_t kDcol = kNA * 64;
 
 struct TcParams {
     int M, N, K, G, gs, sym;
+    int upg;               // blocks of 128 k per scale group (INT4: group_size / 128)
     const float *a_scale;  // INT8 activations: per-token scale
     const float *scale32;  // INT2 weights: per-tensor scale
     int nkb;     // blocks of 128 k
@@ -355,19 +356,21 @@ __global__ void __launch_bounds__(kThreads, 1)
             {
                 const uint16_t *sc = scst + size_t(tl & 1) * 2 * stab_elems;
                 const int n16 = int(((uint32_t(nrows) * p.G * 2u) & ~15u) >> 1);
-                for (int e = threadIdx.x - 64; e < kBW * p.G; e += kDeqWarps * 32) {
-                    const int rl = e / p.G, gi = e - rl * p.G;
-                    uint32_t v = 0;
-                    if (rl < nrows) {
-                        const uint16_t sb = e < n16 ? sc[e] : p.scales16[(size_t)n0 * p.G + e];
-                        uint32_t z = 8;
-                        if (!p.sym) {
-                            const uint16_t zb = e < n16 ? sc[stab_elems + e] : p.zeros[(size_t)n0 * p.G + e];
-                            z = uint32_t(__half2float(__ushort_as_half(zb))) & 15u;
+                for (int rl = warp - 2; rl < kBW; rl += kDeqWarps) {  // a warp per row, lanes over groups
+                    for (int gi = lane; gi < p.G; gi += 32) {
+                        const int e = rl * p.G + gi;
+                        uint32_t v = 0;
+                        if (rl < nrows) {
+                            const uint16_t sb = e < n16 ? sc[e] : p.scales16[(size_t)n0 * p.G + e];
+                            uint32_t z = 8;
+                            if (!p.sym) {
+                                const uint16_t zb = e < n16 ? sc[stab_elems + e] : p.zeros[(size_t)n0 * p.G + e];
+                                z = uint32_t(__half2float(__ushort_as_half(zb))) & 15u;
+                            }
+                            v = uint32_t(sb) | (z << 16);
                         }
-                        v = uint32_t(sb) | (z << 16);
+                        tab[(size_t)gi * p.tab_rs + rl] = v;
                     }
-                    tab[(size_t)gi * p.tab_rs + rl] = v;
                 }
             }
             if (!deq_sync()) break;
@@ -385,7 +388,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const uint32_t sw = uint32_t((r >> 1) & 3);
                     const uint4 w0 = lds128(wrow + ((uint32_t(2 * kh) ^ sw) << 4));
                     const uint4 w1 = lds128(wrow + ((uint32_t(2 * kh + 1) ^ sw) << 4));
-                    const uint32_t z = tab[(size_t)((kb * kKB) / p.gs) * p.tab_rs + r] >> 16;
+                    const uint32_t z = tab[(size_t)(p.upg == 1 ? kb : kb / p.upg) * p.tab_rs + r] >> 16;
                     tc::fence_after_sync();
                     if constexpr (I8) {
                         const uint32_t zc = (0x80u - z) * 0x01010101u;
@@ -471,7 +474,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint32_t db = step % kND, s = step % kNA;
                 float sv = 1.f;  // INT2: the per-tensor scale is applied at the end
                 if constexpr (WB == 4)
-                    sv = __half2float(__ushort_as_half(uint16_t(tab[(size_t)((kb * kKB) / p.gs) * p.tab_rs + r])));
+                    sv = __half2float(__ushort_as_half(uint16_t(tab[(size_t)(p.upg == 1 ? kb : kb / p.upg) * p.tab_rs + r])));
                 if (!tc_wait(&rel[s], (step / kNA) & 1, abort)) { ok = false; break; }
                 tc::fence_after_sync();
 #pragma unroll
@@ -691,6 +694,7 @@ wq_status tc_gemm(int WB, int AM, const void *A, const float *a_scale, const uin
     p.K = int(K);
     p.G = G;
     p.gs = WB == 4 ? c.group_size : int(K);
+    p.upg = WB == 4 ? c.group_size / kKB : 1;
     p.sym = WB == 4 ? c.symmetric : 1;
     p.a_scale = a_scale;
     p.scale32 = static_cast<const float *>(scales);
