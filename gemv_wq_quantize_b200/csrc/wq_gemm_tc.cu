@@ -69,7 +69,7 @@ struct TcParams {
     const float *scale32;  // INT2 weights: per-tensor scale
     int nkb;     // blocks of 128 k
     int ks;      // K slices per tile (split-K when tiles are fewer than SMs)
-    float *ws_part;     // ks > 1: fp32 partial totals [tile][slice][128 rows][128 tokens]
+    float *ws_part;     // ks > 1: fp32 partial totals [tile][slice][128 tokens][128 rows]
     unsigned *ws_cnt;   // ks > 1: per-tile arrival counters (left at zero)
     int TT, NT;  // token tiles, tiles
     int S;       // ring stages
@@ -503,10 +503,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (p.ks > 1) {
                 // split K: publish this slice's totals; the last slice of the tile to arrive adds
                 // all slices in slice order (deterministic) and writes C
-                float *part = p.ws_part + ((size_t(tile) * p.ks + sp) * kBW + r) * kBT + th * 64;
+                // [tile][slice][token][row]: a warp's 32 rows of one token are 128 contiguous bytes
+                float *part = p.ws_part + (size_t(tile) * p.ks + sp) * (kBW * kBT) + size_t(th * 64) * kBW + r;
 #pragma unroll
-                for (int j = 0; j < 64; j += 4)
-                    *reinterpret_cast<float4 *>(part + j) = make_float4(tot[j], tot[j + 1], tot[j + 2], tot[j + 3]);
+                for (int j = 0; j < 64; ++j) __stcg(part + size_t(j) * kBW, tot[j]);
                 __threadfence();
                 if (!fold_sync()) break;
                 if (threadIdx.x == 64 + kDeqWarps * 32) {
@@ -520,15 +520,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int j = 0; j < 64; ++j) tot[j] = 0.f;
                 for (int q2 = 0; q2 < p.ks; ++q2) {
-                    const float *pq = p.ws_part + ((size_t(tile) * p.ks + q2) * kBW + r) * kBT + th * 64;
+                    const float *pq = p.ws_part + (size_t(tile) * p.ks + q2) * (kBW * kBT) + size_t(th * 64) * kBW + r;
 #pragma unroll
-                    for (int j = 0; j < 64; j += 4) {
-                        const float4 v4 = __ldcg(reinterpret_cast<const float4 *>(pq + j));
-                        tot[j] += v4.x;
-                        tot[j + 1] += v4.y;
-                        tot[j + 2] += v4.z;
-                        tot[j + 3] += v4.w;
-                    }
+                    for (int j = 0; j < 64; ++j) tot[j] += __ldcg(pq + size_t(j) * kBW);
                 }
             }
 
