@@ -192,8 +192,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint64_t *full = bars, *rel = bars + kNA;
     uint64_t *afull = bars + 2 * kNA, *dfree = afull + kNA;
     uint64_t *scbar = dfree + kND, *tready = scbar + 2, *tdone = tready + 2, *fin = tdone + 2, *mbar = fin + 1;
-    uint64_t *fbar = mbar + 1;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(fbar + 1);
+    uint64_t *fbar = mbar + 1, *pbar = fbar + 1;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(pbar + 1);
     volatile int *abort = reinterpret_cast<volatile int *>(tmem_slot + 1);
     volatile int *last_flag = abort + 1;
 
@@ -216,6 +216,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_init(fin, 1);
         mbar_init(mbar, kDeqWarps);
         mbar_init(fbar, kFoldWarps);
+        mbar_init(pbar, 1);
         *abort = 0;
         fence_barrier_init();
     }
@@ -451,7 +452,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         grid_dep_wait();  // C and bias belong to this kernel only once the previous one is done
         uint32_t step = 0;
         int tl = 0;
-        uint32_t fphase = 0;
+        uint32_t fphase = 0, pphase = 0;
         auto fold_sync = [&]() -> bool {  // bounded barrier of the folding warps (one arrival per warp)
             __syncwarp();
             if (lane == 0) mbar_arrive(fbar);
@@ -507,6 +508,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 float *part = p.ws_part + (size_t(tile) * p.ks + sp) * (kBW * kBT) + size_t(th * 64) * kBW + r;
 #pragma unroll
                 for (int j = 0; j < 64; ++j) __stcg(part + size_t(j) * kBW, tot[j]);
+                fence_proxy_async_global();  // the last arriver reads the partials by bulk copy
                 __threadfence();
                 if (!fold_sync()) break;
                 if (threadIdx.x == 64 + kDeqWarps * 32) {
@@ -517,12 +519,42 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (!fold_sync()) break;
                 if (!*last_flag) continue;
                 __threadfence();
+                fence_proxy_async_global();
 #pragma unroll
                 for (int j = 0; j < 64; ++j) tot[j] = 0.f;
-                for (int q2 = 0; q2 < p.ks; ++q2) {
-                    const float *pq = p.ws_part + (size_t(tile) * p.ks + q2) * (kBW * kBT) + size_t(th * 64) * kBW + r;
+                constexpr uint32_t kPart = kBW * kBT * 4;  // one slice's partials: 64 KB
+                if (gridDim.x >= p.NT * p.ks) {
+                    // One task per CTA, so the ring is idle now (the tile's MMAs have completed):
+                    // bulk-copy the slices into it, as many at a time as fit, and add them in
+                    // slice order from shared memory.
+                    const int per = int((kNA * kStageBytes) / kPart);
+                    const float *sp0 = reinterpret_cast<const float *>(ring) + size_t(th * 64) * kBW + r;
+                    for (int q0 = 0; q0 < p.ks && ok; q0 += per) {
+                        const int nq = min(per, p.ks - q0);
+                        if (threadIdx.x == 64 + kDeqWarps * 32) {
+                            mbar_arrive_expect_tx(pbar, uint32_t(nq) * kPart);
+                            for (int i = 0; i < nq; ++i)
+                                bulk_load(ring + size_t(i) * kPart,
+                                          p.ws_part + (size_t(tile) * p.ks + q0 + i) * (kBW * kBT), kPart, pbar);
+                        }
+                        if (!tc_wait(pbar, pphase & 1, abort)) ok = false;
+                        ++pphase;
+                        for (int i = 0; i < nq && ok; ++i) {
+                            const float *src = sp0 + size_t(i) * (kBW * kBT);
 #pragma unroll
-                    for (int j = 0; j < 64; ++j) tot[j] += __ldcg(pq + size_t(j) * kBW);
+                            for (int j = 0; j < 64; ++j) tot[j] += src[j * kBW];
+                        }
+                        fence_proxy_async();  // these reads come before the next round's copies
+                        if (!fold_sync()) ok = false;
+                    }
+                    if (!ok) break;
+                } else {
+                    for (int q2 = 0; q2 < p.ks; ++q2) {
+                        const float *pq =
+                            p.ws_part + (size_t(tile) * p.ks + q2) * (kBW * kBT) + size_t(th * 64) * kBW + r;
+#pragma unroll
+                        for (int j = 0; j < 64; ++j) tot[j] += __ldcg(pq + size_t(j) * kBW);
+                    }
                 }
             }
 
