@@ -74,7 +74,9 @@ struct TcParams {
     int TT, NT;  // token tiles, tiles
     int S;       // ring stages
     int scst_off, tab_off, bar_off;
-    int tab_rs;  // table row stride (entries; odd)
+    int tab_rs;    // table row stride (entries; odd)
+    int stage_sc;  // 1: scales / zeros are bulk-copied to shared memory first; 0: read from global
+    int ntab;      // scale tables in shared memory (2: the next tile's is built while one is used)
     const uint16_t *scales16;
     const uint16_t *zeros;
     const void *bias;
@@ -237,6 +239,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             tma_prefetch_desc(&tmap_w);
             auto issue_scales = [&](int n0, int tl) {  // the tile's scale / zero rows: contiguous in [N, G]
                 if constexpr (WB == 4) {
+                    if (!p.stage_sc) return;
                     const int nrows = min(kBW, p.N - n0);
                     const uint32_t bytes16 = (uint32_t(nrows) * p.G * 2u) & ~15u;
                     uint16_t *sc = scst + size_t(tl & 1) * 2 * stab_elems;
@@ -348,11 +351,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int kb0 = sp * p.nkb / p.ks, kb1 = (sp + 1) * p.nkb / p.ks;
             const int n0 = (tile / p.TT) * kBW;
             const int nrows = min(kBW, p.N - n0);
-            uint32_t *tab = tabs + size_t(tl & 1) * tab_elems;
+            const int tb = tl % p.ntab;  // this tile's table buffer
+            uint32_t *tab = tabs + size_t(tb) * tab_elems;
             // ---- scale / zero table of the tile (INT4): [g][row] = fp16 scale bits | z << 16
             if constexpr (WB == 4) {
-            if (!tc_wait(&scbar[tl & 1], (tl >> 1) & 1, abort)) break;
-            if (tl >= 2 && !tc_wait(&tdone[tl & 1], ((tl - 2) >> 1) & 1, abort)) break;  // tile tl-2 folded
+            if (p.stage_sc && !tc_wait(&scbar[tl & 1], (tl >> 1) & 1, abort)) break;
+            // the folding warps are done with tile tl - ntab, the buffer's previous user
+            if (tl >= p.ntab && !tc_wait(&tdone[tb], ((tl - p.ntab) / p.ntab) & 1, abort)) break;
             if (!deq_sync()) break;
             {
                 const uint16_t *sc = scst + size_t(tl & 1) * 2 * stab_elems;
@@ -362,10 +367,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const int e = rl * p.G + gi;
                         uint32_t v = 0;
                         if (rl < nrows) {
-                            const uint16_t sb = e < n16 ? sc[e] : p.scales16[(size_t)n0 * p.G + e];
+                            const bool st = p.stage_sc && e < n16;
+                            const uint16_t sb = st ? sc[e] : p.scales16[(size_t)n0 * p.G + e];
                             uint32_t z = 8;
                             if (!p.sym) {
-                                const uint16_t zb = e < n16 ? sc[stab_elems + e] : p.zeros[(size_t)n0 * p.G + e];
+                                const uint16_t zb = st ? sc[stab_elems + e] : p.zeros[(size_t)n0 * p.G + e];
                                 z = uint32_t(__half2float(__ushort_as_half(zb))) & 15u;
                             }
                             v = uint32_t(sb) | (z << 16);
@@ -375,7 +381,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
             if (!deq_sync()) break;
-            if (threadIdx.x == 64) mbar_arrive(&tready[tl & 1]);
+            if (threadIdx.x == 64) mbar_arrive(&tready[tb]);
             }
 
             for (int kb = kb0; kb < kb1; ++kb, ++step) {
@@ -464,9 +470,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int tile = t / p.ks, sp = t - tile * p.ks;
             const int kb0 = sp * p.nkb / p.ks, kb1 = (sp + 1) * p.nkb / p.ks;
             const int n0 = (tile / p.TT) * kBW, m0 = (tile % p.TT) * kBT;
-            const uint32_t *tab = tabs + size_t(tl & 1) * tab_elems;
+            const int tb = tl % p.ntab;
+            const uint32_t *tab = tabs + size_t(tb) * tab_elems;
             if constexpr (WB == 4)
-                if (!tc_wait(&tready[tl & 1], (tl >> 1) & 1, abort)) break;
+                if (!tc_wait(&tready[tb], (tl / p.ntab) & 1, abort)) break;
             float tot[64];
 #pragma unroll
             for (int j = 0; j < 64; ++j) tot[j] = 0.f;
@@ -499,7 +506,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!ok) break;
             __syncwarp();
             if constexpr (WB == 4)
-                if (lane == 0) mbar_arrive(&tdone[tl & 1]);
+                if (lane == 0) mbar_arrive(&tdone[tb]);
 
             if (p.ks > 1) {
                 // split K: publish this slice's totals; the last slice of the tile to arrive adds
@@ -591,33 +598,40 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 struct TcPlan {
-    int S = 0, scst_off = 0, tab_off = 0, bar_off = 0, tab_rs = 1;
+    int S = 0, scst_off = 0, tab_off = 0, bar_off = 0, tab_rs = 1, stage_sc = 1, ntab = 2;
     size_t smem = 0;
     bool ok = false;
 };
 
 // G: groups of the INT4 scale table (0 for INT2: one per-tensor scale, no table).
+// Preferred: scales staged by bulk copy and two tables (the next tile's built while one is
+// in use).  Long K (many groups) drops the staging, then the second table, to keep the ring.
 TcPlan make_plan(int nkb, int G, int stage, const DeviceInfo &dev)
 {
     TcPlan pl;
-    const size_t scst = (size_t(2) * 2 * kBW * G * 2 + 15) & ~size_t(15);
     pl.tab_rs = kBW + 1;
-    const size_t tab = (size_t(2) * G * pl.tab_rs * 4 + 15) & ~size_t(15);
     const size_t bars = 8 * (3 * kNA + 2 * kND + 12) + 16;
     const size_t budget = size_t(dev.max_smem_optin) - 1024;
-    // the ring has one stage per TMEM A-buffer
-    if (nkb < kNA || budget <= scst + tab + bars || (budget - scst - tab - bars) / size_t(stage) < size_t(kNA))
+    if (nkb < kNA) return pl;  // the ring has one stage per TMEM A-buffer
+    const int forms[3][2] = {{1, 2}, {0, 2}, {0, 1}};
+    for (const auto &f : forms) {
+        const size_t scst = f[0] ? (size_t(2) * 2 * kBW * G * 2 + 15) & ~size_t(15) : 0;
+        const size_t tab = (size_t(f[1]) * G * pl.tab_rs * 4 + 15) & ~size_t(15);
+        if (budget <= scst + tab + bars || (budget - scst - tab - bars) / size_t(stage) < size_t(kNA)) continue;
+        pl.stage_sc = f[0];
+        pl.ntab = f[1];
+        pl.S = kNA;
+        size_t off = size_t(pl.S) * stage;
+        pl.scst_off = int(off);
+        off += scst;
+        pl.tab_off = int(off);
+        off += tab;
+        pl.bar_off = int((off + 7) & ~size_t(7));
+        off = pl.bar_off + bars;
+        pl.smem = ((off + 15) & ~size_t(15)) + 1024;
+        pl.ok = pl.smem <= size_t(dev.max_smem_optin);
         return pl;
-    pl.S = kNA;
-    size_t off = size_t(pl.S) * stage;
-    pl.scst_off = int(off);
-    off += scst;
-    pl.tab_off = int(off);
-    off += tab;
-    pl.bar_off = int((off + 7) & ~size_t(7));
-    off = pl.bar_off + size_t(8) * (3 * kNA + 2 * kND + 12) + 16;
-    pl.smem = ((off + 15) & ~size_t(15)) + 1024;
-    pl.ok = pl.smem <= size_t(dev.max_smem_optin);
+    }
     return pl;
 }
 
@@ -738,6 +752,8 @@ wq_status tc_gemm(int WB, int AM, const void *A, const float *a_scale, const uin
     p.tab_off = pl.tab_off;
     p.bar_off = pl.bar_off;
     p.tab_rs = pl.tab_rs;
+    p.stage_sc = pl.stage_sc;
+    p.ntab = pl.ntab;
     p.scales16 = static_cast<const uint16_t *>(scales);
     p.zeros = static_cast<const uint16_t *>(zeros);
     p.bias = bias;

@@ -280,6 +280,26 @@ def test_a16_split_k_deterministic_and_matches_unsplit(quant, dtype):
     assert rel_fro(bits_np(C0), ref, dtype) <= TOL
 
 
+@pytest.mark.parametrize("quant,dtype,M,N,K", [("asym4", torch.float16, 160, 384, 11008),
+                                                 ("sym4", torch.bfloat16, 640, 4096, 11008)])
+def test_a16_long_k_tensor_core(quant, dtype, M, N, K):
+    # 86 scale groups: the tcgen05 plan keeps one scale table, built from global memory; the
+    # first shape splits K 21 ways, the second gives some CTAs two tiles through that table
+    C, A, _, qc, (oWq, os_, oz) = run_a16(M, N, K, quant, dtype, seed=31)
+    ni = sample_idx(N, 96, 3)
+    adt = oracle.F16 if dtype == torch.float16 else oracle.BF16
+    _, ref = oracle.gemm_a16(bits_np(A), adt, oWq, N, K, qc.bits, qc.symmetric, 128, os_, oz, n_idx=ni)
+    assert rel_fro(bits_np(C)[:, ni], ref, dtype) <= TOL
+
+
+def test_a8_long_k_tensor_core():
+    # 86 scale groups with INT8 activations: two scale tables, built from global memory
+    M, N, K = 200, 384, 11008
+    C, _, qc, (oAq, oasc, oWq, os_, oz), _ = run_a8(M, N, K, "asym4", seed=9, want_acc=False)
+    _, ref, _ = oracle.gemm_a8(oAq, oasc, oWq, N, K, 4, False, 128, os_, oz)
+    assert rel_fro(bits_np(C), ref, torch.float16) <= TOL
+
+
 @pytest.mark.parametrize("use_ws", [True, False])
 def test_a8_bias_and_plans(use_ws):
     M, N, K = 16, 520, 1024
