@@ -131,8 +131,8 @@ SMALL = [(1, 256, 512), (3, 200, 384), (8, 128, 128), (13, 1000, 1024), (16, 384
          (64, 256, 384), (100, 136, 256)]
 
 
-def run_a16(M, N, K, quant, dtype, use_ws=True, bias=False, seed=0, outliers=0.0):
-    qc = qc_of(quant)
+def run_a16(M, N, K, quant, dtype, use_ws=True, bias=False, seed=0, outliers=0.0, gs=128):
+    qc = qc_of(quant, gs)
     W = wq_synth.weights(N, K, seed=seed)
     A = wq_synth.activations(M, K, seed=seed + 1, dtype=dtype, outlier_frac=outliers)
     b = wq_synth.activations(1, N, seed=seed + 2, dtype=dtype)[0] if bias else None
@@ -154,6 +154,27 @@ def test_a16_small_all_outputs(quant, dtype, M, N, K):
     _, ref = oracle.gemm_a16(bits_np(A), adt, oWq, N, K, qc.bits, qc.symmetric, qc.group_size, os_, oz)
     err = rel_fro(bits_np(C), ref, dtype)
     assert err <= TOL, err
+
+
+@pytest.mark.parametrize("gs", [256, 1024, 2048])
+@pytest.mark.parametrize("quant", ["sym4", "asym4"])
+@pytest.mark.parametrize("M", [1, 13, 200])
+def test_a16_group_sizes(gs, quant, M):
+    # groups of several 128-k units (2048 = K: one scale per row), on the few-token kernel
+    # (M = 1, 13) and the tcgen05 kernel (M = 200)
+    N, K = 384, 2048
+    C, A, _, qc, (oWq, os_, oz) = run_a16(M, N, K, quant, torch.float16, seed=M + gs, gs=gs)
+    _, ref = oracle.gemm_a16(bits_np(A), oracle.F16, oWq, N, K, 4, qc.symmetric, gs, os_, oz)
+    assert rel_fro(bits_np(C), ref, torch.float16) <= TOL
+
+
+@pytest.mark.parametrize("gs", [256, 2048])
+@pytest.mark.parametrize("M", [4, 160])
+def test_a8_group_sizes(gs, M):
+    N, K = 384, 2048
+    C, _, qc, (oAq, oasc, oWq, os_, oz), _ = run_a8(M, N, K, "asym4", seed=gs + M, want_acc=False, gs=gs)
+    _, ref, _ = oracle.gemm_a8(oAq, oasc, oWq, N, K, 4, False, gs, os_, oz)
+    assert rel_fro(bits_np(C), ref, torch.float16) <= TOL
 
 
 @pytest.mark.parametrize("use_ws", [True, False])
@@ -181,6 +202,17 @@ def test_a16_bias_and_ragged_tail():
         C, A, b, qc, (oWq, os_, oz) = run_a16(M, N, KK, quant, torch.float16, bias=True)
         _, ref = oracle.gemm_a16(bits_np(A), oracle.F16, oWq, N, KK, qc.bits, qc.symmetric, 128, os_, oz, bits_np(b))
         assert rel_fro(bits_np(C), ref, torch.float16) <= TOL
+
+
+@pytest.mark.parametrize("dtype", [torch.float16, torch.bfloat16])
+@pytest.mark.parametrize("use_ws", [True, False])
+def test_a16_bias_and_ragged_tail_tensor_core(dtype, use_ws):
+    # more than 16 tokens, ragged M and N, with bias; with a workspace K is split
+    M, N, K = 200, 333, 1152
+    C, A, b, qc, (oWq, os_, oz) = run_a16(M, N, K, "asym4", dtype, use_ws=use_ws, bias=True, seed=3)
+    adt = oracle.F16 if dtype == torch.float16 else oracle.BF16
+    _, ref = oracle.gemm_a16(bits_np(A), adt, oWq, N, K, 4, False, 128, os_, oz, bits_np(b))
+    assert rel_fro(bits_np(C), ref, dtype) <= TOL
 
 
 def test_a16_deterministic():
@@ -215,8 +247,8 @@ def test_a16_identity_closed_form():
 
 
 # ------------------------------------------------------------------ W4A8 / W2A8
-def run_a8(M, N, K, quant, seed=0, bias=False, use_ws=True, want_acc=True):
-    qc = qc_of(quant)
+def run_a8(M, N, K, quant, seed=0, bias=False, use_ws=True, want_acc=True, gs=128):
+    qc = qc_of(quant, gs)
     W = wq_synth.weights(N, K, seed=seed)
     A = wq_synth.activations(M, K, seed=seed + 1, outlier_frac=0.01)
     b = wq_synth.activations(1, N, seed=seed + 2)[0] if bias else None
