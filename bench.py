@@ -196,72 +196,106 @@ class Prepared:
         self.ws = wq.make_workspace(wq.workspace_size(c.M, c.N, c.K, self.qc), device)
         self.i = 0
 
-    def launch(self, e2e: bool = False):
+    def launch(self, e2e: bool = False, slot: int = 0):
         import gemv_wq_quantize_b200 as wq
         Wq, s, z = self.weights[self.i % len(self.weights)]
         self.i += 1
         c = self.c
+        A, C = (self.A_slots[slot], self.C_slots[slot]) if e2e else (self.A, self.C)
         if c.mode == "a16":
-            wq.w4a16_gemm(self.A, Wq, s, z, c.N, c.K, self.qc, out=self.C, workspace=self.ws)
+            wq.w4a16_gemm(A, Wq, s, z, c.N, c.K, self.qc, out=C, workspace=self.ws)
         else:
             if e2e:  # the INT8 path starts from the fp16 activations: quantize them too
-                wq.act_quant_int8(self.A, out_q=self.Aq, out_scale=self.a_scale)
-            wq.w4a8_gemm(self.Aq, self.a_scale, Wq, s, z, c.N, c.K, self.qc, out=self.C, workspace=self.ws)
+                wq.act_quant_int8(A, out_q=self.Aq, out_scale=self.a_scale)
+            wq.w4a8_gemm(self.Aq, self.a_scale, Wq, s, z, c.N, c.K, self.qc, out=C, workspace=self.ws)
 
 
 class StepIO:
-    """Every case's activations in one pinned host buffer and one device buffer (outputs
-    likewise), so that an end-to-end step brings its inputs in with one host-to-device copy
-    and reads its results back with one device-to-host copy.  Each case's tensors become views
-    at 256-byte aligned offsets of the device buffers."""
+    """End-to-end input / output staging.  Every case's activations sit in one pinned host
+    buffer, and each step copies them in with one host-to-device copy. Every case's outputs
+    are read back with one device-to-host copy per step.  The device buffers come in two
+    slots (each case's A and C are 256-byte aligned views of them), and the copies run on
+    their own stream.  Step s+1's inputs can then move while step s computes, and step s's
+    results while step s+1 computes, as in a serving loop; a step's kernels wait for its own
+    inputs only."""
+
+    SLOTS = 2
 
     def __init__(self, preps, device):
-        def pack(tensors, hosts):
+        def layout(tensors):
             offs, total = [], 0
             for t in tensors:
                 offs.append(total)
                 total += (t.numel() * t.element_size() + 255) // 256 * 256
-            dev = torch.zeros(total, dtype=torch.uint8, device=device)
-            host = torch.zeros(total, dtype=torch.uint8).pin_memory()
-            views = []
-            for t, h, off in zip(tensors, hosts, offs):
-                n = t.numel() * t.element_size()
-                dv = dev[off:off + n].view(t.dtype).view(t.shape)
-                hv = host[off:off + n].view(t.dtype).view(t.shape)
-                dv.copy_(t)
-                hv.copy_(h)
-                views.append((dv, hv))
-            return dev, host, views
-        self.a_dev, self.a_host, av = pack([p.A for p in preps], [p.A_host for p in preps])
-        self.c_dev, self.c_host, cv = pack([p.C for p in preps], [p.C_host for p in preps])
-        for p, (da, ha), (dc, hc) in zip(preps, av, cv):
-            p.A, p.A_host, p.C, p.C_host = da, ha, dc, hc
-        self.h2d_bytes = self.a_dev.numel()
-        self.d2h_bytes = self.c_dev.numel()
+            return offs, total
 
-    def h2d(self):
-        self.a_dev.copy_(self.a_host, non_blocking=True)
+        def views(buf, tensors, offs):
+            return [buf[o:o + t.numel() * t.element_size()].view(t.dtype).view(t.shape) for t, o in zip(tensors, offs)]
 
-    def d2h(self):
-        self.c_host.copy_(self.c_dev, non_blocking=True)
+        a_offs, a_total = layout([p.A for p in preps])
+        c_offs, c_total = layout([p.C for p in preps])
+        self.a_host = torch.zeros(a_total, dtype=torch.uint8).pin_memory()
+        for hv, p in zip(views(self.a_host, [p.A for p in preps], a_offs), preps):
+            hv.copy_(p.A_host)
+        self.a_dev = [torch.zeros(a_total, dtype=torch.uint8, device=device) for _ in range(self.SLOTS)]
+        self.c_dev = [torch.zeros(c_total, dtype=torch.uint8, device=device) for _ in range(self.SLOTS)]
+        self.c_host = [torch.zeros(c_total, dtype=torch.uint8).pin_memory() for _ in range(self.SLOTS)]
+        for sl in range(self.SLOTS):
+            for p, av, cv in zip(preps, views(self.a_dev[sl], [p.A for p in preps], a_offs),
+                                 views(self.c_dev[sl], [p.C for p in preps], c_offs)):
+                if sl == 0:
+                    p.A_slots, p.C_slots = [], []
+                p.A_slots.append(av)
+                p.C_slots.append(cv)
+        self.h2d_bytes = a_total
+        self.d2h_bytes = c_total
+        self.stream = torch.cuda.Stream(device=device)
+        self.ev = {k: [torch.cuda.Event() for _ in range(self.SLOTS)] for k in ("in", "done", "out")}
+        self.fork = torch.cuda.Event()
 
 
-def run_step(preps, e2e: bool, io=None):
-    """One step: every case once; end to end, the step's inputs are copied in first and its
-    results copied out last."""
-    if e2e:
-        io.h2d()
-    for p in preps:
-        p.launch(e2e)
-    if e2e:
-        io.d2h()
+def run_steps(preps, nsteps: int, e2e: bool, io=None):
+    """`nsteps` steps, each running every case once.  End to end, each step's inputs are
+    copied in from pinned host memory before its kernels and its results copied out after
+    them, pipelined across steps on the copy stream (see StepIO); the launching stream waits
+    for the last copy before it goes on."""
+    if not e2e:
+        for _ in range(nsteps):
+            for p in preps:
+                p.launch(False)
+        return
+    main, cs, ev, S = torch.cuda.current_stream(), io.stream, io.ev, StepIO.SLOTS
+    io.fork.record(main)
+    cs.wait_event(io.fork)
+    with torch.cuda.stream(cs):
+        io.a_dev[0].copy_(io.a_host, non_blocking=True)
+    ev["in"][0].record(cs)
+    for st in range(nsteps):
+        sl = st % S
+        main.wait_event(ev["in"][sl])
+        if st >= S:
+            main.wait_event(ev["out"][sl])  # step st - 2 has read this slot's outputs
+        for p in preps:
+            p.launch(True, sl)
+        ev["done"][sl].record(main)
+        if st + 1 < nsteps:  # the next step's inputs, once step st - 1 no longer reads that slot
+            nx = (st + 1) % S
+            if st >= 1:
+                cs.wait_event(ev["done"][nx])
+            with torch.cuda.stream(cs):
+                io.a_dev[nx].copy_(io.a_host, non_blocking=True)
+            ev["in"][nx].record(cs)
+        cs.wait_event(ev["done"][sl])
+        with torch.cuda.stream(cs):
+            io.c_host[sl].copy_(io.c_dev[sl], non_blocking=True)
+        ev["out"][sl].record(cs)
+    main.wait_event(ev["out"][(nsteps - 1) % S])
 
 
 def capture(preps, nsteps: int, e2e: bool, io=None):
     g = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g):
-        for _ in range(nsteps):
-            run_step(preps, e2e, io)
+        run_steps(preps, nsteps, e2e, io)
     return g
 
 
@@ -279,8 +313,7 @@ def timed_replays(preps, steps: int, warmup: int, e2e: bool, dist_on: bool, samp
         if n == chunk:
             g_chunk.replay()
         else:
-            for _ in range(n):
-                run_step(preps, e2e, io)
+            run_steps(preps, n, e2e, io)
         done += n
     torch.cuda.synchronize()
     if dist_on:
@@ -361,8 +394,8 @@ def run_ours(args, rank, world, local_rank, dist_on):
     wl = wq_synth.WORKLOADS[args.workload]
     preps = [Prepared(c, device, seed_base=0) for c in wl.cases]
     io = StepIO(preps, device)
-    run_step(preps, False)   # first calls configure the kernels outside any capture
-    run_step(preps, True, io)
+    run_steps(preps, 1, False)   # first calls configure the kernels outside any capture
+    run_steps(preps, 2, True, io)
     torch.cuda.synchronize()
     sampler = ClockSampler(device)
     sec = timed_replays(preps, args.steps, args.warmup, False, dist_on, sampler)
