@@ -27,9 +27,12 @@
 // trail them.  The products are exact (|q - z| <= 15 times an f16 / bf16 / int8
 // activation); the only rounding besides fp32 accumulation (int32 for INT8) is the
 // final conversion.  Persistent CTAs walk the (weight tile, token tile) grid token-tile
-// fastest so that concurrent CTAs share weight tiles in L2.  Every wait is bounded; on
-// expiry the CTA records an error, stops, waits for what it has in flight and frees its
-// Tensor Memory.
+// fastest so that concurrent CTAs share weight tiles in L2.  With fewer tiles than SMs, K is
+// split over CTAs: each slice's fp32 partials go to the workspace, and the tile's last CTA
+// to arrive bulk-copies them into its (by then idle) ring and adds them in slice order.
+// Long K (many scale groups) builds the scale tables from global memory, and keeps a single
+// table if shared memory requires it.  Every wait is bounded; on expiry the CTA records an
+// error, stops, waits for what it has in flight and frees its Tensor Memory.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <stdint.h>

@@ -13,11 +13,13 @@
 //    64 packed bytes of a row: 128 k of INT4, 256 k of INT2).
 //  * One TMA box per tile and chunk brings 16 rows x KC units (a 3D box over unit pairs;
 //    a 2D box per unit pair when rows are not a whole number of pairs), written with the
-//    128-byte swizzle so that the warps' 16-byte reads of 8 rows hit 8 different bank
-//    groups.  The boxes of the first S chunks are issued, spread over the warps, before
-//    griddepcontrol.wait: with programmatic dependent launch they stream while the previous
-//    kernel in the stream finishes.  When all chunks fit in shared memory nothing else is
-//    issued; otherwise the last warp to finish a stage refills it.
+//    128-byte swizzle; MMA row g reads tile row (g >> 1) | ((g & 1) << 2), so the two rows of
+//    a quarter-warp fall in opposite bank halves and a 16-byte load per lane is conflict-free.
+//    Thread 0 sends the first chunk's boxes right after setting up the barriers, the other
+//    warps the next S - 1, all before griddepcontrol.wait: with programmatic dependent launch
+//    they stream while the previous kernel in the stream finishes.  When all chunks fit in
+//    shared memory nothing else is issued; otherwise the last warp to finish a stage
+//    refills it.
 //  * The activations are staged once for all of K (one bulk copy per token row) when they
 //    fit, else per chunk by a swizzled 3D TMA box.  The CTA's scales / zero points become a
 //    group-major fp32 table.
