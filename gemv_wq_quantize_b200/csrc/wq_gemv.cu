@@ -23,8 +23,8 @@
 //  * The activations are staged once for all of K (one bulk copy per token row) when they
 //    fit, else per chunk by a swizzled 3D TMA box.  The CTA's scales / zero points become a
 //    group-major fp32 table.
-//  * 16 warps; warp w takes unit w % KC of every chunk and, for 9..16 tokens, every other
-//    tile.  It builds the unit's mma.sync B fragments (activations in the k order of the
+//  * 16 warps; warp w takes unit w % KC of every chunk and, for 9..16 tokens with more than
+//    two tiles per CTA, every other tile.  It builds the unit's mma.sync B fragments (activations in the k order of the
 //    nibble unpack) once and uses them for all its tiles: weights are unpacked with LOP3
 //    into the exact integers q - z, multiplied on the tensor cores, and each unit's fp32 /
 //    int32 sum is folded with its group scale.
@@ -52,10 +52,12 @@ constexpr int kThreads = kCW * 32;
 constexpr int kTileRows = 16;
 constexpr int kPairBytes = 128;                   // two units of a row: one swizzle line
 constexpr int kPairBox = kTileRows * kPairBytes;  // 2 KB
-__host__ __device__ constexpr int wpu_of(int NT) { return NT == 1 ? 1 : 2; }  // warps sharing a unit
-__host__ __device__ constexpr int kc_of(int NT) { return kCW / wpu_of(NT); }  // units per chunk
-__host__ __device__ constexpr int tm_of(int NT) { return NT == 1 ? 6 : 3; }   // tiles per warp and pass
-__host__ __device__ constexpr int ntl_of(int NT) { return NT == 1 ? 2 : 1; }  // tiles per MMA batch
+// Work split by token tiles NT.  `wide` (9..16 tokens, at most two row tiles per CTA): one
+// warp per unit takes both tiles, so each unit's B fragments are built once, not per warp half.
+__host__ __device__ constexpr int wpu_of(int NT, bool wide = false) { return (NT == 1 || wide) ? 1 : 2; }  // warps sharing a unit
+__host__ __device__ constexpr int kc_of(int NT, bool wide = false) { return kCW / wpu_of(NT, wide); }  // units per chunk
+__host__ __device__ constexpr int tm_of(int NT, bool wide = false) { return NT == 1 ? 6 : (wide ? 2 : 3); }  // tiles per warp and pass
+__host__ __device__ constexpr int ntl_of(int NT, bool wide = false) { return (NT == 1 || wide) ? 2 : 1; }  // tiles per MMA batch
 
 struct GemvParams {
     const void *A;
@@ -132,7 +134,7 @@ __device__ __forceinline__ float finish(const GemvParams &p, float total_f, int 
 }
 
 // ACC: also store every INT32 group sum into p.acc_out (W4A8 with group_size 128).
-template <int WB, int AM, int NT, bool ACC>
+template <int WB, int AM, int NT, bool ACC, bool WIDE>
 __global__ void __launch_bounds__(kThreads, 1)
     gemv_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_a,
                 const GemvParams p)
@@ -141,7 +143,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     constexpr int QN = qn_of(WB, AM);
     constexpr int ES = (AM == A_I8) ? 1 : 2;
     constexpr int AU = KU * ES;  // activation bytes of one unit and token
-    constexpr int WPU = wpu_of(NT), KC = kc_of(NT), TM = tm_of(NT), NTL = ntl_of(NT);
+    constexpr int WPU = wpu_of(NT, WIDE), KC = kc_of(NT, WIDE), TM = tm_of(NT, WIDE), NTL = ntl_of(NT, WIDE);
     using Tot = typename std::conditional<AM == A_I8 && WB == 2, int, float>::type;
 
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -467,7 +469,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 // ---------------------------------------------------------------- host side
 struct Plan {
-    int NT = 1, KC = 16, KU = 128, KB = 0, T = 0, P = 0, nch = 0, TPP = 1, S = 1;
+    int NT = 1, wide = 0, KC = 16, KU = 128, KB = 0, T = 0, P = 0, nch = 0, TPP = 1, S = 1;
     int w3d = 0, wtile = 0, wpart = 0, stage = 0;
     int a_whole = 0, a_pitch_b = 0, abox = 0, MB = 8, rows_cap = 0, tab_rs = 1;
     int abuf_off = 0, scst_off = 0, stab_off = 0, red_off = 0, bar_off = 0;
@@ -482,13 +484,14 @@ Plan make_plan(int64_t M, int64_t N, int64_t K, int WB, int AM, int G, const Dev
     Plan pl;
     pl.NT = M <= 8 ? 1 : 2;
     if (WB == 2 && AM != A_I8 && pl.NT == 2) return pl;  // B fragments would not fit in registers
-    pl.KC = kc_of(pl.NT);
     pl.KU = kunit_of(WB);
     pl.KB = int((K + pl.KU - 1) / pl.KU);
     pl.T = int((N + kTileRows - 1) / kTileRows);
     pl.P = std::min(dev.sm_count, pl.T);
     const int ntc_max = (pl.T + pl.P - 1) / pl.P;
-    pl.TPP = std::min(ntc_max, tm_of(pl.NT) * wpu_of(pl.NT));
+    pl.wide = (pl.NT == 2 && AM != A_I8 && ntc_max <= 2) ? 1 : 0;
+    pl.KC = kc_of(pl.NT, pl.wide);
+    pl.TPP = std::min(ntc_max, tm_of(pl.NT, pl.wide) * wpu_of(pl.NT, pl.wide));
     const int npass = (ntc_max + pl.TPP - 1) / pl.TPP;
     pl.nch = (pl.KB + pl.KC - 1) / pl.KC;
     const long long total = (long long)npass * pl.nch;
@@ -546,10 +549,10 @@ Plan make_plan(int64_t M, int64_t N, int64_t K, int WB, int AM, int G, const Dev
     return pl;
 }
 
-template <int WB, int AM, int NT, bool ACC = false>
+template <int WB, int AM, int NT, bool ACC = false, bool WIDE = false>
 wq_status launch(const Plan &pl, const CUtensorMap &tw, const CUtensorMap &ta, const GemvParams &p, cudaStream_t st)
 {
-    auto kern = gemv_kernel<WB, AM, NT, ACC>;
+    auto kern = gemv_kernel<WB, AM, NT, ACC, WIDE>;
     static size_t configured = 0;
     if (pl.smem > configured) {
         if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(pl.smem)) != cudaSuccess)
@@ -650,9 +653,12 @@ wq_status gemv_small_m(int WB, int AM, const void *A, const float *a_scale, cons
     p.C = C;
     p.acc_out = acc_out;
     const bool one = pl.NT == 1;
-    if (WB == 4 && AM == A_F16) return one ? launch<4, A_F16, 1>(pl, tw, ta, p, st) : launch<4, A_F16, 2>(pl, tw, ta, p, st);
+    if (WB == 4 && AM == A_F16)
+        return one ? launch<4, A_F16, 1>(pl, tw, ta, p, st)
+                   : pl.wide ? launch<4, A_F16, 2, false, true>(pl, tw, ta, p, st) : launch<4, A_F16, 2>(pl, tw, ta, p, st);
     if (WB == 4 && AM == A_BF16)
-        return one ? launch<4, A_BF16, 1>(pl, tw, ta, p, st) : launch<4, A_BF16, 2>(pl, tw, ta, p, st);
+        return one ? launch<4, A_BF16, 1>(pl, tw, ta, p, st)
+                   : pl.wide ? launch<4, A_BF16, 2, false, true>(pl, tw, ta, p, st) : launch<4, A_BF16, 2>(pl, tw, ta, p, st);
     if (WB == 4 && acc_out)
         return one ? launch<4, A_I8, 1, true>(pl, tw, ta, p, st) : launch<4, A_I8, 2, true>(pl, tw, ta, p, st);
     if (WB == 4) return one ? launch<4, A_I8, 1>(pl, tw, ta, p, st) : launch<4, A_I8, 2>(pl, tw, ta, p, st);
