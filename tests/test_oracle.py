@@ -468,3 +468,67 @@ def test_gemm_a8_unit_scale_is_integer_matmul():
     s = f16_bits(np.ones((N, 1)))
     Ce, _, _ = oracle.gemm_a8(Aq, np.ones(M, np.float32), Wq, N, K, 4, True, K, s)
     assert np.array_equal(Ce, (Aq.astype(np.int64) @ q.T).astype(np.float64))
+
+
+# ----------------------------------------------------------------- exact ties
+# tests/golden/ties.txt puts exact ties (w / s = k + 1/2 in binary32) in front of every
+# quantizer: "round" read as round-half-to-even must give the fixture's codes, and the
+# fixture also lists the different codes that round-half-away-from-zero would give.
+import tie_inputs  # noqa: E402
+
+
+def test_sym_ties_to_even():
+    fx = tie_inputs.fields()
+    W, q, q_away, s_bits = tie_inputs.sym_case(fx)
+    Wq, s, _ = oracle.quantize_int4(W, 128, True)
+    assert s[0, 0] == s_bits
+    got = oracle.unpack(Wq, 1, 128, 4, True)[0]
+    assert np.array_equal(got, q)
+    assert not np.array_equal(got, q_away)
+
+
+def test_asym_ties_to_even_in_codes_and_zero_point():
+    fx = tie_inputs.fields()
+    W, q, s_bits, z_bits, z_away_bits = tie_inputs.asym_case(fx)
+    Wq, s, z = oracle.quantize_int4(W, 128, False)
+    assert s[0, 0] == s_bits
+    assert z[0, 0] == z_bits and z[0, 0] != z_away_bits
+    assert np.array_equal(oracle.unpack(Wq, 1, 128, 4, False)[0], q)
+
+
+def test_ternary_ties_to_even():
+    fx = tie_inputs.fields()
+    W, q, q_away, s_bits = tie_inputs.tern_case(fx)
+    Wq, s = oracle.quantize_ternary(W)
+    assert s.view(np.uint32)[0] == s_bits
+    got = oracle.unpack(Wq, W.shape[0], W.shape[1], 2, True)
+    assert np.array_equal(got, q) and not np.array_equal(got, q_away)
+
+
+@pytest.mark.parametrize("dtype", [torch.float16, torch.bfloat16])
+def test_act_quant_ties_to_even(dtype):
+    fx = tie_inputs.fields()
+    A, q, q_away, s_bits = tie_inputs.act_case(fx, dtype)
+    Aq, sc = oracle.act_quant_int8(_a_bits(A), oracle.F16 if dtype == torch.float16 else oracle.BF16)
+    assert sc.view(np.uint32)[0] == s_bits
+    assert np.array_equal(Aq[0].astype(np.int64), q) and not np.array_equal(Aq[0].astype(np.int64), q_away)
+
+
+def test_tie_fixture_rejects_half_away_rounding(tmp_path):
+    # The pins above must catch an oracle that rounds ties away from zero: build a copy of
+    # the oracle with every rintf replaced by roundf and check that its codes are the
+    # fixture's *_away codes, not the round-half-to-even ones.
+    import ctypes
+    import subprocess
+    so = str(tmp_path / "liboracle_roundf.so")
+    subprocess.check_call(["gcc", *oracle.CFLAGS, "-Drintf=roundf", "-o", so, oracle._SRC, "-lm"])
+    lib = ctypes.CDLL(so)
+    fx = tie_inputs.fields()
+    W, q, q_away, _ = tie_inputs.sym_case(fx)
+    Wq = np.zeros((1, 64), dtype=np.uint8)
+    s = np.zeros((1, 1), dtype=np.uint16)
+    assert lib.orc_quant_int4_sym(ctypes.c_void_p(W.ctypes.data), ctypes.c_int64(1), ctypes.c_int64(128),
+                                  ctypes.c_int64(128), ctypes.c_void_p(Wq.ctypes.data),
+                                  ctypes.c_void_p(s.ctypes.data)) == 0
+    got = oracle.unpack(Wq, 1, 128, 4, True)[0]
+    assert np.array_equal(got, q_away) and not np.array_equal(got, q)
