@@ -51,13 +51,14 @@ wq_status check_launch(const char *what)
 
 const DeviceInfo &device_info()
 {
+    // A fixed table: references handed out stay valid while other threads add devices.
     static std::mutex mu;
-    static std::vector<DeviceInfo> cache;
+    static DeviceInfo cache[kMaxDevices];
+    static DeviceInfo fallback;
     int dev = 0;
     cudaGetDevice(&dev);
     std::lock_guard<std::mutex> lock(mu);
-    if (int(cache.size()) <= dev) cache.resize(dev + 1);
-    DeviceInfo &d = cache[dev];
+    DeviceInfo &d = (dev >= 0 && dev < kMaxDevices) ? cache[dev] : fallback;
     if (d.device != dev) {
         d.device = dev;
         cudaDeviceGetAttribute(&d.sm_count, cudaDevAttrMultiProcessorCount, dev);

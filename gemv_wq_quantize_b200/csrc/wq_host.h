@@ -23,7 +23,8 @@ struct DeviceInfo {
     int sm_count = 0;
     int max_smem_optin = 0;  // bytes of shared memory a block may opt in to
 };
-// Properties of the current device (cached per device).
+// Properties of the current device (cached per device ordinal below kMaxDevices).
+constexpr int kMaxDevices = 64;
 const DeviceInfo &device_info();
 
 // cuTensorMapEncodeTiled through the runtime's driver entry point (no libcuda link).

@@ -11,9 +11,13 @@
 //
 // The scratch is one array per device, compiled into this translation unit (its module is
 // loaded, and the array created by the driver, on first use).  The first call on a device
-// looks up its address with cudaGetSymbolAddress, with that device current, and clears
-// it; later calls reuse both.  Calls that overlap on the GPU (two streams, or two host
-// threads) share the array and race: serialise them.
+// that needs scratch looks up its address with cudaGetSymbolAddress, with that device
+// current, and clears it; later calls reuse the address.  Every such call also clears the
+// split-K arrival counters at the end of the scratch on its own stream (a memset of a few
+// bytes, which allocates nothing): a kernel that gave up a bounded wait may have left a
+// counter off zero, and later calls must not inherit it.  Shapes that need no scratch (up
+// to 16 tokens) go straight to w4a16_gemm with no set-up at all.  Calls that overlap on
+// the GPU (two streams, or two host threads) share the array and race: serialise them.
 #include <cuda_runtime.h>
 
 #include <mutex>
@@ -26,7 +30,6 @@ namespace {
 // 148 CTAs x 2 slots x 128 rows x 64 tokens x 4 B = 9.25 MiB of partial sums, plus 4 B
 // of arrival counter per 128 weight rows.
 constexpr size_t kScratchBytes = WQ_NOALLOC_SCRATCH_BYTES;
-constexpr int kMaxDevices = 64;
 
 }  // namespace
 
@@ -53,8 +56,7 @@ wq_status scratch_for_current_device(void **out)
         e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
         if (e != cudaSuccess)
             return fail(WQ_ERR_CUDA, "cudaGetSymbolAddress(static scratch): %s", cudaGetErrorString(e));
-        // The split-K arrival counters in the scratch must start at zero; every call
-        // leaves them at zero again, so one clear per device is enough.
+        // Start from a zeroed array; the arrival counters are cleared again by every call.
         e = cudaMemset(p, 0, kScratchBytes);
         if (e == cudaSuccess) e = cudaDeviceSynchronize();
         if (e != cudaSuccess) return fail(WQ_ERR_CUDA, "clearing the static scratch: %s", cudaGetErrorString(e));
@@ -80,8 +82,16 @@ extern "C" wq_status w4a16_gemm_noalloc(const void *A, wq_dtype a_dt, const uint
                     "w4a16_gemm_noalloc: M=%lld N=%lld K=%lld needs %zu bytes of scratch but the static scratch "
                     "holds %zu; call w4a16_gemm with a workspace instead",
                     (long long)M, (long long)N, (long long)K, need, kScratchBytes);
+    // Few tokens: the launch plan needs no scratch, so nothing is set up or cleared.
+    if (need == 0) return w4a16_gemm(A, a_dt, Wq, scales, zeros, bias, C, M, N, K, c, nullptr, 0, stream);
     void *scratch = nullptr;
     const wq_status rc = scratch_for_current_device(&scratch);
     if (rc != WQ_OK) return rc;
+    // The counters follow the partial-sum area; clear them on the caller's stream.
+    const size_t cnt0 = ws_scratch_bytes();
+    if (need > cnt0) {
+        const cudaError_t e = cudaMemsetAsync(static_cast<unsigned char *>(scratch) + cnt0, 0, need - cnt0, stream);
+        if (e != cudaSuccess) return fail(WQ_ERR_CUDA, "clearing the scratch counters: %s", cudaGetErrorString(e));
+    }
     return w4a16_gemm(A, a_dt, Wq, scales, zeros, bias, C, M, N, K, c, scratch, kScratchBytes, stream);
 }

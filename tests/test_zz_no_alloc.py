@@ -56,6 +56,8 @@ def test_noalloc_refuses_a_shape_beyond_its_scratch():
     """N = 2^30 rows needs 4 B of arrival counter per 128 rows (32 MiB) alone: more than
     the 16 MiB static scratch.  The refusal comes before any argument is looked at, so
     NULL pointers are passed and nothing can be launched."""
+    from gemv_wq_quantize_b200 import build
+    build.build(quiet=True)
     lib = wq.load_library()
     qc = wq.QuantConfig(4, 128, True)
     M, N, K = 64, 1 << 30, 128
@@ -65,3 +67,17 @@ def test_noalloc_refuses_a_shape_beyond_its_scratch():
     assert rc == wq.WQ_ERR_WORKSPACE
     msg = lib.wq_last_error().decode()
     assert "static scratch" in msg and str(16 << 20) in msg and str(need) in msg
+
+
+def test_noalloc_few_tokens_need_no_setup():
+    """Up to 16 tokens the launch plan uses no scratch: the call goes straight to the
+    argument checks of w4a16_gemm, with no scratch set-up and no device query, so NULL
+    pointers are refused as invalid arguments (on a machine without a GPU too)."""
+    from gemv_wq_quantize_b200 import build
+    build.build(quiet=True)
+    lib = wq.load_library()
+    qc = wq.QuantConfig(4, 128, True)
+    assert lib.wq_workspace_size(16, 4096, 4096, qc.c()) == 0
+    rc = lib.w4a16_gemm_noalloc(None, wq.WQ_F16, None, None, None, None, None, 16, 4096, 4096, qc.c(), None)
+    assert rc == wq.WQ_ERR_INVALID_ARG
+    assert "non-null" in lib.wq_last_error().decode()
