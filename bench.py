@@ -16,7 +16,12 @@ the measurement through the same C-ABI calls with pinned HOST activations and ou
 every step copies A host->device and C device->host inside the timed region.
 
 Algorithmic bytes per launch: packed weights N*K*b/8 + scales (+ zeros) N*G*2 (each) +
-activations M*K*bytes(A) (+ 4M for INT8 scales) + output M*N*2.
+activations M*K*2 (fp16/bf16; the INT8 paths quantize them per token inside the step) +
+output M*N*2.
+
+The default run also times, in the same process and the same way, the prefill GEMMs
+("gemm": TFLOP/s against the measured bf16 tensor peak, burst and sustained), the W4A8
+workload and the BitNet-3B ternary sweep, each with its per-case breakdown.
 
 ``--impl reference`` times the CPU oracle (plain C, float64) on a bounded sample of the
 same workload on the host cores; it is a deliberately slow baseline, not a target.
@@ -47,6 +52,10 @@ FALLBACK_BF16_TFLOPS = 1590.0
 
 # ------------------------------------------------------------------ workload arithmetic
 def alg_bytes(c: wq_synth.Case) -> int:
+    """Bytes the method must move for one matmul: packed weights, scales (+ zeros), the
+    activations once and the output once.  The INT8 paths start from fp16 activations (the
+    per-token quantization is part of the step), so they too read M*K*2 bytes of A; the
+    INT8 copy of A and its scales are intermediate values, not counted."""
     bits = 2 if c.quant == "tern2" else 4
     w = c.N * c.K * bits // 8
     if bits == 4:
@@ -54,7 +63,7 @@ def alg_bytes(c: wq_synth.Case) -> int:
         w += c.N * G * 2 * (2 if c.quant == "asym4" else 1)
     else:
         w += 4
-    a = c.M * c.K * (1 if c.mode == "a8" else 2) + (4 * c.M if c.mode == "a8" else 0)
+    a = c.M * c.K * 2
     return w + a + c.M * c.N * 2
 
 
@@ -63,7 +72,9 @@ def flops(c: wq_synth.Case) -> int:
 
 
 def launches_per_call(c: wq_synth.Case) -> int:
-    return (c.M + 63) // 64
+    """Kernels one step launches for the case: the matmul, plus the per-token activation
+    quantization on the INT8 paths."""
+    return 2 if c.mode == "a8" else 1
 
 
 def peaks():
@@ -205,8 +216,8 @@ class Prepared:
         if c.mode == "a16":
             wq.w4a16_gemm(A, Wq, s, z, c.N, c.K, self.qc, out=C, workspace=self.ws)
         else:
-            if e2e:  # the INT8 path starts from the fp16 activations: quantize them too
-                wq.act_quant_int8(A, out_q=self.Aq, out_scale=self.a_scale)
+            # the INT8 path starts from the fp16 activations: every step quantizes them per token
+            wq.act_quant_int8(A, out_q=self.Aq, out_scale=self.a_scale)
             wq.w4a8_gemm(self.Aq, self.a_scale, Wq, s, z, c.N, c.K, self.qc, out=C, workspace=self.ws)
 
 
@@ -377,11 +388,117 @@ def per_case_breakdown(preps, reps: int = 200):
         gbs = p.bytes / (us * 1e-6) / 1e9
         tf = flops(p.c) / (us * 1e-6) / 1e12
         peak_tc = pk["bf16_tflops"] * (2.0 if p.c.mode == "a8" else 1.0)
+        peak_tc_s = pk["bf16_tflops_sustained"] * (2.0 if p.c.mode == "a8" else 1.0)
         t_roof = max(p.bytes / (pk["hbm_gbs"] * 1e9), flops(p.c) / (peak_tc * 1e12))
         out.append({"case": p.c.name, "us": round(us, 3), "GB/s": round(gbs, 1), "TFLOP/s": round(tf, 2),
-                    "hbm_frac": round(gbs / pk["hbm_gbs"], 4), "roofline_frac": round(t_roof / (us * 1e-6), 4)})
+                    "hbm_frac": round(gbs / pk["hbm_gbs"], 4), "tensor_frac": round(tf / peak_tc, 4),
+                    "tensor_frac_sustained": round(tf / peak_tc_s, 4),
+                    "roofline_frac": round(t_roof / (us * 1e-6), 4)})
         del g
     return out
+
+
+# Workloads timed beside the headline one in the default run, each as its own object of the
+# JSON line: the prefill GEMMs (the tensor-bound half of the metric), W4A8 and the BitNet sweep.
+EXTRA_WORKLOADS = (("gemm", "prefill-llama7b"), ("w4a8", "w4a8"), ("bitnet3b", "bitnet3b"))
+
+
+def measure_extra(name: str, device, steps: int, warmup: int, dist_on: bool) -> dict:
+    """Device-timed steps of a further workload (same protocol as the headline), with its
+    per-case breakdown and the roofline of its bound: the tensor peak (burst and sustained)
+    for the prefill GEMMs, HBM bandwidth for the rest."""
+    import gemv_wq_quantize_b200 as wq
+    wl = wq_synth.WORKLOADS[name]
+    preps = [Prepared(c, device, seed_base=0) for c in wl.cases]
+    run_steps(preps, 1, False)
+    torch.cuda.synchronize()
+    sampler = ClockSampler(device)
+    sec = timed_replays(preps, steps, warmup, False, dist_on, sampler)
+    assert wq.device_error() == 0, "a kernel gave up a bounded wait"
+    cases = per_case_breakdown(preps)
+    step_bytes = sum(p.bytes for p in preps)
+    step_flops = sum(flops(p.c) for p in preps)
+    pk = peaks()
+    gbs = step_bytes * steps / sec / 1e9
+    tf = step_flops * steps / sec / 1e12
+    out = {"workload": name, "description": wl.description, "steps": steps, "warmup": warmup,
+           "ms_per_step": round(sec / steps * 1e3, 6), "GB/s": round(gbs, 2), "TFLOP/s": round(tf, 2),
+           "gpu_launches": steps * sum(launches_per_call(p.c) for p in preps), "clocks": sampler.report()}
+    if name == "prefill-llama7b":
+        out["roofline"] = {"bound": "tensor", "achieved": round(tf, 2), "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+                           "frac": round(tf / pk["bf16_tflops"], 4), "peak_sustained": pk["bf16_tflops_sustained"],
+                           "frac_sustained": round(tf / pk["bf16_tflops_sustained"], 4),
+                           "traffic": recorded_traffic(name), "peak_source": pk["source"]}
+    else:
+        out["roofline"] = {"bound": "hbm", "achieved": round(gbs, 2), "peak": pk["hbm_gbs"], "unit": "GB/s",
+                           "frac": round(gbs / pk["hbm_gbs"], 4), "traffic": recorded_traffic(name),
+                           "peak_source": pk["source"]}
+    out["cases"] = cases
+    del preps
+    torch.cuda.empty_cache()
+    return out
+
+
+LLAMA7B_LAYER = (("qkv", 12288, 4096), ("o", 4096, 4096), ("gate_up", 22016, 4096), ("down", 4096, 11008))
+
+
+def measure_layer_graph(device, M: int = 1, reps: int = 50) -> dict:
+    """One Llama-7B layer's four decode projections (asymmetric INT4, group 128, fp16) run as
+    one wq_graph per layer, over enough layer copies (6 x 101 MB) that every launch streams
+    its weights from HBM.  Reported per layer step: the graph (one launch per layer), the
+    same four kernels captured by stream capture (device time of the kernels alone), and
+    four direct C-ABI calls per layer issued from this Python process (host-bound)."""
+    import gemv_wq_quantize_b200 as wq
+    qc = wq.QuantConfig(4, 128, False)
+    base = []
+    for i, (name, N, K) in enumerate(LLAMA7B_LAYER):
+        Wq, s, z = wq.quantize_pack(wq_synth.weights(N, K, seed=i).to(device), qc)
+        A = wq_synth.activations(M, K, seed=10 + i, outlier_frac=0.01).to(device)
+        C = torch.empty(M, N, dtype=torch.float16, device=device)
+        base.append((name, N, K, Wq, s, z, A, C))
+    layer_bytes = sum(alg_bytes(wq_synth.Case(M, N, K, "a16", "asym4")) for _, N, K, *_ in base)
+    nlayers = max(2, math.ceil(4 * L2_BYTES / layer_bytes) + 1)
+    layers = [[(name, N, K, Wq.clone(), s.clone(), z.clone(), A, C) for name, N, K, Wq, s, z, A, C in base]
+              for _ in range(nlayers)]
+    graphs = [wq.DecodeGraph([{"A": A, "Wq": Wq, "scales": s, "zeros": z, "N": N, "K": K, "qc": qc, "out": C}
+                              for _, N, K, Wq, s, z, A, C in layer]) for layer in layers]
+
+    def calls():
+        for layer in layers:
+            for _, N, K, Wq, s, z, A, C in layer:
+                wq.w4a16_gemm(A, Wq, s, z, N, K, qc, out=C)
+
+    def timed(fn, n):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0.record()
+        for _ in range(n):
+            fn()
+        t1.record()
+        torch.cuda.synchronize()
+        return t0.elapsed_time(t1) * 1e3 / (n * nlayers)
+
+    def graph_steps():
+        for g in graphs:
+            g.launch()
+
+    us_graph = timed(graph_steps, reps)
+    cap = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(cap):
+        calls()
+    us_captured = timed(cap.replay, reps)
+    us_calls = timed(calls, max(5, reps // 5))
+    for g in graphs:
+        g.close()
+    assert wq.device_error() == 0, "a kernel gave up a bounded wait"
+    pk = peaks()
+    return {"ops": [f"{n}:{N}x{K}" for n, N, K in LLAMA7B_LAYER], "M": M, "layer_copies": nlayers,
+            "bytes_per_layer": layer_bytes, "us_per_layer_graph": round(us_graph, 3),
+            "us_per_layer_stream_captured": round(us_captured, 3), "us_per_layer_direct_calls": round(us_calls, 3),
+            "GB/s_graph": round(layer_bytes / (us_graph * 1e-6) / 1e9, 1),
+            "hbm_frac_graph": round(layer_bytes / (us_graph * 1e-6) / 1e9 / pk["hbm_gbs"], 4)}
 
 
 def run_ours(args, rank, world, local_rank, dist_on):
@@ -436,6 +553,12 @@ def run_ours(args, rank, world, local_rank, dist_on):
     }
     if not args.no_breakdown:
         result["cases"] = per_case_breakdown(preps)
+    del preps, io
+    torch.cuda.empty_cache()
+    if args.workload == "decode-llama7b" and not args.no_extra:
+        for key, name in EXTRA_WORKLOADS:
+            result[key] = measure_extra(name, device, min(args.steps, 2000), args.warmup, dist_on)
+        result["decode_layer_graph"] = measure_layer_graph(device)
     return result
 
 
@@ -534,6 +657,8 @@ def main():
     ap.add_argument("--workload", default="decode-llama7b", choices=sorted(wq_synth.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-breakdown", action="store_true")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="time only the chosen workload (the default run adds the prefill GEMM, W4A8 and BitNet)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=10.0, help="seconds of oracle work for cpu_baseline")
     ap.add_argument("--profile", action="store_true",

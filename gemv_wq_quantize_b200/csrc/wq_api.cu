@@ -24,7 +24,7 @@ wq_status gemv_small_m(int WB, int AM, const void *A, const float *a_scale, cons
                        int64_t K, const wq_qconfig &c, cudaStream_t st);
 int gemv_read_error();
 wq_status tc_gemm(int WB, int AM, const void *A, const float *a_scale, const uint8_t *Wq, const void *scales,
-                  const void *zeros, const void *bias, void *C, int64_t M, int64_t N, int64_t K,
+                  const void *zeros, const void *bias, void *C, int32_t *acc_out, int64_t M, int64_t N, int64_t K,
                   const wq_qconfig &c, void *ws, size_t ws_bytes, cudaStream_t st);
 size_t tc_workspace_size(int64_t M, int64_t N, int64_t K);
 int tc_read_error();
@@ -126,6 +126,23 @@ wq_status encode_tmap(CUtensorMap *map, CUtensorMapDataType dt, int rank, const 
     return WQ_OK;
 }
 
+wq_status launch_prepared(PreparedLaunch &L, cudaStream_t st, const char *what)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = L.grid;
+    cfg.blockDim = L.block;
+    cfg.dynamicSmemBytes = L.smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t e = cudaLaunchKernelExC(&cfg, L.func, L.argp);
+    if (e != cudaSuccess) return fail(WQ_ERR_CUDA, "%s launch: %s", what, cudaGetErrorString(e));
+    return check_launch(what);
+}
+
 int read_device_errors()
 {
     const int a = skinny_read_error(), b = gemv_read_error(), t = tc_read_error();
@@ -133,8 +150,9 @@ int read_device_errors()
 }
 
 namespace {
-// Few tokens go to the weight-streaming GEMV; more tokens to the tcgen05 GEMM, or else (the
-// INT32 group-sum output, shapes without a plan there) to the tiled mma.sync path.
+// Few tokens go to the weight-streaming GEMV; more tokens to the tcgen05 GEMM (the INT32
+// group sums included), or else (shapes without a plan there: K below four 128-k blocks,
+// ternary FP activations at 9..16 tokens) to the tiled mma.sync path.
 wq_status dispatch(int WB, int AM, const void *A, const float *a_scale, const uint8_t *Wq, const void *scales,
                    const void *zeros, const void *bias, void *C, int32_t *acc_out, int64_t M, int64_t N, int64_t K,
                    const wq_qconfig &c, void *ws, size_t ws_bytes, cudaStream_t st)
@@ -142,8 +160,8 @@ wq_status dispatch(int WB, int AM, const void *A, const float *a_scale, const ui
     if (M <= 16) {
         wq_status rc = gemv_small_m(WB, AM, A, a_scale, Wq, scales, zeros, bias, C, acc_out, M, N, K, c, st);
         if (rc != WQ_ERR_UNSUPPORTED) return rc;
-    } else if (!acc_out) {
-        wq_status rc = tc_gemm(WB, AM, A, a_scale, Wq, scales, zeros, bias, C, M, N, K, c, ws, ws_bytes, st);
+    } else {
+        wq_status rc = tc_gemm(WB, AM, A, a_scale, Wq, scales, zeros, bias, C, acc_out, M, N, K, c, ws, ws_bytes, st);
         if (rc != WQ_ERR_UNSUPPORTED) return rc;
     }
     return skinny_gemm(WB, AM, A, a_scale, Wq, scales, zeros, bias, C, acc_out, M, N, K, c, ws, ws_bytes, st);
@@ -207,16 +225,27 @@ extern "C" size_t wq_workspace_size(int64_t M, int64_t N, int64_t K, wq_qconfig 
                      tc_workspace_size(M, N, K)});
 }
 
-extern "C" wq_status w4a16_gemm(const void *A, wq_dtype a_dt, const uint8_t *Wq, const void *scales,
-                                const void *zeros, const void *bias, void *C, int64_t M, int64_t N, int64_t K,
-                                wq_qconfig c, void *workspace, size_t ws_bytes, cudaStream_t stream)
+namespace wq {
+wq_status check_a16(const void *A, wq_dtype a_dt, const uint8_t *Wq, const void *scales, const void *zeros,
+                    const void *bias, const void *C, int64_t M, int64_t N, int64_t K, const wq_qconfig &c)
 {
     wq_status rc = check_weights(Wq, scales, zeros, M, N, K, c);
     if (rc != WQ_OK) return rc;
     if (a_dt != WQ_F16 && a_dt != WQ_BF16) return fail(WQ_ERR_INVALID_ARG, "a_dt must be WQ_F16 or WQ_BF16");
     if (!A || !C) return fail(WQ_ERR_INVALID_ARG, "A and C must be non-null");
-    if (!aligned16(A) || !aligned16(C) || (bias && !aligned16(bias)) || (workspace && !aligned16(workspace)))
-        return fail(WQ_ERR_ALIGNMENT, "A, C, bias and workspace must be 16-byte aligned");
+    if (!aligned16(A) || !aligned16(C) || (bias && !aligned16(bias)))
+        return fail(WQ_ERR_ALIGNMENT, "A, C and bias must be 16-byte aligned");
+    return WQ_OK;
+}
+}  // namespace wq
+
+extern "C" wq_status w4a16_gemm(const void *A, wq_dtype a_dt, const uint8_t *Wq, const void *scales,
+                                const void *zeros, const void *bias, void *C, int64_t M, int64_t N, int64_t K,
+                                wq_qconfig c, void *workspace, size_t ws_bytes, cudaStream_t stream)
+{
+    wq_status rc = check_a16(A, a_dt, Wq, scales, zeros, bias, C, M, N, K, c);
+    if (rc != WQ_OK) return rc;
+    if (workspace && !aligned16(workspace)) return fail(WQ_ERR_ALIGNMENT, "workspace must be 16-byte aligned");
     return dispatch(c.bits, a_dt == WQ_F16 ? 0 : 1, A, nullptr, Wq, scales, c.bits == 4 && !c.symmetric ? zeros : nullptr,
                        bias, C, nullptr, M, N, K, c, workspace, ws_bytes, stream);
 }

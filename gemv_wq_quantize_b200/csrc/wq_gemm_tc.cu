@@ -84,6 +84,7 @@ struct TcParams {
     const uint16_t *zeros;
     const void *bias;
     void *C;
+    int32_t *acc_out;  // ACC: INT32 group sums [M][N][G] (INT4, group 128) or totals [M][N] (INT2)
 };
 
 __device__ __forceinline__ uint64_t globaltimer()
@@ -179,7 +180,11 @@ __device__ __forceinline__ void unpack_word(uint32_t w, uint32_t zc, uint32_t *o
     for (int i = 0; i < 4; ++i) o[i] = BF16 ? bf2_fma(x[i], 0x3F803F80u, zc) : h2_add(x[i], zc);
 }
 
-template <int WB, int AM>
+// ACC (INT8 activations only): also store the exact INT32 sums in p.acc_out.  For INT4
+// with group_size 128 a block of 128 k is one group, so each block accumulator read from
+// Tensor Memory is one acc_g (the zero point is already inside the weight bytes); for
+// ternary INT2 the fp32 totals are exact integers (|sum| < 2^24) and are stored at the end.
+template <int WB, int AM, bool ACC = false>
 __global__ void __launch_bounds__(kThreads, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_w,
                    const TcParams p)
@@ -504,6 +509,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const float dv = I8 ? float(int(d[j])) : __uint_as_float(d[j]);
                         tot[c * 16 + j] = fmaf(sv, dv, tot[c * 16 + j]);
                     }
+                    if constexpr (ACC && WB == 4) {
+                        const int n = n0 + r, mb = m0 + th * 64 + c * 16;
+                        if (n < p.N)
+#pragma unroll
+                            for (int j = 0; j < 16; ++j)
+                                if (mb + j < p.M) p.acc_out[((size_t)(mb + j) * p.N + n) * p.G + kb] = int(d[j]);
+                    }
                 }
             }
             if (!ok) break;
@@ -581,6 +593,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int j = 0; j < 64; ++j) {
                     if (mb + j >= p.M) continue;
+                    if constexpr (ACC && WB == 2) p.acc_out[(size_t)(mb + j) * p.N + n] = int(tot[j]);
                     float v;
                     if constexpr (I8) v = p.a_scale[mb + j] * (WB == 2 ? ws * tot[j] : tot[j]);
                     else v = ws * tot[j];
@@ -638,11 +651,11 @@ TcPlan make_plan(int nkb, int G, int stage, const DeviceInfo &dev)
     return pl;
 }
 
-template <int WB, int AM>
+template <int WB, int AM, bool ACC = false>
 wq_status launch(const TcPlan &pl, const CUtensorMap &ta, const CUtensorMap &tw, const TcParams &p, int grid,
                  cudaStream_t st)
 {
-    auto kern = tc_gemm_kernel<WB, AM>;
+    auto kern = tc_gemm_kernel<WB, AM, ACC>;
     static size_t configured = 0;
     if (pl.smem > configured) {
         if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(pl.smem)) != cudaSuccess)
@@ -698,9 +711,11 @@ size_t tc_workspace_size(int64_t M, int64_t N, int64_t K)
 // The workspace (zero-filled once, see the ABI) is used for split-K partial sums when it
 // is large enough; otherwise every tile covers all of K.
 wq_status tc_gemm(int WB, int AM, const void *A, const float *a_scale, const uint8_t *Wq, const void *scales,
-                  const void *zeros, const void *bias, void *C, int64_t M, int64_t N, int64_t K,
+                  const void *zeros, const void *bias, void *C, int32_t *acc_out, int64_t M, int64_t N, int64_t K,
                   const wq_qconfig &c, void *ws, size_t ws_bytes, cudaStream_t st)
 {
+    if (acc_out && (AM != 2 || (WB == 4 && c.group_size != kKB)))
+        return fail(WQ_ERR_UNSUPPORTED, "tc_gemm: INT32 sums need INT8 activations (and group_size 128 for INT4)");
     if (WB == 4 && (K % kKB || c.group_size % kKB))
         return fail(WQ_ERR_UNSUPPORTED, "tc_gemm: INT4 needs K and group_size multiples of 128");
     const int es = AM == 2 ? 1 : 2;
@@ -761,15 +776,16 @@ wq_status tc_gemm(int WB, int AM, const void *A, const float *a_scale, const uin
     p.zeros = static_cast<const uint16_t *>(zeros);
     p.bias = bias;
     p.C = C;
+    p.acc_out = acc_out;
     const int grid = std::min(dev.sm_count, p.NT * p.ks);
     if (WB == 4) {
         if (AM == 0) return launch<4, 0>(pl, ta, tw, p, grid, st);
         if (AM == 1) return launch<4, 1>(pl, ta, tw, p, grid, st);
-        return launch<4, 2>(pl, ta, tw, p, grid, st);
+        return acc_out ? launch<4, 2, true>(pl, ta, tw, p, grid, st) : launch<4, 2>(pl, ta, tw, p, grid, st);
     }
     if (AM == 0) return launch<2, 0>(pl, ta, tw, p, grid, st);
     if (AM == 1) return launch<2, 1>(pl, ta, tw, p, grid, st);
-    return launch<2, 2>(pl, ta, tw, p, grid, st);
+    return acc_out ? launch<2, 2, true>(pl, ta, tw, p, grid, st) : launch<2, 2>(pl, ta, tw, p, grid, st);
 }
 
 int tc_read_error()

@@ -35,6 +35,7 @@
 #include <stdint.h>
 
 #include <algorithm>
+#include <cstring>
 #include <type_traits>
 
 #include "wq_device.cuh"
@@ -549,8 +550,9 @@ Plan make_plan(int64_t M, int64_t N, int64_t K, int WB, int AM, int G, const Dev
     return pl;
 }
 
+// The kernel instance for the plan, with its dynamic shared memory limit raised as needed.
 template <int WB, int AM, int NT, bool ACC = false, bool WIDE = false>
-wq_status launch(const Plan &pl, const CUtensorMap &tw, const CUtensorMap &ta, const GemvParams &p, cudaStream_t st)
+wq_status kernel_for(const Plan &pl, const void **func)
 {
     auto kern = gemv_kernel<WB, AM, NT, ACC, WIDE>;
     static size_t configured = 0;
@@ -559,27 +561,16 @@ wq_status launch(const Plan &pl, const CUtensorMap &tw, const CUtensorMap &ta, c
             return check_launch("cudaFuncSetAttribute(gemv)");
         configured = pl.smem;
     }
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(pl.P);
-    cfg.blockDim = dim3(kThreads);
-    cfg.dynamicSmemBytes = pl.smem;
-    cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, kern, tw, ta, p);
-    if (e != cudaSuccess) return fail(WQ_ERR_CUDA, "gemv_kernel launch: %s", cudaGetErrorString(e));
-    return check_launch("gemv_kernel");
+    *func = reinterpret_cast<const void *>(kern);
+    return WQ_OK;
 }
 
 }  // namespace
 
-// Few-token path (1 <= M <= 16).  Returns WQ_ERR_UNSUPPORTED if no launch plan fits.
-wq_status gemv_small_m(int WB, int AM, const void *A, const float *a_scale, const uint8_t *Wq, const void *scales,
+// Few-token path (1 <= M <= 16) as a prepared launch.  WQ_ERR_UNSUPPORTED if no plan fits.
+wq_status gemv_prepare(int WB, int AM, const void *A, const float *a_scale, const uint8_t *Wq, const void *scales,
                        const void *zeros, const void *bias, void *C, int32_t *acc_out, int64_t M, int64_t N,
-                       int64_t K, const wq_qconfig &c, cudaStream_t st)
+                       int64_t K, const wq_qconfig &c, PreparedLaunch *out)
 {
     const DeviceInfo &dev = device_info();
     const int G = WB == 4 ? int(K / c.group_size) : 1;
@@ -653,18 +644,43 @@ wq_status gemv_small_m(int WB, int AM, const void *A, const float *a_scale, cons
     p.C = C;
     p.acc_out = acc_out;
     const bool one = pl.NT == 1;
+    const void *func = nullptr;
     if (WB == 4 && AM == A_F16)
-        return one ? launch<4, A_F16, 1>(pl, tw, ta, p, st)
-                   : pl.wide ? launch<4, A_F16, 2, false, true>(pl, tw, ta, p, st) : launch<4, A_F16, 2>(pl, tw, ta, p, st);
-    if (WB == 4 && AM == A_BF16)
-        return one ? launch<4, A_BF16, 1>(pl, tw, ta, p, st)
-                   : pl.wide ? launch<4, A_BF16, 2, false, true>(pl, tw, ta, p, st) : launch<4, A_BF16, 2>(pl, tw, ta, p, st);
-    if (WB == 4 && acc_out)
-        return one ? launch<4, A_I8, 1, true>(pl, tw, ta, p, st) : launch<4, A_I8, 2, true>(pl, tw, ta, p, st);
-    if (WB == 4) return one ? launch<4, A_I8, 1>(pl, tw, ta, p, st) : launch<4, A_I8, 2>(pl, tw, ta, p, st);
-    if (AM == A_F16) return launch<2, A_F16, 1>(pl, tw, ta, p, st);
-    if (AM == A_BF16) return launch<2, A_BF16, 1>(pl, tw, ta, p, st);
-    return one ? launch<2, A_I8, 1>(pl, tw, ta, p, st) : launch<2, A_I8, 2>(pl, tw, ta, p, st);
+        rc = one ? kernel_for<4, A_F16, 1>(pl, &func)
+                 : pl.wide ? kernel_for<4, A_F16, 2, false, true>(pl, &func) : kernel_for<4, A_F16, 2>(pl, &func);
+    else if (WB == 4 && AM == A_BF16)
+        rc = one ? kernel_for<4, A_BF16, 1>(pl, &func)
+                 : pl.wide ? kernel_for<4, A_BF16, 2, false, true>(pl, &func) : kernel_for<4, A_BF16, 2>(pl, &func);
+    else if (WB == 4 && acc_out) rc = one ? kernel_for<4, A_I8, 1, true>(pl, &func) : kernel_for<4, A_I8, 2, true>(pl, &func);
+    else if (WB == 4) rc = one ? kernel_for<4, A_I8, 1>(pl, &func) : kernel_for<4, A_I8, 2>(pl, &func);
+    else if (AM == A_F16) rc = kernel_for<2, A_F16, 1>(pl, &func);
+    else if (AM == A_BF16) rc = kernel_for<2, A_BF16, 1>(pl, &func);
+    else rc = one ? kernel_for<2, A_I8, 1>(pl, &func) : kernel_for<2, A_I8, 2>(pl, &func);
+    if (rc != WQ_OK) return rc;
+    static_assert(sizeof(CUtensorMap) == 128 && sizeof(GemvParams) <= 256, "argument layout");
+    out->func = func;
+    out->grid = dim3(pl.P);
+    out->block = dim3(kThreads);
+    out->smem = pl.smem;
+    memcpy(out->args, &tw, sizeof tw);
+    memcpy(out->args + 128, &ta, sizeof ta);
+    memcpy(out->args + 256, &p, sizeof p);
+    out->argp[0] = out->args;
+    out->argp[1] = out->args + 128;
+    out->argp[2] = out->args + 256;
+    out->nargs = 3;
+    return WQ_OK;
+}
+
+// Few-token path (1 <= M <= 16).  Returns WQ_ERR_UNSUPPORTED if no launch plan fits.
+wq_status gemv_small_m(int WB, int AM, const void *A, const float *a_scale, const uint8_t *Wq, const void *scales,
+                       const void *zeros, const void *bias, void *C, int32_t *acc_out, int64_t M, int64_t N,
+                       int64_t K, const wq_qconfig &c, cudaStream_t st)
+{
+    PreparedLaunch L;
+    const wq_status rc = gemv_prepare(WB, AM, A, a_scale, Wq, scales, zeros, bias, C, acc_out, M, N, K, c, &L);
+    if (rc != WQ_OK) return rc;
+    return launch_prepared(L, st, "gemv_kernel");
 }
 
 int gemv_read_error()

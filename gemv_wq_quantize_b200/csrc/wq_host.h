@@ -45,4 +45,36 @@ inline size_t ws_scratch_bytes() { return size_t(device_info().sm_count) * 65536
 // Reads (and clears) the device error words of all kernels with bounded waits.
 int read_device_errors();
 
+// One prepared kernel launch: the kernel, its shape and a copy of its arguments, usable for a
+// direct launch (launch_prepared) or as a CUDA graph kernel node (node_params).
+struct PreparedLaunch {
+    const void *func = nullptr;
+    dim3 grid, block;
+    size_t smem = 0;
+    alignas(64) unsigned char args[512];  // the kernel's arguments, each at its own offset
+    void *argp[4] = {};                   // pointers into args, in parameter order
+    int nargs = 0;
+    cudaKernelNodeParams node_params()
+    {
+        cudaKernelNodeParams k = {};
+        k.func = const_cast<void *>(func);
+        k.gridDim = grid;
+        k.blockDim = block;
+        k.sharedMemBytes = unsigned(smem);
+        k.kernelParams = argp;
+        return k;
+    }
+};
+// Launches it on `st` with programmatic dependent launch allowed.
+wq_status launch_prepared(PreparedLaunch &L, cudaStream_t st, const char *what);
+
+// Argument checks of w4a16_gemm (all but the workspace).
+wq_status check_a16(const void *A, wq_dtype a_dt, const uint8_t *Wq, const void *scales, const void *zeros,
+                    const void *bias, const void *C, int64_t M, int64_t N, int64_t K, const wq_qconfig &c);
+
+// The few-token matmul (M <= 16) as a prepared launch (see gemv_small_m for the arguments).
+wq_status gemv_prepare(int WB, int AM, const void *A, const float *a_scale, const uint8_t *Wq, const void *scales,
+                       const void *zeros, const void *bias, void *C, int32_t *acc_out, int64_t M, int64_t N,
+                       int64_t K, const wq_qconfig &c, PreparedLaunch *out);
+
 }  // namespace wq

@@ -52,6 +52,30 @@ def rel_fro(gpu_bits, ref_bits, dtype) -> float:
     return float(np.linalg.norm(g - r) / den) if den > 0 else float(np.linalg.norm(g))
 
 
+# Largest single-element error, relative to the largest |C_ref|: both sides round once to the
+# output type, so an element may differ by about one unit in its last place plus the fp32
+# summation error; 4 units of the largest element's last place bound it (2^-9 for binary16,
+# 2^-6 for bfloat16).  A wrong row, column or group shows up here even where the Frobenius
+# norm over many correct outputs would average it away.
+MAX_REL = {torch.float16: 2.0 ** -9, torch.bfloat16: 2.0 ** -6}
+
+
+def max_rel(gpu_bits, ref_bits, dtype) -> float:
+    g, r = out_f64(gpu_bits, dtype), out_f64(ref_bits, dtype)
+    den = np.abs(r).max() if r.size else 0.0
+    return float(np.abs(g - r).max() / den) if den > 0 else float(np.abs(g).max() if g.size else 0.0)
+
+
+def assert_close(gpu_bits, ref_bits, dtype):
+    """The FP parity bar: relative Frobenius error <= 1e-3 and no element off by more than
+    MAX_REL of the largest reference output."""
+    assert np.all(np.isfinite(out_f64(gpu_bits, dtype))), "non-finite output"
+    err = rel_fro(gpu_bits, ref_bits, dtype)
+    assert err <= TOL, f"relative Frobenius error {err}"
+    mr = max_rel(gpu_bits, ref_bits, dtype)
+    assert mr <= MAX_REL[dtype], f"largest element error {mr} of max |C_ref|"
+
+
 def qc_of(quant, gs=128):
     if quant == "tern2":
         return wq.QuantConfig(bits=2)
@@ -152,8 +176,7 @@ def test_a16_small_all_outputs(quant, dtype, M, N, K):
     C, A, _, qc, (oWq, os_, oz) = run_a16(M, N, K, quant, dtype, seed=M + N)
     adt = oracle.F16 if dtype == torch.float16 else oracle.BF16
     _, ref = oracle.gemm_a16(bits_np(A), adt, oWq, N, K, qc.bits, qc.symmetric, qc.group_size, os_, oz)
-    err = rel_fro(bits_np(C), ref, dtype)
-    assert err <= TOL, err
+    assert_close(bits_np(C), ref, dtype)
 
 
 @pytest.mark.parametrize("gs", [256, 1024, 2048])
@@ -165,7 +188,7 @@ def test_a16_group_sizes(gs, quant, M):
     N, K = 384, 2048
     C, A, _, qc, (oWq, os_, oz) = run_a16(M, N, K, quant, torch.float16, seed=M + gs, gs=gs)
     _, ref = oracle.gemm_a16(bits_np(A), oracle.F16, oWq, N, K, 4, qc.symmetric, gs, os_, oz)
-    assert rel_fro(bits_np(C), ref, torch.float16) <= TOL
+    assert_close(bits_np(C), ref, torch.float16)
 
 
 @pytest.mark.parametrize("gs", [256, 2048])
@@ -174,7 +197,7 @@ def test_a8_group_sizes(gs, M):
     N, K = 384, 2048
     C, _, qc, (oAq, oasc, oWq, os_, oz), _ = run_a8(M, N, K, "asym4", seed=gs + M, want_acc=False, gs=gs)
     _, ref, _ = oracle.gemm_a8(oAq, oasc, oWq, N, K, 4, False, gs, os_, oz)
-    assert rel_fro(bits_np(C), ref, torch.float16) <= TOL
+    assert_close(bits_np(C), ref, torch.float16)
 
 
 @pytest.mark.parametrize("use_ws", [True, False])
@@ -182,7 +205,7 @@ def test_a16_plans_agree_with_oracle(use_ws):
     M, N, K = 4, 1024, 2048
     C, A, _, qc, (oWq, os_, oz) = run_a16(M, N, K, "asym4", torch.float16, use_ws=use_ws, outliers=0.01)
     _, ref = oracle.gemm_a16(bits_np(A), oracle.F16, oWq, N, K, 4, False, 128, os_, oz)
-    assert rel_fro(bits_np(C), ref, torch.float16) <= TOL
+    assert_close(bits_np(C), ref, torch.float16)
 
 
 @pytest.mark.parametrize("M,N,K,quant", [(1, 24000, 256, "asym4"), (16, 16000, 256, "sym4"), (4, 24000, 320, "tern2"),
@@ -192,7 +215,7 @@ def test_a16_many_tiles_per_cta(M, N, K, quant):
     C, A, _, qc, (oWq, os_, oz) = run_a16(M, N, K, quant, torch.float16, seed=5)
     ni = np.unique(np.concatenate([np.arange(0, N, 37), [N - 1]]))
     _, ref = oracle.gemm_a16(bits_np(A), oracle.F16, oWq, N, K, qc.bits, qc.symmetric, 128, os_, oz, n_idx=ni)
-    assert rel_fro(bits_np(C)[:, ni], ref, torch.float16) <= TOL
+    assert_close(bits_np(C)[:, ni], ref, torch.float16)
 
 
 def test_a16_bias_and_ragged_tail():
@@ -201,7 +224,7 @@ def test_a16_bias_and_ragged_tail():
         KK = K if quant != "tern2" else 1088
         C, A, b, qc, (oWq, os_, oz) = run_a16(M, N, KK, quant, torch.float16, bias=True)
         _, ref = oracle.gemm_a16(bits_np(A), oracle.F16, oWq, N, KK, qc.bits, qc.symmetric, 128, os_, oz, bits_np(b))
-        assert rel_fro(bits_np(C), ref, torch.float16) <= TOL
+        assert_close(bits_np(C), ref, torch.float16)
 
 
 @pytest.mark.parametrize("dtype", [torch.float16, torch.bfloat16])
@@ -212,7 +235,7 @@ def test_a16_bias_and_ragged_tail_tensor_core(dtype, use_ws):
     C, A, b, qc, (oWq, os_, oz) = run_a16(M, N, K, "asym4", dtype, use_ws=use_ws, bias=True, seed=3)
     adt = oracle.F16 if dtype == torch.float16 else oracle.BF16
     _, ref = oracle.gemm_a16(bits_np(A), adt, oWq, N, K, 4, False, 128, os_, oz, bits_np(b))
-    assert rel_fro(bits_np(C), ref, dtype) <= TOL
+    assert_close(bits_np(C), ref, dtype)
 
 
 def test_a16_deterministic():
@@ -272,8 +295,7 @@ def test_a8_small_bit_exact_sums(quant, M, N, K):
     C, acc, qc, (oAq, oasc, oWq, os_, oz), _ = run_a8(M, N, K, quant, seed=M * 7 + N)
     _, ref, oacc = oracle.gemm_a8(oAq, oasc, oWq, N, K, qc.bits, qc.symmetric, 128, os_, oz, want_acc=True)
     assert np.array_equal(acc.cpu().numpy(), oacc)
-    err = rel_fro(bits_np(C), ref, torch.float16)
-    assert err <= TOL, err
+    assert_close(bits_np(C), ref, torch.float16)
 
 
 @pytest.mark.parametrize("quant", ["sym4", "asym4", "tern2"])
@@ -284,8 +306,7 @@ def test_a8_small_without_group_sums(quant, M, N, K):
         K = max(64, K // 64 * 64)
     C, _, qc, (oAq, oasc, oWq, os_, oz), _ = run_a8(M, N, K, quant, seed=M * 5 + N, want_acc=False)
     _, ref, _ = oracle.gemm_a8(oAq, oasc, oWq, N, K, qc.bits, qc.symmetric, 128, os_, oz)
-    err = rel_fro(bits_np(C), ref, torch.float16)
-    assert err <= TOL, err
+    assert_close(bits_np(C), ref, torch.float16)
 
 
 @pytest.mark.parametrize("use_ws", [True, False])
@@ -294,7 +315,7 @@ def test_a8_split_k_plans(use_ws):
     M, N, K = 128, 512, 2048
     C, _, qc, (oAq, oasc, oWq, os_, oz), b = run_a8(M, N, K, "asym4", bias=True, use_ws=use_ws, want_acc=False)
     _, ref, _ = oracle.gemm_a8(oAq, oasc, oWq, N, K, 4, False, 128, os_, oz, bits_np(b))
-    assert rel_fro(bits_np(C), ref, torch.float16) <= TOL
+    assert_close(bits_np(C), ref, torch.float16)
 
 
 @pytest.mark.parametrize("quant,dtype", [("asym4", torch.bfloat16), ("sym4", torch.float16),
@@ -308,8 +329,8 @@ def test_a16_split_k_deterministic_and_matches_unsplit(quant, dtype):
     assert torch.equal(C1, C2)
     adt = oracle.F16 if dtype == torch.float16 else oracle.BF16
     _, ref = oracle.gemm_a16(bits_np(A), adt, oWq, N, K, qc.bits, qc.symmetric, 128, os_, oz)
-    assert rel_fro(bits_np(C1), ref, dtype) <= TOL
-    assert rel_fro(bits_np(C0), ref, dtype) <= TOL
+    assert_close(bits_np(C1), ref, dtype)
+    assert_close(bits_np(C0), ref, dtype)
 
 
 @pytest.mark.parametrize("quant,dtype,M,N,K", [("asym4", torch.float16, 160, 384, 11008),
@@ -321,7 +342,7 @@ def test_a16_long_k_tensor_core(quant, dtype, M, N, K):
     ni = sample_idx(N, 96, 3)
     adt = oracle.F16 if dtype == torch.float16 else oracle.BF16
     _, ref = oracle.gemm_a16(bits_np(A), adt, oWq, N, K, qc.bits, qc.symmetric, 128, os_, oz, n_idx=ni)
-    assert rel_fro(bits_np(C)[:, ni], ref, dtype) <= TOL
+    assert_close(bits_np(C)[:, ni], ref, dtype)
 
 
 def test_a8_long_k_tensor_core():
@@ -329,7 +350,7 @@ def test_a8_long_k_tensor_core():
     M, N, K = 200, 384, 11008
     C, _, qc, (oAq, oasc, oWq, os_, oz), _ = run_a8(M, N, K, "asym4", seed=9, want_acc=False)
     _, ref, _ = oracle.gemm_a8(oAq, oasc, oWq, N, K, 4, False, 128, os_, oz)
-    assert rel_fro(bits_np(C), ref, torch.float16) <= TOL
+    assert_close(bits_np(C), ref, torch.float16)
 
 
 @pytest.mark.parametrize("use_ws", [True, False])
@@ -338,7 +359,7 @@ def test_a8_bias_and_plans(use_ws):
     C, acc, qc, (oAq, oasc, oWq, os_, oz), b = run_a8(M, N, K, "sym4", bias=True, use_ws=use_ws)
     _, ref, oacc = oracle.gemm_a8(oAq, oasc, oWq, N, K, 4, True, 128, os_, None, bits_np(b), want_acc=True)
     assert np.array_equal(acc.cpu().numpy(), oacc)
-    assert rel_fro(bits_np(C), ref, torch.float16) <= TOL
+    assert_close(bits_np(C), ref, torch.float16)
 
 
 # ------------------------------------------------------------------ full-size workloads
@@ -367,7 +388,7 @@ def test_full_size_sampled(case):
         _, ref = oracle.gemm_a16(bits_np(A), adt, oWq, N, K, qc.bits, qc.symmetric, 128, os_, oz,
                                  m_idx=mi, n_idx=ni)
         got = bits_np(C)[np.ix_(mi, ni)]
-        assert rel_fro(got, ref, case.a_dtype) <= TOL
+        assert_close(got, ref, case.a_dtype)
     else:
         Aq, asc = wq.act_quant_int8(A.cuda())
         G = 1 if qc.bits == 2 else K // 128
@@ -378,8 +399,127 @@ def test_full_size_sampled(case):
         _, ref, oacc = oracle.gemm_a8(oAq, oasc, oWq, N, K, qc.bits, qc.symmetric, 128, os_, oz,
                                       m_idx=mi, n_idx=ni, want_acc=True)
         assert np.array_equal(acc.cpu().numpy()[np.ix_(mi, ni)], oacc)
-        assert rel_fro(bits_np(C)[np.ix_(mi, ni)], ref, torch.float16) <= TOL
+        assert_close(bits_np(C)[np.ix_(mi, ni)], ref, torch.float16)
         # and without the group sums (the tcgen05 kernel when M > 16)
         C2 = wq.w4a8_gemm(Aq, asc, Wq, s, z, N, K, qc, workspace=ws)
-        assert rel_fro(bits_np(C2)[np.ix_(mi, ni)], ref, torch.float16) <= TOL
+        assert_close(bits_np(C2)[np.ix_(mi, ni)], ref, torch.float16)
     torch.cuda.synchronize()
+
+
+# ------------------------------------------------------------------ exact ties on the GPU
+# The hand-worked tie fixture (tests/golden/ties.txt) through the CUDA quantizers: the
+# codes, scales and zero points must equal the fixture's round-half-to-even values (and
+# the oracle's), bit for bit.
+import tie_inputs  # noqa: E402
+
+
+def test_ties_sym_int4_gpu():
+    fx = tie_inputs.fields()
+    W, q, _, s_bits = tie_inputs.sym_case(fx)
+    qc = qc_of("sym4")
+    Wq, s, _, _ = quantize_both(torch.from_numpy(W), qc)
+    assert bits_np(s)[0, 0] == s_bits
+    assert np.array_equal(wq.unpack(Wq, 1, 128, qc).cpu().numpy()[0].astype(np.int64), q)
+
+
+def test_ties_asym_int4_gpu():
+    fx = tie_inputs.fields()
+    W, q, s_bits, z_bits, _ = tie_inputs.asym_case(fx)
+    qc = qc_of("asym4")
+    Wq, s, z, _ = quantize_both(torch.from_numpy(W), qc)
+    assert bits_np(s)[0, 0] == s_bits and bits_np(z)[0, 0] == z_bits
+    assert np.array_equal(wq.unpack(Wq, 1, 128, qc).cpu().numpy()[0].astype(np.int64), q)
+
+
+def test_ties_ternary_gpu():
+    fx = tie_inputs.fields()
+    W, q, _, s_bits = tie_inputs.tern_case(fx)
+    qc = qc_of("tern2")
+    Wq, s, _, _ = quantize_both(torch.from_numpy(W), qc)
+    assert s.cpu().numpy().view(np.uint32)[0] == s_bits
+    assert np.array_equal(wq.unpack(Wq, W.shape[0], W.shape[1], qc).cpu().numpy().astype(np.int64), q)
+
+
+@pytest.mark.parametrize("dtype", [torch.float16, torch.bfloat16])
+def test_ties_act_quant_gpu(dtype):
+    fx = tie_inputs.fields()
+    A, q, _, s_bits = tie_inputs.act_case(fx, dtype)
+    Aq, sc = wq.act_quant_int8(A.cuda())
+    assert sc.cpu().numpy().view(np.uint32)[0] == s_bits
+    assert np.array_equal(Aq.cpu().numpy()[0].astype(np.int64), q)
+    oAq, osc = oracle.act_quant_int8(bits_np(A), oracle.F16 if dtype == torch.float16 else oracle.BF16)
+    assert np.array_equal(Aq.cpu().numpy(), oAq) and np.array_equal(sc.cpu().numpy().view(np.uint32),
+                                                                     osc.view(np.uint32))
+
+
+# ------------------------------------------------------------------ INT32 sums on the tcgen05 path
+@pytest.mark.parametrize("quant", ["sym4", "asym4", "tern2"])
+@pytest.mark.parametrize("M,N,K,use_ws", [(128, 512, 2048, True), (128, 512, 2048, False), (200, 333, 1152, True),
+                                          (200, 333, 1152, False), (17, 136, 640, True), (300, 1000, 768, True)])
+def test_a8_tensor_core_group_sums_bit_exact(quant, M, N, K, use_ws):
+    # more than 16 tokens with acc_out: the tcgen05 kind::i8 kernel stores every block's
+    # int32 accumulator (INT4) or the exact per-output total (ternary); with a workspace
+    # and few tiles, K is split over CTAs
+    C, acc, qc, (oAq, oasc, oWq, os_, oz), _ = run_a8(M, N, K, quant, seed=M + N + K, use_ws=use_ws)
+    _, ref, oacc = oracle.gemm_a8(oAq, oasc, oWq, N, K, qc.bits, qc.symmetric, 128, os_, oz, want_acc=True)
+    assert np.array_equal(acc.cpu().numpy(), oacc)
+    assert_close(bits_np(C), ref, torch.float16)
+
+
+# ------------------------------------------------------------------ degenerate inputs through the matmuls
+@pytest.mark.parametrize("M", [5, 16, 160])
+@pytest.mark.parametrize("quant", ["sym4", "asym4", "tern2"])
+def test_a8_zero_token(M, quant):
+    # an all-zero token has a_scale = 0 and Aq = 0: its outputs are exactly 0 (or the bias)
+    N, K = 384, 1024
+    qc = qc_of(quant)
+    W = wq_synth.weights(N, K, seed=41)
+    A = wq_synth.activations(M, K, seed=42, outlier_frac=0.01)
+    A[1] = 0
+    A[M - 1] = 0
+    Wq, s, z, (oWq, os_, oz) = quantize_both(W, qc)
+    Aq, asc = wq.act_quant_int8(A.cuda())
+    assert float(asc[1]) == 0.0 and int(Aq[1].abs().max()) == 0
+    G = 1 if qc.bits == 2 else K // 128
+    acc = torch.full((M, N, G), 7, dtype=torch.int32, device="cuda")
+    C = wq.w4a8_gemm(Aq, asc, Wq, s, z, N, K, qc, acc_out=acc, workspace=workspace(M, N, K, qc))
+    torch.cuda.synchronize()
+    oAq, oasc = oracle.act_quant_int8(bits_np(A), oracle.F16)
+    _, ref, oacc = oracle.gemm_a8(oAq, oasc, oWq, N, K, qc.bits, qc.symmetric, 128, os_, oz, want_acc=True)
+    assert np.array_equal(acc.cpu().numpy(), oacc)
+    Cb = bits_np(C)
+    assert np.all(Cb[1] == 0) and np.all(Cb[M - 1] == 0)
+    assert_close(Cb, ref, torch.float16)
+
+
+@pytest.mark.parametrize("M", [1, 9, 64, 256])
+@pytest.mark.parametrize("quant", ["sym4", "asym4"])
+@pytest.mark.parametrize("mode", ["a16", "a8"])
+def test_zero_scale_groups(M, quant, mode):
+    # weight groups that are all zero quantize to scale 0 (asymmetric: zero point 0 too);
+    # through both matmul kernels they must contribute exactly nothing
+    N, K = 272, 1024
+    qc = qc_of(quant)
+    W = wq_synth.weights(N, K, seed=43)
+    W[:, 256:384] = 0            # one whole group column
+    W[5, :] = 0                  # one whole row: every group of it
+    W[100, 640:768] = 0
+    Wq, s, z, (oWq, os_, oz) = quantize_both(W, qc)
+    assert np.all(os_[:, 2] == 0) and np.all(os_[5] == 0)
+    A = wq_synth.activations(M, K, seed=44, outlier_frac=0.01)
+    ws = workspace(M, N, K, qc)
+    if mode == "a16":
+        C = wq.w4a16_gemm(A.cuda(), Wq, s, z, N, K, qc, workspace=ws)
+        torch.cuda.synchronize()
+        _, ref = oracle.gemm_a16(bits_np(A), oracle.F16, oWq, N, K, 4, qc.symmetric, 128, os_, oz)
+    else:
+        Aq, asc = wq.act_quant_int8(A.cuda())
+        acc = torch.zeros(M, N, K // 128, dtype=torch.int32, device="cuda")
+        C = wq.w4a8_gemm(Aq, asc, Wq, s, z, N, K, qc, acc_out=acc, workspace=ws)
+        torch.cuda.synchronize()
+        oAq, oasc = oracle.act_quant_int8(bits_np(A), oracle.F16)
+        _, ref, oacc = oracle.gemm_a8(oAq, oasc, oWq, N, K, 4, qc.symmetric, 128, os_, oz, want_acc=True)
+        assert np.array_equal(acc.cpu().numpy(), oacc)
+    Cb = bits_np(C)
+    assert np.all(Cb[:, 5] == 0)
+    assert_close(Cb, ref, torch.float16)
