@@ -71,10 +71,13 @@ def flops(c: wq_synth.Case) -> int:
     return 2 * c.M * c.N * c.K
 
 
-def launches_per_call(c: wq_synth.Case) -> int:
+def launches_per_call(c: wq_synth.Case, fused: bool = True) -> int:
     """Kernels one step launches for the case: the matmul, plus the per-token activation
-    quantization on the INT8 paths."""
-    return 2 if c.mode == "a8" else 1
+    quantization on the INT8 paths, which for small activations (M <= 16, M*K <= 16384) runs
+    inside the matmul kernel (w4a8_gemm_fused) and otherwise as a kernel of its own."""
+    if c.mode != "a8":
+        return 1
+    return 1 if (fused and c.M <= 16 and c.M * c.K <= 16384) else 2
 
 
 def peaks():
@@ -185,14 +188,20 @@ class ClockSampler:
 class Prepared:
     """Quantized weight copies, activations and outputs of one case on the device."""
 
-    def __init__(self, c: wq_synth.Case, device, seed_base: int = 0, copies: int = 0):
+    def __init__(self, c: wq_synth.Case, device, seed_base: int = 0, copies: int = 0, fused: bool = True,
+                 native: bool = False):
+        import dataclasses
         import gemv_wq_quantize_b200 as wq
         self.c = c
+        self.fused = fused
         self.qc = wq.QuantConfig(bits=2) if c.quant == "tern2" else \
             wq.QuantConfig(bits=4, group_size=c.group_size, symmetric=(c.quant == "sym4"))
         W = wq_synth.weights(c.N, c.K, seed=seed_base).to(device)
         Wq, s, z = wq.quantize_pack(W, self.qc)
         del W
+        if native:  # the kernel-native copy of the same weights
+            Wq = wq.repack(Wq, c.N, c.K, self.qc)
+            self.qc = dataclasses.replace(self.qc, layout=wq.LAYOUT_NATIVE)
         self.bytes = alg_bytes(c)
         copies = copies or max(2, math.ceil(4 * L2_BYTES / self.bytes))
         self.weights = [(Wq, s, z)] + [(Wq.clone(), s.clone(), None if z is None else z.clone())
@@ -215,8 +224,12 @@ class Prepared:
         A, C = (self.A_slots[slot], self.C_slots[slot]) if e2e else (self.A, self.C)
         if c.mode == "a16":
             wq.w4a16_gemm(A, Wq, s, z, c.N, c.K, self.qc, out=C, workspace=self.ws)
+        elif self.fused:
+            # the INT8 path starts from the fp16 activations: every step quantizes them per token,
+            # inside the matmul where the few-token kernel allows it
+            wq.w4a8_gemm_fused(A, Wq, s, z, c.N, c.K, self.qc, out=C, out_q=self.Aq, out_scale=self.a_scale,
+                               workspace=self.ws)
         else:
-            # the INT8 path starts from the fp16 activations: every step quantizes them per token
             wq.act_quant_int8(A, out_q=self.Aq, out_scale=self.a_scale)
             wq.w4a8_gemm(self.Aq, self.a_scale, Wq, s, z, c.N, c.K, self.qc, out=C, workspace=self.ws)
 
@@ -434,6 +447,13 @@ def measure_extra(name: str, device, steps: int, warmup: int, dist_on: bool) -> 
                            "frac": round(gbs / pk["hbm_gbs"], 4), "traffic": recorded_traffic(name),
                            "peak_source": pk["source"]}
     out["cases"] = cases
+    if any(p.c.mode == "a8" for p in preps):
+        # the same INT8 cases with the activation quantization as a kernel of its own
+        for p in preps:
+            p.fused = False
+        run_steps(preps, 1, False)
+        torch.cuda.synchronize()
+        out["cases_two_launches"] = [c for c, p in zip(per_case_breakdown(preps), preps) if p.c.mode == "a8"]
     del preps
     torch.cuda.empty_cache()
     return out
@@ -443,11 +463,11 @@ LLAMA7B_LAYER = (("qkv", 12288, 4096), ("o", 4096, 4096), ("gate_up", 22016, 409
 
 
 def measure_layer_graph(device, M: int = 1, reps: int = 50) -> dict:
-    """One Llama-7B layer's four decode projections (asymmetric INT4, group 128, fp16) run as
-    one wq_graph per layer, over enough layer copies (6 x 101 MB) that every launch streams
-    its weights from HBM.  Reported per layer step: the graph (one launch per layer), the
-    same four kernels captured by stream capture (device time of the kernels alone), and
-    four direct C-ABI calls per layer issued from this Python process (host-bound)."""
+    """One Llama-7B layer's four decode projections (asymmetric INT4, group 128, fp16) over
+    enough layer copies (6 x 107 MB) that every launch streams its weights from HBM, run as one
+    wq_graph (built once; one launch per pass over the layers).  Reported per layer: the
+    wq_graph, the same kernels captured by torch stream capture, and four direct C-ABI calls
+    per layer issued from this Python process."""
     import gemv_wq_quantize_b200 as wq
     qc = wq.QuantConfig(4, 128, False)
     base = []
@@ -460,8 +480,9 @@ def measure_layer_graph(device, M: int = 1, reps: int = 50) -> dict:
     nlayers = max(2, math.ceil(4 * L2_BYTES / layer_bytes) + 1)
     layers = [[(name, N, K, Wq.clone(), s.clone(), z.clone(), A, C) for name, N, K, Wq, s, z, A, C in base]
               for _ in range(nlayers)]
-    graphs = [wq.DecodeGraph([{"A": A, "Wq": Wq, "scales": s, "zeros": z, "N": N, "K": K, "qc": qc, "out": C}
-                              for _, N, K, Wq, s, z, A, C in layer]) for layer in layers]
+    # one graph over all layer copies (a decode step runs its layers back to back)
+    graph = wq.DecodeGraph([{"A": A, "Wq": Wq, "scales": s, "zeros": z, "N": N, "K": K, "qc": qc, "out": C}
+                            for layer in layers for _, N, K, Wq, s, z, A, C in layer])
 
     def calls():
         for layer in layers:
@@ -480,25 +501,46 @@ def measure_layer_graph(device, M: int = 1, reps: int = 50) -> dict:
         torch.cuda.synchronize()
         return t0.elapsed_time(t1) * 1e3 / (n * nlayers)
 
-    def graph_steps():
-        for g in graphs:
-            g.launch()
+    us_graph = timed(graph.launch, reps)
 
-    us_graph = timed(graph_steps, reps)
+    def host_us(fn, n):  # host time to enqueue one pass (no synchronisation inside)
+        torch.cuda.synchronize()
+        t = time.perf_counter()
+        for _ in range(n):
+            fn()
+        dt = time.perf_counter() - t
+        torch.cuda.synchronize()
+        return dt * 1e6 / (n * nlayers)
+
+    host_graph = host_us(graph.launch, 20)
+    host_calls = host_us(calls, 5)
     cap = torch.cuda.CUDAGraph()
     with torch.cuda.graph(cap):
         calls()
     us_captured = timed(cap.replay, reps)
     us_calls = timed(calls, max(5, reps // 5))
-    for g in graphs:
-        g.close()
+    graph.close()
     assert wq.device_error() == 0, "a kernel gave up a bounded wait"
     pk = peaks()
     return {"ops": [f"{n}:{N}x{K}" for n, N, K in LLAMA7B_LAYER], "M": M, "layer_copies": nlayers,
             "bytes_per_layer": layer_bytes, "us_per_layer_graph": round(us_graph, 3),
             "us_per_layer_stream_captured": round(us_captured, 3), "us_per_layer_direct_calls": round(us_calls, 3),
+            "host_us_per_layer_graph": round(host_graph, 3), "host_us_per_layer_direct_calls": round(host_calls, 3),
             "GB/s_graph": round(layer_bytes / (us_graph * 1e-6) / 1e9, 1),
             "hbm_frac_graph": round(layer_bytes / (us_graph * 1e-6) / 1e9 / pk["hbm_gbs"], 4)}
+
+
+def measure_native(name: str, device) -> list:
+    """Per-case times of a workload's INT4 cases with the weights in the kernel-native order
+    (wq_repack), to set beside the same cases on the "nt" packing."""
+    wl = wq_synth.WORKLOADS[name]
+    preps = [Prepared(c, device, seed_base=0, native=True) for c in wl.cases if c.quant != "tern2"]
+    run_steps(preps, 1, False)
+    torch.cuda.synchronize()
+    out = per_case_breakdown(preps)
+    del preps
+    torch.cuda.empty_cache()
+    return out
 
 
 def run_ours(args, rank, world, local_rank, dist_on):
@@ -559,6 +601,9 @@ def run_ours(args, rank, world, local_rank, dist_on):
         for key, name in EXTRA_WORKLOADS:
             result[key] = measure_extra(name, device, min(args.steps, 2000), args.warmup, dist_on)
         result["decode_layer_graph"] = measure_layer_graph(device)
+        result["native_layout"] = {"note": "the same cases with the weights repacked into the kernel-native order",
+                                   "decode-llama7b": measure_native("decode-llama7b", device),
+                                   "prefill-llama7b": measure_native("prefill-llama7b", device)}
     return result
 
 

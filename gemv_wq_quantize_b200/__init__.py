@@ -27,7 +27,9 @@ WQ_OK, WQ_ERR_INVALID_ARG, WQ_ERR_ALIGNMENT, WQ_ERR_UNSUPPORTED, WQ_ERR_CUDA, WQ
 WQ_F32, WQ_F16, WQ_BF16, WQ_I8, WQ_I32 = range(5)
 
 EXPORTED = ("wq_quantize_pack", "wq_quantize_workspace_size", "wq_unpack", "act_quant_int8", "w4a16_gemm",
-            "w4a16_gemm_noalloc", "w4a8_gemm", "wq_workspace_size", "wq_status_string", "wq_last_error")
+            "w4a16_gemm_noalloc", "w4a8_gemm", "wq_workspace_size", "wq_status_string", "wq_last_error",
+            "wq_graph_create", "wq_graph_set_io", "wq_graph_launch", "wq_graph_destroy", "w4a8_gemm_fused",
+            "wq_repack")
 
 
 class WqError(RuntimeError):
@@ -38,18 +40,31 @@ class WqError(RuntimeError):
 
 class QConfig(ctypes.Structure):
     _fields_ = [("bits", ctypes.c_int32), ("group_size", ctypes.c_int32), ("symmetric", ctypes.c_int32),
-                ("ternary", ctypes.c_int32)]
+                ("ternary", ctypes.c_int32), ("layout", ctypes.c_int32)]
+
+
+LAYOUT_NT, LAYOUT_NATIVE = 0, 1
 
 
 @dataclass(frozen=True)
 class QuantConfig:
-    """bits 4 (group scales, optional zero points) or 2 (ternary, one scale per tensor)."""
+    """bits 4 (group scales, optional zero points) or 2 (ternary, one scale per tensor);
+    layout LAYOUT_NT (the packing of wq_quantize_pack) or LAYOUT_NATIVE (after repack)."""
     bits: int = 4
     group_size: int = 128
     symmetric: bool = True
+    layout: int = LAYOUT_NT
 
     def c(self) -> QConfig:
-        return QConfig(self.bits, self.group_size, int(self.symmetric), int(self.bits == 2))
+        return QConfig(self.bits, self.group_size, int(self.symmetric), int(self.bits == 2), self.layout)
+
+
+class MatmulDesc(ctypes.Structure):
+    """wq_matmul_desc: the arguments of one w4a16_gemm of a wq_graph chain."""
+    _fields_ = [("A", ctypes.c_void_p), ("a_dt", ctypes.c_int), ("Wq", ctypes.c_void_p),
+                ("scales", ctypes.c_void_p), ("zeros", ctypes.c_void_p), ("bias", ctypes.c_void_p),
+                ("C", ctypes.c_void_p), ("M", ctypes.c_int64), ("N", ctypes.c_int64), ("K", ctypes.c_int64),
+                ("c", QConfig)]
 
 
 _lib = None
@@ -70,6 +85,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.wq_quantize_workspace_size.argtypes = [i64, i64, QConfig]
     lib.wq_quantize_workspace_size.restype = sz
     lib.wq_unpack.argtypes = [vp, i64, i64, QConfig, vp, vp]
+    lib.wq_repack.argtypes = [vp, i64, i64, QConfig, vp, vp]
+    lib.wq_repack.restype = st
     lib.wq_unpack.restype = st
     lib.act_quant_int8.argtypes = [vp, st, i64, i64, vp, vp, vp]
     lib.act_quant_int8.restype = st
@@ -79,6 +96,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.w4a16_gemm_noalloc.restype = st
     lib.w4a8_gemm.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, QConfig, vp, sz, vp]
     lib.w4a8_gemm.restype = st
+    lib.w4a8_gemm_fused.argtypes = [vp, st, vp, vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, QConfig, vp, sz, vp]
+    lib.w4a8_gemm_fused.restype = st
     lib.wq_workspace_size.argtypes = [i64, i64, i64, QConfig]
     lib.wq_workspace_size.restype = sz
     lib.wq_status_string.argtypes = [st]
@@ -87,6 +106,14 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.wq_last_error.restype = ctypes.c_char_p
     lib.wq_device_error.argtypes = []
     lib.wq_device_error.restype = ctypes.c_int
+    lib.wq_graph_create.argtypes = [ctypes.POINTER(MatmulDesc), ctypes.c_int, ctypes.POINTER(ctypes.c_void_p)]
+    lib.wq_graph_create.restype = st
+    lib.wq_graph_set_io.argtypes = [vp, ctypes.c_int, vp, vp]
+    lib.wq_graph_set_io.restype = st
+    lib.wq_graph_launch.argtypes = [vp, vp]
+    lib.wq_graph_launch.restype = st
+    lib.wq_graph_destroy.argtypes = [vp]
+    lib.wq_graph_destroy.restype = None
     _lib = lib
     return lib
 
@@ -158,6 +185,15 @@ def unpack(Wq: torch.Tensor, N: int, K: int, qc: QuantConfig, stream=None) -> to
     return q
 
 
+def repack(Wq: torch.Tensor, N: int, K: int, qc: QuantConfig, out=None, stream=None) -> torch.Tensor:
+    """The kernel-native copy of packed INT4 weights (use it with ``dataclasses.replace(qc,
+    layout=LAYOUT_NATIVE)``); scales and zero points are unchanged."""
+    _dev(Wq, "Wq")
+    o = out if out is not None else torch.empty_like(Wq)
+    _check(load_library().wq_repack(_ptr(Wq), N, K, qc.c(), _ptr(o), _stream(stream)), "wq_repack")
+    return o
+
+
 def act_quant_int8(A: torch.Tensor, out_q=None, out_scale=None, stream=None):
     """Per-token INT8 quantization of A [M,K] fp16/bf16 -> (Aq int8 [M,K], a_scale fp32 [M])."""
     _dev(A, "A")
@@ -217,6 +253,78 @@ def w4a8_gemm(Aq, a_scale, Wq, scales, zeros, N: int, K: int, qc: QuantConfig, b
                                   _ptr(acc_out), M, N, K, qc.c(), _ptr(workspace), wsb, _stream(stream))
     _check(rc, "w4a8_gemm")
     return C
+
+
+class DecodeGraph:
+    """A chain of few-token W4A16 matmuls (for example one layer's QKV, output, gate/up and
+    down projections at decode time) run as one CUDA graph (wq_graph_create).
+
+    ``ops`` is a list of dicts with the keys of :func:`w4a16_gemm`: ``A``, ``Wq``,
+    ``scales``, ``zeros``, ``N``, ``K``, ``qc``, ``out`` (required: the graph writes into
+    it) and optionally ``bias``.  The graph keeps the tensors' device pointers: keep them
+    alive until :meth:`close`.  :meth:`set_io` points one matmul at new activation /
+    output tensors (same shapes) for the following launches; :meth:`launch` runs the chain.
+    """
+
+    def __init__(self, ops):
+        self._keep = []
+        descs = (MatmulDesc * len(ops))()
+        for d, op in zip(descs, ops):
+            A, C = op["A"], op["out"]
+            for t, n in ((A, "A"), (op["Wq"], "Wq"), (op["scales"], "scales"), (op.get("zeros"), "zeros"),
+                         (op.get("bias"), "bias"), (C, "out")):
+                _dev(t, n)
+            d.A, d.a_dt, d.Wq = A.data_ptr(), _DT[A.dtype], op["Wq"].data_ptr()
+            d.scales = op["scales"].data_ptr()
+            d.zeros = None if op.get("zeros") is None else op["zeros"].data_ptr()
+            d.bias = None if op.get("bias") is None else op["bias"].data_ptr()
+            d.C, d.M, d.N, d.K, d.c = C.data_ptr(), A.shape[0], op["N"], op["K"], op["qc"].c()
+            self._keep.append(op)
+        h = ctypes.c_void_p()
+        _check(load_library().wq_graph_create(descs, len(ops), ctypes.byref(h)), "wq_graph_create")
+        self._h = h
+
+    def set_io(self, i: int, A, out):
+        _dev(A, "A")
+        _dev(out, "out")
+        _check(load_library().wq_graph_set_io(self._h, i, _ptr(A), _ptr(out)), "wq_graph_set_io")
+        self._keep[i] = dict(self._keep[i], A=A, out=out)
+
+    def launch(self, stream=None):
+        _check(load_library().wq_graph_launch(self._h, _stream(stream)), "wq_graph_launch")
+
+    def close(self):
+        if getattr(self, "_h", None):
+            load_library().wq_graph_destroy(self._h)
+            self._h = None
+            self._keep = []
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def w4a8_gemm_fused(A, Wq, scales, zeros, N: int, K: int, qc: QuantConfig, bias=None, out=None, out_q=None,
+                    out_scale=None, acc_out=None, workspace=None, stream=None):
+    """W4A8 from fp16/bf16 activations with the per-token INT8 quantization fused in.
+
+    Returns (C fp16 [M,N], Aq int8 [M,K], a_scale fp32 [M]); bit-identical to
+    ``act_quant_int8`` followed by ``w4a8_gemm``."""
+    for t, n in ((A, "A"), (Wq, "Wq"), (scales, "scales"), (zeros, "zeros"), (bias, "bias"), (out, "out"),
+                 (out_q, "out_q"), (out_scale, "out_scale"), (acc_out, "acc_out")):
+        _dev(t, n)
+    M = A.shape[0]
+    C = out if out is not None else torch.empty(M, N, dtype=torch.float16, device=A.device)
+    Aq = out_q if out_q is not None else torch.empty(M, K, dtype=torch.int8, device=A.device)
+    sc = out_scale if out_scale is not None else torch.empty(M, dtype=torch.float32, device=A.device)
+    wsb = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    rc = load_library().w4a8_gemm_fused(_ptr(A), _DT[A.dtype], _ptr(Wq), _ptr(scales), _ptr(zeros), _ptr(bias),
+                                        _ptr(C), _ptr(Aq), _ptr(sc), _ptr(acc_out), M, N, K, qc.c(), _ptr(workspace),
+                                        wsb, _stream(stream))
+    _check(rc, "w4a8_gemm_fused")
+    return C, Aq, sc
 
 
 def device_error() -> int:

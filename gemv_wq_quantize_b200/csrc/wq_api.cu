@@ -164,6 +164,9 @@ wq_status dispatch(int WB, int AM, const void *A, const float *a_scale, const ui
         wq_status rc = tc_gemm(WB, AM, A, a_scale, Wq, scales, zeros, bias, C, acc_out, M, N, K, c, ws, ws_bytes, st);
         if (rc != WQ_ERR_UNSUPPORTED) return rc;
     }
+    if (c.layout == WQ_LAYOUT_NATIVE)
+        return fail(WQ_ERR_UNSUPPORTED, "native layout: no launch plan for M=%lld K=%lld (use WQ_LAYOUT_NT)",
+                    (long long)M, (long long)K);
     return skinny_gemm(WB, AM, A, a_scale, Wq, scales, zeros, bias, C, acc_out, M, N, K, c, ws, ws_bytes, st);
 }
 }  // namespace
@@ -178,6 +181,8 @@ wq_status check_weights(const uint8_t *Wq, const void *scales, const void *zeros
     if (!Wq || !scales) return fail(WQ_ERR_INVALID_ARG, "Wq and scales must be non-null");
     if (!aligned16(Wq) || !aligned16(scales) || (zeros && !aligned16(zeros)))
         return fail(WQ_ERR_ALIGNMENT, "Wq, scales and zeros must be 16-byte aligned");
+    if (c.layout != WQ_LAYOUT_NT && c.layout != WQ_LAYOUT_NATIVE) return fail(WQ_ERR_INVALID_ARG, "unknown layout");
+    if (c.layout == WQ_LAYOUT_NATIVE && c.bits != 4) return fail(WQ_ERR_UNSUPPORTED, "the native layout is INT4 only");
     if (c.bits == 4) {
         if (K % 128) return fail(WQ_ERR_INVALID_ARG, "INT4 needs K %% 128 == 0");
         if (c.group_size <= 0 || K % c.group_size) return fail(WQ_ERR_INVALID_ARG, "K %% group_size != 0");
@@ -248,6 +253,39 @@ extern "C" wq_status w4a16_gemm(const void *A, wq_dtype a_dt, const uint8_t *Wq,
     if (workspace && !aligned16(workspace)) return fail(WQ_ERR_ALIGNMENT, "workspace must be 16-byte aligned");
     return dispatch(c.bits, a_dt == WQ_F16 ? 0 : 1, A, nullptr, Wq, scales, c.bits == 4 && !c.symmetric ? zeros : nullptr,
                        bias, C, nullptr, M, N, K, c, workspace, ws_bytes, stream);
+}
+
+// W4A8 from FP activations: the per-token INT8 quantization inside the few-token matmul
+// when the activations are small and its launch plan stages them whole, else
+// act_quant_int8 then w4a8_gemm.
+constexpr int64_t kFusedMaxElems = 16384;
+extern "C" wq_status w4a8_gemm_fused(const void *A, wq_dtype a_dt, const uint8_t *Wq, const void *scales,
+                                     const void *zeros, const void *bias, void *C, int8_t *Aq, float *a_scale,
+                                     int32_t *acc_out, int64_t M, int64_t N, int64_t K, wq_qconfig c, void *workspace,
+                                     size_t ws_bytes, cudaStream_t stream)
+{
+    wq_status rc = check_weights(Wq, scales, zeros, M, N, K, c);
+    if (rc != WQ_OK) return rc;
+    if (a_dt != WQ_F16 && a_dt != WQ_BF16) return fail(WQ_ERR_INVALID_ARG, "a_dt must be WQ_F16 or WQ_BF16");
+    if (!A || !C || !Aq || !a_scale) return fail(WQ_ERR_INVALID_ARG, "A, C, Aq and a_scale must be non-null");
+    if (!aligned16(A) || !aligned16(Aq) || !aligned16(C) || (bias && !aligned16(bias)) ||
+        (workspace && !aligned16(workspace)))
+        return fail(WQ_ERR_ALIGNMENT, "A, Aq, C, bias and workspace must be 16-byte aligned");
+    if (acc_out && c.bits == 4 && c.group_size != 128)
+        return fail(WQ_ERR_UNSUPPORTED, "acc_out needs group_size == 128");
+    // Every CTA of the fused kernel reads all of A twice from L2 (maximum, then codes): worth it
+    // while A is small; beyond that the separate quantization kernel is faster.
+    if (M <= 16 && M * K <= kFusedMaxElems) {
+        const FusedActQuant fa{A, a_dt == WQ_BF16, Aq, a_scale};
+        PreparedLaunch L;
+        rc = gemv_prepare(c.bits, 2, Aq, a_scale, Wq, scales, c.bits == 4 && !c.symmetric ? zeros : nullptr, bias, C,
+                          acc_out, M, N, K, c, &L, &fa);
+        if (rc == WQ_OK) return launch_prepared(L, stream, "gemv_kernel");
+        if (rc != WQ_ERR_UNSUPPORTED) return rc;
+    }
+    rc = act_quant_int8(A, a_dt, M, K, Aq, a_scale, stream);
+    if (rc != WQ_OK) return rc;
+    return w4a8_gemm(Aq, a_scale, Wq, scales, zeros, bias, C, acc_out, M, N, K, c, workspace, ws_bytes, stream);
 }
 
 extern "C" wq_status w4a8_gemm(const int8_t *Aq, const float *a_scale, const uint8_t *Wq, const void *scales,

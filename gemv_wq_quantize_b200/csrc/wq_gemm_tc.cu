@@ -85,6 +85,7 @@ struct TcParams {
     const void *bias;
     void *C;
     int32_t *acc_out;  // ACC: INT32 group sums [M][N][G] (INT4, group 128) or totals [M][N] (INT2)
+    int nat;           // INT4 weights in the kernel-native order
 };
 
 __device__ __forceinline__ uint64_t globaltimer()
@@ -184,6 +185,37 @@ __device__ __forceinline__ void unpack_word(uint32_t w, uint32_t zc, uint32_t *o
 // with group_size 128 a block of 128 k is one group, so each block accumulator read from
 // Tensor Memory is one acc_g (the zero point is already inside the weight bytes); for
 // ternary INT2 the fp32 totals are exact integers (|sum| < 2^24) and are stored at the end.
+// Kernel-native INT4 order (nibble i of a word = element 0,2,4,6,1,3,5,7): the masks give the
+// natural pairs directly.  f16: (x & 0x000F000F) | magic = 1024 + q of (k, k+1);
+// (x & 0x00F000F0) | magic = 1024 + 16 q of (k+2, k+3), made q - z by one fma with 1/16;
+// the upper byte the same after one shift.  bf16 has 7 mantissa bits, so its odd pairs are
+// shifted into place instead of scaled.
+template <bool BF16>
+__device__ __forceinline__ void unpack_word_nat(uint32_t w, uint32_t z, uint32_t *o)
+{
+    if constexpr (BF16) {
+        const uint32_t c1 = 0xC300u | z, cc = c1 | (c1 << 16);  // -(128 + z)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) o[i] = bf2_fma(and_or(w >> (4 * i), 0x000F000Fu, 0x43004300u), 0x3F803F80u, cc);
+    } else {
+        const uint32_t a1 = 0xE400u | z, clo = a1 | (a1 << 16);                // -(1024 + z)
+        const uint32_t b1 = 0xD400u | (z << 4), chi = b1 | (b1 << 16);         // -(64 + z)
+        const uint32_t w8 = w >> 8;
+        o[0] = h2_add(and_or(w, 0x000F000Fu, 0x64006400u), clo);
+        o[1] = h2_fma(and_or(w, 0x00F000F0u, 0x64006400u), 0x2C002C00u, chi);
+        o[2] = h2_add(and_or(w8, 0x000F000Fu, 0x64006400u), clo);
+        o[3] = h2_fma(and_or(w8, 0x00F000F0u, 0x64006400u), 0x2C002C00u, chi);
+    }
+}
+
+// Kernel-native INT4, INT8 activations: one word -> 8 signed bytes q - z in natural k order.
+__device__ __forceinline__ void unpack_word_s8_nat(uint32_t w, uint32_t zc, uint32_t *o)
+{
+    const uint32_t lo = w & 0x0F0F0F0Fu, hi = (w >> 4) & 0x0F0F0F0Fu;  // k0 k4 k1 k5 / k2 k6 k3 k7
+    o[0] = (prmt(lo, hi, 0x6420) + zc) ^ 0x80808080u;  // k0 k1 k2 k3
+    o[1] = (prmt(lo, hi, 0x7531) + zc) ^ 0x80808080u;  // k4 .. k7
+}
+
 template <int WB, int AM, bool ACC = false>
 __global__ void __launch_bounds__(kThreads, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_w,
@@ -408,27 +440,27 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if constexpr (I8) {
                         const uint32_t zc = (0x80u - z) * 0x01010101u;
                         uint32_t v[16];
-                        unpack_word_s8(w0.x, zc, v + 0);
-                        unpack_word_s8(w0.y, zc, v + 2);
-                        unpack_word_s8(w0.z, zc, v + 4);
-                        unpack_word_s8(w0.w, zc, v + 6);
-                        unpack_word_s8(w1.x, zc, v + 8);
-                        unpack_word_s8(w1.y, zc, v + 10);
-                        unpack_word_s8(w1.z, zc, v + 12);
-                        unpack_word_s8(w1.w, zc, v + 14);
+                        const uint32_t wd[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+                        if (p.nat) {
+#pragma unroll
+                            for (int i = 0; i < 8; ++i) unpack_word_s8_nat(wd[i], zc, v + 2 * i);
+                        } else {
+#pragma unroll
+                            for (int i = 0; i < 8; ++i) unpack_word_s8(wd[i], zc, v + 2 * i);
+                        }
                         tc::st_32x32b_x16(tlane + kAcol + s * 64 + kh * 16, v);
                     } else {
                         const uint32_t zc1 = magic_z | z;
                         const uint32_t zc = zc1 | (zc1 << 16);
                         uint32_t v[32];
-                        unpack_word<BF16>(w0.x, zc, v + 0);
-                        unpack_word<BF16>(w0.y, zc, v + 4);
-                        unpack_word<BF16>(w0.z, zc, v + 8);
-                        unpack_word<BF16>(w0.w, zc, v + 12);
-                        unpack_word<BF16>(w1.x, zc, v + 16);
-                        unpack_word<BF16>(w1.y, zc, v + 20);
-                        unpack_word<BF16>(w1.z, zc, v + 24);
-                        unpack_word<BF16>(w1.w, zc, v + 28);
+                        const uint32_t wd[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+                        if (p.nat) {
+#pragma unroll
+                            for (int i = 0; i < 8; ++i) unpack_word_nat<BF16>(wd[i], z, v + 4 * i);
+                        } else {
+#pragma unroll
+                            for (int i = 0; i < 8; ++i) unpack_word<BF16>(wd[i], zc, v + 4 * i);
+                        }
                         tc::st_32x32b_x32(tlane + kAcol + s * 64 + kh * 32, v);
                     }
                 } else {
@@ -777,6 +809,7 @@ wq_status tc_gemm(int WB, int AM, const void *A, const float *a_scale, const uin
     p.bias = bias;
     p.C = C;
     p.acc_out = acc_out;
+    p.nat = WB == 4 && c.layout == WQ_LAYOUT_NATIVE;
     const int grid = std::min(dev.sm_count, p.NT * p.ks);
     if (WB == 4) {
         if (AM == 0) return launch<4, 0>(pl, ta, tw, p, grid, st);

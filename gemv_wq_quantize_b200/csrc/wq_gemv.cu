@@ -82,6 +82,13 @@ struct GemvParams {
     const float *a_scale;
     void *C;
     int32_t *acc_out;
+    // fused per-token INT8 quantization of FP activations (FS != 0): source, outputs and
+    // the shared-memory offset of the tokens' scales and their reciprocals
+    const void *A_src;
+    int8_t *Aq_out;
+    float *a_scale_out;
+    int fs_off;
+    int nat;  // INT4 weights in the kernel-native order
 };
 
 __device__ __forceinline__ uint64_t globaltimer()
@@ -122,11 +129,10 @@ __device__ __forceinline__ float bias_at(const void *bias, int n)
 }
 
 template <int WB, int AM>
-__device__ __forceinline__ float finish(const GemvParams &p, float total_f, int total_i, int n, int m)
+__device__ __forceinline__ float finish(const GemvParams &p, float total_f, int total_i, int n, float as)
 {
     float v;
     if constexpr (AM == A_I8) {
-        const float as = p.a_scale[m];
         v = (WB == 2) ? as * (p.scale32[0] * float(total_i)) : as * total_f;
     } else {
         v = (WB == 2) ? p.scale32[0] * total_f : total_f;
@@ -134,12 +140,39 @@ __device__ __forceinline__ float finish(const GemvParams &p, float total_f, int 
     return v + bias_at<AM>(p.bias, n);
 }
 
+// Per-token INT8 code of one activation, exactly clip(rint(a / s), -127, 127) with the IEEE
+// binary32 quotient ("Accelerating LLM inference with CUDA Graph and INT4 quantization",
+// part 1, step 2), without a division per element: y = a * r with r the correctly rounded
+// 1/s is within |a/s| * 2^-23 <= 1.6e-5 of a/s, and the correctly rounded quotient within
+// 2^-18 of it, so both round to the same integer unless a/s lies within 2^-12 of a tie
+// (k + 1/2); only there is the quotient formed by division.
+__device__ __forceinline__ int quant_i8(float a, float s, float r)
+{
+    if (s == 0.f) return 0;
+    const float y = a * r;
+    float k = rintf(y);
+    if (fabsf(fabsf(y - k) - 0.5f) < 0x1p-12f) k = rintf(__fdiv_rn(a, s));
+    return int(fminf(fmaxf(k, -127.f), 127.f));
+}
+
+template <int FS>
+__device__ __forceinline__ float src_at(const uint4 &raw, int i)
+{
+    const uint16_t h = reinterpret_cast<const uint16_t *>(&raw)[i];
+    if constexpr (FS == 2) return __bfloat162float(__ushort_as_bfloat16(h));
+    return __half2float(__ushort_as_half(h));
+}
+
 // ACC: also store every INT32 group sum into p.acc_out (W4A8 with group_size 128).
-template <int WB, int AM, int NT, bool ACC, bool WIDE>
+// FS: 0, or the FP activations to quantize per token first (1: binary16, 2: bfloat16; INT8
+// mode and whole-K activation staging only): the "fused kernel" of the same page's section
+// on combining the strategies, here the quantization done in the matmul's prologue.
+template <int WB, int AM, int NT, bool ACC, bool WIDE, int FS = 0>
 __global__ void __launch_bounds__(kThreads, 1)
     gemv_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_a,
                 const GemvParams p)
 {
+    static_assert(FS == 0 || AM == A_I8, "the fused quantization feeds the INT8 path");
     constexpr int KU = kunit_of(WB);
     constexpr int QN = qn_of(WB, AM);
     constexpr int ES = (AM == A_I8) ? 1 : 2;
@@ -256,9 +289,49 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 
     grid_dep_wait();  // activations, a_scale and bias may be written by the previous kernel
+    float *fsc = reinterpret_cast<float *>(smem + p.fs_off);  // FS: [16] token scales, [16] their reciprocals
+    if constexpr (FS != 0) {
+        // per-token absolute maximum (a warp per token), then the codes of all of A into the
+        // activation buffer; each 8-element chunk of Aq is also written out by one CTA
+        if (threadIdx.x == 0) {
+            const int kpad = p.KB * KU;
+            for (int m = 0; m < p.M; ++m)
+                for (int k = p.K; k < kpad; ++k) abuf[(size_t)m * p.a_pitch_b + k] = 0;
+        }
+        const int K8 = p.K / 8;
+        const uint4 *src = static_cast<const uint4 *>(p.A_src);
+        for (int m = warp; m < p.M; m += kCW) {
+            float amax = 0.f;
+            for (int j = lane; j < K8; j += 32) {
+                const uint4 raw = __ldg(src + (size_t)m * K8 + j);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(src_at<FS>(raw, i)));
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+            if (lane == 0) {
+                const float sc = __fdiv_rn(amax, 127.0f);
+                fsc[m] = sc;
+                fsc[16 + m] = sc != 0.f ? __frcp_rn(sc) : 0.f;
+                if (blockIdx.x == 0) p.a_scale_out[m] = sc;
+            }
+        }
+        __syncthreads();
+        for (int e = threadIdx.x; e < p.M * K8; e += kThreads) {
+            const int m = e / K8, j = e - m * K8;
+            const uint4 raw = __ldg(src + (size_t)m * K8 + j);
+            const float sc = fsc[m], rc = fsc[16 + m];
+            uint32_t w[2] = {0u, 0u};
+#pragma unroll
+            for (int i = 0; i < 8; ++i) w[i >> 2] |= (uint32_t(quant_i8(src_at<FS>(raw, i), sc, rc)) & 0xffu) << (8 * (i & 3));
+            *reinterpret_cast<uint2 *>(abuf + (size_t)m * p.a_pitch_b + 8 * j) = make_uint2(w[0], w[1]);
+            if (int(e % gridDim.x) == blockIdx.x)
+                reinterpret_cast<uint2 *>(p.Aq_out + (size_t)m * p.K)[j] = make_uint2(w[0], w[1]);
+        }
+    }
     if (lane == 0 && !p.a_whole)
         for (int it = warp; it < pro; it += kCW) issue_a(it);
-    if (p.a_whole && threadIdx.x == 0) {
+    if (FS == 0 && p.a_whole && threadIdx.x == 0) {
         // all of K, one bulk copy per token row; zeros past K up to the last unit
         const int kpad = p.KB * KU;
         for (int m = 0; m < p.M; ++m)
@@ -273,7 +346,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                       abar);
     }
     __syncthreads();  // table (and activation padding) visible; no early exit before this point
-    if (p.a_whole && !wait_bar(abar, 0)) return;
+    if (FS == 0 && p.a_whole && !wait_bar(abar, 0)) return;
 
     uint32_t cphase = 0;
     auto csync = [&]() -> bool {  // bounded barrier of all threads (one arrival per warp)
@@ -319,7 +392,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const int pitch = p.a_pitch_b;
                     auto addr = [=](int m, int o) { return ablk + m * pitch + o; };
 #pragma unroll
-                    for (int j = 0; j < NT; ++j) build_bfrag<WB, AM>(addr, p.M, j, lane, bf[j], asum[j]);
+                    for (int j = 0; j < NT; ++j) build_bfrag<WB, AM>(addr, p.M, j, lane, bf[j], asum[j], p.nat != 0);
                 } else {
                     const uint8_t *abase = st + p.wpart_bytes;
                     const int MB = p.MB;
@@ -328,7 +401,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         return abase + swz128(((x >> 7) * MB + m) * 128u + (x & 127u));
                     };
 #pragma unroll
-                    for (int j = 0; j < NT; ++j) build_bfrag<WB, AM>(addr, p.M, j, lane, bf[j], asum[j]);
+                    for (int j = 0; j < NT; ++j) build_bfrag<WB, AM>(addr, p.M, j, lane, bf[j], asum[j], p.nat != 0);
                 }
                 int sA[NT][2];
                 if constexpr (AM == A_I8) {
@@ -460,7 +533,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 sf += v;
                 si += __float_as_int(v);
             }
-            store_out<AM>(p.C, (long long)m * p.N + n, finish<WB, AM>(p, sf, si, n, m));
+            const float as = (AM != A_I8) ? 1.f : (FS != 0 ? fsc[m] : p.a_scale[m]);
+            store_out<AM>(p.C, (long long)m * p.N + n, finish<WB, AM>(p, sf, si, n, as));
             if constexpr (AM == A_I8 && WB == 2)
                 if (p.acc_out) p.acc_out[(long long)m * p.N + n] = si;
         }
@@ -473,7 +547,7 @@ struct Plan {
     int NT = 1, wide = 0, KC = 16, KU = 128, KB = 0, T = 0, P = 0, nch = 0, TPP = 1, S = 1;
     int w3d = 0, wtile = 0, wpart = 0, stage = 0;
     int a_whole = 0, a_pitch_b = 0, abox = 0, MB = 8, rows_cap = 0, tab_rs = 1;
-    int abuf_off = 0, scst_off = 0, stab_off = 0, red_off = 0, bar_off = 0;
+    int abuf_off = 0, scst_off = 0, stab_off = 0, red_off = 0, fs_off = 0, bar_off = 0;
     size_t smem = 0;
     bool ok = false;
 };
@@ -507,7 +581,7 @@ Plan make_plan(int64_t M, int64_t N, int64_t K, int WB, int AM, int G, const Dev
     const size_t scst = (WB == 4) ? up(size_t(pl.rows_cap) * G * 2 * 2, 16) : 0;
     const size_t table = (WB == 4) ? up(size_t(pl.tab_rs) * G * 8, 16) : 0;
     const size_t red = up(size_t(pl.TPP) * pl.KC * kTileRows * M * 4, 16);
-    const size_t tail = scst + table + red + 8 * 19 + 4 * 16 + 64;  // + barriers (S <= 16), counters
+    const size_t tail = scst + table + red + 128 + 8 * 19 + 4 * 16 + 64;  // + fused scales, barriers (S <= 16), counters
     const size_t budget = size_t(dev.max_smem_optin) - 1024;  // 1 KB for the alignment of the base
     auto stages_for = [&](size_t stage, size_t extra) -> long long {
         if (budget <= tail + extra) return 0;
@@ -543,6 +617,8 @@ Plan make_plan(int64_t M, int64_t N, int64_t K, int WB, int AM, int G, const Dev
     off += table;
     pl.red_off = int(off);
     off += red;
+    pl.fs_off = int(up(off, 16));  // fused quantization: 16 token scales and their reciprocals
+    off = pl.fs_off + 128;
     pl.bar_off = int(up(off, 8));
     off = pl.bar_off + size_t(8) * (pl.S + 3) + size_t(4) * pl.S;
     pl.smem = up(off, 16) + 1024;
@@ -551,10 +627,10 @@ Plan make_plan(int64_t M, int64_t N, int64_t K, int WB, int AM, int G, const Dev
 }
 
 // The kernel instance for the plan, with its dynamic shared memory limit raised as needed.
-template <int WB, int AM, int NT, bool ACC = false, bool WIDE = false>
+template <int WB, int AM, int NT, bool ACC = false, bool WIDE = false, int FS = 0>
 wq_status kernel_for(const Plan &pl, const void **func)
 {
-    auto kern = gemv_kernel<WB, AM, NT, ACC, WIDE>;
+    auto kern = gemv_kernel<WB, AM, NT, ACC, WIDE, FS>;
     static size_t configured = 0;
     if (pl.smem > configured) {
         if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(pl.smem)) != cudaSuccess)
@@ -570,12 +646,15 @@ wq_status kernel_for(const Plan &pl, const void **func)
 // Few-token path (1 <= M <= 16) as a prepared launch.  WQ_ERR_UNSUPPORTED if no plan fits.
 wq_status gemv_prepare(int WB, int AM, const void *A, const float *a_scale, const uint8_t *Wq, const void *scales,
                        const void *zeros, const void *bias, void *C, int32_t *acc_out, int64_t M, int64_t N,
-                       int64_t K, const wq_qconfig &c, PreparedLaunch *out)
+                       int64_t K, const wq_qconfig &c, PreparedLaunch *out, const FusedActQuant *fa)
 {
     const DeviceInfo &dev = device_info();
     const int G = WB == 4 ? int(K / c.group_size) : 1;
     Plan pl = make_plan(M, N, K, WB, AM, G, dev);
     if (!pl.ok) return fail(WQ_ERR_UNSUPPORTED, "no few-token plan for M=%lld K=%lld", (long long)M, (long long)K);
+    if (fa && (AM != A_I8 || !pl.a_whole))
+        return fail(WQ_ERR_UNSUPPORTED, "the activations of M=%lld K=%lld are not staged whole", (long long)M,
+                    (long long)K);
     CUtensorMap tw, ta;
     const uint64_t row_bytes = uint64_t(K) * WB / 8;
     wq_status rc = WQ_ERR_UNSUPPORTED;
@@ -643,8 +722,25 @@ wq_status gemv_prepare(int WB, int AM, const void *A, const float *a_scale, cons
     p.a_scale = a_scale;
     p.C = C;
     p.acc_out = acc_out;
+    p.fs_off = pl.fs_off;
+    p.nat = WB == 4 && c.layout == WQ_LAYOUT_NATIVE;
     const bool one = pl.NT == 1;
     const void *func = nullptr;
+    if (fa) {
+        p.A_src = fa->A;
+        p.Aq_out = fa->Aq;
+        p.a_scale_out = fa->a_scale;
+        const bool bf = fa->bf16;
+        if (WB == 4 && acc_out)
+            rc = bf ? (one ? kernel_for<4, A_I8, 1, true, false, 2>(pl, &func) : kernel_for<4, A_I8, 2, true, false, 2>(pl, &func))
+                    : (one ? kernel_for<4, A_I8, 1, true, false, 1>(pl, &func) : kernel_for<4, A_I8, 2, true, false, 1>(pl, &func));
+        else if (WB == 4)
+            rc = bf ? (one ? kernel_for<4, A_I8, 1, false, false, 2>(pl, &func) : kernel_for<4, A_I8, 2, false, false, 2>(pl, &func))
+                    : (one ? kernel_for<4, A_I8, 1, false, false, 1>(pl, &func) : kernel_for<4, A_I8, 2, false, false, 1>(pl, &func));
+        else
+            rc = bf ? (one ? kernel_for<2, A_I8, 1, false, false, 2>(pl, &func) : kernel_for<2, A_I8, 2, false, false, 2>(pl, &func))
+                    : (one ? kernel_for<2, A_I8, 1, false, false, 1>(pl, &func) : kernel_for<2, A_I8, 2, false, false, 1>(pl, &func));
+    } else
     if (WB == 4 && AM == A_F16)
         rc = one ? kernel_for<4, A_F16, 1>(pl, &func)
                  : pl.wide ? kernel_for<4, A_F16, 2, false, true>(pl, &func) : kernel_for<4, A_F16, 2>(pl, &func);

@@ -72,9 +72,20 @@ wq_status launch_prepared(PreparedLaunch &L, cudaStream_t st, const char *what);
 wq_status check_a16(const void *A, wq_dtype a_dt, const uint8_t *Wq, const void *scales, const void *zeros,
                     const void *bias, const void *C, int64_t M, int64_t N, int64_t K, const wq_qconfig &c);
 
-// The few-token matmul (M <= 16) as a prepared launch (see gemv_small_m for the arguments).
+// FP activations that the few-token INT8 matmul quantizes per token itself (written to Aq
+// and a_scale exactly as act_quant_int8 writes them).
+struct FusedActQuant {
+    const void *A;
+    bool bf16;
+    int8_t *Aq;
+    float *a_scale;
+};
+
+// The few-token matmul (M <= 16) as a prepared launch (see gemv_small_m for the arguments);
+// with `fa`, INT8 mode starting from FP activations (WQ_ERR_UNSUPPORTED when the launch
+// plan does not stage the activations whole).
 wq_status gemv_prepare(int WB, int AM, const void *A, const float *a_scale, const uint8_t *Wq, const void *scales,
                        const void *zeros, const void *bias, void *C, int32_t *acc_out, int64_t M, int64_t N,
-                       int64_t K, const wq_qconfig &c, PreparedLaunch *out);
+                       int64_t K, const wq_qconfig &c, PreparedLaunch *out, const FusedActQuant *fa = nullptr);
 
 }  // namespace wq

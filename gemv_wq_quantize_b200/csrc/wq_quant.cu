@@ -17,6 +17,7 @@
 
 #include <algorithm>
 
+#include "wq_device.cuh"
 #include "wq_host.h"
 
 namespace wq {
@@ -236,6 +237,36 @@ __global__ void __launch_bounds__(256) unpack_kernel(const uint8_t *__restrict__
     }
 }
 
+// Kernel-native order: nibble i of every 32-bit word holds element kNativePos[i] of the word's
+// 8 elements (the inverse, kNativeSlot[e], is the nibble that holds element e).
+__device__ __constant__ int kNativePos[8] = {0, 2, 4, 6, 1, 3, 5, 7};
+__device__ __constant__ int kNativeSlot[8] = {0, 4, 1, 5, 2, 6, 3, 7};
+
+__global__ void __launch_bounds__(256) repack_kernel(const uint32_t *__restrict__ in, int64_t nwords,
+                                                     uint32_t *__restrict__ out)
+{
+    const int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (i >= nwords) return;
+    const uint32_t w = in[i];
+    uint32_t o = 0;
+#pragma unroll
+    for (int s = 0; s < 8; ++s) o |= ((w >> (4 * kNativePos[s])) & 15u) << (4 * s);
+    out[i] = o;
+}
+
+__global__ void __launch_bounds__(256) unpack_native_kernel(const uint32_t *__restrict__ in, int64_t nwords, int sym,
+                                                            int8_t *__restrict__ q)
+{
+    const int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (i >= nwords) return;
+    const uint32_t w = in[i];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+        const int v = int((w >> (4 * kNativeSlot[e])) & 15u);
+        q[8 * i + e] = int8_t(sym ? v - 8 : v);
+    }
+}
+
 // One block per token row: absmax, a_scale = absmax / 127, codes.  8 elements per access.
 template <typename T>
 __global__ void __launch_bounds__(256) act_quant_kernel(const T *__restrict__ A, int64_t K, int8_t *__restrict__ Aq,
@@ -244,6 +275,10 @@ __global__ void __launch_bounds__(256) act_quant_kernel(const T *__restrict__ A,
     const int64_t m = blockIdx.x;
     const T *a = A + m * K;
     const int64_t K8 = K / 8;
+    // programmatic dependent launch: the matmul that reads Aq may start its prologue (its
+    // weights do not depend on this kernel); A may be written by the previous kernel
+    grid_dep_launch();
+    grid_dep_wait();
     float amax = 0.f;
     for (int64_t j = threadIdx.x; j < K8; j += blockDim.x) {
         uint4 raw = __ldg(reinterpret_cast<const uint4 *>(a) + j);
@@ -326,6 +361,8 @@ extern "C" wq_status wq_quantize_pack(const void *W, wq_dtype w_dt, int64_t N, i
 {
     if (N <= 0 || K <= 0) return fail(WQ_ERR_INVALID_ARG, "N and K must be positive");
     if (!W || !Wq || !scales) return fail(WQ_ERR_INVALID_ARG, "W, Wq and scales must be non-null");
+    if (c.layout != WQ_LAYOUT_NT)
+        return fail(WQ_ERR_UNSUPPORTED, "quantize with layout WQ_LAYOUT_NT, then wq_repack");
     if (w_dt != WQ_F32 && w_dt != WQ_F16 && w_dt != WQ_BF16)
         return fail(WQ_ERR_INVALID_ARG, "w_dt must be WQ_F32, WQ_F16 or WQ_BF16");
     if (!aligned16(W) || !aligned16(Wq) || (zeros && !aligned16(zeros)) || !aligned16(scales))
@@ -353,8 +390,31 @@ extern "C" wq_status wq_unpack(const uint8_t *Wq, int64_t N, int64_t K, wq_qconf
     if (c.bits != 4 && c.bits != 2) return fail(WQ_ERR_INVALID_ARG, "bits must be 4 or 2");
     if (K % (8 / c.bits)) return fail(WQ_ERR_INVALID_ARG, "K must fill whole bytes");
     const int64_t nbytes = N * K * c.bits / 8;
+    if (c.layout == WQ_LAYOUT_NATIVE) {
+        if (c.bits != 4) return fail(WQ_ERR_UNSUPPORTED, "the native layout is INT4 only");
+        if (K % 8 || !aligned16(Wq)) return fail(WQ_ERR_INVALID_ARG, "native layout: K %% 8 == 0, Wq 16-byte aligned");
+        const int64_t nwords = nbytes / 4;
+        unpack_native_kernel<<<blocks_for(nwords), 256, 0, stream>>>(reinterpret_cast<const uint32_t *>(Wq), nwords,
+                                                                     c.symmetric, q);
+        return check_launch("unpack_native_kernel");
+    }
+    if (c.layout != WQ_LAYOUT_NT) return fail(WQ_ERR_INVALID_ARG, "unknown layout %d", int(c.layout));
     unpack_kernel<<<blocks_for(nbytes), 256, 0, stream>>>(Wq, nbytes, c.bits, c.bits == 4 ? c.symmetric : 1, q);
     return check_launch("unpack_kernel");
+}
+
+extern "C" wq_status wq_repack(const uint8_t *Wq, int64_t N, int64_t K, wq_qconfig c, uint8_t *Wq_native,
+                               cudaStream_t stream)
+{
+    if (N <= 0 || K <= 0 || !Wq || !Wq_native) return fail(WQ_ERR_INVALID_ARG, "bad sizes or null pointer");
+    if (c.bits != 4) return fail(WQ_ERR_UNSUPPORTED, "the native layout is INT4 only");
+    if (c.layout != WQ_LAYOUT_NT) return fail(WQ_ERR_INVALID_ARG, "wq_repack reads weights in WQ_LAYOUT_NT");
+    if (K % 8) return fail(WQ_ERR_INVALID_ARG, "K %% 8 != 0");
+    if (!aligned16(Wq) || !aligned16(Wq_native)) return fail(WQ_ERR_ALIGNMENT, "Wq and Wq_native must be 16-byte aligned");
+    const int64_t nwords = N * K / 8;
+    repack_kernel<<<blocks_for(nwords), 256, 0, stream>>>(reinterpret_cast<const uint32_t *>(Wq), nwords,
+                                                          reinterpret_cast<uint32_t *>(Wq_native));
+    return check_launch("repack_kernel");
 }
 
 extern "C" wq_status act_quant_int8(const void *A, wq_dtype a_dt, int64_t M, int64_t K, int8_t *Aq, float *a_scale,
@@ -365,10 +425,21 @@ extern "C" wq_status act_quant_int8(const void *A, wq_dtype a_dt, int64_t M, int
     if (K % 8) return fail(WQ_ERR_INVALID_ARG, "K %% 8 != 0");
     if (!aligned16(A) || !aligned16(Aq)) return fail(WQ_ERR_ALIGNMENT, "A and Aq must be 16-byte aligned");
     if (M > 0x7fffffff) return fail(WQ_ERR_INVALID_ARG, "M too large");
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(unsigned(M));
+    cfg.blockDim = dim3(256);
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e;
     if (a_dt == WQ_F16)
-        act_quant_kernel<__half><<<unsigned(M), 256, 0, stream>>>(static_cast<const __half *>(A), K, Aq, a_scale);
+        e = cudaLaunchKernelEx(&cfg, act_quant_kernel<__half>, static_cast<const __half *>(A), K, Aq, a_scale);
     else
-        act_quant_kernel<__nv_bfloat16><<<unsigned(M), 256, 0, stream>>>(static_cast<const __nv_bfloat16 *>(A), K, Aq,
-                                                                         a_scale);
+        e = cudaLaunchKernelEx(&cfg, act_quant_kernel<__nv_bfloat16>, static_cast<const __nv_bfloat16 *>(A), K, Aq,
+                               a_scale);
+    if (e != cudaSuccess) return fail(WQ_ERR_CUDA, "act_quant_kernel launch: %s", cudaGetErrorString(e));
     return check_launch("act_quant_kernel");
 }

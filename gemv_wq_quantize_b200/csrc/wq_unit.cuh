@@ -8,7 +8,9 @@
 // k order: the nibble unpack of a 32-bit word naturally yields pairs (k, k+4) of INT4
 // (pairs (k, k+8) of INT2; byte quads (k, k+2, k+4, k+6) for INT8 activations).  Since
 // an MMA sums over k, the activations (B operand) are loaded in the same permuted order,
-// so the weights are used straight from the packed layout with no reordering.
+// so the weights are used straight from the packed layout with no reordering.  INT4 weights
+// in the kernel-native order (see wq_repack) unpack to pairs (k, k+1), the activations'
+// own order, and their B fragments need no permutation.
 #pragma once
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -35,9 +37,11 @@ __host__ __device__ constexpr int qn_of(int WB, int AM) { return steps_of(WB, AM
 // of the unit (o < KU * element size, 16-byte chunks contiguous); tokens >= M give zeros.
 // For INT8 activations `asum` receives this lane's partial sum of the token's activations
 // over the unit (the quad of lanes sharing a token adds up to the token's sum).
+// nat: INT4 weights in the kernel-native order (nibble i of a word = element 0,2,4,6,1,3,5,7),
+// whose unpack yields the pairs (k, k+1) (FP) or the byte quads (k, k+4, k+1, k+5) (INT8).
 template <int WB, int AM, typename Addr>
 __device__ __forceinline__ void build_bfrag(Addr addr, int M, int nt, int lane, uint4 (&bf)[qn_of(WB, AM)],
-                                            int &asum)
+                                            int &asum, bool nat = false)
 {
     constexpr int QN = qn_of(WB, AM);
     const int g = lane >> 2, t = lane & 3;
@@ -53,11 +57,16 @@ __device__ __forceinline__ void build_bfrag(Addr addr, int M, int nt, int lane, 
         uint4 r;
         if constexpr (AM != A_I8 && WB == 4) {
             // k-steps 2q, 2q+1 use halves 32t + 8q + {0..7} as pairs (0,4),(1,5) / (2,6),(3,7)
+            // (native order: (0,1),(2,3) / (4,5),(6,7), the halves as they lie)
             const uint4 v = lds128(addr(m, (32 * t + 8 * q) * 2));
-            r.x = prmt(v.x, v.z, 0x5410);
-            r.y = prmt(v.x, v.z, 0x7632);
-            r.z = prmt(v.y, v.w, 0x5410);
-            r.w = prmt(v.y, v.w, 0x7632);
+            if (nat) {
+                r = v;
+            } else {
+                r.x = prmt(v.x, v.z, 0x5410);
+                r.y = prmt(v.x, v.z, 0x7632);
+                r.z = prmt(v.y, v.w, 0x5410);
+                r.w = prmt(v.y, v.w, 0x7632);
+            }
         } else if constexpr (AM != A_I8 && WB == 2) {
             // k-steps 4j + 2hh (+1): pairs (i, i+8) of halves 64t + 16j + 4hh + {0..3, 8..11}
             const int j = q >> 1, hh = q & 1;
@@ -70,11 +79,13 @@ __device__ __forceinline__ void build_bfrag(Addr addr, int M, int nt, int lane, 
             r.w = prmt(lo.y, hi.y, 0x7632);
         } else if constexpr (WB == 4) {
             // k-steps 2q, 2q+1 (k32): bytes 32t + 16q + {0..15} as quads (0,2,4,6),(1,3,5,7)
+            // (native order: (0,4,1,5),(2,6,3,7))
             const uint4 v = lds128(addr(m, 32 * t + 16 * q));
-            r.x = prmt(v.x, v.y, 0x6420);
-            r.y = prmt(v.x, v.y, 0x7531);
-            r.z = prmt(v.z, v.w, 0x6420);
-            r.w = prmt(v.z, v.w, 0x7531);
+            const uint32_t s0 = nat ? 0x5140u : 0x6420u, s1 = nat ? 0x7362u : 0x7531u;
+            r.x = prmt(v.x, v.y, s0);
+            r.y = prmt(v.x, v.y, s1);
+            r.z = prmt(v.z, v.w, s0);
+            r.w = prmt(v.z, v.w, s1);
             asum = __dp4a(int(v.x), 0x01010101, asum);
             asum = __dp4a(int(v.y), 0x01010101, asum);
             asum = __dp4a(int(v.z), 0x01010101, asum);

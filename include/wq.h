@@ -81,7 +81,12 @@ typedef struct {
                          /* INT2: ignored (one scale per tensor).                          */
     int32_t symmetric;   /* INT4: 1 = symmetric (q + 8 stored, no zeros), 0 = zero points.  */
     int32_t ternary;     /* INT2: must be 1 (codes -1, 0, 1 from the ternary quantizer).    */
+    int32_t layout;      /* INT4 only: WQ_LAYOUT_NT (0), the packing described above, or     */
+                         /* WQ_LAYOUT_NATIVE (1), the order written by wq_repack.           */
 } wq_qconfig;
+
+#define WQ_LAYOUT_NT 0
+#define WQ_LAYOUT_NATIVE 1
 
 /* Weight quantization and packing ("Accelerating LLM inference with CUDA Graph and INT4
  * quantization", part 1, step 1; BitBLAS guide, "Advanced features 2").
@@ -97,6 +102,21 @@ wq_status wq_quantize_pack(const void *W, wq_dtype w_dt, int64_t N, int64_t K, w
                            uint8_t *Wq, void *scales, void *zeros,
                            void *workspace, size_t ws_bytes, cudaStream_t stream);
 size_t wq_quantize_workspace_size(int64_t N, int64_t K, wq_qconfig c);
+
+/* Kernel-native weight layout ("BitBLAS practical guide", "use the BitBLAS compressed format":
+ * weights stored offline in the order the kernels consume them).  Within every 32-bit word
+ * (8 codes of k = 8j .. 8j+7), nibble i holds element 8j + p(i) with p = 0, 2, 4, 6, 1, 3, 5, 7,
+ * so that masking the word with 0x000F000F / 0x00F000F0 yields the half pairs (k, k+1) in
+ * natural order (one LOP3 per pair in the tensor-core unpack, and activation fragments that
+ * need no byte permutation).  Scales and zero points are unchanged.
+ *   Wq [N, K/2] INT4 in WQ_LAYOUT_NT (c.layout 0); Wq_native [N, K/2] written (may equal Wq).
+ *   Matmuls given c.layout = WQ_LAYOUT_NATIVE read it.  Their results are bit-identical to the
+ *   "nt" call on the INT8 paths (exact sums) and above 16 tokens (the tensor-core unpack yields
+ *   the same values in the same order); up to 16 tokens on the FP path each MMA step sums a
+ *   different grouping of k, so results agree within the FP accuracy bar, not bit for bit.
+ * INT4 only (WQ_ERR_UNSUPPORTED for INT2); K % 8 == 0. */
+wq_status wq_repack(const uint8_t *Wq, int64_t N, int64_t K, wq_qconfig c, uint8_t *Wq_native,
+                    cudaStream_t stream);
 
 /* Inverse of the packing: signed codes q [N,K] int8 (symmetric INT4: nibble - 8; asymmetric
  * INT4: nibble; INT2: two's complement).  For tests and debugging ("Accelerating LLM
@@ -140,6 +160,23 @@ wq_status w4a8_gemm(const int8_t *Aq, const float *a_scale, const uint8_t *Wq, c
                     int64_t M, int64_t N, int64_t K, wq_qconfig c,
                     void *workspace, size_t ws_bytes, cudaStream_t stream);
 
+/* W4A8 from FP16 / BF16 activations, with the per-token INT8 quantization fused into the
+ * matmul ("Accelerating LLM inference with CUDA Graph and INT4 quantization", part 1, steps 2-4,
+ * and the fused-kernel item of its section on combining the strategies).  Results are
+ * bit-identical to act_quant_int8(A, a_dt, M, K, Aq, a_scale) followed by
+ * w4a8_gemm(Aq, a_scale, Wq, scales, zeros, bias, C, acc_out, ...).
+ *   A [M,K] a_dt (WQ_F16 or WQ_BF16), K % 8 == 0.
+ *   Aq [M,K] int8 and a_scale [M] binary32: required outputs, written with the values
+ *   act_quant_int8 writes.  C, bias, acc_out, workspace as for w4a8_gemm.
+ * When M <= 16, M * K <= 16384 and the few-token kernel stages the activations whole, this is
+ * ONE launch: every CTA forms the per-token scales and codes itself in its prologue (no second
+ * kernel, no INT8 round trip through memory).  Otherwise it enqueues act_quant_int8 and
+ * w4a8_gemm (each CTA would read all of a larger A twice). */
+wq_status w4a8_gemm_fused(const void *A, wq_dtype a_dt, const uint8_t *Wq, const void *scales,
+                          const void *zeros, const void *bias, void *C, int8_t *Aq, float *a_scale,
+                          int32_t *acc_out, int64_t M, int64_t N, int64_t K, wq_qconfig c,
+                          void *workspace, size_t ws_bytes, cudaStream_t stream);
+
 /* Bytes of workspace that lets w4a16_gemm / w4a8_gemm use their split-K plans on the
  * current device. */
 size_t wq_workspace_size(int64_t M, int64_t N, int64_t K, wq_qconfig c);
@@ -165,6 +202,51 @@ size_t wq_workspace_size(int64_t M, int64_t N, int64_t K, wq_qconfig c);
 wq_status w4a16_gemm_noalloc(const void *A, wq_dtype a_dt, const uint8_t *Wq, const void *scales,
                              const void *zeros, const void *bias, void *C,
                              int64_t M, int64_t N, int64_t K, wq_qconfig c, cudaStream_t stream);
+
+/* ---- A decode step as one CUDA graph ("Accelerating LLM inference with CUDA Graph and INT4
+ * quantization", part 2: capture the step's kernels in a graph once, update the arguments that
+ * change from step to step, and launch the whole step with one call).
+ *
+ * A wq_graph holds a chain of up to WQ_GRAPH_MAX_OPS W4A16 / W2A16 matmuls of at most 16
+ * tokens each (for example the QKV, output, gate/up and down projections of one transformer
+ * layer at decode time), as kernel nodes of one CUDA graph in the given order.  Consecutive
+ * nodes are joined by programmatic-dependent-launch edges, so each matmul streams its weights
+ * while the previous one finishes; a node may read the output of an earlier one.
+ *   ops[i]: the arguments of w4a16_gemm for matmul i (same meaning, layouts and checks;
+ *           M <= 16, else WQ_ERR_UNSUPPORTED).  The weights, scales, zeros and bias stay
+ *           fixed for the graph's life; A and C can be changed per step with wq_graph_set_io.
+ *   Each launch computes exactly what w4a16_gemm computes for the same arguments (the same
+ *   kernels and launch plans: bit-identical outputs).
+ * Ownership: the graph keeps the device pointers it was given (the caller keeps those buffers
+ * alive and unchanged in shape until wq_graph_destroy).  Creating it captures the launches on a
+ * private stream (created and destroyed inside the call; nothing runs) and allocates host
+ * memory and the driver's graph objects, never device memory.  One wq_graph is used by one
+ * host thread at a time.  Errors as for w4a16_gemm; a failed create returns no
+ * graph. */
+#define WQ_GRAPH_MAX_OPS 64
+typedef struct {
+    const void *A;
+    wq_dtype a_dt;
+    const uint8_t *Wq;
+    const void *scales;
+    const void *zeros;
+    const void *bias;
+    void *C;
+    int64_t M, N, K;
+    wq_qconfig c;
+} wq_matmul_desc;
+
+typedef struct wq_graph wq_graph;
+
+wq_status wq_graph_create(const wq_matmul_desc *ops, int n_ops, wq_graph **out);
+/* New activation and output pointers for matmul `op` (16-byte aligned device pointers of the
+ * same shapes), taking effect from the next wq_graph_launch: the node's arguments are
+ * rewritten in the instantiated graph (cudaGraphExecKernelNodeSetParams); nothing is
+ * re-instantiated.  Launches already enqueued keep the pointers they were launched with. */
+wq_status wq_graph_set_io(wq_graph *g, int op, const void *A, void *C);
+/* Enqueues one run of the whole chain on `stream` (asynchronous). */
+wq_status wq_graph_launch(wq_graph *g, cudaStream_t stream);
+void wq_graph_destroy(wq_graph *g);
 
 const char *wq_status_string(wq_status s);
 

@@ -94,6 +94,32 @@ def test_alignment_and_null_checks(lib):
     assert lib.wq_unpack(FAKE, 4, 7, qc, FAKE, None) == wq.WQ_ERR_INVALID_ARG
 
 
+def test_fused_w4a8_checks(lib):
+    qc = _qc()
+    # Aq and a_scale are required outputs
+    assert lib.w4a8_gemm_fused(FAKE, wq.WQ_F16, FAKE, FAKE, None, None, FAKE, None, FAKE, None, 1, 128, 128, qc,
+                               None, 0, None) == wq.WQ_ERR_INVALID_ARG
+    assert lib.w4a8_gemm_fused(FAKE, wq.WQ_I8, FAKE, FAKE, None, None, FAKE, FAKE, FAKE, None, 1, 128, 128, qc,
+                               None, 0, None) == wq.WQ_ERR_INVALID_ARG
+    assert lib.w4a8_gemm_fused(FAKE_MIS, wq.WQ_F16, FAKE, FAKE, None, None, FAKE, FAKE, FAKE, None, 1, 128, 128,
+                               qc, None, 0, None) == wq.WQ_ERR_ALIGNMENT
+
+
+def test_native_layout_checks(lib):
+    nt, nat = _qc(), wq.QConfig(4, 128, 1, 0, wq.LAYOUT_NATIVE)
+    assert lib.wq_repack(FAKE, 4, 128, _qc(bits=2), FAKE, None) == wq.WQ_ERR_UNSUPPORTED
+    assert lib.wq_repack(FAKE, 4, 128, nat, FAKE, None) == wq.WQ_ERR_INVALID_ARG      # input must be "nt"
+    assert lib.wq_repack(FAKE, 4, 100, nt, FAKE, None) == wq.WQ_ERR_INVALID_ARG       # K % 8
+    assert lib.wq_repack(FAKE_MIS, 4, 128, nt, FAKE, None) == wq.WQ_ERR_ALIGNMENT
+    assert lib.wq_quantize_pack(FAKE, wq.WQ_F32, 4, 128, nat, FAKE, FAKE, None, None, 0, None) == wq.WQ_ERR_UNSUPPORTED
+    bad = wq.QConfig(4, 128, 1, 0, 7)
+    assert lib.w4a16_gemm(FAKE, wq.WQ_F16, FAKE, FAKE, None, None, FAKE, 1, 128, 128, bad, None, 0, None) \
+        == wq.WQ_ERR_INVALID_ARG
+    tern_nat = wq.QConfig(2, 128, 1, 1, wq.LAYOUT_NATIVE)
+    assert lib.w4a16_gemm(FAKE, wq.WQ_F16, FAKE, FAKE, None, None, FAKE, 1, 128, 128, tern_nat, None, 0, None) \
+        == wq.WQ_ERR_UNSUPPORTED
+
+
 def test_quantize_workspace_size(lib):
     assert lib.wq_quantize_workspace_size(4, 128, _qc()) == 0
     assert lib.wq_quantize_workspace_size(4, 128, _qc(bits=2)) >= 2048

@@ -523,3 +523,118 @@ def test_zero_scale_groups(M, quant, mode):
     Cb = bits_np(C)
     assert np.all(Cb[:, 5] == 0)
     assert_close(Cb, ref, torch.float16)
+
+
+# ------------------------------------------------------------------ W4A8 with fused activation quantization
+def _fused_case(M, N, K, quant, dtype, seed):
+    qc = qc_of(quant)
+    W = wq_synth.weights(N, K, seed=seed)
+    A = wq_synth.activations(M, K, seed=seed + 1, dtype=dtype, outlier_frac=0.01)
+    if M > 2:
+        A[1] = 0                                   # a token whose scale is 0
+    fx = tie_inputs.fields()
+    At, _, _, _ = tie_inputs.act_case(fx, dtype)   # exact ties in the last token's first 128 k
+    A[M - 1, :128] = At[0]
+    A[M - 1, 128:] = 0
+    Wq, s, z, (oWq, os_, oz) = quantize_both(W, qc)
+    return qc, A, Wq, s, z, (oWq, os_, oz)
+
+
+@pytest.mark.parametrize("dtype", [torch.float16, torch.bfloat16])
+@pytest.mark.parametrize("quant", ["sym4", "asym4", "tern2"])
+@pytest.mark.parametrize("M,N,K", [(1, 256, 512), (1, 520, 11008), (4, 1000, 1024), (12, 300, 1024),
+                                   (9, 384, 2048), (16, 4096, 4096), (16, 520, 11008), (40, 384, 1024)])
+def test_w4a8_fused_matches_two_launches_and_oracle(dtype, quant, M, N, K):
+    # small activations (M <= 16, M*K <= 16384): one launch quantizes in the matmul's prologue;
+    # otherwise the call runs two launches.  Either way C, Aq, a_scale and the INT32 sums must
+    # equal act_quant_int8 + w4a8_gemm bit for bit, and the oracle
+    if quant == "tern2":
+        K = K // 64 * 64
+    qc, A, Wq, s, z, (oWq, os_, oz) = _fused_case(M, N, K, quant, dtype, seed=M + N)
+    G = 1 if qc.bits == 2 else K // 128
+    ws = workspace(M, N, K, qc)
+    Ad = A.cuda()
+    acc1 = torch.full((M, N, G), 7, dtype=torch.int32, device="cuda")
+    C1, Aq1, sc1 = wq.w4a8_gemm_fused(Ad, Wq, s, z, N, K, qc, acc_out=acc1, workspace=ws)
+    Aq2, sc2 = wq.act_quant_int8(Ad)
+    acc2 = torch.full((M, N, G), 7, dtype=torch.int32, device="cuda")
+    C2 = wq.w4a8_gemm(Aq2, sc2, Wq, s, z, N, K, qc, acc_out=acc2, workspace=ws)
+    torch.cuda.synchronize()
+    assert torch.equal(Aq1, Aq2)
+    assert torch.equal(sc1.view(torch.int32), sc2.view(torch.int32))
+    assert torch.equal(acc1, acc2)
+    assert torch.equal(C1.view(torch.int16), C2.view(torch.int16))
+    oAq, oasc = oracle.act_quant_int8(bits_np(A), oracle.F16 if dtype == torch.float16 else oracle.BF16)
+    assert np.array_equal(Aq1.cpu().numpy(), oAq)
+    assert np.array_equal(sc1.cpu().numpy().view(np.uint32), oasc.view(np.uint32))
+    _, ref, oacc = oracle.gemm_a8(oAq, oasc, oWq, N, K, qc.bits, qc.symmetric, 128, os_, oz, want_acc=True)
+    assert np.array_equal(acc1.cpu().numpy(), oacc)
+    assert_close(bits_np(C1), ref, torch.float16)
+
+
+# ------------------------------------------------------------------ kernel-native weight layout
+def _native_perm_numpy(Wq):
+    """The layout wq_repack documents, written out independently: nibble i of every 32-bit
+    word takes the code of element (0, 2, 4, 6, 1, 3, 5, 7)[i] of that word."""
+    w = Wq.reshape(-1, 4)
+    nib = np.empty((w.shape[0], 8), dtype=np.uint8)
+    nib[:, 0::2] = w & 15
+    nib[:, 1::2] = w >> 4
+    out_nib = nib[:, [0, 2, 4, 6, 1, 3, 5, 7]]
+    return (out_nib[:, 0::2] | (out_nib[:, 1::2] << 4)).astype(np.uint8).reshape(Wq.shape)
+
+
+@pytest.mark.parametrize("quant", ["sym4", "asym4"])
+def test_repack_layout_and_unpack(quant):
+    qc = qc_of(quant)
+    N, K = 77, 1024
+    Wq = wq_synth.uniform_bytes((N, K // 2), seed=33)
+    Wn = wq.repack(Wq.cuda(), N, K, qc)
+    torch.cuda.synchronize()
+    assert np.array_equal(Wn.cpu().numpy(), _native_perm_numpy(Wq.numpy()))
+    import dataclasses
+    qn = dataclasses.replace(qc, layout=wq.LAYOUT_NATIVE)
+    q = wq.unpack(Wn, N, K, qn)
+    assert np.array_equal(q.cpu().numpy(), oracle.unpack(Wq.numpy(), N, K, 4, qc.symmetric))
+
+
+@pytest.mark.parametrize("quant", ["sym4", "asym4"])
+@pytest.mark.parametrize("mode,dtype", [("a16", torch.float16), ("a16", torch.bfloat16), ("a8", torch.float16)])
+@pytest.mark.parametrize("M,N,K", [(1, 4096, 4096), (5, 333, 1152), (13, 1000, 2048), (16, 4096, 11008),
+                                   (64, 256, 640), (200, 384, 4096), (512, 4096, 4096)])
+def test_native_layout_matches_nt_layout(quant, mode, dtype, M, N, K):
+    # every kernel reading the native order (few-token, fused INT8, tcgen05 with and without
+    # split K) matches the same call on the "nt" packing: bit for bit where the arithmetic
+    # is the same -- the INT8 paths (exact int32 sums) and the tcgen05 path (the unpack puts
+    # the same values in the same k order into Tensor Memory) -- and within the FP bar on the
+    # few-token FP path, whose MMAs sum the k's of a step in another grouping there
+    import dataclasses
+    qc = qc_of(quant)
+    qn = dataclasses.replace(qc, layout=wq.LAYOUT_NATIVE)
+    W = wq_synth.weights(N, K, seed=M + K)
+    Wq, s, z = wq.quantize_pack(W.cuda(), qc)
+    Wn = wq.repack(Wq, N, K, qc)
+    A = wq_synth.activations(M, K, seed=M + 3, dtype=dtype, outlier_frac=0.01)
+    Ad = A.cuda()
+    ws = workspace(M, N, K, qc)
+    if mode == "a16":
+        C0 = wq.w4a16_gemm(Ad, Wq, s, z, N, K, qc, workspace=ws)
+        C1 = wq.w4a16_gemm(Ad, Wn, s, z, N, K, qn, workspace=ws)
+        torch.cuda.synchronize()
+        if M > 16:
+            assert torch.equal(C0.view(torch.int16), C1.view(torch.int16))
+        else:
+            ni = sample_idx(N, 256, 7)
+            adt = oracle.F16 if dtype == torch.float16 else oracle.BF16
+            _, ref = oracle.gemm_a16(bits_np(A), adt, Wq.cpu().numpy(), N, K, 4, qc.symmetric, 128,
+                                     bits_np(s), None if z is None else bits_np(z), n_idx=ni)
+            assert_close(bits_np(C1)[:, ni], ref, dtype)
+            assert_close(bits_np(C0)[:, ni], ref, dtype)
+    else:
+        acc0 = torch.zeros(M, N, K // 128, dtype=torch.int32, device="cuda")
+        acc1 = torch.zeros_like(acc0)
+        C0, _, _ = wq.w4a8_gemm_fused(Ad, Wq, s, z, N, K, qc, acc_out=acc0, workspace=ws)
+        C1, _, _ = wq.w4a8_gemm_fused(Ad, Wn, s, z, N, K, qn, acc_out=acc1, workspace=ws)
+        torch.cuda.synchronize()
+        assert torch.equal(acc0, acc1)
+        assert torch.equal(C0.view(torch.int16), C1.view(torch.int16))
