@@ -13,7 +13,9 @@ as the two source pages define it:
   accumulation, then the (weight_scale x activation_scale) dequantization;
 * "BitBLAS practical guide: mixed-precision compute in vLLM" (mlqm): the
   problem statement, the "nt" layout, group_size=128 with scales and
-  "original" zero points, FP16/INT8 x INT2 (BitNet-b1.58 ternary) weights.
+  "original" zero points, FP16/INT8 x INT2 (BitNet-b1.58 ternary) weights,
+  and the other weight types of its "Main features" list: FP16 x FP4 (e2m1),
+  FP16 x FP8 (e4m3), FP16 / INT8 x INT1 (binary).
 
 Only the test suite, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
 ``bench.py`` may import this package.  It never imports the CUDA library and
@@ -36,6 +38,7 @@ _SRC = os.path.join(_HERE, "wq_oracle.c")
 _LIB = os.path.join(_HERE, "_build", "liboracle.so")
 
 F16, BF16 = 1, 2
+FMT_INT, FMT_E2M1, FMT_E4M3 = 0, 1, 2
 OK, ERR_ARG, ERR_OVERFLOW = 0, 1, 2
 
 CFLAGS = ["-O2", "-std=c11", "-ffp-contract=off", "-fno-fast-math", "-fPIC", "-shared", "-pthread"]
@@ -70,12 +73,17 @@ def _L():
         lib.orc_exact_abs_sum_f32.restype = dbl
         lib.orc_exact_abs_sum_f32.argtypes = [vp, i64]
         lib.orc_pack.argtypes = [vp, i64, i64, i32, vp]
-        lib.orc_unpack.argtypes = [vp, i64, i64, i32, i32, vp]
+        lib.orc_unpack.argtypes = [vp, i64, i64, i32, i32, i32, vp]
+        lib.orc_minifloat_value.restype = dbl
+        lib.orc_minifloat_value.argtypes = [i32, i32]
+        lib.orc_minifloat_encode.argtypes = [i32, dbl]
         lib.orc_quant_int4_sym.argtypes = [vp, i64, i64, i64, vp, vp]
         lib.orc_quant_int4_asym.argtypes = [vp, i64, i64, i64, vp, vp, vp]
         lib.orc_quant_ternary.argtypes = [vp, i64, i64, vp, vp]
+        lib.orc_quant_minifloat.argtypes = [vp, i64, i64, i64, i32, vp, vp]
+        lib.orc_quant_binary.argtypes = [vp, i64, i64, vp, vp]
         lib.orc_act_quant_int8.argtypes = [vp, i32, i64, i64, vp, vp]
-        lib.orc_gemm_a16.argtypes = [vp, i32, i64, i64, vp, i64, i32, i32, i64, vp, vp, vp,
+        lib.orc_gemm_a16.argtypes = [vp, i32, i64, i64, vp, i64, i32, i32, i32, i64, vp, vp, vp,
                                      vp, i64, vp, i64, vp, vp, i32]
         lib.orc_gemm_a8.argtypes = [vp, vp, i64, i64, vp, i64, i32, i32, i64, vp, vp, vp,
                                     vp, i64, vp, i64, vp, vp, vp, i32]
@@ -118,6 +126,16 @@ def bf16_bits_to_f64(h) -> np.ndarray:
     return np.array([L.orc_bf16_to_f64(int(v)) for v in h.ravel()], dtype=np.float64).reshape(h.shape)
 
 
+def minifloat_value(fmt: int, code: int) -> float:
+    """Value of an e2m1 (FMT_E2M1, codes 0..15) or e4m3 (FMT_E4M3, codes 0..255) code."""
+    return _L().orc_minifloat_value(fmt, int(code))
+
+
+def minifloat_encode(fmt: int, x: float) -> int:
+    """Code of the format's value nearest to x (|x| <= 6 or 448), ties to even, +0 for zero."""
+    return _L().orc_minifloat_encode(fmt, float(x))
+
+
 def exact_abs_sum_f32(x) -> float:
     x = np.ascontiguousarray(x, dtype=np.float32)
     return _L().orc_exact_abs_sum_f32(_p(x), x.size)
@@ -125,7 +143,7 @@ def exact_abs_sum_f32(x) -> float:
 
 # ---------------------------------------------------------------- packing
 def pack(fields, bits: int) -> np.ndarray:
-    """Pack unsigned field values [N,K] (0..15 or 0..3) into bytes [N, K*bits/8]."""
+    """Pack unsigned field values [N,K] (0..2^bits - 1; bits 8, 4, 2 or 1) into bytes [N, K*bits/8]."""
     f = np.ascontiguousarray(fields, dtype=np.uint8)
     N, K = f.shape
     out = np.zeros((N, K * bits // 8), dtype=np.uint8)
@@ -133,11 +151,12 @@ def pack(fields, bits: int) -> np.ndarray:
     return out
 
 
-def unpack(Wq, N: int, K: int, bits: int, symmetric: bool) -> np.ndarray:
-    """Signed codes [N,K]: symmetric INT4 nibble-8, asymmetric INT4 nibble, INT2 two's complement."""
+def unpack(Wq, N: int, K: int, bits: int, symmetric: bool, fmt: int = FMT_INT) -> np.ndarray:
+    """Integer formats: signed codes [N,K] (symmetric INT4 nibble-8, asymmetric INT4 nibble,
+    INT2 two's complement, INT1 2c-1).  e2m1 / e4m3: the raw codes, as int8 storage."""
     Wq = np.ascontiguousarray(Wq, dtype=np.uint8)
     q = np.zeros((N, K), dtype=np.int8)
-    _check(_L().orc_unpack(_p(Wq), N, K, bits, int(bool(symmetric)), _p(q)), "unpack")
+    _check(_L().orc_unpack(_p(Wq), N, K, bits, fmt, int(bool(symmetric)), _p(q)), "unpack")
     return q
 
 
@@ -167,6 +186,27 @@ def quantize_ternary(W):
     return Wq, s
 
 
+def quantize_minifloat(W, group_size: int = 128, fmt: int = FMT_E2M1):
+    """e2m1 (packed two per byte, like INT4) or e4m3 (one byte each) codes with per-group
+    binary16 scales.  Returns (Wq uint8 [N, K/2] or [N, K], scales f16-bits uint16 [N, G])."""
+    W = np.ascontiguousarray(W, dtype=np.float32)
+    N, K = W.shape
+    Wq = np.zeros((N, K // 2 if fmt == FMT_E2M1 else K), dtype=np.uint8)
+    s = np.zeros((N, K // group_size), dtype=np.uint16)
+    _check(_L().orc_quant_minifloat(_p(W), N, K, group_size, fmt, _p(Wq), _p(s)), "quant_minifloat")
+    return Wq, s
+
+
+def quantize_binary(W):
+    """INT1: returns (Wq uint8 [N, K/8], scale float32 array of shape [1])."""
+    W = np.ascontiguousarray(W, dtype=np.float32)
+    N, K = W.shape
+    Wq = np.zeros((N, K // 8), dtype=np.uint8)
+    s = np.zeros(1, dtype=np.float32)
+    _check(_L().orc_quant_binary(_p(W), N, K, _p(Wq), _p(s)), "quant_binary")
+    return Wq, s
+
+
 def act_quant_int8(A_bits, a_dtype: int = F16):
     """A: uint16 bit patterns [M,K] of binary16 (F16) or bfloat16 (BF16).
     Returns (Aq int8 [M,K], a_scale float32 [M])."""
@@ -187,7 +227,7 @@ def _idx(sel):
 
 
 def gemm_a16(A_bits, a_dtype, Wq, N, K, bits, symmetric, group_size, scales, zeros=None, bias_bits=None,
-             m_idx=None, n_idx=None, threads=None):
+             m_idx=None, n_idx=None, threads=None, fmt: int = FMT_INT):
     """Returns (C_exact float64 [m,n], C_out uint16 bits [m,n] in A's dtype)."""
     A = np.ascontiguousarray(A_bits, dtype=np.uint16)
     M = A.shape[0]
@@ -197,11 +237,12 @@ def gemm_a16(A_bits, a_dtype, Wq, N, K, bits, symmetric, group_size, scales, zer
     nc = nc if ni is not None else N
     Ce = np.zeros((mc, nc), dtype=np.float64)
     Co = np.zeros((mc, nc), dtype=np.uint16)
-    sc = np.ascontiguousarray(scales, dtype=np.float32 if bits == 2 else np.uint16)
+    per_tensor = fmt == FMT_INT and bits <= 2
+    sc = np.ascontiguousarray(scales, dtype=np.float32 if per_tensor else np.uint16)
     z = None if zeros is None else np.ascontiguousarray(zeros, dtype=np.uint16)
     b = None if bias_bits is None else np.ascontiguousarray(bias_bits, dtype=np.uint16)
     Wq = np.ascontiguousarray(Wq, dtype=np.uint8)
-    rc = _L().orc_gemm_a16(_p(A), a_dtype, M, K, _p(Wq), N, bits, int(bool(symmetric)), group_size,
+    rc = _L().orc_gemm_a16(_p(A), a_dtype, M, K, _p(Wq), N, bits, fmt, int(bool(symmetric)), group_size,
                            _p(sc), _p(z), _p(b), _p(mi), mc, _p(ni), nc, _p(Ce), _p(Co),
                            threads or os.cpu_count() or 1)
     _check(rc, "gemm_a16")
@@ -218,11 +259,11 @@ def gemm_a8(Aq, a_scale, Wq, N, K, bits, symmetric, group_size, scales, zeros=No
     ni, nc = _idx(n_idx)
     mc = mc if mi is not None else M
     nc = nc if ni is not None else N
-    G = 1 if bits == 2 else K // group_size
+    G = 1 if bits <= 2 else K // group_size
     Ce = np.zeros((mc, nc), dtype=np.float64)
     Co = np.zeros((mc, nc), dtype=np.uint16)
     acc = np.zeros((mc, nc, G), dtype=np.int32) if want_acc else None
-    sc = np.ascontiguousarray(scales, dtype=np.float32 if bits == 2 else np.uint16)
+    sc = np.ascontiguousarray(scales, dtype=np.float32 if bits <= 2 else np.uint16)
     z = None if zeros is None else np.ascontiguousarray(zeros, dtype=np.uint16)
     b = None if bias_bits is None else np.ascontiguousarray(bias_bits, dtype=np.uint16)
     Wq = np.ascontiguousarray(Wq, dtype=np.uint8)

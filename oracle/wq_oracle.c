@@ -52,6 +52,22 @@
  *     in bits 4..7 (INT2: element 4j+i in bits 2i..2i+1);
  *   - degenerate groups (scale 0) quantize to code 0 (nibble 8 when symmetric).
  *
+ * The other weight types of [BB] "Main features" (FP16 x FP8 / FP4 / INT1 and
+ * INT8 x INT1; "Core advantages 3": INT1 is 1/16 of the FP16 bytes).  The page
+ * names the types only; the readings are:
+ *   - FP4 = e2m1 (1 sign, 2 exponent bits with bias 1, 1 mantissa bit; values
+ *     0, 0.5, 1, 1.5, 2, 3, 4, 6 and their negatives), FP8 = e4m3 (1 sign,
+ *     4 exponent bits with bias 7, 3 mantissa bits, no infinities, largest
+ *     finite 448);  per group of gs elements along K: scale = binary16 of
+ *     absmax / 6 (e2m1) or absmax / 448 (e4m3), the stored value used; code =
+ *     the format's value nearest to w / scale (binary32 quotient, clipped to
+ *     the largest finite value), ties to the even last mantissa bit; a
+ *     magnitude that rounds to 0 is the code +0; scale 0 gives code 0.  FP4
+ *     packs like INT4, FP8 is one byte per element;
+ *   - INT1 = binary weights: one binary32 scale per tensor equal to mean |w|
+ *     (as for ternary), code c = 1 when w >= 0 else 0, value (2c - 1) * scale;
+ *     element 8j+i in bit i of byte j.
+ *
  * Build: gcc -O2 -std=c11 -ffp-contract=off -fno-fast-math -fPIC -shared -pthread
  * (IEEE binary32 / binary64 arithmetic on SSE, round to nearest even).
  */
@@ -66,6 +82,8 @@
 #define ORC_ERR_OVERFLOW 2
 
 enum { ORC_F16 = 1, ORC_BF16 = 2 };
+/* weight formats: integer codes (INT4 / INT2 / INT1 by `bits`), e2m1, e4m3 */
+enum { ORC_FMT_INT = 0, ORC_FMT_E2M1 = 1, ORC_FMT_E4M3 = 2 };
 
 /* ------------------------------------------------------------------------ */
 /* binary16 / bfloat16 rounding, from the IEEE 754 definition                */
@@ -129,6 +147,37 @@ double orc_bf16_to_f64(uint16_t h)
     return (double)f;
 }
 
+/* e2m1 / e4m3 (sign | exponent | mantissa, the layouts of the readings above):
+ * value of a code from the definition of a binary format with a subnormal
+ * binade, and the code of a value the format holds (searched in the code
+ * table, so that encode and decode cannot disagree). */
+double orc_minifloat_value(int fmt, int code)
+{
+    int eb = fmt == ORC_FMT_E2M1 ? 2 : 4, mb = fmt == ORC_FMT_E2M1 ? 1 : 3;
+    int bias = fmt == ORC_FMT_E2M1 ? 1 : 7;
+    int sign = (code >> (eb + mb)) & 1, e = (code >> mb) & ((1 << eb) - 1), m = code & ((1 << mb) - 1);
+    if (fmt == ORC_FMT_E4M3 && e == 15 && m == 7) return NAN;
+    double v = e == 0 ? ldexp((double)m, 1 - bias - mb)                    /* subnormal: m * 2^(1-bias-mb) */
+                      : ldexp((double)((1 << mb) + m), e - bias - mb);     /* (1 + m / 2^mb) * 2^(e-bias) */
+    return sign ? -v : v;
+}
+
+static double minifloat_max(int fmt) { return fmt == ORC_FMT_E2M1 ? 6.0 : 448.0; }
+
+/* Round x (|x| <= the format's largest finite value) to the format: nearest,
+ * ties to even (the generic binary rounding above with p = mantissa bits + 1
+ * and the smallest normal 2^(1-bias)); returns the code, +0 for a zero result. */
+int orc_minifloat_encode(int fmt, double x)
+{
+    int p = fmt == ORC_FMT_E2M1 ? 2 : 4, emin = fmt == ORC_FMT_E2M1 ? 0 : -6;
+    int ncode = fmt == ORC_FMT_E2M1 ? 16 : 256;
+    double r = round_to_format(x, p, emin, minifloat_max(fmt));
+    if (r == 0.0) return 0;
+    for (int c = 0; c < ncode; ++c)
+        if (orc_minifloat_value(fmt, c) == r) return c;
+    return -1;                                      /* not reached for |x| <= max */
+}
+
 static double act_value(const uint16_t *A, int dt, int64_t i)
 {
     return dt == ORC_BF16 ? orc_bf16_to_f64(A[i]) : orc_f16_to_f64(A[i]);
@@ -165,34 +214,63 @@ int orc_pack(const uint8_t *fields, int64_t N, int64_t K, int bits, uint8_t *out
             }
         return ORC_OK;
     }
+    if (bits == 1) {
+        if (K % 8) return ORC_ERR_ARG;
+        for (int64_t n = 0; n < N; ++n)
+            for (int64_t j = 0; j < K / 8; ++j) {
+                uint8_t b = 0;
+                for (int i = 0; i < 8; ++i) b |= (uint8_t)((fields[n * K + 8 * j + i] & 1) << i);
+                out[n * (K / 8) + j] = b;
+            }
+        return ORC_OK;
+    }
+    if (bits == 8) {
+        memcpy(out, fields, (size_t)(N * K));
+        return ORC_OK;
+    }
     return ORC_ERR_ARG;
 }
 
 /* Field value of element k of row n. */
 static int field_at(const uint8_t *Wq, int64_t K, int bits, int64_t n, int64_t k)
 {
+    if (bits == 8) return Wq[n * K + k];
     if (bits == 4) {
         uint8_t b = Wq[n * (K / 2) + k / 2];
         return (k & 1) ? (b >> 4) : (b & 15);
     }
+    if (bits == 1) return (Wq[n * (K / 8) + k / 8] >> (k & 7)) & 1;
     uint8_t b = Wq[n * (K / 4) + k / 4];
     return (b >> (2 * (k & 3))) & 3;
 }
 
-/* Signed code of a field: symmetric INT4 nibble - 8, asymmetric INT4 nibble
- * unchanged, INT2 two's complement. */
+/* Signed code of an integer field: symmetric INT4 nibble - 8, asymmetric INT4
+ * nibble unchanged, INT2 two's complement, INT1 2c - 1. */
 static int code_of(int field, int bits, int symmetric)
 {
     if (bits == 4) return symmetric ? field - 8 : field;
+    if (bits == 1) return 2 * field - 1;
     return field >= 2 ? field - 4 : field;
 }
 
-int orc_unpack(const uint8_t *Wq, int64_t N, int64_t K, int bits, int symmetric, int8_t *q)
+/* Bits per element of a weight format, 0 if the pair is not one. */
+static int format_bits(int fmt, int bits)
 {
-    if ((bits != 4 && bits != 2) || K % (8 / bits)) return ORC_ERR_ARG;
+    if (fmt == ORC_FMT_INT) return (bits == 4 || bits == 2 || bits == 1) ? bits : 0;
+    if (fmt == ORC_FMT_E2M1) return bits == 4 ? 4 : 0;
+    if (fmt == ORC_FMT_E4M3) return bits == 8 ? 8 : 0;
+    return 0;
+}
+
+/* Integer formats: the signed codes; e2m1 / e4m3: the raw codes (as bytes). */
+int orc_unpack(const uint8_t *Wq, int64_t N, int64_t K, int bits, int fmt, int symmetric, int8_t *q)
+{
+    if (!format_bits(fmt, bits) || K % (8 / (bits < 8 ? bits : 8))) return ORC_ERR_ARG;
     for (int64_t n = 0; n < N; ++n)
-        for (int64_t k = 0; k < K; ++k)
-            q[n * K + k] = (int8_t)code_of(field_at(Wq, K, bits, n, k), bits, symmetric);
+        for (int64_t k = 0; k < K; ++k) {
+            int f = field_at(Wq, K, bits, n, k);
+            q[n * K + k] = (int8_t)(fmt == ORC_FMT_INT ? code_of(f, bits, symmetric) : f);
+        }
     return ORC_OK;
 }
 
@@ -324,6 +402,50 @@ int orc_quant_ternary(const float *W, int64_t N, int64_t K, uint8_t *Wq, float *
     return rc;
 }
 
+/* e2m1 / e4m3 per group of gs elements along K ([BB] "Main features", with
+ * the group scheme of "Advanced features 2"). scales: binary16 bits [N, K/gs]. */
+int orc_quant_minifloat(const float *W, int64_t N, int64_t K, int64_t gs, int fmt, uint8_t *Wq, uint16_t *scales)
+{
+    if ((fmt != ORC_FMT_E2M1 && fmt != ORC_FMT_E4M3) || gs <= 0 || K % gs || K % 2) return ORC_ERR_ARG;
+    int64_t G = K / gs;
+    float fmax = (float)minifloat_max(fmt);
+    uint8_t *fields = (uint8_t *)malloc((size_t)(N * K));
+    if (!fields) return ORC_ERR_ARG;
+    for (int64_t n = 0; n < N; ++n)
+        for (int64_t g = 0; g < G; ++g) {
+            const float *w = W + n * K + g * gs;
+            float amax = 0.0f;
+            for (int64_t i = 0; i < gs; ++i) amax = fmaxf(amax, fabsf(w[i]));
+            uint16_t sh = orc_f64_to_f16((double)(amax / fmax));
+            float s = (float)orc_f16_to_f64(sh);
+            scales[n * G + g] = sh;
+            for (int64_t i = 0; i < gs; ++i) {
+                int c = 0;
+                if (s != 0.0f) c = orc_minifloat_encode(fmt, (double)clampf(w[i] / s, -fmax, fmax));
+                if (c < 0) { free(fields); return ORC_ERR_ARG; }
+                fields[n * K + g * gs + i] = (uint8_t)c;
+            }
+        }
+    int rc = orc_pack(fields, N, K, fmt == ORC_FMT_E2M1 ? 4 : 8, Wq);
+    free(fields);
+    return rc;
+}
+
+/* Binary (INT1) quantization with one binary32 scale per tensor:
+ * scale_out[0] = mean |w| (as for ternary); bit 1 for w >= 0, eight per byte. */
+int orc_quant_binary(const float *W, int64_t N, int64_t K, uint8_t *Wq, float *scale_out)
+{
+    if (K % 8) return ORC_ERR_ARG;
+    double sum = orc_exact_abs_sum_f32(W, N * K);
+    scale_out[0] = (float)(sum / (double)(N * K));
+    uint8_t *fields = (uint8_t *)malloc((size_t)(N * K));
+    if (!fields) return ORC_ERR_ARG;
+    for (int64_t i = 0; i < N * K; ++i) fields[i] = W[i] >= 0.0f ? 1 : 0;
+    int rc = orc_pack(fields, N, K, 1, Wq);
+    free(fields);
+    return rc;
+}
+
 /* ------------------------------------------------------------------------ */
 /* activation quantization ([CG] step 2), per token                          */
 /* ------------------------------------------------------------------------ */
@@ -354,7 +476,7 @@ typedef struct {
     const uint16_t *A; int a_dt;                 /* A16 */
     const int8_t *Aq; const float *a_scale;      /* A8 */
     int64_t M, N, K;
-    const uint8_t *Wq; int bits, symmetric; int64_t gs;
+    const uint8_t *Wq; int bits, fmt, symmetric; int64_t gs;
     const uint16_t *scales16; const float *scale32; const uint16_t *zeros; const uint16_t *bias;
     /* selection */
     const int64_t *m_idx; int64_t m_cnt;
@@ -367,12 +489,18 @@ typedef struct {
 
 static int64_t sel(const int64_t *idx, int64_t j) { return idx ? idx[j] : j; }
 
-/* Dequantized weight w[n,k] = (q - z) * s, exact in binary64 (|q - z| <= 15,
+/* Dequantized weight w[n,k] = (q - z) * s, or value(code) * s for e2m1 / e4m3,
+ * exact in binary64 (|q - z| <= 15, a code value has at most 4 significant bits,
  * s a binary16 or binary32 value). */
 static double dequant_weight(const job_t *J, int64_t n, int64_t k)
 {
-    int c = code_of(field_at(J->Wq, J->K, J->bits, n, k), J->bits, J->symmetric);
-    if (J->bits == 2) return (double)c * (double)J->scale32[0];
+    int f = field_at(J->Wq, J->K, J->bits, n, k);
+    if (J->fmt != ORC_FMT_INT) {
+        int64_t G = J->K / J->gs;
+        return orc_minifloat_value(J->fmt, f) * orc_f16_to_f64(J->scales16[n * G + k / J->gs]);
+    }
+    int c = code_of(f, J->bits, J->symmetric);
+    if (J->bits <= 2) return (double)c * (double)J->scale32[0];
     int64_t G = J->K / J->gs, g = k / J->gs;
     double s = orc_f16_to_f64(J->scales16[n * G + g]);
     double z = (J->symmetric || !J->zeros) ? 0.0 : orc_f16_to_f64(J->zeros[n * G + g]);
@@ -403,8 +531,8 @@ static void *run_a16(void *arg)
 static void *run_a8(void *arg)
 {
     job_t *J = (job_t *)arg;
-    int64_t G = J->bits == 2 ? 1 : J->K / J->gs;
-    int64_t glen = J->bits == 2 ? J->K : J->gs;
+    int64_t G = J->bits <= 2 ? 1 : J->K / J->gs;
+    int64_t glen = J->bits <= 2 ? J->K : J->gs;
     int32_t *qz = (int32_t *)malloc((size_t)J->K * sizeof(int32_t));
     if (!qz) { J->status = ORC_ERR_ARG; return NULL; }
     for (int64_t j = J->j0; j < J->j1; ++j) {
@@ -429,7 +557,7 @@ static void *run_a8(void *arg)
                     acc += (int64_t)J->Aq[m * J->K + k] * (int64_t)qz[k];
                 if (acc > INT32_MAX || acc < INT32_MIN) J->status = ORC_ERR_OVERFLOW;
                 if (J->acc_out) J->acc_out[(i * J->n_cnt + j) * G + g] = (int32_t)acc;
-                double s = J->bits == 2 ? (double)J->scale32[0] : orc_f16_to_f64(J->scales16[n * G + g]);
+                double s = J->bits <= 2 ? (double)J->scale32[0] : orc_f16_to_f64(J->scales16[n * G + g]);
                 total += s * (double)acc;
             }
             double c = (double)J->a_scale[m] * total;   /* (w_scale * a_scale) dequantization */
@@ -463,30 +591,31 @@ static int run_threads(job_t *proto, void *(*fn)(void *), int threads)
     return rc;
 }
 
-static int check_weights(int64_t K, int bits, int64_t gs)
+static int check_weights(int64_t K, int bits, int fmt, int64_t gs)
 {
-    if (bits == 4) return (gs > 0 && K % gs == 0 && K % 2 == 0) ? ORC_OK : ORC_ERR_ARG;
-    if (bits == 2) return K % 4 == 0 ? ORC_OK : ORC_ERR_ARG;
-    return ORC_ERR_ARG;
+    if (!format_bits(fmt, bits)) return ORC_ERR_ARG;
+    if (fmt != ORC_FMT_INT || bits == 4) return (gs > 0 && K % gs == 0 && K % 2 == 0) ? ORC_OK : ORC_ERR_ARG;
+    return K % (8 / bits) == 0 ? ORC_OK : ORC_ERR_ARG;
 }
 
-/* W4A16 / W2A16:  C[m,n] = sum_k A[m,k] * (q[n,k] - z[n,g(k)]) * s[n,g(k)]  (+ bias[n])
- * accumulated in binary64 in k order, then rounded once to A's dtype.
- * scales: binary16 [N, K/gs] (INT4) or one binary32 (INT2). zeros: binary16 or NULL.
- * m_idx / n_idx select the computed rows / columns (NULL = all);
+/* W4A16 / W2A16 / W1A16:  C[m,n] = sum_k A[m,k] * (q[n,k] - z[n,g(k)]) * s[n,g(k)]  (+ bias[n])
+ * accumulated in binary64 in k order, then rounded once to A's dtype; for e2m1 / e4m3
+ * weights (q - z) is the code's value.
+ * scales: binary16 [N, K/gs] (INT4, e2m1, e4m3) or one binary32 (INT2, INT1).
+ * zeros: binary16 or NULL.  m_idx / n_idx select the computed rows / columns (NULL = all);
  * outputs are [m_cnt, n_cnt]. */
 int orc_gemm_a16(const uint16_t *A, int a_dt, int64_t M, int64_t K,
-                 const uint8_t *Wq, int64_t N, int bits, int symmetric, int64_t gs,
+                 const uint8_t *Wq, int64_t N, int bits, int fmt, int symmetric, int64_t gs,
                  const void *scales, const uint16_t *zeros, const uint16_t *bias,
                  const int64_t *m_idx, int64_t m_cnt, const int64_t *n_idx, int64_t n_cnt,
                  double *C_exact, uint16_t *C_out, int threads)
 {
-    if ((a_dt != ORC_F16 && a_dt != ORC_BF16) || check_weights(K, bits, gs) || M < 0 || N < 0)
+    if ((a_dt != ORC_F16 && a_dt != ORC_BF16) || check_weights(K, bits, fmt, gs) || M < 0 || N < 0)
         return ORC_ERR_ARG;
     job_t J;
     memset(&J, 0, sizeof J);
     J.A = A; J.a_dt = a_dt; J.M = M; J.N = N; J.K = K;
-    J.Wq = Wq; J.bits = bits; J.symmetric = symmetric; J.gs = gs;
+    J.Wq = Wq; J.bits = bits; J.fmt = fmt; J.symmetric = symmetric; J.gs = gs;
     J.scales16 = (const uint16_t *)scales; J.scale32 = (const float *)scales;
     J.zeros = zeros; J.bias = bias;
     J.m_idx = m_idx; J.m_cnt = m_idx ? m_cnt : M;
@@ -495,11 +624,11 @@ int orc_gemm_a16(const uint16_t *A, int a_dt, int64_t M, int64_t K,
     return run_threads(&J, run_a16, threads);
 }
 
-/* W4A8 / W2A8:  acc_g[m,n] = sum_{k in group g} Aq[m,k] * (q[n,k] - z[n,g])   (exact integer)
+/* W4A8 / W2A8 / W1A8:  acc_g[m,n] = sum_{k in group g} Aq[m,k] * (q[n,k] - z[n,g])   (exact integer)
  *               C[m,n] = fp16( a_scale[m] * sum_g s[n,g] * acc_g[m,n]  (+ bias[n]) )
  * The integer dot product is the DP4A definition; the float scale is applied
- * after integer accumulation.  INT2 weights have one group spanning all of K
- * and one binary32 scale.  acc_out (optional): int32 [m_cnt, n_cnt, G].
+ * after integer accumulation.  INT2 and INT1 weights have one group spanning all
+ * of K and one binary32 scale.  acc_out (optional): int32 [m_cnt, n_cnt, G].
  * Returns ORC_ERR_OVERFLOW if some group sum leaves the int32 range. */
 int orc_gemm_a8(const int8_t *Aq, const float *a_scale, int64_t M, int64_t K,
                 const uint8_t *Wq, int64_t N, int bits, int symmetric, int64_t gs,
@@ -507,7 +636,7 @@ int orc_gemm_a8(const int8_t *Aq, const float *a_scale, int64_t M, int64_t K,
                 const int64_t *m_idx, int64_t m_cnt, const int64_t *n_idx, int64_t n_cnt,
                 double *C_exact, uint16_t *C_out, int32_t *acc_out, int threads)
 {
-    if (check_weights(K, bits, gs) || M < 0 || N < 0) return ORC_ERR_ARG;
+    if (check_weights(K, bits, ORC_FMT_INT, gs) || M < 0 || N < 0) return ORC_ERR_ARG;
     job_t J;
     memset(&J, 0, sizeof J);
     J.Aq = Aq; J.a_scale = a_scale; J.M = M; J.N = N; J.K = K;
