@@ -56,13 +56,13 @@ def alg_bytes(c: wq_synth.Case) -> int:
     activations once and the output once.  The INT8 paths start from fp16 activations (the
     per-token quantization is part of the step), so they too read M*K*2 bytes of A; the
     INT8 copy of A and its scales are intermediate values, not counted."""
-    bits = 2 if c.quant == "tern2" else 4
+    bits = wq_synth.QUANT_BITS[c.quant]
     w = c.N * c.K * bits // 8
-    if bits == 4:
+    if c.quant in ("tern2", "int1"):
+        w += 4  # one binary32 scale
+    else:
         G = c.K // c.group_size
         w += c.N * G * 2 * (2 if c.quant == "asym4" else 1)
-    else:
-        w += 4
     a = c.M * c.K * 2
     return w + a + c.M * c.N * 2
 
@@ -185,6 +185,19 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------------ our arm
+def quant_config(c: wq_synth.Case):
+    import gemv_wq_quantize_b200 as wq
+    if c.quant == "tern2":
+        return wq.QuantConfig(bits=2)
+    if c.quant == "int1":
+        return wq.QuantConfig(bits=1)
+    if c.quant == "e2m1":
+        return wq.QuantConfig(bits=4, group_size=c.group_size, format=wq.FMT_E2M1)
+    if c.quant == "e4m3":
+        return wq.QuantConfig(bits=8, group_size=c.group_size, format=wq.FMT_E4M3)
+    return wq.QuantConfig(bits=4, group_size=c.group_size, symmetric=(c.quant == "sym4"))
+
+
 class Prepared:
     """Quantized weight copies, activations and outputs of one case on the device."""
 
@@ -194,8 +207,7 @@ class Prepared:
         import gemv_wq_quantize_b200 as wq
         self.c = c
         self.fused = fused
-        self.qc = wq.QuantConfig(bits=2) if c.quant == "tern2" else \
-            wq.QuantConfig(bits=4, group_size=c.group_size, symmetric=(c.quant == "sym4"))
+        self.qc = quant_config(c)
         W = wq_synth.weights(c.N, c.K, seed=seed_base).to(device)
         Wq, s, z = wq.quantize_pack(W, self.qc)
         del W
@@ -412,8 +424,11 @@ def per_case_breakdown(preps, reps: int = 200):
 
 
 # Workloads timed beside the headline one in the default run, each as its own object of the
-# JSON line: the prefill GEMMs (the tensor-bound half of the metric), W4A8 and the BitNet sweep.
-EXTRA_WORKLOADS = (("gemm", "prefill-llama7b"), ("w4a8", "w4a8"), ("bitnet3b", "bitnet3b"))
+# JSON line: the prefill GEMMs (the tensor-bound half of the metric), W4A8, the BitNet sweep
+# and the other weight types (FP4, FP8, INT1) at decode and at prefill.
+EXTRA_WORKLOADS = (("gemm", "prefill-llama7b"), ("w4a8", "w4a8"), ("bitnet3b", "bitnet3b"),
+                   ("formats_decode", "formats-decode"), ("formats_prefill", "formats-prefill"))
+TENSOR_BOUND = ("prefill-llama7b", "formats-prefill")
 
 
 def measure_extra(name: str, device, steps: int, warmup: int, dist_on: bool) -> dict:
@@ -437,7 +452,7 @@ def measure_extra(name: str, device, steps: int, warmup: int, dist_on: bool) -> 
     out = {"workload": name, "description": wl.description, "steps": steps, "warmup": warmup,
            "ms_per_step": round(sec / steps * 1e3, 6), "GB/s": round(gbs, 2), "TFLOP/s": round(tf, 2),
            "gpu_launches": steps * sum(launches_per_call(p.c) for p in preps), "clocks": sampler.report()}
-    if name == "prefill-llama7b":
+    if name in TENSOR_BOUND:
         out["roofline"] = {"bound": "tensor", "achieved": round(tf, 2), "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
                            "frac": round(tf / pk["bf16_tflops"], 4), "peak_sustained": pk["bf16_tflops_sustained"],
                            "frac_sustained": round(tf / pk["bf16_tflops_sustained"], 4),
@@ -614,31 +629,44 @@ def oracle_sample(wl, budget_s: float, threads: int):
     import oracle
     oracle.build()
     prepared = []
+    max_frac = 1.0 / 16  # the sample never covers more output columns than this
     for c in wl.cases:
-        W = wq_synth.weights(c.N, c.K, seed=0).numpy()
+        # only the weight rows a sample can use are quantized (codes and group scales are
+        # per row; the per-tensor scale of INT2 / INT1 then comes from these rows)
+        W = wq_synth.weights(c.N, c.K, seed=0).numpy()[:max(1, math.ceil(c.N * max_frac))]
         A = wq_synth.activations(c.M, c.K, seed=1, dtype=c.a_dtype, outlier_frac=c.outlier_frac)
         Abits = A.contiguous().view(torch.int16).numpy().view(np.uint16)
+        fmt = oracle.FMT_INT
         if c.quant == "tern2":
             Wq, s = oracle.quantize_ternary(W)
             z, bits, sym = None, 2, True
+        elif c.quant == "int1":
+            Wq, s = oracle.quantize_binary(W)
+            z, bits, sym = None, 1, True
+        elif c.quant in ("e2m1", "e4m3"):
+            fmt = oracle.FMT_E2M1 if c.quant == "e2m1" else oracle.FMT_E4M3
+            Wq, s = oracle.quantize_minifloat(W, c.group_size, fmt)
+            z, bits, sym = None, wq_synth.QUANT_BITS[c.quant], True
         else:
             Wq, s, z = oracle.quantize_int4(W, c.group_size, c.quant == "sym4")
             bits, sym = 4, c.quant == "sym4"
-        prepared.append((c, Abits, Wq, s, z, bits, sym))
+        prepared.append((c, Abits, Wq, s, z, bits, sym, fmt))
 
     def run(frac):
         t = 0.0
         covered = 0.0
-        for c, Abits, Wq, s, z, bits, sym in prepared:
-            n_cnt = max(1, int(round(c.N * frac)))
-            ni = np.arange(n_cnt) * (c.N // n_cnt)
+        for c, Abits, Wq, s, z, bits, sym, fmt in prepared:
+            rows = Wq.shape[0]
+            n_cnt = min(rows, max(1, int(round(c.N * frac))))
+            ni = np.arange(n_cnt)
             t0 = time.perf_counter()
             if c.mode == "a16":
                 adt = oracle.F16 if c.a_dtype == torch.float16 else oracle.BF16
-                oracle.gemm_a16(Abits, adt, Wq, c.N, c.K, bits, sym, c.group_size, s, z, n_idx=ni, threads=threads)
+                oracle.gemm_a16(Abits, adt, Wq, rows, c.K, bits, sym, c.group_size, s, z, n_idx=ni, threads=threads,
+                                fmt=fmt)
             else:
                 Aq, asc = oracle.act_quant_int8(Abits, oracle.F16)
-                oracle.gemm_a8(Aq, asc, Wq, c.N, c.K, bits, sym, c.group_size, s, z, n_idx=ni, threads=threads)
+                oracle.gemm_a8(Aq, asc, Wq, rows, c.K, bits, sym, c.group_size, s, z, n_idx=ni, threads=threads)
             t += time.perf_counter() - t0
             covered += alg_bytes(c) * n_cnt / c.N
         return covered, t
@@ -646,7 +674,7 @@ def oracle_sample(wl, budget_s: float, threads: int):
     frac = 1.0 / 512
     covered, t = run(frac)
     if t < budget_s / 4:
-        frac = min(1.0, frac * budget_s / max(t, 1e-3) / 2)
+        frac = min(max_frac, frac * budget_s / max(t, 1e-3) / 2)
         covered, t = run(frac)
     desc = f"oracle on {frac:.4%} of the output columns of every case (all tokens), {threads} threads"
     return covered, t, desc

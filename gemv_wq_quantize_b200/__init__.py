@@ -1,4 +1,4 @@
-"""Python binding of libwq: INT4 / INT2 weight-quantized matmul on B200 (sm_100a).
+"""Python binding of libwq: INT4 / INT2 / INT1 / FP4 / FP8 weight-quantized matmul on B200 (sm_100a).
 
 Thin ctypes marshalling over the C ABI declared in ``include/wq.h``: it checks
 tensor devices / dtypes, allocates outputs with torch, passes raw device pointers
@@ -40,23 +40,33 @@ class WqError(RuntimeError):
 
 class QConfig(ctypes.Structure):
     _fields_ = [("bits", ctypes.c_int32), ("group_size", ctypes.c_int32), ("symmetric", ctypes.c_int32),
-                ("ternary", ctypes.c_int32), ("layout", ctypes.c_int32)]
+                ("ternary", ctypes.c_int32), ("layout", ctypes.c_int32), ("format", ctypes.c_int32)]
 
 
 LAYOUT_NT, LAYOUT_NATIVE = 0, 1
+FMT_INT, FMT_E2M1, FMT_E4M3 = 0, 1, 2
 
 
 @dataclass(frozen=True)
 class QuantConfig:
-    """bits 4 (group scales, optional zero points) or 2 (ternary, one scale per tensor);
-    layout LAYOUT_NT (the packing of wq_quantize_pack) or LAYOUT_NATIVE (after repack)."""
+    """Integer codes (format FMT_INT): bits 4 (group scales, optional zero points), 2 (ternary)
+    or 1 (binary), the last two with one scale per tensor.  format FMT_E2M1 (bits 4) or
+    FMT_E4M3 (bits 8): FP4 / FP8 codes with group scales.  layout LAYOUT_NT (the packing of
+    wq_quantize_pack) or LAYOUT_NATIVE (INT4 after repack)."""
     bits: int = 4
     group_size: int = 128
     symmetric: bool = True
     layout: int = LAYOUT_NT
+    format: int = FMT_INT
+
+    @property
+    def per_tensor_scale(self) -> bool:
+        """One binary32 scale for the tensor (INT2, INT1) instead of binary16 group scales."""
+        return self.format == FMT_INT and self.bits <= 2
 
     def c(self) -> QConfig:
-        return QConfig(self.bits, self.group_size, int(self.symmetric), int(self.bits == 2), self.layout)
+        return QConfig(self.bits, self.group_size, int(self.symmetric), int(self.bits == 2), self.layout,
+                       self.format)
 
 
 class MatmulDesc(ctypes.Structure):
@@ -157,16 +167,17 @@ def make_workspace(nbytes: int, device=None) -> torch.Tensor:
 def quantize_pack(W: torch.Tensor, qc: QuantConfig = QuantConfig(), stream=None):
     """Quantize and pack W [N,K] (fp32/fp16/bf16, CUDA).
 
-    Returns (Wq uint8 [N, K*bits/8], scales, zeros): scales fp16 [N, K/g] for INT4
-    (fp32 [1] for INT2), zeros fp16 [N, K/g] for asymmetric INT4 else None."""
+    Returns (Wq uint8 [N, K*bits/8], scales, zeros): scales fp16 [N, K/g] for INT4, FP4 and FP8
+    (fp32 [1] for INT2 and INT1), zeros fp16 [N, K/g] for asymmetric INT4 else None."""
     _dev(W, "W")
     N, K = W.shape
     L = load_library()
     Wq = torch.empty(N, K * qc.bits // 8, dtype=torch.uint8, device=W.device)
-    if qc.bits == 4:
+    if not qc.per_tensor_scale:
         G = K // qc.group_size if qc.group_size > 0 else 0
         scales = torch.empty(N, max(G, 1), dtype=torch.float16, device=W.device)
-        zeros = None if qc.symmetric else torch.empty(N, max(G, 1), dtype=torch.float16, device=W.device)
+        int4_asym = qc.format == FMT_INT and qc.bits == 4 and not qc.symmetric
+        zeros = torch.empty(N, max(G, 1), dtype=torch.float16, device=W.device) if int4_asym else None
     else:
         scales = torch.empty(4, dtype=torch.float32, device=W.device)[:1]
         zeros = None
@@ -179,6 +190,7 @@ def quantize_pack(W: torch.Tensor, qc: QuantConfig = QuantConfig(), stream=None)
 
 
 def unpack(Wq: torch.Tensor, N: int, K: int, qc: QuantConfig, stream=None) -> torch.Tensor:
+    """Signed integer codes [N,K] int8 (INT1: +-1), or the raw FP4 / FP8 codes (one per byte)."""
     _dev(Wq, "Wq")
     q = torch.empty(N, K, dtype=torch.int8, device=Wq.device)
     _check(load_library().wq_unpack(_ptr(Wq), N, K, qc.c(), _ptr(q), _stream(stream)), "wq_unpack")

@@ -10,6 +10,7 @@
 #include <mutex>
 #include <vector>
 
+#include "wq_format.h"
 #include "wq_host.h"
 
 namespace wq {
@@ -152,22 +153,26 @@ int read_device_errors()
 namespace {
 // Few tokens go to the weight-streaming GEMV; more tokens to the tcgen05 GEMM (the INT32
 // group sums included), or else (shapes without a plan there: K below four 128-k blocks,
-// ternary FP activations at 9..16 tokens) to the tiled mma.sync path.
-wq_status dispatch(int WB, int AM, const void *A, const float *a_scale, const uint8_t *Wq, const void *scales,
+// ternary FP activations at 9..16 tokens) to the tiled mma.sync path, which serves INT4 and
+// INT2 only.  WF: the weight format (wq_format.h).
+wq_status dispatch(int WF, int AM, const void *A, const float *a_scale, const uint8_t *Wq, const void *scales,
                    const void *zeros, const void *bias, void *C, int32_t *acc_out, int64_t M, int64_t N, int64_t K,
                    const wq_qconfig &c, void *ws, size_t ws_bytes, cudaStream_t st)
 {
     if (M <= 16) {
-        wq_status rc = gemv_small_m(WB, AM, A, a_scale, Wq, scales, zeros, bias, C, acc_out, M, N, K, c, st);
+        wq_status rc = gemv_small_m(WF, AM, A, a_scale, Wq, scales, zeros, bias, C, acc_out, M, N, K, c, st);
         if (rc != WQ_ERR_UNSUPPORTED) return rc;
     } else {
-        wq_status rc = tc_gemm(WB, AM, A, a_scale, Wq, scales, zeros, bias, C, acc_out, M, N, K, c, ws, ws_bytes, st);
+        wq_status rc = tc_gemm(WF, AM, A, a_scale, Wq, scales, zeros, bias, C, acc_out, M, N, K, c, ws, ws_bytes, st);
         if (rc != WQ_ERR_UNSUPPORTED) return rc;
     }
+    if (WF != WF_I4 && WF != WF_I2)
+        return fail(WQ_ERR_UNSUPPORTED, "no launch plan for M=%lld N=%lld K=%lld with these weights (%s)", (long long)M,
+                    (long long)N, (long long)K, wq_last_error());
     if (c.layout == WQ_LAYOUT_NATIVE)
         return fail(WQ_ERR_UNSUPPORTED, "native layout: no launch plan for M=%lld K=%lld (use WQ_LAYOUT_NT)",
                     (long long)M, (long long)K);
-    return skinny_gemm(WB, AM, A, a_scale, Wq, scales, zeros, bias, C, acc_out, M, N, K, c, ws, ws_bytes, st);
+    return skinny_gemm(WF, AM, A, a_scale, Wq, scales, zeros, bias, C, acc_out, M, N, K, c, ws, ws_bytes, st);
 }
 }  // namespace
 
@@ -182,8 +187,17 @@ wq_status check_weights(const uint8_t *Wq, const void *scales, const void *zeros
     if (!aligned16(Wq) || !aligned16(scales) || (zeros && !aligned16(zeros)))
         return fail(WQ_ERR_ALIGNMENT, "Wq, scales and zeros must be 16-byte aligned");
     if (c.layout != WQ_LAYOUT_NT && c.layout != WQ_LAYOUT_NATIVE) return fail(WQ_ERR_INVALID_ARG, "unknown layout");
-    if (c.layout == WQ_LAYOUT_NATIVE && c.bits != 4) return fail(WQ_ERR_UNSUPPORTED, "the native layout is INT4 only");
-    if (c.bits == 4) {
+    if (c.format != WQ_FMT_INT && c.format != WQ_FMT_E2M1 && c.format != WQ_FMT_E4M3)
+        return fail(WQ_ERR_INVALID_ARG, "unknown weight format %d", int(c.format));
+    if (c.layout == WQ_LAYOUT_NATIVE && (c.bits != 4 || c.format != WQ_FMT_INT))
+        return fail(WQ_ERR_UNSUPPORTED, "the native layout is INT4 only");
+    if (c.format != WQ_FMT_INT) {
+        if (c.bits != (c.format == WQ_FMT_E2M1 ? 4 : 8))
+            return fail(WQ_ERR_INVALID_ARG, "FP4 (e2m1) weights have bits 4, FP8 (e4m3) bits 8");
+        if (K % 128) return fail(WQ_ERR_INVALID_ARG, "FP4 / FP8 weights need K %% 128 == 0");
+        if (c.group_size <= 0 || K % c.group_size) return fail(WQ_ERR_INVALID_ARG, "K %% group_size != 0");
+        if (c.group_size % 128) return fail(WQ_ERR_UNSUPPORTED, "group_size must be a multiple of 128");
+    } else if (c.bits == 4) {
         if (K % 128) return fail(WQ_ERR_INVALID_ARG, "INT4 needs K %% 128 == 0");
         if (c.group_size <= 0 || K % c.group_size) return fail(WQ_ERR_INVALID_ARG, "K %% group_size != 0");
         if (c.group_size % 128) return fail(WQ_ERR_UNSUPPORTED, "group_size must be a multiple of 128");
@@ -191,9 +205,22 @@ wq_status check_weights(const uint8_t *Wq, const void *scales, const void *zeros
     } else if (c.bits == 2) {
         if (!c.ternary) return fail(WQ_ERR_UNSUPPORTED, "INT2 weights must be ternary");
         if (K % 64) return fail(WQ_ERR_INVALID_ARG, "INT2 needs K %% 64 == 0");
+    } else if (c.bits == 1) {
+        if (K % 128) return fail(WQ_ERR_INVALID_ARG, "INT1 needs K %% 128 == 0");
     } else {
-        return fail(WQ_ERR_INVALID_ARG, "bits must be 4 or 2");
+        return fail(WQ_ERR_INVALID_ARG, "bits must be 4, 2 or 1 (integer codes)");
     }
+    return WQ_OK;
+}
+
+// The activation paths of each weight type: the pairs of the BitBLAS guide's list (FP16 x
+// FP8 / FP4 / INT4 / INT2 / INT1, INT8 x INT4 / INT2 / INT1), plus BF16 with INT4 / INT2.
+wq_status check_pair(int wf, int am)
+{
+    if (am == 1 && wf != WF_I4 && wf != WF_I2)
+        return fail(WQ_ERR_UNSUPPORTED, "BF16 activations take INT4 or INT2 weights");
+    if (am == 2 && (wf == WF_E2M1 || wf == WF_E4M3))
+        return fail(WQ_ERR_UNSUPPORTED, "FP4 / FP8 weights take FP16 activations (no INT8 path)");
     return WQ_OK;
 }
 
@@ -223,10 +250,14 @@ extern "C" int wq_device_error(void) { return read_device_errors(); }
 
 extern "C" size_t wq_workspace_size(int64_t M, int64_t N, int64_t K, wq_qconfig c)
 {
-    if (M <= 0 || N <= 0 || K <= 0 || (c.bits != 4 && c.bits != 2)) return 0;
+    const bool known = (c.format == WQ_FMT_INT && (c.bits == 4 || c.bits == 2 || c.bits == 1)) ||
+                       (c.format == WQ_FMT_E2M1 && c.bits == 4) || (c.format == WQ_FMT_E4M3 && c.bits == 8);
+    if (M <= 0 || N <= 0 || K <= 0 || !known) return 0;
     // the INT8 path has the smaller activation blocks; size for the larger of the two
     if (M <= 16) return 0;  // the few-token kernel needs no workspace
-    return std::max({skinny_workspace_size(c.bits, 0, M, N, K), skinny_workspace_size(c.bits, 2, M, N, K),
+    const int wf = wf_of(c);
+    if (wf != WF_I4 && wf != WF_I2) return tc_workspace_size(M, N, K);  // no mma.sync fallback
+    return std::max({skinny_workspace_size(wf, 0, M, N, K), skinny_workspace_size(wf, 2, M, N, K),
                      tc_workspace_size(M, N, K)});
 }
 
@@ -237,6 +268,8 @@ wq_status check_a16(const void *A, wq_dtype a_dt, const uint8_t *Wq, const void 
     wq_status rc = check_weights(Wq, scales, zeros, M, N, K, c);
     if (rc != WQ_OK) return rc;
     if (a_dt != WQ_F16 && a_dt != WQ_BF16) return fail(WQ_ERR_INVALID_ARG, "a_dt must be WQ_F16 or WQ_BF16");
+    rc = check_pair(wf_of(c), a_dt == WQ_F16 ? 0 : 1);
+    if (rc != WQ_OK) return rc;
     if (!A || !C) return fail(WQ_ERR_INVALID_ARG, "A and C must be non-null");
     if (!aligned16(A) || !aligned16(C) || (bias && !aligned16(bias)))
         return fail(WQ_ERR_ALIGNMENT, "A, C and bias must be 16-byte aligned");
@@ -251,8 +284,9 @@ extern "C" wq_status w4a16_gemm(const void *A, wq_dtype a_dt, const uint8_t *Wq,
     wq_status rc = check_a16(A, a_dt, Wq, scales, zeros, bias, C, M, N, K, c);
     if (rc != WQ_OK) return rc;
     if (workspace && !aligned16(workspace)) return fail(WQ_ERR_ALIGNMENT, "workspace must be 16-byte aligned");
-    return dispatch(c.bits, a_dt == WQ_F16 ? 0 : 1, A, nullptr, Wq, scales, c.bits == 4 && !c.symmetric ? zeros : nullptr,
-                       bias, C, nullptr, M, N, K, c, workspace, ws_bytes, stream);
+    const int wf = wf_of(c);
+    return dispatch(wf, a_dt == WQ_F16 ? 0 : 1, A, nullptr, Wq, scales, wf == WF_I4 && !c.symmetric ? zeros : nullptr,
+                    bias, C, nullptr, M, N, K, c, workspace, ws_bytes, stream);
 }
 
 // W4A8 from FP activations: the per-token INT8 quantization inside the few-token matmul
@@ -271,14 +305,17 @@ extern "C" wq_status w4a8_gemm_fused(const void *A, wq_dtype a_dt, const uint8_t
     if (!aligned16(A) || !aligned16(Aq) || !aligned16(C) || (bias && !aligned16(bias)) ||
         (workspace && !aligned16(workspace)))
         return fail(WQ_ERR_ALIGNMENT, "A, Aq, C, bias and workspace must be 16-byte aligned");
-    if (acc_out && c.bits == 4 && c.group_size != 128)
+    const int wf = wf_of(c);
+    rc = check_pair(wf, 2);
+    if (rc != WQ_OK) return rc;
+    if (acc_out && wf == WF_I4 && c.group_size != 128)
         return fail(WQ_ERR_UNSUPPORTED, "acc_out needs group_size == 128");
     // Every CTA of the fused kernel reads all of A twice from L2 (maximum, then codes): worth it
     // while A is small; beyond that the separate quantization kernel is faster.
     if (M <= 16 && M * K <= kFusedMaxElems) {
         const FusedActQuant fa{A, a_dt == WQ_BF16, Aq, a_scale};
         PreparedLaunch L;
-        rc = gemv_prepare(c.bits, 2, Aq, a_scale, Wq, scales, c.bits == 4 && !c.symmetric ? zeros : nullptr, bias, C,
+        rc = gemv_prepare(wf, 2, Aq, a_scale, Wq, scales, wf == WF_I4 && !c.symmetric ? zeros : nullptr, bias, C,
                           acc_out, M, N, K, c, &L, &fa);
         if (rc == WQ_OK) return launch_prepared(L, stream, "gemv_kernel");
         if (rc != WQ_ERR_UNSUPPORTED) return rc;
@@ -297,8 +334,11 @@ extern "C" wq_status w4a8_gemm(const int8_t *Aq, const float *a_scale, const uin
     if (!Aq || !a_scale || !C) return fail(WQ_ERR_INVALID_ARG, "Aq, a_scale and C must be non-null");
     if (!aligned16(Aq) || !aligned16(C) || (bias && !aligned16(bias)) || (workspace && !aligned16(workspace)))
         return fail(WQ_ERR_ALIGNMENT, "Aq, C, bias and workspace must be 16-byte aligned");
-    if (acc_out && c.bits == 4 && c.group_size != 128)
+    const int wf = wf_of(c);
+    rc = check_pair(wf, 2);
+    if (rc != WQ_OK) return rc;
+    if (acc_out && wf == WF_I4 && c.group_size != 128)
         return fail(WQ_ERR_UNSUPPORTED, "acc_out needs group_size == 128");
-    return dispatch(c.bits, 2, Aq, a_scale, Wq, scales, c.bits == 4 && !c.symmetric ? zeros : nullptr, bias, C,
-                       acc_out, M, N, K, c, workspace, ws_bytes, stream);
+    return dispatch(wf, 2, Aq, a_scale, Wq, scales, wf == WF_I4 && !c.symmetric ? zeros : nullptr, bias, C, acc_out,
+                    M, N, K, c, workspace, ws_bytes, stream);
 }

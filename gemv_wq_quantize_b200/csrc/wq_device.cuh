@@ -260,6 +260,55 @@ __device__ __forceinline__ void mma_u8s8(int (&d)[4], const uint32_t (&a)[4], ui
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
+// D = A(16x32 s8, row) * B(32x8 s8, col) + C, exact int32 accumulators.
+__device__ __forceinline__ void mma_s8s8(int (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1)
+{
+    asm volatile(
+        "mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// Binary weights: bits 15 and 31 of t (1 -> +1, 0 -> -1) as a pair of binary16 +-1.0
+// (0x3C00 / 0xBC00): (~t & 0x80008000) | 0x3C003C00 in one LOP3.
+__device__ __forceinline__ uint32_t pm1_f16x2(uint32_t t)
+{
+    uint32_t d;
+    asm("lop3.b32 %0, %1, %2, %3, 0xAE;" : "=r"(d) : "r"(t), "r"(0x80008000u), "r"(0x3C003C00u));
+    return d;
+}
+
+// Two FP4 e2m1 codes (byte B of w: element 2B + 0 in its low nibble, 2B + 1 in its high
+// nibble) -> the binary16 pair (element 2B + 0 in the low half), exact.
+template <int B>
+__device__ __forceinline__ uint32_t e2m1x2_to_f16x2(uint32_t w)
+{
+    uint32_t d;
+    if constexpr (B == 0)
+        asm("{\n.reg .b8 t0, t1, t2, t3;\nmov.b32 {t0, t1, t2, t3}, %1;\ncvt.rn.f16x2.e2m1x2 %0, t0;\n}" : "=r"(d) : "r"(w));
+    else if constexpr (B == 1)
+        asm("{\n.reg .b8 t0, t1, t2, t3;\nmov.b32 {t0, t1, t2, t3}, %1;\ncvt.rn.f16x2.e2m1x2 %0, t1;\n}" : "=r"(d) : "r"(w));
+    else if constexpr (B == 2)
+        asm("{\n.reg .b8 t0, t1, t2, t3;\nmov.b32 {t0, t1, t2, t3}, %1;\ncvt.rn.f16x2.e2m1x2 %0, t2;\n}" : "=r"(d) : "r"(w));
+    else
+        asm("{\n.reg .b8 t0, t1, t2, t3;\nmov.b32 {t0, t1, t2, t3}, %1;\ncvt.rn.f16x2.e2m1x2 %0, t3;\n}" : "=r"(d) : "r"(w));
+    return d;
+}
+
+// Two FP8 e4m3 codes (half H of w: element 2H + 0 in its low byte) -> the binary16 pair
+// (element 2H + 0 in the low half), exact (every e4m3 value is a binary16 value).
+template <int H>
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t w)
+{
+    uint32_t d;
+    if constexpr (H == 0)
+        asm("{\n.reg .b16 lo, hi;\nmov.b32 {lo, hi}, %1;\ncvt.rn.f16x2.e4m3x2 %0, lo;\n}" : "=r"(d) : "r"(w));
+    else
+        asm("{\n.reg .b16 lo, hi;\nmov.b32 {lo, hi}, %1;\ncvt.rn.f16x2.e4m3x2 %0, hi;\n}" : "=r"(d) : "r"(w));
+    return d;
+}
+
 __device__ __forceinline__ uint4 lds128(const void *p)
 {
     uint4 v;

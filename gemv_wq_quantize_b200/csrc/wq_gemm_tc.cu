@@ -1,5 +1,6 @@
 // wq_gemm_tc.cu -- many-token weight-quantized matmul on the 5th-generation tensor cores
-// (tcgen05), for INT4 (group scales, optional zero points) and ternary INT2 weights.
+// (tcgen05), for INT4 (group scales, optional zero points), ternary INT2 and binary INT1
+// weights (one scale per tensor), and FP4 e2m1 / FP8 e4m3 weights (group scales).
 //
 // C[M,N] = A[M,K] x dequant(Wq[N,K])^T: "BitBLAS practical guide", "What is BitBLAS",
 // "Weight group quantization" and the FP16 x INT4 / INT2 and INT8 x INT4 / INT2 rows of its
@@ -14,9 +15,10 @@
 // MMA's K-major descriptor expects.  Per block of 128 k:
 //  * a producer warp TMAs the block's activations and packed weights into a 4-stage ring;
 //  * eight unpacking warps turn the packed weights of their own row (thread = weight row,
-//    warp pairs split the 128 k) into exact integers in natural k order -- q - z (INT4) or
-//    the ternary value (INT2), as f16 / bf16 pairs, or as signed bytes for INT8
-//    activations -- and store them to the stage's TMEM A-buffer (tcgen05.st);
+//    warp pairs split the 128 k) into exact values in natural k order -- q - z (INT4), the
+//    ternary value (INT2), +-1 (INT1) or the e2m1 / e4m3 value (hardware conversion), as
+//    f16 / bf16 pairs, or as signed bytes for INT8 activations -- and store them to the
+//    stage's TMEM A-buffer (tcgen05.st);
 //  * one thread issues the block's MMAs (8 of k 16, or 4 of k 32 for INT8) into a TMEM
 //    accumulator of that block alone, and one tcgen05.commit frees the stage, its A-buffer
 //    and announces the accumulator;
@@ -38,8 +40,10 @@
 #include <stdint.h>
 
 #include <algorithm>
+#include <type_traits>
 
 #include "wq_device.cuh"
+#include "wq_format.h"
 #include "wq_host.h"
 #include "wq_tc.cuh"
 
@@ -57,8 +61,9 @@ constexpr int kFoldWarps = 8;  // fold block accumulators into the totals, write
 constexpr int kThreads = (2 + kDeqWarps + kFoldWarps) * 32;  // + warp 0 TMA, warp 1 MMA / TMEM
 constexpr int kActBox = kBT * 128;  // one box of activations: 128 rows x 128 B (64 k FP, 128 k INT8)
 __host__ __device__ constexpr int act_bytes(int AM) { return AM == 2 ? kActBox : 2 * kActBox; }
-__host__ __device__ constexpr int w_bytes(int WB) { return kBW * kKB * WB / 8; }  // 8 KB / 4 KB packed
-__host__ __device__ constexpr int stage_bytes(int WB, int AM) { return act_bytes(AM) + w_bytes(WB); }
+// packed weights of a block: 16 KB FP8, 8 KB INT4 / FP4, 4 KB INT2, 2 KB INT1
+__host__ __device__ constexpr int w_bytes(int WF) { return kBW * kKB * wf_bits(WF) / 8; }
+__host__ __device__ constexpr int stage_bytes(int WF, int AM) { return act_bytes(AM) + w_bytes(WF); }
 constexpr uint32_t kTmemCols = 512;
 constexpr int kNA = 4;          // TMEM A-buffers: unpacked weights of a block, 64 columns each
 constexpr int kND = 2;          // TMEM accumulators of a block, 128 columns each
@@ -67,9 +72,9 @@ constexpr uint32_t kDcol = kNA * 64;
 
 struct TcParams {
     int M, N, K, G, gs, sym;
-    int upg;               // blocks of 128 k per scale group (INT4: group_size / 128)
+    int upg;               // blocks of 128 k per scale group (group_size / 128)
     const float *a_scale;  // INT8 activations: per-token scale
-    const float *scale32;  // INT2 weights: per-tensor scale
+    const float *scale32;  // INT2 / INT1 weights: per-tensor scale
     int nkb;     // blocks of 128 k
     int ks;      // K slices per tile (split-K when tiles are fewer than SMs)
     float *ws_part;     // ks > 1: fp32 partial totals [tile][slice][128 tokens][128 rows]
@@ -84,7 +89,7 @@ struct TcParams {
     const uint16_t *zeros;
     const void *bias;
     void *C;
-    int32_t *acc_out;  // ACC: INT32 group sums [M][N][G] (INT4, group 128) or totals [M][N] (INT2)
+    int32_t *acc_out;  // ACC: INT32 group sums [M][N][G] (INT4, group 128) or totals [M][N] (INT2, INT1)
     int nat;           // INT4 weights in the kernel-native order
 };
 
@@ -216,18 +221,52 @@ __device__ __forceinline__ void unpack_word_s8_nat(uint32_t w, uint32_t zc, uint
     o[1] = (prmt(lo, hi, 0x7531) + zc) ^ 0x80808080u;  // k4 .. k7
 }
 
-template <int WB, int AM, bool ACC = false>
+// (a & m) | (b & ~m) in one LOP3.
+__device__ __forceinline__ uint32_t bitsel(uint32_t a, uint32_t b, uint32_t m)
+{
+    uint32_t d;
+    asm("lop3.b32 %0, %1, %2, %3, 0xE4;" : "=r"(d) : "r"(a), "r"(b), "r"(m));
+    return d;
+}
+
+// INT1, FP16 activations: one word (32 bits, k0 in bit 0) -> 16 binary16 pairs (k0,k1) ..
+// (k30,k31) of +-1: bit 2p moved to bit 15 and bit 2p+1 to bit 31, then one LOP3.
+__device__ __forceinline__ void unpack1_word(uint32_t w, uint32_t *o)
+{
+#pragma unroll
+    for (int p = 0; p < 16; ++p) {
+        const uint32_t lo = p <= 7 ? (w << (15 - 2 * p)) : (w >> (2 * p - 15));
+        const uint32_t hi = w << (30 - 2 * p);
+        o[p] = pm1_f16x2(bitsel(lo, hi, 0x0000FFFFu));
+    }
+}
+
+// INT1, INT8 activations: one word -> 32 signed bytes +-1 in natural k order.  Nibble i
+// times 0x00204081 puts its bits at 0, 8, 16 and 24 (no carries); 2c + 0x7F, ^0x80 -> -1 / +1.
+__device__ __forceinline__ void unpack1_word_s8(uint32_t w, uint32_t *o)
+{
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const uint32_t x = (((w >> (4 * i)) & 15u) * 0x00204081u) & 0x01010101u;
+        o[i] = ((x << 1) + 0x7F7F7F7Fu) ^ 0x80808080u;
+    }
+}
+
+template <int WF, int AM, bool ACC = false>
 __global__ void __launch_bounds__(kThreads, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_w,
                    const TcParams p)
 {
     constexpr bool BF16 = AM == 1, I8 = AM == 2;
-    constexpr int kActBytes = act_bytes(AM), kStageBytes = stage_bytes(WB, AM);
+    constexpr bool GROUPED = wf_grouped(WF);
+    constexpr int kActBytes = act_bytes(AM), kStageBytes = stage_bytes(WF, AM);
+    // scale table entries: binary16 scale | zero point << 16 (INT4), the scale alone (FP4 / FP8)
+    using TabT = typename std::conditional<WF == WF_I4, uint32_t, uint16_t>::type;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *ring = smem;  // kNA x (activations | packed weights)
     uint16_t *scst = reinterpret_cast<uint16_t *>(smem + p.scst_off);  // 2 x (scales, zeros) [128][G]
-    uint32_t *tabs = reinterpret_cast<uint32_t *>(smem + p.tab_off);   // 2 x [G][tab_rs]: scale | z << 16
+    TabT *tabs = reinterpret_cast<TabT *>(smem + p.tab_off);           // 2 x [G][tab_rs]
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + p.bar_off);
     // rel[s]: the MMAs of the step in stage s have completed: stage s and A-buffer s are free
     // and accumulator step % kND holds the block's sums
@@ -278,7 +317,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             tma_prefetch_desc(&tmap_a);
             tma_prefetch_desc(&tmap_w);
             auto issue_scales = [&](int n0, int tl) {  // the tile's scale / zero rows: contiguous in [N, G]
-                if constexpr (WB == 4) {
+                if constexpr (GROUPED) {
                     if (!p.stage_sc) return;
                     const int nrows = min(kBW, p.N - n0);
                     const uint32_t bytes16 = (uint32_t(nrows) * p.G * 2u) & ~15u;
@@ -302,7 +341,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int i = 0; i < npre; ++i) {
                     uint8_t *st = ring + size_t(i) * kStageBytes;
                     mbar_arrive_expect_tx(&full[i], kStageBytes);
-                    tma_load_2d(st + kActBytes, &tmap_w, (kb0 + i) * (kKB * WB / 8), n0, &full[i]);
+                    tma_load_2d(st + kActBytes, &tmap_w, (kb0 + i) * (kKB * wf_bits(WF) / 8), n0, &full[i]);
                 }
             }
             grid_dep_wait();  // activations may be written by the previous kernel
@@ -320,7 +359,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (!pre) {
                         if (!tc_wait(&rel[s], ((step / kNA) & 1) ^ 1, abort)) break;
                         mbar_arrive_expect_tx(&full[s], kStageBytes);
-                        tma_load_2d(st + kActBytes, &tmap_w, kb * (kKB * WB / 8), n0, &full[s]);
+                        tma_load_2d(st + kActBytes, &tmap_w, kb * (kKB * wf_bits(WF) / 8), n0, &full[s]);
                     }
                     tma_load_2d(st, &tmap_a, kb * kKB, m0, &full[s]);
                     if constexpr (!I8) tma_load_2d(st + kActBox, &tmap_a, kb * kKB + 64, m0, &full[s]);
@@ -392,9 +431,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int n0 = (tile / p.TT) * kBW;
             const int nrows = min(kBW, p.N - n0);
             const int tb = tl % p.ntab;  // this tile's table buffer
-            uint32_t *tab = tabs + size_t(tb) * tab_elems;
-            // ---- scale / zero table of the tile (INT4): [g][row] = fp16 scale bits | z << 16
-            if constexpr (WB == 4) {
+            TabT *tab = tabs + size_t(tb) * tab_elems;
+            // ---- scale / zero table of the tile: [g][row] = fp16 scale bits (| z << 16 for INT4)
+            if constexpr (GROUPED) {
             if (p.stage_sc && !tc_wait(&scbar[tl & 1], (tl >> 1) & 1, abort)) break;
             // the folding warps are done with tile tl - ntab, the buffer's previous user
             if (tl >= p.ntab && !tc_wait(&tdone[tb], ((tl - p.ntab) / p.ntab) & 1, abort)) break;
@@ -416,7 +455,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                             }
                             v = uint32_t(sb) | (z << 16);
                         }
-                        tab[(size_t)gi * p.tab_rs + rl] = v;
+                        tab[(size_t)gi * p.tab_rs + rl] = TabT(v);
                     }
                 }
             }
@@ -429,7 +468,58 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // full also tells that the MMAs of step - kNA (stage and A-buffer s) have completed
                 if (!tc_wait(&full[s], (step / kNA) & 1, abort)) break;
                 const uint8_t *wst = ring + size_t(s) * kStageBytes + kActBytes;
-                if constexpr (WB == 4) {
+                if constexpr (WF == WF_E2M1) {
+                    // this row's 32 packed bytes of the k half (64-byte rows, 64-byte swizzle)
+                    const uint8_t *wrow = wst + r * 64;
+                    const uint32_t sw = uint32_t((r >> 1) & 3);
+                    const uint4 w0 = lds128(wrow + ((uint32_t(2 * kh) ^ sw) << 4));
+                    const uint4 w1 = lds128(wrow + ((uint32_t(2 * kh + 1) ^ sw) << 4));
+                    tc::fence_after_sync();
+                    uint32_t v[32];
+                    const uint32_t wd[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        v[4 * i + 0] = e2m1x2_to_f16x2<0>(wd[i]);
+                        v[4 * i + 1] = e2m1x2_to_f16x2<1>(wd[i]);
+                        v[4 * i + 2] = e2m1x2_to_f16x2<2>(wd[i]);
+                        v[4 * i + 3] = e2m1x2_to_f16x2<3>(wd[i]);
+                    }
+                    tc::st_32x32b_x32(tlane + kAcol + s * 64 + kh * 32, v);
+                } else if constexpr (WF == WF_E4M3) {
+                    // this row's 64 bytes of the k half (128-byte rows, 128-byte swizzle)
+                    const uint8_t *wrow = wst + r * 128;
+                    const uint32_t sw = uint32_t(r & 7);
+                    uint4 c4[4];
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) c4[i] = lds128(wrow + ((uint32_t(4 * kh + i) ^ sw) << 4));
+                    tc::fence_after_sync();
+                    uint32_t v[32];
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const uint32_t wd[4] = {c4[i].x, c4[i].y, c4[i].z, c4[i].w};
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            v[8 * i + 2 * j] = e4m3x2_to_f16x2<0>(wd[j]);
+                            v[8 * i + 2 * j + 1] = e4m3x2_to_f16x2<1>(wd[j]);
+                        }
+                    }
+                    tc::st_32x32b_x32(tlane + kAcol + s * 64 + kh * 32, v);
+                } else if constexpr (WF == WF_I1) {
+                    // this row's 8 packed bytes of the k half (16-byte rows, not swizzled)
+                    const uint2 w = lds64(wst + r * 16 + kh * 8);
+                    tc::fence_after_sync();
+                    if constexpr (I8) {
+                        uint32_t v[16];
+                        unpack1_word_s8(w.x, v);
+                        unpack1_word_s8(w.y, v + 8);
+                        tc::st_32x32b_x16(tlane + kAcol + s * 64 + kh * 16, v);
+                    } else {
+                        uint32_t v[32];
+                        unpack1_word(w.x, v);
+                        unpack1_word(w.y, v + 16);
+                        tc::st_32x32b_x32(tlane + kAcol + s * 64 + kh * 32, v);
+                    }
+                } else if constexpr (WF == WF_I4) {
                     // this row's 32 packed bytes of the k half (64-byte rows, 64-byte swizzle)
                     const uint8_t *wrow = wst + r * 64;
                     const uint32_t sw = uint32_t((r >> 1) & 3);
@@ -511,8 +601,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int kb0 = sp * p.nkb / p.ks, kb1 = (sp + 1) * p.nkb / p.ks;
             const int n0 = (tile / p.TT) * kBW, m0 = (tile % p.TT) * kBT;
             const int tb = tl % p.ntab;
-            const uint32_t *tab = tabs + size_t(tb) * tab_elems;
-            if constexpr (WB == 4)
+            const TabT *tab = tabs + size_t(tb) * tab_elems;
+            if constexpr (GROUPED)
                 if (!tc_wait(&tready[tb], (tl / p.ntab) & 1, abort)) break;
             float tot[64];
 #pragma unroll
@@ -520,8 +610,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             bool ok = true;
             for (int kb = kb0; kb < kb1; ++kb, ++step) {
                 const uint32_t db = step % kND, s = step % kNA;
-                float sv = 1.f;  // INT2: the per-tensor scale is applied at the end
-                if constexpr (WB == 4)
+                float sv = 1.f;  // INT2 / INT1: the per-tensor scale is applied at the end
+                if constexpr (GROUPED)
                     sv = __half2float(__ushort_as_half(uint16_t(tab[(size_t)(p.upg == 1 ? kb : kb / p.upg) * p.tab_rs + r])));
                 if (!tc_wait(&rel[s], (step / kNA) & 1, abort)) { ok = false; break; }
                 tc::fence_after_sync();
@@ -541,7 +631,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const float dv = I8 ? float(int(d[j])) : __uint_as_float(d[j]);
                         tot[c * 16 + j] = fmaf(sv, dv, tot[c * 16 + j]);
                     }
-                    if constexpr (ACC && WB == 4) {
+                    if constexpr (ACC && WF == WF_I4) {
                         const int n = n0 + r, mb = m0 + th * 64 + c * 16;
                         if (n < p.N)
 #pragma unroll
@@ -552,7 +642,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             if (!ok) break;
             __syncwarp();
-            if constexpr (WB == 4)
+            if constexpr (GROUPED)
                 if (lane == 0) mbar_arrive(&tdone[tb]);
 
             if (p.ks > 1) {
@@ -620,14 +710,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if constexpr (BF16) b = __bfloat162float(static_cast<const __nv_bfloat16 *>(p.bias)[n]);
                     else b = __half2float(static_cast<const __half *>(p.bias)[n]);
                 }
-                const float ws = (WB == 2) ? p.scale32[0] : 1.f;
+                const float ws = wf_per_tensor(WF) ? p.scale32[0] : 1.f;
                 const int mb = m0 + th * 64;
 #pragma unroll
                 for (int j = 0; j < 64; ++j) {
                     if (mb + j >= p.M) continue;
-                    if constexpr (ACC && WB == 2) p.acc_out[(size_t)(mb + j) * p.N + n] = int(tot[j]);
+                    if constexpr (ACC && wf_per_tensor(WF)) p.acc_out[(size_t)(mb + j) * p.N + n] = int(tot[j]);
                     float v;
-                    if constexpr (I8) v = p.a_scale[mb + j] * (WB == 2 ? ws * tot[j] : tot[j]);
+                    if constexpr (I8) v = p.a_scale[mb + j] * (wf_per_tensor(WF) ? ws * tot[j] : tot[j]);
                     else v = ws * tot[j];
                     store_out<BF16>(p.C, (long long)(mb + j) * p.N + n, v + b);
                 }
@@ -651,10 +741,11 @@ struct TcPlan {
     bool ok = false;
 };
 
-// G: groups of the INT4 scale table (0 for INT2: one per-tensor scale, no table).
-// Preferred: scales staged by bulk copy and two tables (the next tile's built while one is
-// in use).  Long K (many groups) drops the staging, then the second table, to keep the ring.
-TcPlan make_plan(int nkb, int G, int stage, const DeviceInfo &dev)
+// G: groups of the scale table (0 for INT2 / INT1: one per-tensor scale, no table); tab_es:
+// bytes per table entry.  Preferred: scales staged by bulk copy and two tables (the next
+// tile's built while one is in use).  Long K (many groups) drops the staging, then the
+// second table, to keep the ring.
+TcPlan make_plan(int nkb, int G, int stage, int tab_es, const DeviceInfo &dev)
 {
     TcPlan pl;
     pl.tab_rs = kBW + 1;
@@ -664,7 +755,7 @@ TcPlan make_plan(int nkb, int G, int stage, const DeviceInfo &dev)
     const int forms[3][2] = {{1, 2}, {0, 2}, {0, 1}};
     for (const auto &f : forms) {
         const size_t scst = f[0] ? (size_t(2) * 2 * kBW * G * 2 + 15) & ~size_t(15) : 0;
-        const size_t tab = (size_t(f[1]) * G * pl.tab_rs * 4 + 15) & ~size_t(15);
+        const size_t tab = (size_t(f[1]) * G * pl.tab_rs * tab_es + 15) & ~size_t(15);
         if (budget <= scst + tab + bars || (budget - scst - tab - bars) / size_t(stage) < size_t(kNA)) continue;
         pl.stage_sc = f[0];
         pl.ntab = f[1];
@@ -683,11 +774,11 @@ TcPlan make_plan(int nkb, int G, int stage, const DeviceInfo &dev)
     return pl;
 }
 
-template <int WB, int AM, bool ACC = false>
+template <int WF, int AM, bool ACC = false>
 wq_status launch(const TcPlan &pl, const CUtensorMap &ta, const CUtensorMap &tw, const TcParams &p, int grid,
                  cudaStream_t st)
 {
-    auto kern = tc_gemm_kernel<WB, AM, ACC>;
+    auto kern = tc_gemm_kernel<WF, AM, ACC>;
     static size_t configured = 0;
     if (pl.smem > configured) {
         if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(pl.smem)) != cudaSuccess)
@@ -736,28 +827,29 @@ size_t tc_workspace_size(int64_t M, int64_t N, int64_t K)
     return split_bytes(M, N, choose_slices(M, N, K, device_info().sm_count));
 }
 
-// Many-token path on the tcgen05 tensor cores: INT4 (group size a multiple of 128) or ternary
-// INT2 weights, FP16 / BF16 (AM 0 / 1) or INT8 (AM 2, with a_scale) activations.
+// Many-token path on the tcgen05 tensor cores: INT4, FP4 or FP8 (group size a multiple of 128),
+// ternary INT2 or binary INT1 weights, FP16 / BF16 (AM 0 / 1) or INT8 (AM 2, with a_scale)
+// activations (the entry points admit the pairs listed in the ABI).
 // WQ_ERR_UNSUPPORTED when the configuration has no plan here (the caller then uses the
 // tiled mma.sync path).
 // The workspace (zero-filled once, see the ABI) is used for split-K partial sums when it
 // is large enough; otherwise every tile covers all of K.
-wq_status tc_gemm(int WB, int AM, const void *A, const float *a_scale, const uint8_t *Wq, const void *scales,
+wq_status tc_gemm(int WF, int AM, const void *A, const float *a_scale, const uint8_t *Wq, const void *scales,
                   const void *zeros, const void *bias, void *C, int32_t *acc_out, int64_t M, int64_t N, int64_t K,
                   const wq_qconfig &c, void *ws, size_t ws_bytes, cudaStream_t st)
 {
-    if (acc_out && (AM != 2 || (WB == 4 && c.group_size != kKB)))
+    if (acc_out && (AM != 2 || (WF == WF_I4 && c.group_size != kKB)))
         return fail(WQ_ERR_UNSUPPORTED, "tc_gemm: INT32 sums need INT8 activations (and group_size 128 for INT4)");
-    if (WB == 4 && (K % kKB || c.group_size % kKB))
-        return fail(WQ_ERR_UNSUPPORTED, "tc_gemm: INT4 needs K and group_size multiples of 128");
+    if (wf_grouped(WF) && (K % kKB || c.group_size % kKB))
+        return fail(WQ_ERR_UNSUPPORTED, "tc_gemm: group-scaled weights need K and group_size multiples of 128");
+    if (WF == WF_I1 && K % kKB) return fail(WQ_ERR_UNSUPPORTED, "tc_gemm: INT1 needs K %% 128 == 0");
     const int es = AM == 2 ? 1 : 2;
     if ((K * es) % 16) return fail(WQ_ERR_UNSUPPORTED, "tc_gemm: activation rows must be 16-byte multiples");
     const DeviceInfo &dev = device_info();
-    const int G = WB == 4 ? int(K / c.group_size) : 0;
+    const int G = wf_grouped(WF) ? int(K / c.group_size) : 0;
     const int nkb = int((K + kKB - 1) / kKB);
-    const int stage = WB == 4 ? (AM == 2 ? stage_bytes(4, 2) : stage_bytes(4, 0))
-                              : (AM == 2 ? stage_bytes(2, 2) : stage_bytes(2, 0));
-    const TcPlan pl = make_plan(nkb, G, stage, dev);
+    const int stage = act_bytes(AM == 2 ? 2 : 0) + w_bytes(WF);
+    const TcPlan pl = make_plan(nkb, G, stage, WF == WF_I4 ? 4 : 2, dev);
     if (!pl.ok) return fail(WQ_ERR_UNSUPPORTED, "tc_gemm: no shared-memory plan for K=%lld", (long long)K);
     CUtensorMap ta, tw;
     {
@@ -770,12 +862,15 @@ wq_status tc_gemm(int WB, int AM, const void *A, const float *a_scale, const uin
         if (rc != WQ_OK) return rc;
     }
     {
-        // packed weights [N][K*WB/8]: one box = 128 rows x one block (64 B INT4 / 32 B INT2)
-        const uint64_t row_bytes = uint64_t(K) * WB / 8;
+        // packed weights [N][K*bits/8]: one box = 128 rows x one block (128 B FP8, 64 B INT4 / FP4,
+        // 32 B INT2, 16 B INT1), swizzled as the unpacking warps read it
+        const int blk = kKB * wf_bits(WF) / 8;
+        const uint64_t row_bytes = uint64_t(K) * wf_bits(WF) / 8;
         const uint64_t dims[2] = {row_bytes, uint64_t(N)};
         const uint64_t strides[1] = {row_bytes};
-        const uint32_t box[2] = {uint32_t(kKB * WB / 8), uint32_t(kBW)};
-        wq_status rc = encode_tmap(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, Wq, dims, strides, box, WB == 4 ? 64 : 0);
+        const uint32_t box[2] = {uint32_t(blk), uint32_t(kBW)};
+        wq_status rc = encode_tmap(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, Wq, dims, strides, box,
+                                   blk == 128 ? 128 : blk == 64 ? 64 : 0);
         if (rc != WQ_OK) return rc;
     }
     TcParams p{};
@@ -783,9 +878,9 @@ wq_status tc_gemm(int WB, int AM, const void *A, const float *a_scale, const uin
     p.N = int(N);
     p.K = int(K);
     p.G = G;
-    p.gs = WB == 4 ? c.group_size : int(K);
-    p.upg = WB == 4 ? c.group_size / kKB : 1;
-    p.sym = WB == 4 ? c.symmetric : 1;
+    p.gs = wf_grouped(WF) ? c.group_size : int(K);
+    p.upg = wf_grouped(WF) ? c.group_size / kKB : 1;
+    p.sym = WF == WF_I4 ? c.symmetric : 1;
     p.a_scale = a_scale;
     p.scale32 = static_cast<const float *>(scales);
     p.nkb = nkb;
@@ -809,9 +904,18 @@ wq_status tc_gemm(int WB, int AM, const void *A, const float *a_scale, const uin
     p.bias = bias;
     p.C = C;
     p.acc_out = acc_out;
-    p.nat = WB == 4 && c.layout == WQ_LAYOUT_NATIVE;
+    p.nat = WF == WF_I4 && c.layout == WQ_LAYOUT_NATIVE;
     const int grid = std::min(dev.sm_count, p.NT * p.ks);
-    if (WB == 4) {
+    if (WF == WF_E2M1) return AM == 0 ? launch<WF_E2M1, 0>(pl, ta, tw, p, grid, st)
+                                      : fail(WQ_ERR_UNSUPPORTED, "tc_gemm: FP4 weights take FP16 activations");
+    if (WF == WF_E4M3) return AM == 0 ? launch<WF_E4M3, 0>(pl, ta, tw, p, grid, st)
+                                      : fail(WQ_ERR_UNSUPPORTED, "tc_gemm: FP8 weights take FP16 activations");
+    if (WF == WF_I1) {
+        if (AM == 0) return launch<WF_I1, 0>(pl, ta, tw, p, grid, st);
+        if (AM == 1) return fail(WQ_ERR_UNSUPPORTED, "tc_gemm: INT1 weights take FP16 or INT8 activations");
+        return acc_out ? launch<WF_I1, 2, true>(pl, ta, tw, p, grid, st) : launch<WF_I1, 2>(pl, ta, tw, p, grid, st);
+    }
+    if (WF == WF_I4) {
         if (AM == 0) return launch<4, 0>(pl, ta, tw, p, grid, st);
         if (AM == 1) return launch<4, 1>(pl, ta, tw, p, grid, st);
         return acc_out ? launch<4, 2, true>(pl, ta, tw, p, grid, st) : launch<4, 2>(pl, ta, tw, p, grid, st);

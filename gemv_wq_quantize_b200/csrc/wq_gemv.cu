@@ -1,4 +1,5 @@
-// wq_gemv.cu -- decode GEMV / few-token matmul (M <= 16) over packed INT4 / INT2 weights.
+// wq_gemv.cu -- decode GEMV / few-token matmul (M <= 16) over packed INT4 / INT2 / INT1 /
+// FP4 / FP8 weights.
 //
 // C[M,N] = A[M,K] x dequant(Wq[N,K])^T ("BitBLAS practical guide", "What is BitBLAS",
 // layout "nt"), FP16 / BF16 activations (W4A16) or per-token INT8 activations with exact
@@ -10,7 +11,8 @@
 // byte once it arrives:
 //  * Rows are cut into 16-row tiles; CTA c (one per SM) owns a contiguous run of tiles and all
 //    of K, so no CTA needs another's result.  K is walked in chunks of KC units (a unit =
-//    64 packed bytes of a row: 128 k of INT4, 256 k of INT2).
+//    64 packed bytes of a row: 128 k of INT4 or FP4, 256 k of INT2, 512 k of INT1, 64 k of
+//    FP8).
 //  * One TMA box per tile and chunk brings 16 rows x KC units (a 3D box over unit pairs;
 //    a 2D box per unit pair when rows are not a whole number of pairs), written with the
 //    128-byte swizzle; MMA row g reads tile row (g >> 1) | ((g & 1) << 2), so the two rows of
@@ -128,14 +130,14 @@ __device__ __forceinline__ float bias_at(const void *bias, int n)
     return __half2float(static_cast<const __half *>(bias)[n]);
 }
 
-template <int WB, int AM>
+template <int WF, int AM>
 __device__ __forceinline__ float finish(const GemvParams &p, float total_f, int total_i, int n, float as)
 {
     float v;
     if constexpr (AM == A_I8) {
-        v = (WB == 2) ? as * (p.scale32[0] * float(total_i)) : as * total_f;
+        v = wf_per_tensor(WF) ? as * (p.scale32[0] * float(total_i)) : as * total_f;
     } else {
-        v = (WB == 2) ? p.scale32[0] * total_f : total_f;
+        v = wf_per_tensor(WF) ? p.scale32[0] * total_f : total_f;
     }
     return v + bias_at<AM>(p.bias, n);
 }
@@ -167,18 +169,19 @@ __device__ __forceinline__ float src_at(const uint4 &raw, int i)
 // FS: 0, or the FP activations to quantize per token first (1: binary16, 2: bfloat16; INT8
 // mode and whole-K activation staging only): the "fused kernel" of the same page's section
 // on combining the strategies, here the quantization done in the matmul's prologue.
-template <int WB, int AM, int NT, bool ACC, bool WIDE, int FS = 0>
+template <int WF, int AM, int NT, bool ACC, bool WIDE, int FS = 0>
 __global__ void __launch_bounds__(kThreads, 1)
     gemv_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_a,
                 const GemvParams p)
 {
     static_assert(FS == 0 || AM == A_I8, "the fused quantization feeds the INT8 path");
-    constexpr int KU = kunit_of(WB);
-    constexpr int QN = qn_of(WB, AM);
+    constexpr int KU = kunit_of(WF);
+    constexpr int QN = qn_of(WF, AM);
+    constexpr bool GROUPED = wf_grouped(WF);
     constexpr int ES = (AM == A_I8) ? 1 : 2;
     constexpr int AU = KU * ES;  // activation bytes of one unit and token
     constexpr int WPU = wpu_of(NT, WIDE), KC = kc_of(NT, WIDE), TM = tm_of(NT, WIDE), NTL = ntl_of(NT, WIDE);
-    using Tot = typename std::conditional<AM == A_I8 && WB == 2, int, float>::type;
+    using Tot = typename std::conditional<AM == A_I8 && wf_per_tensor(WF), int, float>::type;
 
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -234,7 +237,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // the CTA's scale / zero rows are contiguous in [N, G]: one bulk copy each (a ragged
     // tail of < 16 bytes is read directly below)
     const int nrows = min(ntc * kTileRows, p.N - r0);
-    const uint32_t sc_bytes = (WB == 4) ? uint32_t(nrows) * p.G * 2u : 0u;
+    const uint32_t sc_bytes = GROUPED ? uint32_t(nrows) * p.G * 2u : 0u;
     const uint32_t sc16 = sc_bytes & ~15u;
     const int pro = min(S, total_it);
     // Thread 0 sets up the barriers and at once sends the first stage's weights, which are on
@@ -251,7 +254,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_prefetch_desc(&tmap_w);
         if (!p.a_whole) tma_prefetch_desc(&tmap_a);
         issue_w(0);
-        if constexpr (WB == 4) {
+        if constexpr (GROUPED) {
             mbar_arrive_expect_tx(scbar, sc16 * (p.sym ? 1u : 2u));
             if (sc16) {
                 bulk_load(sc_st, p.scales16 + (size_t)r0 * p.G, sc16, scbar);
@@ -266,7 +269,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (it > 0) issue_w(it);
 
     // ---- scale / zero table of the CTA's rows, group-major: {scale, zero point as integer bits}
-    if constexpr (WB == 4) {
+    if constexpr (GROUPED) {
         wait_bar(scbar, 0);  // on expiry the error is recorded; carry on to the next barrier
         const int nsm = int(sc16 >> 1);
         const int nrow_t = ntc * kTileRows;  // a warp per row, its lanes over the groups
@@ -387,12 +390,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (kb < p.KB && nmine > 0) {
                 uint4 bf[NT][QN];
                 int asum[NT];
-                if (p.a_whole) {
+                if constexpr (WF == WF_I1) {
+                    // fragments are formed per word inside unit_mma_b1
+                } else if (p.a_whole) {
                     const uint8_t *ablk = abuf + (size_t)kb * AU;
                     const int pitch = p.a_pitch_b;
                     auto addr = [=](int m, int o) { return ablk + m * pitch + o; };
 #pragma unroll
-                    for (int j = 0; j < NT; ++j) build_bfrag<WB, AM>(addr, p.M, j, lane, bf[j], asum[j], p.nat != 0);
+                    for (int j = 0; j < NT; ++j) build_bfrag<WF, AM>(addr, p.M, j, lane, bf[j], asum[j], p.nat != 0);
                 } else {
                     const uint8_t *abase = st + p.wpart_bytes;
                     const int MB = p.MB;
@@ -401,10 +406,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                         return abase + swz128(((x >> 7) * MB + m) * 128u + (x & 127u));
                     };
 #pragma unroll
-                    for (int j = 0; j < NT; ++j) build_bfrag<WB, AM>(addr, p.M, j, lane, bf[j], asum[j], p.nat != 0);
+                    for (int j = 0; j < NT; ++j) build_bfrag<WF, AM>(addr, p.M, j, lane, bf[j], asum[j], p.nat != 0);
                 }
                 int sA[NT][2];
-                if constexpr (AM == A_I8) {
+                if constexpr (AM == A_I8 && WF != WF_I1) {
 #pragma unroll
                     for (int j = 0; j < NT; ++j) {
                         int v = asum[j];
@@ -414,7 +419,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         sA[j][1] = __shfl_sync(0xffffffffu, v, (2 * t + 1) * 4);
                     }
                 }
-                const int gi = (WB == 4) ? (p.upg == 1 ? kb : kb / p.upg) : 0;
+                const int gi = GROUPED ? (p.upg == 1 ? kb : kb / p.upg) : 0;
                 const float2 *srow = stab + (size_t)gi * p.tab_rs + pass * p.TPP * kTileRows + gr;
                 // a batch of B tiles (jp .. jp + B - 1); an odd last tile runs alone
                 auto batch = [&](int jp, auto nb) {
@@ -430,7 +435,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         wb[l] = lds128(wt + off_hi);
                         s_lo[l] = s_hi[l] = 0.f;
                         zl[l] = zh[l] = 8;
-                        if constexpr (WB == 4) {
+                        if constexpr (GROUPED) {
                             const uint2 v_lo = lds64(srow + i * kTileRows);
                             const uint2 v_hi = lds64(srow + i * kTileRows + 8);
                             s_lo[l] = __uint_as_float(v_lo.x);
@@ -448,7 +453,20 @@ __global__ void __launch_bounds__(kThreads, 1)
                             for (int j = 0; j < NT; ++j)
 #pragma unroll
                                 for (int e = 0; e < 4; ++e) ua[a][l][j][e] = acc_t<AM>(0);
-                    unit_mma<WB, AM, NT, B>(wa, wb, bf, zl, zh, ua);
+                    if constexpr (WF == WF_I1) {
+                        const bool whole = p.a_whole != 0;
+                        const uint8_t *ablk = abuf + (size_t)kb * AU;
+                        const uint8_t *abase = st + p.wpart_bytes;
+                        const int pitch = p.a_pitch_b, MB = p.MB;
+                        auto addr = [=](int m, int o) -> const uint8_t * {
+                            if (whole) return ablk + m * pitch + o;
+                            const uint32_t x = uint32_t(us * AU + o);
+                            return abase + swz128(((x >> 7) * MB + m) * 128u + (x & 127u));
+                        };
+                        unit_mma_b1<AM, NT, B>(wa, wb, addr, p.M, lane, ua);
+                    } else {
+                        unit_mma<WF, AM, NT, B>(wa, wb, bf, zl, zh, ua);
+                    }
 #pragma unroll
                     for (int l = 0; l < B; ++l) {
                         const int i = hf + WPU * (jp + l);
@@ -458,7 +476,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                             for (int e = 0; e < 4; ++e) {
                                 const acc_t<AM> v = ua[0][l][j][e] + ua[1][l][j][e];
                                 const float sc_e = (e < 2) ? s_lo[l] : s_hi[l];
-                                if constexpr (AM == A_I8 && WB == 2) {
+                                if constexpr (AM == A_I8 && WF == WF_I1) {
+                                    tot[jp + l][j][e] += v;  // signed +-1 weights: no correction
+                                } else if constexpr (AM == A_I8 && WF == WF_I2) {
                                     tot[jp + l][j][e] += v - 2 * sA[j][e & 1];
                                 } else if constexpr (AM == A_I8) {
                                     const int corr = v - int((e < 2) ? zl[l] : zh[l]) * sA[j][e & 1];
@@ -468,7 +488,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                         if (n < p.N && m < p.M) p.acc_out[((long long)m * p.N + n) * p.G + kb] = corr;
                                     }
                                     tot[jp + l][j][e] = fmaf(sc_e, float(corr), tot[jp + l][j][e]);
-                                } else if constexpr (WB == 2) {
+                                } else if constexpr (wf_per_tensor(WF)) {
                                     tot[jp + l][j][e] += v;
                                 } else {
                                     tot[jp + l][j][e] = fmaf(sc_e, v, tot[jp + l][j][e]);
@@ -512,7 +532,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const int r = gr + ((e & 2) ? 8 : 0);
                     if (m < p.M) {
                         float v;
-                        if constexpr (AM == A_I8 && WB == 2) v = __int_as_float(tot[jj][j][e]);
+                        if constexpr (AM == A_I8 && wf_per_tensor(WF)) v = __int_as_float(tot[jj][j][e]);
                         else v = tot[jj][j][e];
                         red[((size_t)(m * p.TPP + i) * KC + us) * kTileRows + r] = v;
                     }
@@ -534,8 +554,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 si += __float_as_int(v);
             }
             const float as = (AM != A_I8) ? 1.f : (FS != 0 ? fsc[m] : p.a_scale[m]);
-            store_out<AM>(p.C, (long long)m * p.N + n, finish<WB, AM>(p, sf, si, n, as));
-            if constexpr (AM == A_I8 && WB == 2)
+            store_out<AM>(p.C, (long long)m * p.N + n, finish<WF, AM>(p, sf, si, n, as));
+            if constexpr (AM == A_I8 && wf_per_tensor(WF))
                 if (p.acc_out) p.acc_out[(long long)m * p.N + n] = si;
         }
         if (pass + 1 < npass && !csync()) return;  // red is reused by the next pass
@@ -554,17 +574,17 @@ struct Plan {
 
 size_t up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
-Plan make_plan(int64_t M, int64_t N, int64_t K, int WB, int AM, int G, const DeviceInfo &dev)
+Plan make_plan(int64_t M, int64_t N, int64_t K, int WF, int AM, int G, const DeviceInfo &dev)
 {
     Plan pl;
     pl.NT = M <= 8 ? 1 : 2;
-    if (WB == 2 && AM != A_I8 && pl.NT == 2) return pl;  // B fragments would not fit in registers
-    pl.KU = kunit_of(WB);
+    if (WF == WF_I2 && AM != A_I8 && pl.NT == 2) return pl;  // B fragments would not fit in registers
+    pl.KU = kunit_of(WF);
     pl.KB = int((K + pl.KU - 1) / pl.KU);
     pl.T = int((N + kTileRows - 1) / kTileRows);
     pl.P = std::min(dev.sm_count, pl.T);
     const int ntc_max = (pl.T + pl.P - 1) / pl.P;
-    pl.wide = (pl.NT == 2 && AM != A_I8 && ntc_max <= 2) ? 1 : 0;
+    pl.wide = (WF == WF_I4 && pl.NT == 2 && AM != A_I8 && ntc_max <= 2) ? 1 : 0;
     pl.KC = kc_of(pl.NT, pl.wide);
     pl.TPP = std::min(ntc_max, tm_of(pl.NT, pl.wide) * wpu_of(pl.NT, pl.wide));
     const int npass = (ntc_max + pl.TPP - 1) / pl.TPP;
@@ -572,14 +592,14 @@ Plan make_plan(int64_t M, int64_t N, int64_t K, int WB, int AM, int G, const Dev
     const long long total = (long long)npass * pl.nch;
     const int es = AM == A_I8 ? 1 : 2;
     const int au = pl.KU * es;
-    const int64_t row_bytes = K * WB / 8;
+    const int64_t row_bytes = K * wf_bits(WF) / 8;
     pl.w3d = (row_bytes % kPairBytes) == 0 ? 1 : 0;
     pl.wtile = pl.KC * kTileRows * 64;
     pl.wpart = pl.TPP * pl.wtile;
     pl.rows_cap = ntc_max * kTileRows;
     pl.tab_rs = pl.rows_cap | 1;
-    const size_t scst = (WB == 4) ? up(size_t(pl.rows_cap) * G * 2 * 2, 16) : 0;
-    const size_t table = (WB == 4) ? up(size_t(pl.tab_rs) * G * 8, 16) : 0;
+    const size_t scst = wf_grouped(WF) ? up(size_t(pl.rows_cap) * G * 2 * 2, 16) : 0;
+    const size_t table = wf_grouped(WF) ? up(size_t(pl.tab_rs) * G * 8, 16) : 0;
     const size_t red = up(size_t(pl.TPP) * pl.KC * kTileRows * M * 4, 16);
     const size_t tail = scst + table + red + 128 + 8 * 19 + 4 * 16 + 64;  // + fused scales, barriers (S <= 16), counters
     const size_t budget = size_t(dev.max_smem_optin) - 1024;  // 1 KB for the alignment of the base
@@ -627,10 +647,10 @@ Plan make_plan(int64_t M, int64_t N, int64_t K, int WB, int AM, int G, const Dev
 }
 
 // The kernel instance for the plan, with its dynamic shared memory limit raised as needed.
-template <int WB, int AM, int NT, bool ACC = false, bool WIDE = false, int FS = 0>
+template <int WF, int AM, int NT, bool ACC = false, bool WIDE = false, int FS = 0>
 wq_status kernel_for(const Plan &pl, const void **func)
 {
-    auto kern = gemv_kernel<WB, AM, NT, ACC, WIDE, FS>;
+    auto kern = gemv_kernel<WF, AM, NT, ACC, WIDE, FS>;
     static size_t configured = 0;
     if (pl.smem > configured) {
         if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(pl.smem)) != cudaSuccess)
@@ -644,19 +664,19 @@ wq_status kernel_for(const Plan &pl, const void **func)
 }  // namespace
 
 // Few-token path (1 <= M <= 16) as a prepared launch.  WQ_ERR_UNSUPPORTED if no plan fits.
-wq_status gemv_prepare(int WB, int AM, const void *A, const float *a_scale, const uint8_t *Wq, const void *scales,
+wq_status gemv_prepare(int WF, int AM, const void *A, const float *a_scale, const uint8_t *Wq, const void *scales,
                        const void *zeros, const void *bias, void *C, int32_t *acc_out, int64_t M, int64_t N,
                        int64_t K, const wq_qconfig &c, PreparedLaunch *out, const FusedActQuant *fa)
 {
     const DeviceInfo &dev = device_info();
-    const int G = WB == 4 ? int(K / c.group_size) : 1;
-    Plan pl = make_plan(M, N, K, WB, AM, G, dev);
+    const int G = wf_grouped(WF) ? int(K / c.group_size) : 1;
+    Plan pl = make_plan(M, N, K, WF, AM, G, dev);
     if (!pl.ok) return fail(WQ_ERR_UNSUPPORTED, "no few-token plan for M=%lld K=%lld", (long long)M, (long long)K);
     if (fa && (AM != A_I8 || !pl.a_whole))
         return fail(WQ_ERR_UNSUPPORTED, "the activations of M=%lld K=%lld are not staged whole", (long long)M,
                     (long long)K);
     CUtensorMap tw, ta;
-    const uint64_t row_bytes = uint64_t(K) * WB / 8;
+    const uint64_t row_bytes = uint64_t(K) * wf_bits(WF) / 8;
     wq_status rc = WQ_ERR_UNSUPPORTED;
     if (pl.w3d) {
         // (128-byte unit pair, row, pair): one box = 16 rows x KC units
@@ -691,9 +711,9 @@ wq_status gemv_prepare(int WB, int AM, const void *A, const float *a_scale, cons
     p.N = int(N);
     p.K = int(K);
     p.G = G;
-    p.gs = WB == 4 ? c.group_size : int(K);
-    p.upg = WB == 4 ? c.group_size / kunit_of(WB) : 1;
-    p.sym = WB == 4 ? c.symmetric : 1;
+    p.gs = wf_grouped(WF) ? c.group_size : int(K);
+    p.upg = wf_grouped(WF) ? c.group_size / kunit_of(WF) : 1;
+    p.sym = WF == WF_I4 ? c.symmetric : 1;
     p.KB = pl.KB;
     p.T = pl.T;
     p.P = pl.P;
@@ -723,7 +743,7 @@ wq_status gemv_prepare(int WB, int AM, const void *A, const float *a_scale, cons
     p.C = C;
     p.acc_out = acc_out;
     p.fs_off = pl.fs_off;
-    p.nat = WB == 4 && c.layout == WQ_LAYOUT_NATIVE;
+    p.nat = WF == WF_I4 && c.layout == WQ_LAYOUT_NATIVE;
     const bool one = pl.NT == 1;
     const void *func = nullptr;
     if (fa) {
@@ -731,24 +751,34 @@ wq_status gemv_prepare(int WB, int AM, const void *A, const float *a_scale, cons
         p.Aq_out = fa->Aq;
         p.a_scale_out = fa->a_scale;
         const bool bf = fa->bf16;
-        if (WB == 4 && acc_out)
+        if (WF == WF_I1)
+            rc = bf ? (one ? kernel_for<1, A_I8, 1, false, false, 2>(pl, &func) : kernel_for<1, A_I8, 2, false, false, 2>(pl, &func))
+                    : (one ? kernel_for<1, A_I8, 1, false, false, 1>(pl, &func) : kernel_for<1, A_I8, 2, false, false, 1>(pl, &func));
+        else if (WF == WF_I4 && acc_out)
             rc = bf ? (one ? kernel_for<4, A_I8, 1, true, false, 2>(pl, &func) : kernel_for<4, A_I8, 2, true, false, 2>(pl, &func))
                     : (one ? kernel_for<4, A_I8, 1, true, false, 1>(pl, &func) : kernel_for<4, A_I8, 2, true, false, 1>(pl, &func));
-        else if (WB == 4)
+        else if (WF == WF_I4)
             rc = bf ? (one ? kernel_for<4, A_I8, 1, false, false, 2>(pl, &func) : kernel_for<4, A_I8, 2, false, false, 2>(pl, &func))
                     : (one ? kernel_for<4, A_I8, 1, false, false, 1>(pl, &func) : kernel_for<4, A_I8, 2, false, false, 1>(pl, &func));
         else
             rc = bf ? (one ? kernel_for<2, A_I8, 1, false, false, 2>(pl, &func) : kernel_for<2, A_I8, 2, false, false, 2>(pl, &func))
                     : (one ? kernel_for<2, A_I8, 1, false, false, 1>(pl, &func) : kernel_for<2, A_I8, 2, false, false, 1>(pl, &func));
-    } else
-    if (WB == 4 && AM == A_F16)
+    } else if (WF == WF_E2M1)
+        rc = one ? kernel_for<WF_E2M1, A_F16, 1>(pl, &func) : kernel_for<WF_E2M1, A_F16, 2>(pl, &func);
+    else if (WF == WF_E4M3)
+        rc = one ? kernel_for<WF_E4M3, A_F16, 1>(pl, &func) : kernel_for<WF_E4M3, A_F16, 2>(pl, &func);
+    else if (WF == WF_I1 && AM == A_F16)
+        rc = one ? kernel_for<WF_I1, A_F16, 1>(pl, &func) : kernel_for<WF_I1, A_F16, 2>(pl, &func);
+    else if (WF == WF_I1)
+        rc = one ? kernel_for<WF_I1, A_I8, 1>(pl, &func) : kernel_for<WF_I1, A_I8, 2>(pl, &func);
+    else if (WF == WF_I4 && AM == A_F16)
         rc = one ? kernel_for<4, A_F16, 1>(pl, &func)
                  : pl.wide ? kernel_for<4, A_F16, 2, false, true>(pl, &func) : kernel_for<4, A_F16, 2>(pl, &func);
-    else if (WB == 4 && AM == A_BF16)
+    else if (WF == WF_I4 && AM == A_BF16)
         rc = one ? kernel_for<4, A_BF16, 1>(pl, &func)
                  : pl.wide ? kernel_for<4, A_BF16, 2, false, true>(pl, &func) : kernel_for<4, A_BF16, 2>(pl, &func);
-    else if (WB == 4 && acc_out) rc = one ? kernel_for<4, A_I8, 1, true>(pl, &func) : kernel_for<4, A_I8, 2, true>(pl, &func);
-    else if (WB == 4) rc = one ? kernel_for<4, A_I8, 1>(pl, &func) : kernel_for<4, A_I8, 2>(pl, &func);
+    else if (WF == WF_I4 && acc_out) rc = one ? kernel_for<4, A_I8, 1, true>(pl, &func) : kernel_for<4, A_I8, 2, true>(pl, &func);
+    else if (WF == WF_I4) rc = one ? kernel_for<4, A_I8, 1>(pl, &func) : kernel_for<4, A_I8, 2>(pl, &func);
     else if (AM == A_F16) rc = kernel_for<2, A_F16, 1>(pl, &func);
     else if (AM == A_BF16) rc = kernel_for<2, A_BF16, 1>(pl, &func);
     else rc = one ? kernel_for<2, A_I8, 1>(pl, &func) : kernel_for<2, A_I8, 2>(pl, &func);
@@ -769,12 +799,12 @@ wq_status gemv_prepare(int WB, int AM, const void *A, const float *a_scale, cons
 }
 
 // Few-token path (1 <= M <= 16).  Returns WQ_ERR_UNSUPPORTED if no launch plan fits.
-wq_status gemv_small_m(int WB, int AM, const void *A, const float *a_scale, const uint8_t *Wq, const void *scales,
+wq_status gemv_small_m(int WF, int AM, const void *A, const float *a_scale, const uint8_t *Wq, const void *scales,
                        const void *zeros, const void *bias, void *C, int32_t *acc_out, int64_t M, int64_t N,
                        int64_t K, const wq_qconfig &c, cudaStream_t st)
 {
     PreparedLaunch L;
-    const wq_status rc = gemv_prepare(WB, AM, A, a_scale, Wq, scales, zeros, bias, C, acc_out, M, N, K, c, &L);
+    const wq_status rc = gemv_prepare(WF, AM, A, a_scale, Wq, scales, zeros, bias, C, acc_out, M, N, K, c, &L);
     if (rc != WQ_OK) return rc;
     return launch_prepared(L, st, "gemv_kernel");
 }

@@ -36,7 +36,8 @@ wq_status prepare_op(const wq_matmul_desc &d, PreparedLaunch *L)
     if (rc != WQ_OK) return rc;
     if (d.M > 16) return fail(WQ_ERR_UNSUPPORTED, "wq_graph: matmuls of at most 16 tokens (M=%lld)", (long long)d.M);
     const int am = d.a_dt == WQ_F16 ? 0 : 1;
-    return gemv_prepare(d.c.bits, am, d.A, nullptr, d.Wq, d.scales, d.c.bits == 4 && !d.c.symmetric ? d.zeros : nullptr,
+    const int wf = wf_of(d.c);
+    return gemv_prepare(wf, am, d.A, nullptr, d.Wq, d.scales, wf == WF_I4 && !d.c.symmetric ? d.zeros : nullptr,
                         d.bias, d.C, nullptr, d.M, d.N, d.K, d.c, L);
 }
 

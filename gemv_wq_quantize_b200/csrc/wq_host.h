@@ -9,6 +9,7 @@
 #include <cstdio>
 
 #include "wq.h"
+#include "wq_format.h"
 
 namespace wq {
 

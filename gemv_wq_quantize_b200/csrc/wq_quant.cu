@@ -5,7 +5,9 @@
 // (cnblogs), part 1: step 1 (absmax scale, round, clip, two INT4 per byte) and
 // step 2 (q = round(a / a_scale)); "BitBLAS practical guide: mixed-precision
 // compute in vLLM" (mlqm): "Advanced features 2" (group_size 128, scales,
-// "original" zero points) and the BitNet-b1.58 ternary weights of "Real-world case".
+// "original" zero points), the BitNet-b1.58 ternary weights of "Real-world case", and the
+// FP4 / FP8 / INT1 weights of "Main features" (e2m1 / e4m3 codes with binary16 group scales;
+// binary weights with one mean-|w| scale).
 //
 // Every decision that turns a float into an integer code is taken in binary32
 // with IEEE division (__fdiv_rn) and round-half-to-even (rintf), and the scale is
@@ -123,6 +125,77 @@ __global__ void __launch_bounds__(256) quant_int4_kernel(const T *__restrict__ W
     }
 }
 
+// ---- FP4 e2m1 / FP8 e4m3 codes -----------------------------------------------
+// Nearest value of the format to x (|x| <= its largest finite value), ties to even, as a
+// code (sign | exponent | mantissa), +0 for a zero result.  Below the smallest normal the
+// value is a multiple of the subnormal step; above it x is scaled by an exact power of two so
+// that rintf rounds to the format's mantissa bits (a result of 2^(m+1) moves to the next
+// binade).
+template <int FMT>
+__device__ __forceinline__ uint32_t minifloat_code(float x)
+{
+    constexpr int MB = FMT == WQ_FMT_E2M1 ? 1 : 3;       // mantissa bits
+    constexpr int BIAS = FMT == WQ_FMT_E2M1 ? 1 : 7;
+    constexpr float kMinNormal = FMT == WQ_FMT_E2M1 ? 1.0f : 0x1p-6f;
+    constexpr float kSubStep = FMT == WQ_FMT_E2M1 ? 0.5f : 0x1p-9f;
+    const float a = fabsf(x);
+    uint32_t code;
+    if (a < kMinNormal) {
+        code = uint32_t(rintf(__fdiv_rn(a, kSubStep)));  // a power of two: exact; 2^MB is the smallest normal
+    } else {
+        int e = int((__float_as_uint(a) >> 23) & 0xffu) - 127;                   // floor(log2 a)
+        const float scaled = __fmul_rn(a, __uint_as_float(uint32_t(127 + MB - e) << 23));  // in [2^MB, 2^(MB+1))
+        uint32_t q = uint32_t(rintf(scaled));
+        if (q == (2u << MB)) {
+            q = 1u << MB;
+            ++e;
+        }
+        code = (uint32_t(e + BIAS) << MB) | (q - (1u << MB));
+    }
+    if (code != 0u && x < 0.f) code |= FMT == WQ_FMT_E2M1 ? 0x8u : 0x80u;
+    return code;
+}
+
+// One warp per (row n, group g), lane l on elements c*128 + 4l .. +3 of each 128-chunk c:
+// scale = fp16(absmax / 6 or 448), codes of clip(w / scale, -max, max).
+template <typename T, int FMT>
+__global__ void __launch_bounds__(256) quant_minifloat_kernel(const T *__restrict__ W, int64_t N, int64_t K, int gs,
+                                                              uint8_t *__restrict__ Wq, __half *__restrict__ scales)
+{
+    constexpr float kMax = FMT == WQ_FMT_E2M1 ? 6.0f : 448.0f;
+    const int64_t G = K / gs;
+    const int64_t warp = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+    const int lane = threadIdx.x & 31;
+    if (warp >= N * G) return;
+    const int64_t n = warp / G, g = warp % G;
+    const T *w = W + n * K + g * gs;
+    const int chunks = gs / 128;
+    float amax = 0.f;
+    for (int c = 0; c < chunks; ++c) {
+        float v[4];
+        load4(w + c * 128 + 4 * lane, v);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) amax = fmaxf(amax, fabsf(v[i]));
+    }
+    amax = warp_max(amax);
+    const __half sh = __float2half_rn(__fdiv_rn(amax, kMax));
+    const float s = __half2float(sh);
+    if (lane == 0) scales[n * G + g] = sh;
+    for (int c = 0; c < chunks; ++c) {
+        float v[4];
+        load4(w + c * 128 + 4 * lane, v);
+        uint32_t packed = 0;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const uint32_t code = s != 0.f ? minifloat_code<FMT>(clampf(__fdiv_rn(v[i], s), -kMax, kMax)) : 0u;
+            packed |= code << ((FMT == WQ_FMT_E2M1 ? 4 : 8) * i);
+        }
+        const int64_t e0 = g * gs + c * 128 + 4 * lane;
+        if (FMT == WQ_FMT_E2M1) *reinterpret_cast<uint16_t *>(Wq + n * (K / 2) + e0 / 2) = uint16_t(packed);
+        else *reinterpret_cast<uint32_t *>(Wq + n * K + e0) = packed;
+    }
+}
+
 // ---- ternary: exact mean |w| via per-exponent integer bins ----------------
 // |w| = m * 2^(E-149) with integer m < 2^24 and E = max(biased exponent, 1) - 1,
 // so sum|w| = (sum_E bins[E] * 2^E) * 2^-149 exactly, where bins[E] sums the m's.
@@ -218,13 +291,40 @@ __global__ void __launch_bounds__(256) pack_ternary_kernel(const T *__restrict__
     reinterpret_cast<uint32_t *>(Wq)[t] = word;
 }
 
+// Binary (INT1) weights: 32 consecutive elements per thread -> one word, bit i = (w >= 0).
+template <typename T>
+__global__ void __launch_bounds__(256) pack_binary_kernel(const T *__restrict__ W, int64_t count,
+                                                          uint32_t *__restrict__ Wq)
+{
+    const int64_t t = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (t * 32 >= count) return;
+    uint32_t word = 0;
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+        float v[4];
+        load4(W + t * 32 + 4 * c, v);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) word |= (v[i] >= 0.f ? 1u : 0u) << (4 * c + i);
+    }
+    Wq[t] = word;
+}
+
+// bits 4 / 2 / 1: signed integer codes; raw: FP4 nibbles / FP8 bytes as they are.
 __global__ void __launch_bounds__(256) unpack_kernel(const uint8_t *__restrict__ Wq, int64_t nbytes, int bits, int sym,
-                                                     int8_t *__restrict__ q)
+                                                     int raw, int8_t *__restrict__ q)
 {
     const int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
     if (i >= nbytes) return;
     const uint32_t b = Wq[i];
-    if (bits == 4) {
+    if (bits == 8) {
+        q[i] = int8_t(b);
+    } else if (bits == 4 && raw) {
+        q[2 * i] = int8_t(b & 15);
+        q[2 * i + 1] = int8_t(b >> 4);
+    } else if (bits == 1) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) q[8 * i + j] = int8_t(((b >> j) & 1u) ? 1 : -1);
+    } else if (bits == 4) {
         int lo = b & 15, hi = b >> 4;
         q[2 * i] = int8_t(sym ? lo - 8 : lo);
         q[2 * i + 1] = int8_t(sym ? hi - 8 : hi);
@@ -317,6 +417,17 @@ template <typename T>
 wq_status quantize_typed(const T *W, int64_t N, int64_t K, wq_qconfig c, uint8_t *Wq, void *scales, void *zeros,
                          void *ws, size_t ws_bytes, cudaStream_t st)
 {
+    if (c.format != WQ_FMT_INT) {
+        const int64_t warps = N * (K / c.group_size);
+        const int grid = blocks_for(warps * 32);
+        if (c.format == WQ_FMT_E2M1)
+            quant_minifloat_kernel<T, WQ_FMT_E2M1><<<grid, 256, 0, st>>>(W, N, K, c.group_size, Wq,
+                                                                          static_cast<__half *>(scales));
+        else
+            quant_minifloat_kernel<T, WQ_FMT_E4M3><<<grid, 256, 0, st>>>(W, N, K, c.group_size, Wq,
+                                                                          static_cast<__half *>(scales));
+        return check_launch("quant_minifloat_kernel");
+    }
     if (c.bits == 4) {
         const int64_t G = K / c.group_size;
         const int64_t warps = N * G;
@@ -330,10 +441,10 @@ wq_status quantize_typed(const T *W, int64_t N, int64_t K, wq_qconfig c, uint8_t
                                                               static_cast<__half *>(zeros));
         return check_launch("quant_int4_kernel");
     }
-    // ternary
+    // ternary / binary: one mean-|w| scale for the tensor
     auto *bins = static_cast<unsigned long long *>(ws);
     if (!bins || ws_bytes < kBins * sizeof(unsigned long long))
-        return fail(WQ_ERR_WORKSPACE, "ternary quantization needs %zu bytes of workspace",
+        return fail(WQ_ERR_WORKSPACE, "ternary / binary quantization needs %zu bytes of workspace",
                     size_t(kBins * sizeof(unsigned long long)));
     const int64_t count = N * K;
     if (cudaMemsetAsync(bins, 0, kBins * sizeof(unsigned long long), st) != cudaSuccess)
@@ -341,6 +452,10 @@ wq_status quantize_typed(const T *W, int64_t N, int64_t K, wq_qconfig c, uint8_t
     const int grid = int(std::min<int64_t>(4 * device_info().sm_count, blocks_for(count)));
     abs_bins_kernel<T><<<grid, 256, 0, st>>>(W, count, bins);
     ternary_scale_kernel<<<1, 32, 0, st>>>(bins, count, static_cast<float *>(scales));
+    if (c.bits == 1) {
+        pack_binary_kernel<T><<<blocks_for(count / 32), 256, 0, st>>>(W, count, reinterpret_cast<uint32_t *>(Wq));
+        return check_launch("binary quantization kernels");
+    }
     pack_ternary_kernel<T><<<blocks_for(count / 16), 256, 0, st>>>(W, count, static_cast<const float *>(scales), Wq);
     return check_launch("ternary quantization kernels");
 }
@@ -352,7 +467,7 @@ using namespace wq;
 
 extern "C" size_t wq_quantize_workspace_size(int64_t, int64_t, wq_qconfig c)
 {
-    return c.bits == 2 ? kBins * sizeof(unsigned long long) : 0;
+    return (c.format == WQ_FMT_INT && (c.bits == 2 || c.bits == 1)) ? kBins * sizeof(unsigned long long) : 0;
 }
 
 extern "C" wq_status wq_quantize_pack(const void *W, wq_dtype w_dt, int64_t N, int64_t K, wq_qconfig c, uint8_t *Wq,
@@ -367,15 +482,24 @@ extern "C" wq_status wq_quantize_pack(const void *W, wq_dtype w_dt, int64_t N, i
         return fail(WQ_ERR_INVALID_ARG, "w_dt must be WQ_F32, WQ_F16 or WQ_BF16");
     if (!aligned16(W) || !aligned16(Wq) || (zeros && !aligned16(zeros)) || !aligned16(scales))
         return fail(WQ_ERR_ALIGNMENT, "device pointers must be 16-byte aligned");
-    if (c.bits == 4) {
+    if (c.format == WQ_FMT_E2M1 || c.format == WQ_FMT_E4M3) {
+        if (c.bits != (c.format == WQ_FMT_E2M1 ? 4 : 8))
+            return fail(WQ_ERR_INVALID_ARG, "FP4 (e2m1) weights have bits 4, FP8 (e4m3) bits 8");
+        if (c.group_size <= 0 || K % c.group_size) return fail(WQ_ERR_INVALID_ARG, "K %% group_size != 0");
+        if (c.group_size % 128) return fail(WQ_ERR_UNSUPPORTED, "group_size must be a multiple of 128");
+    } else if (c.format != WQ_FMT_INT) {
+        return fail(WQ_ERR_INVALID_ARG, "unknown weight format %d", int(c.format));
+    } else if (c.bits == 4) {
         if (c.group_size <= 0 || K % c.group_size) return fail(WQ_ERR_INVALID_ARG, "K %% group_size != 0");
         if (c.group_size % 128) return fail(WQ_ERR_UNSUPPORTED, "group_size must be a multiple of 128");
         if (!c.symmetric && !zeros) return fail(WQ_ERR_INVALID_ARG, "asymmetric INT4 needs a zeros buffer");
     } else if (c.bits == 2) {
         if (!c.ternary) return fail(WQ_ERR_UNSUPPORTED, "INT2 weights are produced by the ternary quantizer only");
         if (K % 64) return fail(WQ_ERR_INVALID_ARG, "INT2 needs K %% 64 == 0");
+    } else if (c.bits == 1) {
+        if (K % 128) return fail(WQ_ERR_INVALID_ARG, "INT1 needs K %% 128 == 0");
     } else {
-        return fail(WQ_ERR_INVALID_ARG, "bits must be 4 or 2");
+        return fail(WQ_ERR_INVALID_ARG, "bits must be 4, 2 or 1 (integer codes)");
     }
     switch (w_dt) {
     case WQ_F32: return quantize_typed(static_cast<const float *>(W), N, K, c, Wq, scales, zeros, workspace, ws_bytes, stream);
@@ -387,11 +511,13 @@ extern "C" wq_status wq_quantize_pack(const void *W, wq_dtype w_dt, int64_t N, i
 extern "C" wq_status wq_unpack(const uint8_t *Wq, int64_t N, int64_t K, wq_qconfig c, int8_t *q, cudaStream_t stream)
 {
     if (N <= 0 || K <= 0 || !Wq || !q) return fail(WQ_ERR_INVALID_ARG, "bad sizes or null pointer");
-    if (c.bits != 4 && c.bits != 2) return fail(WQ_ERR_INVALID_ARG, "bits must be 4 or 2");
-    if (K % (8 / c.bits)) return fail(WQ_ERR_INVALID_ARG, "K must fill whole bytes");
+    const bool ok = (c.format == WQ_FMT_INT && (c.bits == 4 || c.bits == 2 || c.bits == 1)) ||
+                    (c.format == WQ_FMT_E2M1 && c.bits == 4) || (c.format == WQ_FMT_E4M3 && c.bits == 8);
+    if (!ok) return fail(WQ_ERR_INVALID_ARG, "bits / format: INT 4, 2 or 1; E2M1 4; E4M3 8");
+    if (c.bits < 8 && K % (8 / c.bits)) return fail(WQ_ERR_INVALID_ARG, "K must fill whole bytes");
     const int64_t nbytes = N * K * c.bits / 8;
     if (c.layout == WQ_LAYOUT_NATIVE) {
-        if (c.bits != 4) return fail(WQ_ERR_UNSUPPORTED, "the native layout is INT4 only");
+        if (c.bits != 4 || c.format != WQ_FMT_INT) return fail(WQ_ERR_UNSUPPORTED, "the native layout is INT4 only");
         if (K % 8 || !aligned16(Wq)) return fail(WQ_ERR_INVALID_ARG, "native layout: K %% 8 == 0, Wq 16-byte aligned");
         const int64_t nwords = nbytes / 4;
         unpack_native_kernel<<<blocks_for(nwords), 256, 0, stream>>>(reinterpret_cast<const uint32_t *>(Wq), nwords,
@@ -399,7 +525,8 @@ extern "C" wq_status wq_unpack(const uint8_t *Wq, int64_t N, int64_t K, wq_qconf
         return check_launch("unpack_native_kernel");
     }
     if (c.layout != WQ_LAYOUT_NT) return fail(WQ_ERR_INVALID_ARG, "unknown layout %d", int(c.layout));
-    unpack_kernel<<<blocks_for(nbytes), 256, 0, stream>>>(Wq, nbytes, c.bits, c.bits == 4 ? c.symmetric : 1, q);
+    unpack_kernel<<<blocks_for(nbytes), 256, 0, stream>>>(Wq, nbytes, c.bits, c.bits == 4 ? c.symmetric : 1,
+                                                          c.format != WQ_FMT_INT ? 1 : 0, q);
     return check_launch("unpack_kernel");
 }
 
@@ -407,7 +534,7 @@ extern "C" wq_status wq_repack(const uint8_t *Wq, int64_t N, int64_t K, wq_qconf
                                cudaStream_t stream)
 {
     if (N <= 0 || K <= 0 || !Wq || !Wq_native) return fail(WQ_ERR_INVALID_ARG, "bad sizes or null pointer");
-    if (c.bits != 4) return fail(WQ_ERR_UNSUPPORTED, "the native layout is INT4 only");
+    if (c.bits != 4 || c.format != WQ_FMT_INT) return fail(WQ_ERR_UNSUPPORTED, "the native layout is INT4 only");
     if (c.layout != WQ_LAYOUT_NT) return fail(WQ_ERR_INVALID_ARG, "wq_repack reads weights in WQ_LAYOUT_NT");
     if (K % 8) return fail(WQ_ERR_INVALID_ARG, "K %% 8 != 0");
     if (!aligned16(Wq) || !aligned16(Wq_native)) return fail(WQ_ERR_ALIGNMENT, "Wq and Wq_native must be 16-byte aligned");

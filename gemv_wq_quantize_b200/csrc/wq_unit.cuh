@@ -1,5 +1,6 @@
 // wq_unit.cuh -- the arithmetic of one weight "unit" (16 rows x 64 packed bytes per row:
-// 128 k of INT4 or 256 k of INT2) on mma.sync, shared by the few-token kernels.
+// 128 k of INT4 or FP4, 256 k of INT2, 512 k of INT1, 64 k of FP8) on mma.sync, shared by
+// the few-token kernels.
 //
 // Exactness: weights enter the tensor cores as the integers q - z (|q - z| <= 15), which
 // f16, bf16 and int8 represent exactly, so every product is exact; FP paths accumulate in
@@ -10,7 +11,10 @@
 // an MMA sums over k, the activations (B operand) are loaded in the same permuted order,
 // so the weights are used straight from the packed layout with no reordering.  INT4 weights
 // in the kernel-native order (see wq_repack) unpack to pairs (k, k+1), the activations'
-// own order, and their B fragments need no permutation.
+// own order, and their B fragments need no permutation.  FP4 (e2m1) and FP8 (e4m3) codes are
+// turned into exact binary16 values by the hardware conversions, pairs (k, k+1) in natural
+// order; INT1 bits become +-1 (pairs (k, k+16) of a word, whose activation pairs are formed
+// per word).
 #pragma once
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -19,18 +23,17 @@
 #include <type_traits>
 
 #include "wq_device.cuh"
+#include "wq_format.h"
 
 namespace wq {
 
 enum AMode { A_F16 = 0, A_BF16 = 1, A_I8 = 2 };
 
-__host__ __device__ constexpr int kunit_of(int WB) { return WB == 4 ? 128 : 256; }
+// k of one unit (64 packed bytes of a row) for weight format WF
+__host__ __device__ constexpr int kunit_of(int WF) { return 512 / wf_bits(WF); }
 // mma k-steps per unit (k16 for f16/bf16, k32 for int8)
-__host__ __device__ constexpr int steps_of(int WB, int AM)
-{
-    return AM == A_I8 ? (WB == 4 ? 4 : 8) : (WB == 4 ? 8 : 16);
-}
-__host__ __device__ constexpr int qn_of(int WB, int AM) { return steps_of(WB, AM) / 2; }
+__host__ __device__ constexpr int steps_of(int WF, int AM) { return AM == A_I8 ? kunit_of(WF) / 32 : kunit_of(WF) / 16; }
+__host__ __device__ constexpr int qn_of(int WF, int AM) { return steps_of(WF, AM) / 2; }
 
 // B fragments of one unit for the n8 token tile `nt`: bf[q] holds {b0, b1} of k-steps 2q
 // and 2q+1.  addr(m, o) gives the shared-memory address of byte o of token m's activations
@@ -39,11 +42,13 @@ __host__ __device__ constexpr int qn_of(int WB, int AM) { return steps_of(WB, AM
 // over the unit (the quad of lanes sharing a token adds up to the token's sum).
 // nat: INT4 weights in the kernel-native order (nibble i of a word = element 0,2,4,6,1,3,5,7),
 // whose unpack yields the pairs (k, k+1) (FP) or the byte quads (k, k+4, k+1, k+5) (INT8).
-template <int WB, int AM, typename Addr>
-__device__ __forceinline__ void build_bfrag(Addr addr, int M, int nt, int lane, uint4 (&bf)[qn_of(WB, AM)],
+// FP4 weights unpack to the pairs (k, k+1) like native INT4; FP8 lanes hold 16 consecutive k.
+// (INT1 builds its fragments per word inside unit_mma_b1.)
+template <int WF, int AM, typename Addr>
+__device__ __forceinline__ void build_bfrag(Addr addr, int M, int nt, int lane, uint4 (&bf)[qn_of(WF, AM)],
                                             int &asum, bool nat = false)
 {
-    constexpr int QN = qn_of(WB, AM);
+    constexpr int QN = qn_of(WF, AM);
     const int g = lane >> 2, t = lane & 3;
     const int m = nt * 8 + g;
     asum = 0;
@@ -55,11 +60,14 @@ __device__ __forceinline__ void build_bfrag(Addr addr, int M, int nt, int lane, 
 #pragma unroll
     for (int q = 0; q < QN; ++q) {
         uint4 r;
-        if constexpr (AM != A_I8 && WB == 4) {
+        if constexpr (AM != A_I8 && WF == WF_E4M3) {
+            // k-steps 2q, 2q+1 use halves 16t + 8q + {0..7} as the pairs (0,1),(2,3) / (4,5),(6,7)
+            r = lds128(addr(m, (16 * t + 8 * q) * 2));
+        } else if constexpr (AM != A_I8 && (WF == WF_I4 || WF == WF_E2M1)) {
             // k-steps 2q, 2q+1 use halves 32t + 8q + {0..7} as pairs (0,4),(1,5) / (2,6),(3,7)
-            // (native order: (0,1),(2,3) / (4,5),(6,7), the halves as they lie)
+            // (native order and FP4: (0,1),(2,3) / (4,5),(6,7), the halves as they lie)
             const uint4 v = lds128(addr(m, (32 * t + 8 * q) * 2));
-            if (nat) {
+            if (WF == WF_E2M1 || nat) {
                 r = v;
             } else {
                 r.x = prmt(v.x, v.z, 0x5410);
@@ -67,7 +75,7 @@ __device__ __forceinline__ void build_bfrag(Addr addr, int M, int nt, int lane, 
                 r.z = prmt(v.y, v.w, 0x5410);
                 r.w = prmt(v.y, v.w, 0x7632);
             }
-        } else if constexpr (AM != A_I8 && WB == 2) {
+        } else if constexpr (AM != A_I8 && WF == WF_I2) {
             // k-steps 4j + 2hh (+1): pairs (i, i+8) of halves 64t + 16j + 4hh + {0..3, 8..11}
             const int j = q >> 1, hh = q & 1;
             const int o = (64 * t + 16 * j + 4 * hh) * 2;
@@ -77,7 +85,7 @@ __device__ __forceinline__ void build_bfrag(Addr addr, int M, int nt, int lane, 
             r.y = prmt(lo.x, hi.x, 0x7632);
             r.z = prmt(lo.y, hi.y, 0x5410);
             r.w = prmt(lo.y, hi.y, 0x7632);
-        } else if constexpr (WB == 4) {
+        } else if constexpr (WF == WF_I4) {
             // k-steps 2q, 2q+1 (k32): bytes 32t + 16q + {0..15} as quads (0,2,4,6),(1,3,5,7)
             // (native order: (0,4,1,5),(2,6,3,7))
             const uint4 v = lds128(addr(m, 32 * t + 16 * q));
@@ -121,12 +129,61 @@ __device__ __forceinline__ void build_bfrag(Addr addr, int M, int nt, int lane, 
 template <int AM>
 using acc_t = typename std::conditional<AM == A_I8, int, float>::type;
 
-template <int WB, int AM, int NT, int NTL>
+template <int WF, int AM, int NT, int NTL>
 __device__ __forceinline__ void unit_mma(const uint4 (&wa)[NTL], const uint4 (&wb)[NTL],
-                                         const uint4 (&bf)[NT][qn_of(WB, AM)], const uint32_t (&z_lo)[NTL],
+                                         const uint4 (&bf)[NT][qn_of(WF, AM)], const uint32_t (&z_lo)[NTL],
                                          const uint32_t (&z_hi)[NTL], acc_t<AM> (&acc)[2][NTL][NT][4])
 {
-    if constexpr (AM == A_F16 && WB == 4) {
+    if constexpr (AM == A_F16 && WF == WF_E2M1) {
+        // byte b of word j -> the exact binary16 pair (8j + 2b, 8j + 2b + 1); no zero point
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+#pragma unroll
+                for (int l = 0; l < NTL; ++l) {
+                    const uint32_t wl = j == 0 ? wa[l].x : j == 1 ? wa[l].y : j == 2 ? wa[l].z : wa[l].w;
+                    const uint32_t wh = j == 0 ? wb[l].x : j == 1 ? wb[l].y : j == 2 ? wb[l].z : wb[l].w;
+                    uint32_t a[4];
+                    if (h == 0) {
+                        a[0] = e2m1x2_to_f16x2<0>(wl);
+                        a[1] = e2m1x2_to_f16x2<0>(wh);
+                        a[2] = e2m1x2_to_f16x2<1>(wl);
+                        a[3] = e2m1x2_to_f16x2<1>(wh);
+                    } else {
+                        a[0] = e2m1x2_to_f16x2<2>(wl);
+                        a[1] = e2m1x2_to_f16x2<2>(wh);
+                        a[2] = e2m1x2_to_f16x2<3>(wl);
+                        a[3] = e2m1x2_to_f16x2<3>(wh);
+                    }
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt)
+                        mma_f16(acc[(j & 1)][l][nt], a, h ? bf[nt][j].z : bf[nt][j].x, h ? bf[nt][j].w : bf[nt][j].y);
+                }
+            }
+        }
+    } else if constexpr (AM == A_F16 && WF == WF_E4M3) {
+        // word j holds k = 16t + 4j .. 4j + 3: halves 0 / 1 -> the exact binary16 pairs (4j, 4j+1) /
+        // (4j+2, 4j+3) of k-step j
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+#pragma unroll
+            for (int l = 0; l < NTL; ++l) {
+                const uint32_t wl = j == 0 ? wa[l].x : j == 1 ? wa[l].y : j == 2 ? wa[l].z : wa[l].w;
+                const uint32_t wh = j == 0 ? wb[l].x : j == 1 ? wb[l].y : j == 2 ? wb[l].z : wb[l].w;
+                uint32_t a[4];
+                a[0] = e4m3x2_to_f16x2<0>(wl);
+                a[1] = e4m3x2_to_f16x2<0>(wh);
+                a[2] = e4m3x2_to_f16x2<1>(wl);
+                a[3] = e4m3x2_to_f16x2<1>(wh);
+                const int q = j >> 1;
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt)
+                    mma_f16(acc[(j & 1)][l][nt], a, (j & 1) ? bf[nt][q].z : bf[nt][q].x,
+                            (j & 1) ? bf[nt][q].w : bf[nt][q].y);
+            }
+        }
+    } else if constexpr (AM == A_F16 && WF == WF_I4) {
         // x = 1024 + nibble (low nibbles) or 1024 + 16 * nibble (high nibbles), made the
         // exact integer q - z by one half2 add / fma
         uint32_t clo0[NTL], clo1[NTL], chi0[NTL], chi1[NTL];
@@ -161,7 +218,7 @@ __device__ __forceinline__ void unit_mma(const uint4 (&wa)[NTL], const uint4 (&w
                 }
             }
         }
-    } else if constexpr (AM == A_BF16 && WB == 4) {
+    } else if constexpr (AM == A_BF16 && WF == WF_I4) {
         // x = 128 + nibble in bf16 (shifted nibbles), minus 128 + z
         uint32_t cc0[NTL], cc1[NTL];
 #pragma unroll
@@ -190,7 +247,7 @@ __device__ __forceinline__ void unit_mma(const uint4 (&wa)[NTL], const uint4 (&w
                 }
             }
         }
-    } else if constexpr (AM != A_I8 && WB == 2) {
+    } else if constexpr (AM != A_I8 && WF == WF_I2) {
         // 2-bit field f, c' = f ^ 2 in [0,3], value c' - 2.  Field pairs (i, i+8) of a word.
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
@@ -235,7 +292,7 @@ __device__ __forceinline__ void unit_mma(const uint4 (&wa)[NTL], const uint4 (&w
                 }
             }
         }
-    } else if constexpr (AM == A_I8 && WB == 4) {
+    } else if constexpr (AM == A_I8 && WF == WF_I4) {
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
 #pragma unroll
@@ -271,6 +328,109 @@ __device__ __forceinline__ void unit_mma(const uint4 (&wa)[NTL], const uint4 (&w
 #pragma unroll
                     for (int nt = 0; nt < NT; ++nt)
                         mma_u8s8(acc[h][l][nt], a, h ? bf[nt][j].z : bf[nt][j].x, h ? bf[nt][j].w : bf[nt][j].y);
+                }
+            }
+        }
+    }
+}
+
+// INT1 (binary) weights, one unit = 512 k: lane t holds k = 128t .. 128t + 127 of each of its
+// two rows as four words, bit i of word j being k = 128t + 32j + i (value 2c - 1).
+//  FP16 activations: k-step s of word j pairs (2s, 2s+16) and (2s+1, 2s+17), so one shift and
+//  one LOP3 give each +-1 pair, and the activation pairs are formed from the word's 32 halves
+//  by one byte permute each.
+//  INT8 activations: (w >> i) & 0x01010101 gives the quad (i, i+8, i+16, i+24) of bits, made
+//  signed bytes +-1; k-step s of word j uses quads 2s and 2s+1, the activation quads likewise.
+// addr(m, o): byte o of token m's activations of the unit; tokens >= M give zeros.
+template <int AM, int NT, int NTL, typename Addr>
+__device__ __forceinline__ void unit_mma_b1(const uint4 (&wa)[NTL], const uint4 (&wb)[NTL], Addr addr, int M,
+                                            int lane, acc_t<AM> (&acc)[2][NTL][NT][4])
+{
+    const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        if constexpr (AM == A_F16) {
+            uint32_t R[NT][16];
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+                const int m = nt * 8 + g;
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const uint4 v = m < M ? lds128(addr(m, (128 * t + 32 * j) * 2 + 16 * i)) : make_uint4(0, 0, 0, 0);
+                    R[nt][4 * i + 0] = v.x;
+                    R[nt][4 * i + 1] = v.y;
+                    R[nt][4 * i + 2] = v.z;
+                    R[nt][4 * i + 3] = v.w;
+                }
+            }
+#pragma unroll
+            for (int s2 = 0; s2 < 8; ++s2) {
+                uint32_t b0[NT], b1[NT];
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) {
+                    b0[nt] = prmt(R[nt][s2], R[nt][s2 + 8], 0x5410);  // halves 2s, 2s + 16
+                    b1[nt] = prmt(R[nt][s2], R[nt][s2 + 8], 0x7632);  // halves 2s + 1, 2s + 17
+                }
+#pragma unroll
+                for (int l = 0; l < NTL; ++l) {
+                    const uint32_t wl = j == 0 ? wa[l].x : j == 1 ? wa[l].y : j == 2 ? wa[l].z : wa[l].w;
+                    const uint32_t wh = j == 0 ? wb[l].x : j == 1 ? wb[l].y : j == 2 ? wb[l].z : wb[l].w;
+                    uint32_t a[4];
+                    a[0] = pm1_f16x2(wl << (15 - 2 * s2));
+                    a[1] = pm1_f16x2(wh << (15 - 2 * s2));
+                    a[2] = pm1_f16x2(wl << (14 - 2 * s2));
+                    a[3] = pm1_f16x2(wh << (14 - 2 * s2));
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt) mma_f16(acc[s2 & 1][l][nt], a, b0[nt], b1[nt]);
+                }
+            }
+        } else {
+            static_assert(AM == A_I8, "INT1 weights take FP16 or INT8 activations");
+            uint32_t R[NT][8];
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+                const int m = nt * 8 + g;
+#pragma unroll
+                for (int i = 0; i < 2; ++i) {
+                    const uint4 v = m < M ? lds128(addr(m, 128 * t + 32 * j + 16 * i)) : make_uint4(0, 0, 0, 0);
+                    R[nt][4 * i + 0] = v.x;
+                    R[nt][4 * i + 1] = v.y;
+                    R[nt][4 * i + 2] = v.z;
+                    R[nt][4 * i + 3] = v.w;
+                }
+            }
+#pragma unroll
+            for (int a2 = 0; a2 < 2; ++a2) {
+                uint32_t E0[NT], E1[NT], O0[NT], O1[NT];
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) {
+                    E0[nt] = prmt(R[nt][a2], R[nt][a2 + 2], 0x6420);
+                    E1[nt] = prmt(R[nt][a2 + 4], R[nt][a2 + 6], 0x6420);
+                    O0[nt] = prmt(R[nt][a2], R[nt][a2 + 2], 0x7531);
+                    O1[nt] = prmt(R[nt][a2 + 4], R[nt][a2 + 6], 0x7531);
+                }
+#pragma unroll
+                for (int hs = 0; hs < 2; ++hs) {
+                    const int s2 = 2 * a2 + hs;  // activation bytes 2s + 8u (b0) and 2s + 1 + 8u (b1)
+                    uint32_t b0[NT], b1[NT];
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt) {
+                        b0[nt] = prmt(E0[nt], E1[nt], hs ? 0x7531 : 0x6420);
+                        b1[nt] = prmt(O0[nt], O1[nt], hs ? 0x7531 : 0x6420);
+                    }
+#pragma unroll
+                    for (int l = 0; l < NTL; ++l) {
+                        const uint32_t wl = j == 0 ? wa[l].x : j == 1 ? wa[l].y : j == 2 ? wa[l].z : wa[l].w;
+                        const uint32_t wh = j == 0 ? wb[l].x : j == 1 ? wb[l].y : j == 2 ? wb[l].z : wb[l].w;
+                        // bits -> bytes 0 / 1 -> 2c + 0x7F -> ^0x80: signed bytes -1 / +1 (no carries)
+                        uint32_t a[4];
+                        a[0] = ((((wl >> (2 * s2)) & 0x01010101u) << 1) + 0x7F7F7F7Fu) ^ 0x80808080u;
+                        a[1] = ((((wh >> (2 * s2)) & 0x01010101u) << 1) + 0x7F7F7F7Fu) ^ 0x80808080u;
+                        a[2] = ((((wl >> (2 * s2 + 1)) & 0x01010101u) << 1) + 0x7F7F7F7Fu) ^ 0x80808080u;
+                        a[3] = ((((wh >> (2 * s2 + 1)) & 0x01010101u) << 1) + 0x7F7F7F7Fu) ^ 0x80808080u;
+#pragma unroll
+                        for (int nt = 0; nt < NT; ++nt) mma_s8s8(acc[s2 & 1][l][nt], a, b0[nt], b1[nt]);
+                    }
                 }
             }
         }

@@ -1,5 +1,6 @@
 /*
- * wq.h -- C ABI of libwq: INT4 / INT2 weight-quantized matmul on NVIDIA B200 (sm_100a).
+ * wq.h -- C ABI of libwq: INT4 / INT2 / INT1 / FP4 / FP8 weight-quantized matmul on NVIDIA
+ * B200 (sm_100a).
  *
  * The operation (statement of the problem in "BitBLAS practical guide: mixed-precision
  * compute in vLLM" (mlqm), section "What is BitBLAS"):
@@ -20,7 +21,9 @@
  *
  * and the same two paths for ternary / INT2 weights with one scale per tensor
  * (BitBLAS guide, "Core advantages 2" FP16xINT2 and INT8xINT2, "Real-world case"
- * BitNet-b1.58).
+ * BitNet-b1.58).  The other weight types of the guide's "Main features" list:
+ *   FP16 x FP4 (e2m1) and FP16 x FP8 (e4m3) with group scales (W4A16 path only), and
+ *   FP16 x INT1 / INT8 x INT1 (binary weights, one scale per tensor; both paths).
  *
  * Data formats (fixed):
  *   - all matrices row-major; A [M,K], W [N,K], C [M,N];
@@ -28,7 +31,13 @@
  *     symmetric weights store q + 8 (q in [-7,7]); asymmetric weights store q in [0,15]
  *     and dequantize as (q - z) * s;
  *   - INT2 (ternary): element 4j+i in bits 2i..2i+1 of byte j, 2-bit two's complement;
- *   - scales / zeros: binary16 [N, K/group_size] row-major (INT4); one binary32 (INT2).
+ *   - INT1 (binary): element 8j+i in bit i of byte j; bit c stands for the value 2c - 1;
+ *   - FP4: e2m1 codes (bit 3 sign, bits 2..1 exponent with bias 1, bit 0 mantissa: values
+ *     0, 0.5, 1, 1.5, 2, 3, 4, 6 and negatives), packed two per byte as INT4;
+ *   - FP8: e4m3 codes (sign, 4 exponent bits with bias 7, 3 mantissa bits, largest finite
+ *     448, no infinities), one per byte;
+ *   - scales / zeros: binary16 [N, K/group_size] row-major (INT4, FP4, FP8); one binary32
+ *     (INT2, INT1).
  *
  * Quantization readings (the pages print an INT8 range inside the INT4 passage):
  *   symmetric  s = fp16(absmax/7), q = clip(rint(w/s), -7, 7);
@@ -36,6 +45,9 @@
  *              q = clip(rint(w/s) + z, 0, 15);
  *   ternary    s = mean|w| (exact sum rounded once to binary64, / count, -> binary32),
  *              q = clip(rint(w/s), -1, 1);
+ *   binary     s = mean|w| as for ternary, c = (w >= 0) (so -0 and +0 give 1);
+ *   FP4 / FP8  s = fp16(absmax/6) / fp16(absmax/448), code = the format's value nearest to
+ *              clip(w/s, -max, max), ties to the even last mantissa bit, +0 for a zero result;
  *   activations a_scale[m] = absmax_k|A[m,k]| / 127 (binary32), Aq = clip(rint(A/a_scale), -127, 127).
  * rint is round-half-to-even; divisions are IEEE binary32 divisions; the stored binary16 scale
  * is the one used to quantize.  Scale 0 gives code 0.
@@ -75,29 +87,35 @@ typedef enum {
 typedef enum { WQ_F32 = 0, WQ_F16 = 1, WQ_BF16 = 2, WQ_I8 = 3, WQ_I32 = 4 } wq_dtype;
 
 typedef struct {
-    int32_t bits;        /* 4 (INT4) or 2 (INT2 / ternary)                                    */
-    int32_t group_size;  /* INT4: elements of K per scale, a multiple of 128 dividing K;     */
-                         /*       K itself means one scale per output channel.              */
-                         /* INT2: ignored (one scale per tensor).                          */
+    int32_t bits;        /* WQ_FMT_INT: 4 (INT4), 2 (INT2 / ternary) or 1 (INT1 / binary);   */
+                         /* WQ_FMT_E2M1: 4; WQ_FMT_E4M3: 8.                                  */
+    int32_t group_size;  /* INT4, FP4, FP8: elements of K per scale, a multiple of 128        */
+                         /*       dividing K; K itself means one scale per output channel.  */
+                         /* INT2, INT1: ignored (one scale per tensor).                    */
     int32_t symmetric;   /* INT4: 1 = symmetric (q + 8 stored, no zeros), 0 = zero points.  */
+                         /* Ignored for the other types (no zero points).                  */
     int32_t ternary;     /* INT2: must be 1 (codes -1, 0, 1 from the ternary quantizer).    */
     int32_t layout;      /* INT4 only: WQ_LAYOUT_NT (0), the packing described above, or     */
                          /* WQ_LAYOUT_NATIVE (1), the order written by wq_repack.           */
+    int32_t format;      /* WQ_FMT_INT (0), WQ_FMT_E2M1 (1) or WQ_FMT_E4M3 (2).             */
 } wq_qconfig;
 
 #define WQ_LAYOUT_NT 0
 #define WQ_LAYOUT_NATIVE 1
+#define WQ_FMT_INT 0
+#define WQ_FMT_E2M1 1
+#define WQ_FMT_E4M3 2
 
 /* Weight quantization and packing ("Accelerating LLM inference with CUDA Graph and INT4
  * quantization", part 1, step 1; BitBLAS guide, "Advanced features 2").
  *   W       [N,K] device, dtype w_dt in {WQ_F32, WQ_F16, WQ_BF16}.
  *   Wq      [N, K*bits/8] bytes, device, written.
- *   scales  INT4: binary16 [N, K/group_size]; INT2: one binary32. Written.
+ *   scales  INT4, FP4, FP8: binary16 [N, K/group_size]; INT2, INT1: one binary32. Written.
  *   zeros   INT4 asymmetric: binary16 [N, K/group_size] (integers 0..15), written; else NULL.
- *   workspace / ws_bytes: scratch for the INT2 per-tensor mean (wq_quantize_workspace_size
- *   bytes); unused for INT4 (may be NULL).
- * Requires K % group_size == 0 (INT4) or K % 64 == 0 (INT2), N >= 1, K >= 1.
- * Bit-exact with the CPU reference of the same readings. */
+ *   workspace / ws_bytes: scratch for the INT2 / INT1 per-tensor mean
+ *   (wq_quantize_workspace_size bytes); unused otherwise (may be NULL).
+ * Requires K % group_size == 0 (INT4, FP4, FP8), K % 64 == 0 (INT2) or K % 128 == 0 (INT1),
+ * N >= 1, K >= 1.  Bit-exact with the CPU reference of the same readings. */
 wq_status wq_quantize_pack(const void *W, wq_dtype w_dt, int64_t N, int64_t K, wq_qconfig c,
                            uint8_t *Wq, void *scales, void *zeros,
                            void *workspace, size_t ws_bytes, cudaStream_t stream);
@@ -119,7 +137,8 @@ wq_status wq_repack(const uint8_t *Wq, int64_t N, int64_t K, wq_qconfig c, uint8
                     cudaStream_t stream);
 
 /* Inverse of the packing: signed codes q [N,K] int8 (symmetric INT4: nibble - 8; asymmetric
- * INT4: nibble; INT2: two's complement).  For tests and debugging ("Accelerating LLM
+ * INT4: nibble; INT2: two's complement; INT1: 2c - 1), or for FP4 / FP8 the raw e2m1 / e4m3
+ * code of every element (one per byte).  For tests and debugging ("Accelerating LLM
  * inference...", part 1, step 3: unpack each byte into two INT4 values). */
 wq_status wq_unpack(const uint8_t *Wq, int64_t N, int64_t K, wq_qconfig c, int8_t *q,
                     cudaStream_t stream);
@@ -130,9 +149,13 @@ wq_status wq_unpack(const uint8_t *Wq, int64_t N, int64_t K, wq_qconfig c, int8_
 wq_status act_quant_int8(const void *A, wq_dtype a_dt, int64_t M, int64_t K,
                          int8_t *Aq, float *a_scale, cudaStream_t stream);
 
-/* W4A16 (and W2A16):  C[m,n] = sum_k A[m,k] * (q[n,k] - z[n,g]) * s[n,g]  (+ bias[n]),
- * accumulated in binary32 and rounded once to a_dt.
- *   A      [M,K] a_dt in {WQ_F16, WQ_BF16};  C [M,N] a_dt;  bias [N] a_dt or NULL.
+/* W4A16 (and W2A16, W1A16, FP4 / FP8 weights):
+ *     C[m,n] = sum_k A[m,k] * (q[n,k] - z[n,g]) * s[n,g]  (+ bias[n]),
+ * with (q - z) the code's value for FP4 / FP8 and 2c - 1 for INT1, accumulated in binary32
+ * and rounded once to a_dt.
+ *   A      [M,K] a_dt in {WQ_F16, WQ_BF16} (INT4, INT2); WQ_F16 only for INT1, FP4 and FP8
+ *          (the pairs of the BitBLAS guide's list; WQ_ERR_UNSUPPORTED otherwise);
+ *          C [M,N] a_dt;  bias [N] a_dt or NULL.
  *   Wq, scales, zeros as written by wq_quantize_pack (zeros NULL unless asymmetric INT4).
  *   workspace: device scratch of at least wq_workspace_size(M,N,K,c) bytes, ZERO-FILLED
  *   once before its first use.  It holds split-K partial sums (overwritten by every call)
@@ -140,20 +163,24 @@ wq_status act_quant_int8(const void *A, wq_dtype a_dt, int64_t M, int64_t K,
  *   later calls of any shape without clearing.  A workspace that is NULL or too small is
  *   allowed: the call then uses a launch plan that needs none (possibly slower).  Calls
  *   that share one workspace must not overlap on the GPU.
- * Requires K % 128 == 0 for INT4 (K % 64 == 0 for INT2), M, N >= 1. */
+ * Requires K % 128 == 0 for INT4, FP4, FP8 and INT1 (K % 64 == 0 for INT2), M, N >= 1.
+ * Above 16 tokens INT1, FP4 and FP8 need K >= 512 (the tensor-core kernel's shortest K);
+ * shorter K gives WQ_ERR_UNSUPPORTED. */
 wq_status w4a16_gemm(const void *A, wq_dtype a_dt, const uint8_t *Wq, const void *scales,
                      const void *zeros, const void *bias, void *C,
                      int64_t M, int64_t N, int64_t K, wq_qconfig c,
                      void *workspace, size_t ws_bytes, cudaStream_t stream);
 
-/* W4A8 (and W2A8):
+/* W4A8 (and W2A8, W1A8):
  *   acc_g[m,n] = sum_{k in group g} Aq[m,k] * (q[n,k] - z[n,g])        exact INT32
  *   C[m,n]     = fp16( a_scale[m] * sum_g s[n,g] * acc_g[m,n]  (+ bias[n]) )
- * INT2 weights have a single group spanning K and a single binary32 scale.
+ * INT2 and INT1 weights have a single group spanning K and a single binary32 scale; FP4 and
+ * FP8 weights are not in this path (WQ_ERR_UNSUPPORTED).
  *   Aq [M,K] int8, a_scale [M] binary32 (from act_quant_int8); C [M,N] binary16;
  *   bias [N] binary16 or NULL; zeros (asymmetric INT4) must hold integers.
  *   acc_out: NULL, or int32 [M, N, G] receiving every acc_g (G = K/128 for INT4, which
- *   then requires group_size == 128; G = 1 for INT2), bit-exact with the CPU reference.
+ *   then requires group_size == 128; G = 1 for INT2 and INT1), bit-exact with the CPU
+ *   reference.
  *   workspace: as for w4a16_gemm. */
 wq_status w4a8_gemm(const int8_t *Aq, const float *a_scale, const uint8_t *Wq, const void *scales,
                     const void *zeros, const void *bias, void *C, int32_t *acc_out,

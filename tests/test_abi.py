@@ -129,3 +129,48 @@ def test_binding_refuses_cpu_tensors(lib):
     import torch
     with pytest.raises(ValueError):
         wq.act_quant_int8(torch.zeros(2, 128, dtype=torch.float16))
+
+
+def _fq(bits, fmt, gs=128):
+    return wq.QConfig(bits, gs, 1, 0, wq.LAYOUT_NT, fmt)
+
+
+def test_weight_format_checks(lib):
+    E2M1, E4M3, INT = wq.FMT_E2M1, wq.FMT_E4M3, wq.FMT_INT
+
+    def a16(qc, K=256, dt=wq.WQ_F16):
+        return lib.w4a16_gemm(FAKE, dt, FAKE, FAKE, None, None, FAKE, 1, 128, K, qc, None, 0, None)
+
+    assert a16(_fq(8, E2M1)) == wq.WQ_ERR_INVALID_ARG          # e2m1 codes are 4 bits
+    assert a16(_fq(4, E4M3)) == wq.WQ_ERR_INVALID_ARG          # e4m3 codes are 8 bits
+    assert a16(_fq(4, 5)) == wq.WQ_ERR_INVALID_ARG             # unknown format
+    assert a16(_fq(1, INT), K=64) == wq.WQ_ERR_INVALID_ARG     # INT1 K % 128
+    assert a16(_fq(4, E2M1, gs=64)) == wq.WQ_ERR_UNSUPPORTED    # groups are multiples of 128
+    # the pairs of the BitBLAS guide's list: FP16 only for FP4 / FP8 / INT1
+    for qc in (_fq(4, E2M1), _fq(8, E4M3), _fq(1, INT)):
+        assert a16(qc, dt=wq.WQ_BF16) == wq.WQ_ERR_UNSUPPORTED
+    # no INT8 path for FP4 / FP8 weights
+    for qc in (_fq(4, E2M1), _fq(8, E4M3)):
+        assert lib.w4a8_gemm(FAKE, FAKE, FAKE, FAKE, None, None, FAKE, None, 1, 128, 256, qc, None, 0, None) \
+            == wq.WQ_ERR_UNSUPPORTED
+        assert lib.w4a8_gemm_fused(FAKE, wq.WQ_F16, FAKE, FAKE, None, None, FAKE, FAKE, FAKE, None, 1, 128, 256, qc,
+                                   None, 0, None) == wq.WQ_ERR_UNSUPPORTED
+    nat = wq.QConfig(4, 128, 1, 0, wq.LAYOUT_NATIVE, E2M1)
+    assert a16(nat) == wq.WQ_ERR_UNSUPPORTED                    # the native layout is INT4 only
+    assert lib.wq_repack(FAKE, 4, 128, _fq(4, E2M1), FAKE, None) == wq.WQ_ERR_UNSUPPORTED
+    # quantization: binary weights need the scratch of the exact mean; FP groups of 128
+    assert lib.wq_quantize_pack(FAKE, wq.WQ_F32, 4, 128, _fq(1, INT), FAKE, FAKE, None, None, 0, None) \
+        == wq.WQ_ERR_WORKSPACE
+    assert lib.wq_quantize_pack(FAKE, wq.WQ_F32, 4, 256, _fq(4, E2M1, gs=64), FAKE, FAKE, None, None, 0, None) \
+        == wq.WQ_ERR_UNSUPPORTED
+    assert lib.wq_unpack(FAKE, 4, 128, _fq(4, E4M3), FAKE, None) == wq.WQ_ERR_INVALID_ARG
+    assert lib.wq_quantize_workspace_size(4, 128, _fq(1, INT)) >= 2048
+    assert lib.wq_quantize_workspace_size(4, 128, _fq(4, E2M1)) == 0
+    assert lib.wq_quantize_workspace_size(4, 128, _fq(8, E4M3)) == 0
+
+
+def test_quant_config_carries_the_format():
+    qc = wq.QuantConfig(bits=8, format=wq.FMT_E4M3).c()
+    assert (qc.bits, qc.format, qc.ternary) == (8, wq.FMT_E4M3, 0)
+    assert wq.QuantConfig(bits=1).per_tensor_scale and not wq.QuantConfig(bits=4, format=wq.FMT_E2M1).per_tensor_scale
+    assert ctypes.sizeof(wq.QConfig) == 24

@@ -1,0 +1,276 @@
+"""GPU parity of the other weight types against the CPU oracle: FP4 e2m1 and FP8 e4m3 weights
+with group scales (FP16 activations), INT1 binary weights with one scale per tensor (FP16 and
+INT8 activations) -- "BitBLAS practical guide: mixed-precision compute in vLLM", "Main
+features" (FP16 x FP8 / FP4 / INT1, INT8 x INT1).
+
+* quantization, packing and unpacking, and the INT8 x INT1 INT32 sums: bit-exact;
+* matmul outputs: the FP parity bar of the other GPU tests (relative Frobenius error <= 1e-3
+  and no element off by more than 4 units in the last place of the largest output);
+* an identity product with power-of-two scales, where every output is exact.
+
+Small cases run the oracle on every output (both kernels: up to 16 tokens and more, ragged
+N / M and, for INT1, a partial 512-k unit); full-size Llama-7B shapes compare sampled outputs.
+"""
+import numpy as np
+import pytest
+import torch
+
+import gemv_wq_quantize_b200 as wq
+import oracle
+import wq_synth
+
+pytestmark = pytest.mark.gpu
+
+TOL = 1e-3
+MAX_REL = 2.0 ** -9  # binary16 outputs
+
+KINDS = ["e2m1", "e4m3", "int1"]
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from gemv_wq_quantize_b200 import build
+    build.build(quiet=True)
+    wq.load_library()
+    oracle.build()
+    yield
+    torch.cuda.synchronize()
+    assert wq.device_error() == 0
+
+
+def bits_np(t: torch.Tensor) -> np.ndarray:
+    return t.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+def f16(bits):
+    return np.asarray(bits, dtype=np.uint16).view(np.float16).astype(np.float64)
+
+
+def assert_close(gpu_bits, ref_bits):
+    g, r = f16(gpu_bits), f16(ref_bits)
+    assert np.all(np.isfinite(g)), "non-finite output"
+    den = np.linalg.norm(r)
+    err = float(np.linalg.norm(g - r) / den) if den > 0 else float(np.linalg.norm(g))
+    assert err <= TOL, f"relative Frobenius error {err}"
+    top = np.abs(r).max()
+    mr = float(np.abs(g - r).max() / top) if top > 0 else float(np.abs(g).max())
+    assert mr <= MAX_REL, f"largest element error {mr} of max |C_ref|"
+
+
+def qc_of(kind, gs=128):
+    if kind == "e2m1":
+        return wq.QuantConfig(bits=4, group_size=gs, format=wq.FMT_E2M1)
+    if kind == "e4m3":
+        return wq.QuantConfig(bits=8, group_size=gs, format=wq.FMT_E4M3)
+    return wq.QuantConfig(bits=1)
+
+
+def ofmt(kind):
+    return {"e2m1": oracle.FMT_E2M1, "e4m3": oracle.FMT_E4M3, "int1": oracle.FMT_INT}[kind]
+
+
+def quantize_both(W, kind, gs=128):
+    """GPU quantization, asserted bit-exact against the oracle's; returns GPU and oracle tensors."""
+    qc = qc_of(kind, gs)
+    Wq, s, z = wq.quantize_pack(W.cuda(), qc)
+    torch.cuda.synchronize()
+    assert z is None
+    Wf = W.float().numpy()
+    if kind == "int1":
+        oWq, os_ = oracle.quantize_binary(Wf)
+        assert np.array_equal(s.cpu().numpy().view(np.uint32), os_.view(np.uint32))
+    else:
+        oWq, os_ = oracle.quantize_minifloat(Wf, gs, ofmt(kind))
+        assert np.array_equal(bits_np(s), os_)
+    assert np.array_equal(Wq.cpu().numpy(), oWq)
+    return qc, Wq, s, (oWq, os_)
+
+
+def ref_a16(A, oWq, os_, kind, N, K, gs=128, bias=None, m_idx=None, n_idx=None):
+    qc = qc_of(kind, gs)
+    _, ref = oracle.gemm_a16(bits_np(A), oracle.F16, oWq, N, K, qc.bits, True, gs, os_, None,
+                             None if bias is None else bits_np(bias), m_idx=m_idx, n_idx=n_idx, fmt=ofmt(kind))
+    return ref
+
+
+def workspace(M, N, K, qc):
+    return wq.make_workspace(wq.workspace_size(M, N, K, qc))
+
+
+# ------------------------------------------------------------------ quantizers
+@pytest.mark.parametrize("kind", KINDS)
+@pytest.mark.parametrize("N,K", [(1, 128), (37, 256), (300, 1024), (64, 640)])
+def test_quantize_pack_bit_exact(kind, N, K):
+    W = wq_synth.weights(N, K, seed=200 + N)
+    W[0, :128] = 0.0                     # a degenerate group: scale 0, codes 0
+    if N > 2:
+        W[1, 128:256] = -0.37            # a one-sided group
+        W[2, 3] = -1e-12                 # rounds to zero: code +0
+    quantize_both(W, kind)
+
+
+@pytest.mark.parametrize("kind", KINDS)
+@pytest.mark.parametrize("dtype", [torch.float16, torch.bfloat16])
+def test_quantize_from_half_inputs(kind, dtype):
+    quantize_both(wq_synth.weights(96, 512, seed=17).to(dtype), kind)
+
+
+@pytest.mark.parametrize("kind", ["e2m1", "e4m3"])
+def test_quantize_ties_to_even(kind):
+    # every group holds +-max * 2^j (so the scale is exactly 2^j) and the midpoints between
+    # neighbouring format values times 2^j: each quotient is an exact tie
+    top = 6.0 if kind == "e2m1" else 448.0
+    fmt = ofmt(kind)
+    ncode = 8 if kind == "e2m1" else 127
+    vals = np.array(sorted({abs(oracle.minifloat_value(fmt, c)) for c in range(ncode)}))
+    mids = (vals[1:] + vals[:-1]) / 2
+    row = np.concatenate([[top], mids, -mids])
+    row = np.resize(row, 128)
+    row[0] = top
+    W = np.stack([row * 2.0 ** -j for j in range(4, 12)]).astype(np.float32)
+    qc, Wq, s, (oWq, os_) = quantize_both(torch.from_numpy(W), kind)
+    # the reading: ties go to the code with the even last mantissa bit
+    codes = oracle.unpack(oWq, W.shape[0], 128, qc.bits, True, fmt).view(np.uint8)
+    assert np.all(codes[:, 1:1 + len(mids)] % 2 == 0)
+
+
+@pytest.mark.parametrize("kind", KINDS)
+def test_unpack_bit_exact(kind):
+    qc = qc_of(kind)
+    N, K = 50, 1024
+    Wq = wq_synth.uniform_bytes((N, K * qc.bits // 8), seed=19)
+    q = wq.unpack(Wq.cuda(), N, K, qc)
+    assert np.array_equal(q.cpu().numpy(), oracle.unpack(Wq.numpy(), N, K, qc.bits, True, ofmt(kind)))
+
+
+# ------------------------------------------------------------------ FP16 activations
+# up to 16 tokens: the few-token kernel (one and two token tiles); more: the tcgen05 kernel
+SMALL = [(1, 256, 512), (3, 200, 384), (8, 128, 128), (9, 130, 1024), (16, 384, 256),
+         (17, 256, 512), (64, 200, 640), (200, 136, 1024)]
+
+
+@pytest.mark.parametrize("kind", KINDS)
+@pytest.mark.parametrize("M,N,K", SMALL)
+def test_a16_small_all_outputs(kind, M, N, K):
+    W = wq_synth.weights(N, K, seed=M + N)
+    A = wq_synth.activations(M, K, seed=M + 1, outlier_frac=0.01)
+    qc, Wq, s, (oWq, os_) = quantize_both(W, kind)
+    C = wq.w4a16_gemm(A.cuda(), Wq, s, None, N, K, qc, workspace=workspace(M, N, K, qc))
+    torch.cuda.synchronize()
+    assert_close(bits_np(C), ref_a16(A, oWq, os_, kind, N, K))
+
+
+@pytest.mark.parametrize("kind", KINDS)
+@pytest.mark.parametrize("M", [5, 160])
+def test_a16_bias_ragged_and_groups(kind, M):
+    # ragged N, bias, groups of 256 k (FP4 / FP8), K not a whole number of 512-k INT1 units
+    N, K, gs = 333, 1280, 256 if kind != "int1" else 128
+    W = wq_synth.weights(N, K, seed=23)
+    A = wq_synth.activations(M, K, seed=24)
+    b = wq_synth.activations(1, N, seed=25)[0]
+    qc, Wq, s, (oWq, os_) = quantize_both(W, kind, gs)
+    C = wq.w4a16_gemm(A.cuda(), Wq, s, None, N, K, qc, bias=b.cuda(), workspace=workspace(M, N, K, qc))
+    torch.cuda.synchronize()
+    assert_close(bits_np(C), ref_a16(A, oWq, os_, kind, N, K, gs, bias=b))
+
+
+@pytest.mark.parametrize("use_ws", [True, False])
+@pytest.mark.parametrize("kind", KINDS)
+def test_a16_tensor_core_split_k(kind, use_ws):
+    # few 128 x 128 tiles: with a workspace K is split over CTAs; results equal either way
+    M, N, K = 128, 384, 4096
+    W = wq_synth.weights(N, K, seed=26)
+    A = wq_synth.activations(M, K, seed=27).cuda()
+    qc, Wq, s, (oWq, os_) = quantize_both(W, kind)
+    C = wq.w4a16_gemm(A, Wq, s, None, N, K, qc, workspace=workspace(M, N, K, qc) if use_ws else None)
+    torch.cuda.synchronize()
+    ni = np.arange(0, N, 3)
+    mi = np.arange(0, M, 5)
+    assert_close(bits_np(C)[np.ix_(mi, ni)], ref_a16(A.cpu(), oWq, os_, kind, N, K, m_idx=mi, n_idx=ni))
+
+
+@pytest.mark.parametrize("kind", ["e2m1", "e4m3"])
+@pytest.mark.parametrize("M", [4, 256])
+def test_a16_identity_closed_form(kind, M):
+    # A = I (rows of it): C[m, n] = value(code[n, m]) * scale, exact for power-of-two scales
+    fmt = ofmt(kind)
+    qc = qc_of(kind)
+    N, K = 256, 512
+    rng = np.random.default_rng(28)
+    ncode = 16 if kind == "e2m1" else 256
+    ok = [c for c in range(ncode) if np.isfinite(oracle.minifloat_value(fmt, c))]
+    codes = rng.choice(ok, (N, K))
+    sc = 2.0 ** rng.integers(-10, -4, (N, K // 128))
+    fields = codes.astype(np.uint8)
+    Wq = torch.from_numpy(oracle.pack(fields, qc.bits)).cuda()
+    s = torch.from_numpy(sc.astype(np.float16)).cuda()
+    A = torch.eye(K, dtype=torch.float16)[:M].contiguous().cuda()
+    C = wq.w4a16_gemm(A, Wq, s, None, N, K, qc, workspace=workspace(M, N, K, qc))
+    vals = np.vectorize(lambda c: oracle.minifloat_value(fmt, int(c)))(codes)
+    w = vals * np.repeat(sc, 128, axis=1)
+    assert np.array_equal(C.cpu().numpy().astype(np.float64), w.T[:M] + 0.0)
+
+
+@pytest.mark.parametrize("kind", KINDS)
+@pytest.mark.parametrize("M,N,K", [(1, 11008, 4096), (16, 4096, 11008), (512, 4096, 4096)])
+def test_a16_full_size_sampled(kind, M, N, K):
+    W = wq_synth.weights(N, K, seed=29)
+    A = wq_synth.activations(M, K, seed=30, outlier_frac=0.01)
+    qc, Wq, s, (oWq, os_) = quantize_both(W, kind)
+    C = wq.w4a16_gemm(A.cuda(), Wq, s, None, N, K, qc, workspace=workspace(M, N, K, qc))
+    torch.cuda.synchronize()
+    rng = np.random.default_rng(31)
+    mi = np.unique(np.concatenate([rng.choice(M, min(M, 24), replace=False), [M - 1]]))
+    ni = np.unique(np.concatenate([rng.choice(N, 192, replace=False), [0, N - 1]]))
+    assert_close(bits_np(C)[np.ix_(mi, ni)], ref_a16(A, oWq, os_, kind, N, K, m_idx=mi, n_idx=ni))
+
+
+# ------------------------------------------------------------------ INT8 x INT1
+@pytest.mark.parametrize("M,N,K", [(1, 256, 512), (5, 130, 1024), (16, 384, 256), (17, 256, 512),
+                                   (128, 384, 1024), (200, 136, 1152)])
+@pytest.mark.parametrize("want_acc", [True, False])
+def test_a8_int1_bit_exact_sums(M, N, K, want_acc):
+    W = wq_synth.weights(N, K, seed=M + 40)
+    A = wq_synth.activations(M, K, seed=M + 41, outlier_frac=0.01)
+    b = wq_synth.activations(1, N, seed=42)[0]
+    qc, Wq, s, (oWq, os_) = quantize_both(W, "int1")
+    Aq, asc = wq.act_quant_int8(A.cuda())
+    acc = torch.zeros(M, N, 1, dtype=torch.int32, device="cuda") if want_acc else None
+    C = wq.w4a8_gemm(Aq, asc, Wq, s, None, N, K, qc, bias=b.cuda(), acc_out=acc, workspace=workspace(M, N, K, qc))
+    torch.cuda.synchronize()
+    oAq, oasc = oracle.act_quant_int8(bits_np(A), oracle.F16)
+    assert np.array_equal(Aq.cpu().numpy(), oAq)
+    _, ref, oacc = oracle.gemm_a8(oAq, oasc, oWq, N, K, 1, True, 128, os_, None, bits_np(b), want_acc=True)
+    if want_acc:
+        assert np.array_equal(acc.cpu().numpy(), oacc)
+    assert_close(bits_np(C), ref)
+
+
+@pytest.mark.parametrize("M,K", [(1, 4096), (4, 3200), (12, 1024)])
+def test_a8_int1_fused_matches_two_step(M, K):
+    # the per-token quantization fused into the few-token kernel: identical outputs
+    N = 640
+    W = wq_synth.weights(N, K, seed=43)
+    A = wq_synth.activations(M, K, seed=44, outlier_frac=0.01).cuda()
+    qc, Wq, s, _ = quantize_both(W, "int1")
+    acc1 = torch.zeros(M, N, 1, dtype=torch.int32, device="cuda")
+    acc2 = torch.zeros_like(acc1)
+    C1, Aq1, sc1 = wq.w4a8_gemm_fused(A, Wq, s, None, N, K, qc, acc_out=acc1)
+    Aq2, sc2 = wq.act_quant_int8(A)
+    C2 = wq.w4a8_gemm(Aq2, sc2, Wq, s, None, N, K, qc, acc_out=acc2)
+    torch.cuda.synchronize()
+    assert torch.equal(Aq1, Aq2) and torch.equal(sc1, sc2)
+    assert torch.equal(acc1, acc2) and torch.equal(C1, C2)
+
+
+# ------------------------------------------------------------------ shapes without a plan
+def test_tensor_core_short_k_is_refused():
+    # more than 16 tokens with K below four 128-k blocks: no launch plan for these weights
+    N, K, M = 128, 256, 64
+    W = wq_synth.weights(N, K, seed=45)
+    qc, Wq, s, _ = quantize_both(W, "e4m3")
+    with pytest.raises(wq.WqError) as e:
+        wq.w4a16_gemm(torch.zeros(M, K, dtype=torch.float16, device="cuda"), Wq, s, None, N, K, qc)
+    assert e.value.status == wq.WQ_ERR_UNSUPPORTED

@@ -50,8 +50,9 @@ def uniform_bytes(shape, seed: int) -> torch.Tensor:
 # --------------------------------------------------------------------------
 # Workload shapes.  mode: "a16" (fp16/bf16 activations) or "a8" (int8 per-token
 # activations); quant: "sym4" (symmetric INT4, group scales), "asym4"
-# (INT4 with group scales and zero points) or "tern2" (ternary, 2-bit codes,
-# one scale per tensor).
+# (INT4 with group scales and zero points), "tern2" (ternary, 2-bit codes,
+# one scale per tensor), "int1" (binary, 1-bit codes, one scale per tensor),
+# "e2m1" (FP4 codes, group scales) or "e4m3" (FP8 codes, group scales).
 # --------------------------------------------------------------------------
 @dataclass(frozen=True)
 class Case:
@@ -81,6 +82,8 @@ class Workload:
 
 LLAMA7B_NK = ((4096, 4096), (11008, 4096), (4096, 11008))
 BITNET3B_NK = ((3200, 3200), (8640, 3200), (3200, 8640))
+# bits per weight of each quant kind
+QUANT_BITS = {"sym4": 4, "asym4": 4, "tern2": 2, "int1": 1, "e2m1": 4, "e4m3": 8}
 
 WORKLOADS = {
     "gemv-small": Workload(
@@ -108,4 +111,17 @@ WORKLOADS = {
         "M in {1,128}, (N,K) in {(3200,3200),(8640,3200),(3200,8640)}, fp16 and INT8 activations",
         tuple(Case(M, N, K, mode, "tern2")
               for mode in ("a16", "a8") for M in (1, 128) for (N, K) in BITNET3B_NK)),
+    "formats-decode": Workload(
+        "formats-decode",
+        "The other weight types at decode: FP16 x FP4 (e2m1, g128 scales), FP16 x FP8 (e4m3, g128 "
+        "scales) and FP16 x INT1 (binary, one scale) at M=1 on the Llama-7B shapes, and INT8 x INT1 "
+        "(M=1, N=K=4096); fp16 activations with 1% outlier channels x20",
+        tuple(Case(1, N, K, "a16", q, outlier_frac=0.01) for q in ("e2m1", "e4m3", "int1")
+              for (N, K) in LLAMA7B_NK) + (Case(1, 4096, 4096, "a8", "int1", outlier_frac=0.01),)),
+    "formats-prefill": Workload(
+        "formats-prefill",
+        "The other weight types at prefill: FP16 x FP4 (e2m1), FP16 x FP8 (e4m3) and FP16 x INT1 at "
+        "M=512, (N,K) in {(4096,4096),(11008,4096)}, and INT8 x INT1 at M=128, N=K=4096",
+        tuple(Case(512, N, K, "a16", q) for q in ("e2m1", "e4m3", "int1")
+              for (N, K) in ((4096, 4096), (11008, 4096))) + (Case(128, 4096, 4096, "a8", "int1"),)),
 }
