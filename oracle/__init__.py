@@ -87,6 +87,8 @@ def _L():
                                      vp, i64, vp, i64, vp, vp, i32]
         lib.orc_gemm_a8.argtypes = [vp, vp, i64, i64, vp, i64, i32, i32, i64, vp, vp, vp,
                                     vp, i64, vp, i64, vp, vp, vp, i32]
+        lib.orc_act_quant_e4m3.argtypes = [vp, i32, i64, i64, vp, vp]
+        lib.orc_gemm_f8.argtypes = [vp, vp, i64, i64, vp, i64, i64, vp, vp, vp, i64, vp, i64, vp, vp, i32]
         _lib = lib
     return _lib
 
@@ -272,3 +274,35 @@ def gemm_a8(Aq, a_scale, Wq, N, K, bits, symmetric, group_size, scales, zeros=No
                           threads or os.cpu_count() or 1)
     _check(rc, "gemm_a8")
     return Ce, Co, acc
+
+
+def act_quant_e4m3(A_bits, a_dtype: int = F16):
+    """FP8 activations per token: A uint16 bit patterns [M,K] (binary16 or bfloat16).
+    Returns (Aq uint8 e4m3 codes [M,K], a_scale float32 [M]) with a_scale = absmax / 448."""
+    A = np.ascontiguousarray(A_bits, dtype=np.uint16)
+    M, K = A.shape
+    Aq = np.zeros((M, K), dtype=np.uint8)
+    sc = np.zeros(M, dtype=np.float32)
+    _check(_L().orc_act_quant_e4m3(_p(A), a_dtype, M, K, _p(Aq), _p(sc)), "act_quant_e4m3")
+    return Aq, sc
+
+
+def gemm_f8(Aq, a_scale, Wq, N, K, group_size, scales, bias_bits=None, m_idx=None, n_idx=None, threads=None):
+    """W8A8 FP8: e4m3 codes Aq [M,K] and Wq [N,K], a_scale [M] binary32, scales binary16 [N,G].
+    Returns (C_exact float64 [m,n], C_out f16 bits [m,n])."""
+    Aq = np.ascontiguousarray(Aq, dtype=np.uint8)
+    a_scale = np.ascontiguousarray(a_scale, dtype=np.float32)
+    M = Aq.shape[0]
+    mi, mc = _idx(m_idx)
+    ni, nc = _idx(n_idx)
+    mc = mc if mi is not None else M
+    nc = nc if ni is not None else N
+    Ce = np.zeros((mc, nc), dtype=np.float64)
+    Co = np.zeros((mc, nc), dtype=np.uint16)
+    sc = np.ascontiguousarray(scales, dtype=np.uint16)
+    b = None if bias_bits is None else np.ascontiguousarray(bias_bits, dtype=np.uint16)
+    Wq = np.ascontiguousarray(Wq, dtype=np.uint8)
+    rc = _L().orc_gemm_f8(_p(Aq), _p(a_scale), M, K, _p(Wq), N, group_size, _p(sc), _p(b), _p(mi), mc, _p(ni), nc,
+                          _p(Ce), _p(Co), threads or os.cpu_count() or 1)
+    _check(rc, "gemm_f8")
+    return Ce, Co

@@ -67,6 +67,12 @@
  *   - INT1 = binary weights: one binary32 scale per tensor equal to mean |w|
  *     (as for ternary), code c = 1 when w >= 0 else 0, value (2c - 1) * scale;
  *     element 8j+i in bit i of byte j.
+ * The page's data-type table also lists FP8_E4M3 x FP8_E4M3 -> FP32 -> FP16: FP8
+ * activations with FP8 weights.  Reading: the activations are quantized per token
+ * like the INT8 ones, scale = absmax / 448 in binary32, code = e4m3 of a / scale
+ * (the weight rounding above); the products of code values are summed per weight
+ * group, times the group's weight scale, and the token's scale is applied last:
+ *     C[m,n] = fp16( a_scale[m] * sum_g s[n,g] * sum_{k in g} v(Aq[m,k]) v(Wq[n,k])  (+ bias) ).
  *
  * Build: gcc -O2 -std=c11 -ffp-contract=off -fno-fast-math -fPIC -shared -pthread
  * (IEEE binary32 / binary64 arithmetic on SSE, round to nearest even).
@@ -467,6 +473,26 @@ int orc_act_quant_int8(const uint16_t *A, int a_dt, int64_t M, int64_t K, int8_t
     return ORC_OK;
 }
 
+/* FP8 activations per token ([BB] data-type table, FP8_E4M3 x FP8_E4M3):
+ * a_scale[m] = absmax / 448 (binary32), Aq = e4m3 code of clip(a / a_scale, -448, 448). */
+int orc_act_quant_e4m3(const uint16_t *A, int a_dt, int64_t M, int64_t K, uint8_t *Aq, float *a_scale)
+{
+    if (a_dt != ORC_F16 && a_dt != ORC_BF16) return ORC_ERR_ARG;
+    for (int64_t m = 0; m < M; ++m) {
+        float amax = 0.0f;
+        for (int64_t k = 0; k < K; ++k) amax = fmaxf(amax, fabsf((float)act_value(A, a_dt, m * K + k)));
+        float sc = amax / 448.0f;
+        a_scale[m] = sc;
+        for (int64_t k = 0; k < K; ++k) {
+            int c = 0;
+            if (sc != 0.0f) c = orc_minifloat_encode(ORC_FMT_E4M3, (double)clampf((float)act_value(A, a_dt, m * K + k) / sc, -448.0f, 448.0f));
+            if (c < 0) return ORC_ERR_ARG;
+            Aq[m * K + k] = (uint8_t)c;
+        }
+    }
+    return ORC_OK;
+}
+
 /* ------------------------------------------------------------------------ */
 /* reference matmuls ([BB] "What is BitBLAS"; [CG] steps 3-4)                */
 /* ------------------------------------------------------------------------ */
@@ -570,6 +596,37 @@ static void *run_a8(void *arg)
     return NULL;
 }
 
+/* FP8 x FP8: per group, the sum of products of the code values (binary64), times the
+ * weight group scale; the token scale last. */
+static void *run_f8(void *arg)
+{
+    job_t *J = (job_t *)arg;
+    int64_t G = J->K / J->gs;
+    const uint8_t *Aq = (const uint8_t *)J->Aq;
+    double *w = (double *)malloc((size_t)J->K * sizeof(double));
+    if (!w) { J->status = ORC_ERR_ARG; return NULL; }
+    for (int64_t j = J->j0; j < J->j1; ++j) {
+        int64_t n = sel(J->n_idx, j);
+        for (int64_t k = 0; k < J->K; ++k) w[k] = orc_minifloat_value(ORC_FMT_E4M3, J->Wq[n * J->K + k]);
+        for (int64_t i = 0; i < J->m_cnt; ++i) {
+            int64_t m = sel(J->m_idx, i);
+            double total = 0.0;
+            for (int64_t g = 0; g < G; ++g) {
+                double acc = 0.0;
+                for (int64_t k = g * J->gs; k < (g + 1) * J->gs; ++k)
+                    acc += orc_minifloat_value(ORC_FMT_E4M3, Aq[m * J->K + k]) * w[k];
+                total += orc_f16_to_f64(J->scales16[n * G + g]) * acc;
+            }
+            double c = (double)J->a_scale[m] * total;
+            if (J->bias) c += orc_f16_to_f64(J->bias[n]);
+            if (J->C_exact) J->C_exact[i * J->n_cnt + j] = c;
+            if (J->C_out) J->C_out[i * J->n_cnt + j] = orc_f64_to_f16(c);
+        }
+    }
+    free(w);
+    return NULL;
+}
+
 static int run_threads(job_t *proto, void *(*fn)(void *), int threads)
 {
     if (threads < 1) threads = 1;
@@ -647,4 +704,25 @@ int orc_gemm_a8(const int8_t *Aq, const float *a_scale, int64_t M, int64_t K,
     J.n_idx = n_idx; J.n_cnt = n_idx ? n_cnt : N;
     J.C_exact = C_exact; J.C_out = C_out; J.acc_out = acc_out;
     return run_threads(&J, run_a8, threads);
+}
+
+/* W8A8 FP8 (e4m3 weights with binary16 group scales, e4m3 activations with per-token
+ * binary32 scales):
+ *   C[m,n] = fp16( a_scale[m] * sum_g s[n,g] * sum_{k in g} v(Aq[m,k]) * v(Wq[n,k])  (+ bias[n]) )
+ * summed in binary64.  Wq [N,K] and Aq [M,K] are e4m3 codes (bytes). */
+int orc_gemm_f8(const uint8_t *Aq, const float *a_scale, int64_t M, int64_t K,
+                const uint8_t *Wq, int64_t N, int64_t gs, const uint16_t *scales, const uint16_t *bias,
+                const int64_t *m_idx, int64_t m_cnt, const int64_t *n_idx, int64_t n_cnt,
+                double *C_exact, uint16_t *C_out, int threads)
+{
+    if (gs <= 0 || K % gs || M < 0 || N < 0) return ORC_ERR_ARG;
+    job_t J;
+    memset(&J, 0, sizeof J);
+    J.Aq = (const int8_t *)Aq; J.a_scale = a_scale; J.M = M; J.N = N; J.K = K;
+    J.Wq = Wq; J.bits = 8; J.fmt = ORC_FMT_E4M3; J.symmetric = 1; J.gs = gs;
+    J.scales16 = scales; J.bias = bias;
+    J.m_idx = m_idx; J.m_cnt = m_idx ? m_cnt : M;
+    J.n_idx = n_idx; J.n_cnt = n_idx ? n_cnt : N;
+    J.C_exact = C_exact; J.C_out = C_out;
+    return run_threads(&J, run_f8, threads);
 }

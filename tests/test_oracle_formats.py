@@ -263,3 +263,57 @@ def test_gemm_rejects_bad_format_pairs():
         oracle.gemm_a16(A, oracle.F16, Wq, 1, 128, 8, True, 128, s, fmt=E2M1)
     with pytest.raises(ValueError):
         oracle.gemm_a16(A, oracle.F16, Wq, 1, 128, 4, True, 128, s, fmt=E4M3)
+
+
+# ------------------------------------------------------------------ FP8 x FP8 (e4m3 activations)
+@pytest.mark.parametrize("dtype", [torch.float16, torch.bfloat16])
+def test_act_quant_e4m3_matches_recomputation(dtype):
+    A = wq_synth.activations(6, 1024, seed=50, dtype=dtype, outlier_frac=0.01)
+    A[2] = 0.0                              # all-zero token: scale 0, codes 0
+    A[3, 7] = -1e-7                         # rounds to zero: code +0
+    Aq, sc = oracle.act_quant_e4m3(a_bits(A), oracle.F16 if dtype == torch.float16 else oracle.BF16)
+    a = A.float().numpy()
+    amax = np.abs(a).max(axis=1).astype(np.float32)
+    want_sc = (amax / np.float32(448.0)).astype(np.float32)
+    assert np.array_equal(sc.view(np.uint32), want_sc.view(np.uint32))
+    with np.errstate(divide="ignore", invalid="ignore"):
+        x = np.where(want_sc[:, None] != 0, np.clip(a / want_sc[:, None], -448, 448), 0).astype(np.float32)
+    ref = torch.tensor(x).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    ref = np.where(ref == 0x80, 0, ref)
+    assert np.array_equal(Aq, ref)
+    assert np.all(Aq[2] == 0) and Aq[3, 7] == 0
+    # the token's largest magnitude is the code of +-448 (0x7E / 0xFE)
+    for m in (0, 1, 4, 5):
+        assert (Aq[m] & 0x7F).max() == 0x7E
+
+
+@pytest.mark.parametrize("M,N,K,gs", [(1, 3, 128, 128), (5, 8, 256, 128), (3, 4, 512, 256)])
+def test_gemm_f8_brute_force(M, N, K, gs):
+    W = wq_synth.weights(N, K, seed=51).numpy()
+    A = wq_synth.activations(M, K, seed=52, outlier_frac=0.01)
+    bias = wq_synth.activations(1, N, seed=53)[0]
+    Wq, s = oracle.quantize_minifloat(W, gs, E4M3)
+    Aq, asc = oracle.act_quant_e4m3(a_bits(A), oracle.F16)
+    Ce, Co = oracle.gemm_f8(Aq, asc, Wq, N, K, gs, s, a_bits(bias))
+    tab = e4m3_table()
+    av = tab[Aq] * asc.astype(np.float64)[:, None]
+    wv = tab[Wq] * np.repeat(f16_val(s), gs, axis=1)
+    ref = av @ wv.T + bias.double().numpy()
+    assert np.allclose(Ce, ref, rtol=1e-12, atol=1e-12)
+    assert np.array_equal(Co, Ce.astype(np.float16).view(np.uint16))
+
+
+def test_gemm_f8_constant_token_closed_form():
+    # a token of equal values quantizes to +-448 codes with scale |a| / 448, so
+    # C[m, n] = a * sum_k s[n, g(k)] * v(Wq[n, k]): the row sums of the dequantized weights
+    N, K, gs = 6, 256, 128
+    W = wq_synth.weights(N, K, seed=54).numpy()
+    Wq, s = oracle.quantize_minifloat(W, gs, E4M3)
+    A = torch.full((2, K), 0.75, dtype=torch.float16)
+    A[1] = -0.75
+    Aq, asc = oracle.act_quant_e4m3(a_bits(A), oracle.F16)
+    assert np.all(Aq[0] == 0x7E) and np.all(Aq[1] == 0xFE)
+    Ce, _ = oracle.gemm_f8(Aq, asc, Wq, N, K, gs, s)
+    wsum = (e4m3_table()[Wq] * np.repeat(f16_val(s), gs, axis=1)).sum(axis=1)
+    scale = float(np.float32(0.75) / np.float32(448.0)) * 448.0
+    assert np.allclose(Ce[0], scale * wsum, rtol=1e-12) and np.allclose(Ce[1], -scale * wsum, rtol=1e-12)
