@@ -75,6 +75,8 @@ def launches_per_call(c: wq_synth.Case, fused: bool = True) -> int:
     """Kernels one step launches for the case: the matmul, plus the per-token activation
     quantization on the INT8 paths, which for small activations (M <= 16, M*K <= 16384) runs
     inside the matmul kernel (w4a8_gemm_fused) and otherwise as a kernel of its own."""
+    if c.mode == "f8":
+        return 2  # act_quant_fp8, then w8a8_fp8_gemm
     if c.mode != "a8":
         return 1
     return 1 if (fused and c.M <= 16 and c.M * c.K <= 16384) else 2
@@ -223,7 +225,9 @@ class Prepared:
         self.A_host = A.pin_memory()
         if c.mode == "a8":
             self.Aq, self.a_scale = wq.act_quant_int8(self.A)
-        self.C = torch.empty(c.M, c.N, dtype=torch.float16 if c.mode == "a8" else c.a_dtype, device=device)
+        elif c.mode == "f8":
+            self.Aq, self.a_scale = wq.act_quant_fp8(self.A)
+        self.C = torch.empty(c.M, c.N, dtype=torch.float16 if c.mode in ("a8", "f8") else c.a_dtype, device=device)
         self.C_host = torch.empty(self.C.shape, dtype=self.C.dtype).pin_memory()
         self.ws = wq.make_workspace(wq.workspace_size(c.M, c.N, c.K, self.qc), device)
         self.i = 0
@@ -236,6 +240,10 @@ class Prepared:
         A, C = (self.A_slots[slot], self.C_slots[slot]) if e2e else (self.A, self.C)
         if c.mode == "a16":
             wq.w4a16_gemm(A, Wq, s, z, c.N, c.K, self.qc, out=C, workspace=self.ws)
+        elif c.mode == "f8":
+            # FP8 x FP8: the step quantizes the fp16 activations per token, then multiplies
+            wq.act_quant_fp8(A, out_q=self.Aq, out_scale=self.a_scale)
+            wq.w8a8_fp8_gemm(self.Aq, self.a_scale, Wq, s, c.N, c.K, self.qc, out=C, workspace=self.ws)
         elif self.fused:
             # the INT8 path starts from the fp16 activations: every step quantizes them per token,
             # inside the matmul where the few-token kernel allows it
@@ -412,8 +420,8 @@ def per_case_breakdown(preps, reps: int = 200):
         us = t0.elapsed_time(t1) * 1e3 / reps
         gbs = p.bytes / (us * 1e-6) / 1e9
         tf = flops(p.c) / (us * 1e-6) / 1e12
-        peak_tc = pk["bf16_tflops"] * (2.0 if p.c.mode == "a8" else 1.0)
-        peak_tc_s = pk["bf16_tflops_sustained"] * (2.0 if p.c.mode == "a8" else 1.0)
+        peak_tc = pk["bf16_tflops"] * (2.0 if p.c.mode in ("a8", "f8") else 1.0)
+        peak_tc_s = pk["bf16_tflops_sustained"] * (2.0 if p.c.mode in ("a8", "f8") else 1.0)
         t_roof = max(p.bytes / (pk["hbm_gbs"] * 1e9), flops(p.c) / (peak_tc * 1e12))
         out.append({"case": p.c.name, "us": round(us, 3), "GB/s": round(gbs, 1), "TFLOP/s": round(tf, 2),
                     "hbm_frac": round(gbs / pk["hbm_gbs"], 4), "tensor_frac": round(tf / peak_tc, 4),
@@ -664,6 +672,9 @@ def oracle_sample(wl, budget_s: float, threads: int):
                 adt = oracle.F16 if c.a_dtype == torch.float16 else oracle.BF16
                 oracle.gemm_a16(Abits, adt, Wq, rows, c.K, bits, sym, c.group_size, s, z, n_idx=ni, threads=threads,
                                 fmt=fmt)
+            elif c.mode == "f8":
+                Aq, asc = oracle.act_quant_e4m3(Abits, oracle.F16)
+                oracle.gemm_f8(Aq, asc, Wq, rows, c.K, c.group_size, s, n_idx=ni, threads=threads)
             else:
                 Aq, asc = oracle.act_quant_int8(Abits, oracle.F16)
                 oracle.gemm_a8(Aq, asc, Wq, rows, c.K, bits, sym, c.group_size, s, z, n_idx=ni, threads=threads)

@@ -29,7 +29,7 @@ WQ_F32, WQ_F16, WQ_BF16, WQ_I8, WQ_I32 = range(5)
 EXPORTED = ("wq_quantize_pack", "wq_quantize_workspace_size", "wq_unpack", "act_quant_int8", "w4a16_gemm",
             "w4a16_gemm_noalloc", "w4a8_gemm", "wq_workspace_size", "wq_status_string", "wq_last_error",
             "wq_graph_create", "wq_graph_set_io", "wq_graph_launch", "wq_graph_destroy", "w4a8_gemm_fused",
-            "wq_repack")
+            "wq_repack", "act_quant_fp8", "w8a8_fp8_gemm")
 
 
 class WqError(RuntimeError):
@@ -100,6 +100,10 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.wq_unpack.restype = st
     lib.act_quant_int8.argtypes = [vp, st, i64, i64, vp, vp, vp]
     lib.act_quant_int8.restype = st
+    lib.act_quant_fp8.argtypes = [vp, st, i64, i64, vp, vp, vp]
+    lib.act_quant_fp8.restype = st
+    lib.w8a8_fp8_gemm.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, i64, QConfig, vp, sz, vp]
+    lib.w8a8_fp8_gemm.restype = st
     lib.w4a16_gemm.argtypes = [vp, st, vp, vp, vp, vp, vp, i64, i64, i64, QConfig, vp, sz, vp]
     lib.w4a16_gemm.restype = st
     lib.w4a16_gemm_noalloc.argtypes = [vp, st, vp, vp, vp, vp, vp, i64, i64, i64, QConfig, vp]
@@ -217,6 +221,34 @@ def act_quant_int8(A: torch.Tensor, out_q=None, out_scale=None, stream=None):
     _check(load_library().act_quant_int8(_ptr(A), _DT[A.dtype], M, K, _ptr(Aq), _ptr(sc), _stream(stream)),
            "act_quant_int8")
     return Aq, sc
+
+
+def act_quant_fp8(A: torch.Tensor, out_q=None, out_scale=None, stream=None):
+    """Per-token FP8 quantization of A [M,K] fp16/bf16 -> (Aq e4m3 codes uint8 [M,K], a_scale fp32 [M])."""
+    _dev(A, "A")
+    M, K = A.shape
+    Aq = out_q if out_q is not None else torch.empty(M, K, dtype=torch.uint8, device=A.device)
+    sc = out_scale if out_scale is not None else torch.empty(M, dtype=torch.float32, device=A.device)
+    _dev(Aq, "out_q")
+    _dev(sc, "out_scale")
+    _check(load_library().act_quant_fp8(_ptr(A), _DT[A.dtype], M, K, _ptr(Aq), _ptr(sc), _stream(stream)),
+           "act_quant_fp8")
+    return Aq, sc
+
+
+def w8a8_fp8_gemm(Aq, a_scale, Wq, scales, N: int, K: int, qc: QuantConfig, bias=None, out=None, workspace=None,
+                  stream=None) -> torch.Tensor:
+    """C[M,N] = fp16(a_scale[m] * sum_g s[n,g] * sum_k v(Aq) v(Wq) (+ bias)): FP8 (e4m3) activations
+    and weights (qc: bits 8, format FMT_E4M3)."""
+    for t, n in ((Aq, "Aq"), (a_scale, "a_scale"), (Wq, "Wq"), (scales, "scales"), (bias, "bias"), (out, "out")):
+        _dev(t, n)
+    M = Aq.shape[0]
+    C = out if out is not None else torch.empty(M, N, dtype=torch.float16, device=Aq.device)
+    wsb = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    rc = load_library().w8a8_fp8_gemm(_ptr(Aq), _ptr(a_scale), _ptr(Wq), _ptr(scales), _ptr(bias), _ptr(C), M, N, K,
+                                      qc.c(), _ptr(workspace), wsb, _stream(stream))
+    _check(rc, "w8a8_fp8_gemm")
+    return C
 
 
 def w4a16_gemm(A, Wq, scales, zeros, N: int, K: int, qc: QuantConfig, bias=None, out=None, workspace=None,

@@ -214,9 +214,11 @@ wq_status check_weights(const uint8_t *Wq, const void *scales, const void *zeros
 }
 
 // The activation paths of each weight type: the pairs of the BitBLAS guide's list (FP16 x
-// FP8 / FP4 / INT4 / INT2 / INT1, INT8 x INT4 / INT2 / INT1), plus BF16 with INT4 / INT2.
+// FP8 / FP4 / INT4 / INT2 / INT1, INT8 x INT4 / INT2 / INT1, FP8 x FP8), plus BF16 with
+// INT4 / INT2.  am: 0 FP16, 1 BF16, 2 INT8, 3 FP8 (e4m3).
 wq_status check_pair(int wf, int am)
 {
+    if (am == 3 && wf != WF_E4M3) return fail(WQ_ERR_UNSUPPORTED, "FP8 activations take FP8 (e4m3) weights");
     if (am == 1 && wf != WF_I4 && wf != WF_I2)
         return fail(WQ_ERR_UNSUPPORTED, "BF16 activations take INT4 or INT2 weights");
     if (am == 2 && (wf == WF_E2M1 || wf == WF_E4M3))
@@ -341,4 +343,19 @@ extern "C" wq_status w4a8_gemm(const int8_t *Aq, const float *a_scale, const uin
         return fail(WQ_ERR_UNSUPPORTED, "acc_out needs group_size == 128");
     return dispatch(wf, 2, Aq, a_scale, Wq, scales, wf == WF_I4 && !c.symmetric ? zeros : nullptr, bias, C, acc_out,
                     M, N, K, c, workspace, ws_bytes, stream);
+}
+
+extern "C" wq_status w8a8_fp8_gemm(const uint8_t *Aq, const float *a_scale, const uint8_t *Wq, const void *scales,
+                                   const void *bias, void *C, int64_t M, int64_t N, int64_t K, wq_qconfig c,
+                                   void *workspace, size_t ws_bytes, cudaStream_t stream)
+{
+    wq_status rc = check_weights(Wq, scales, nullptr, M, N, K, c);
+    if (rc != WQ_OK) return rc;
+    rc = check_pair(wf_of(c), 3);
+    if (rc != WQ_OK) return rc;
+    if (!Aq || !a_scale || !C) return fail(WQ_ERR_INVALID_ARG, "Aq, a_scale and C must be non-null");
+    if (!aligned16(Aq) || !aligned16(C) || (bias && !aligned16(bias)) || (workspace && !aligned16(workspace)))
+        return fail(WQ_ERR_ALIGNMENT, "Aq, C, bias and workspace must be 16-byte aligned");
+    return dispatch(WF_E4M3, 3, Aq, a_scale, Wq, scales, nullptr, bias, C, nullptr, M, N, K, c, workspace, ws_bytes,
+                    stream);
 }

@@ -5,6 +5,7 @@
 // C[M,N] = A[M,K] x dequant(Wq[N,K])^T: "BitBLAS practical guide", "What is BitBLAS",
 // "Weight group quantization" and the FP16 x INT4 / INT2 and INT8 x INT4 / INT2 rows of its
 // data-type table.  FP16 / BF16 activations use kind::f16 MMAs with fp32 accumulation;
+// FP8 (e4m3) activations with FP8 weights use kind::f8f6f4 MMAs on the codes as they are;
 // per-token INT8 activations ("Accelerating LLM inference with CUDA Graph and INT4
 // quantization", part 1, steps 2-4) use kind::i8 MMAs whose int32 group sums are exact,
 // followed by the (a_scale x w_scale) epilogue.
@@ -60,7 +61,8 @@ constexpr int kDeqWarps = 8;   // unpack weights into TMEM (two per TMEM lane qu
 constexpr int kFoldWarps = 8;  // fold block accumulators into the totals, write C
 constexpr int kThreads = (2 + kDeqWarps + kFoldWarps) * 32;  // + warp 0 TMA, warp 1 MMA / TMEM
 constexpr int kActBox = kBT * 128;  // one box of activations: 128 rows x 128 B (64 k FP, 128 k INT8)
-__host__ __device__ constexpr int act_bytes(int AM) { return AM == 2 ? kActBox : 2 * kActBox; }
+// AM: 0 binary16, 1 bfloat16, 2 int8, 3 e4m3 activations (the last two one byte each)
+__host__ __device__ constexpr int act_bytes(int AM) { return AM >= 2 ? kActBox : 2 * kActBox; }
 // packed weights of a block: 16 KB FP8, 8 KB INT4 / FP4, 4 KB INT2, 2 KB INT1
 __host__ __device__ constexpr int w_bytes(int WF) { return kBW * kKB * wf_bits(WF) / 8; }
 __host__ __device__ constexpr int stage_bytes(int WF, int AM) { return act_bytes(AM) + w_bytes(WF); }
@@ -257,7 +259,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_w,
                    const TcParams p)
 {
-    constexpr bool BF16 = AM == 1, I8 = AM == 2;
+    constexpr bool BF16 = AM == 1, I8 = AM == 2, F8 = AM == 3, B8 = I8 || F8;
     constexpr bool GROUPED = wf_grouped(WF);
     constexpr int kActBytes = act_bytes(AM), kStageBytes = stage_bytes(WF, AM);
     // scale table entries: binary16 scale | zero point << 16 (INT4), the scale alone (FP4 / FP8)
@@ -362,7 +364,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         tma_load_2d(st + kActBytes, &tmap_w, kb * (kKB * wf_bits(WF) / 8), n0, &full[s]);
                     }
                     tma_load_2d(st, &tmap_a, kb * kKB, m0, &full[s]);
-                    if constexpr (!I8) tma_load_2d(st + kActBox, &tmap_a, kb * kKB + 64, m0, &full[s]);
+                    if constexpr (!B8) tma_load_2d(st + kActBox, &tmap_a, kb * kKB + 64, m0, &full[s]);
                 }
             }
             // nothing may land in shared memory after the CTA exits: wait for the last stages
@@ -372,7 +374,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
-            const uint32_t idesc = I8 ? tc::idesc_i8(kBW, kBT) : tc::idesc_f16(BF16, kBW, kBT);
+            const uint32_t idesc = I8 ? tc::idesc_i8(kBW, kBT) : F8 ? tc::idesc_f8(kBW, kBT) : tc::idesc_f16(BF16, kBW, kBT);
             uint64_t desc0[kNA];  // descriptor of each stage's activations (k step 0)
 #pragma unroll
             for (int b = 0; b < kNA; ++b) desc0[b] = tc::sdesc_sw128(smem_u32(ring + size_t(b) * kStageBytes));
@@ -393,6 +395,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                         for (int kk = 0; kk < kKB / 32; ++kk)  // k 32: 32 bytes per step
                             tc::mma_i8_ts(dcol, acol + kk * 8, d0 + uint64_t((kk * 32) >> 4), idesc, kk > 0 ? 1u : 0u);
+                    } else if constexpr (F8) {
+#pragma unroll
+                        for (int kk = 0; kk < kKB / 32; ++kk)  // k 32: 32 bytes per step
+                            tc::mma_f8_ts(dcol, acol + kk * 8, d0 + uint64_t((kk * 32) >> 4), idesc, kk > 0 ? 1u : 0u);
                     } else {
 #pragma unroll
                         for (int kk = 0; kk < kKB / 16; ++kk)  // k 16: 32 bytes per step
@@ -468,7 +474,24 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // full also tells that the MMAs of step - kNA (stage and A-buffer s) have completed
                 if (!tc_wait(&full[s], (step / kNA) & 1, abort)) break;
                 const uint8_t *wst = ring + size_t(s) * kStageBytes + kActBytes;
-                if constexpr (WF == WF_E2M1) {
+                if constexpr (F8) {
+                    // FP8 weights for e4m3 activations: this row's 64 code bytes of the k half
+                    // (128-byte rows, 128-byte swizzle), stored to Tensor Memory as they are
+                    static_assert(WF == WF_E4M3, "FP8 activations take FP8 weights");
+                    const uint8_t *wrow = wst + r * 128;
+                    const uint32_t sw = uint32_t(r & 7);
+                    uint32_t v[16];
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const uint4 c = lds128(wrow + ((uint32_t(4 * kh + i) ^ sw) << 4));
+                        v[4 * i + 0] = c.x;
+                        v[4 * i + 1] = c.y;
+                        v[4 * i + 2] = c.z;
+                        v[4 * i + 3] = c.w;
+                    }
+                    tc::fence_after_sync();
+                    tc::st_32x32b_x16(tlane + kAcol + s * 64 + kh * 16, v);
+                } else if constexpr (WF == WF_E2M1) {
                     // this row's 32 packed bytes of the k half (64-byte rows, 64-byte swizzle)
                     const uint8_t *wrow = wst + r * 64;
                     const uint32_t sw = uint32_t((r >> 1) & 3);
@@ -717,7 +740,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (mb + j >= p.M) continue;
                     if constexpr (ACC && wf_per_tensor(WF)) p.acc_out[(size_t)(mb + j) * p.N + n] = int(tot[j]);
                     float v;
-                    if constexpr (I8) v = p.a_scale[mb + j] * (wf_per_tensor(WF) ? ws * tot[j] : tot[j]);
+                    if constexpr (B8) v = p.a_scale[mb + j] * (wf_per_tensor(WF) ? ws * tot[j] : tot[j]);
                     else v = ws * tot[j];
                     store_out<BF16>(p.C, (long long)(mb + j) * p.N + n, v + b);
                 }
@@ -843,12 +866,12 @@ wq_status tc_gemm(int WF, int AM, const void *A, const float *a_scale, const uin
     if (wf_grouped(WF) && (K % kKB || c.group_size % kKB))
         return fail(WQ_ERR_UNSUPPORTED, "tc_gemm: group-scaled weights need K and group_size multiples of 128");
     if (WF == WF_I1 && K % kKB) return fail(WQ_ERR_UNSUPPORTED, "tc_gemm: INT1 needs K %% 128 == 0");
-    const int es = AM == 2 ? 1 : 2;
+    const int es = AM >= 2 ? 1 : 2;
     if ((K * es) % 16) return fail(WQ_ERR_UNSUPPORTED, "tc_gemm: activation rows must be 16-byte multiples");
     const DeviceInfo &dev = device_info();
     const int G = wf_grouped(WF) ? int(K / c.group_size) : 0;
     const int nkb = int((K + kKB - 1) / kKB);
-    const int stage = act_bytes(AM == 2 ? 2 : 0) + w_bytes(WF);
+    const int stage = act_bytes(AM >= 2 ? 2 : 0) + w_bytes(WF);
     const TcPlan pl = make_plan(nkb, G, stage, WF == WF_I4 ? 4 : 2, dev);
     if (!pl.ok) return fail(WQ_ERR_UNSUPPORTED, "tc_gemm: no shared-memory plan for K=%lld", (long long)K);
     CUtensorMap ta, tw;
@@ -908,8 +931,9 @@ wq_status tc_gemm(int WF, int AM, const void *A, const float *a_scale, const uin
     const int grid = std::min(dev.sm_count, p.NT * p.ks);
     if (WF == WF_E2M1) return AM == 0 ? launch<WF_E2M1, 0>(pl, ta, tw, p, grid, st)
                                       : fail(WQ_ERR_UNSUPPORTED, "tc_gemm: FP4 weights take FP16 activations");
-    if (WF == WF_E4M3) return AM == 0 ? launch<WF_E4M3, 0>(pl, ta, tw, p, grid, st)
-                                      : fail(WQ_ERR_UNSUPPORTED, "tc_gemm: FP8 weights take FP16 activations");
+    if (WF == WF_E4M3) return AM == 0   ? launch<WF_E4M3, 0>(pl, ta, tw, p, grid, st)
+                              : AM == 3 ? launch<WF_E4M3, 3>(pl, ta, tw, p, grid, st)
+                                        : fail(WQ_ERR_UNSUPPORTED, "tc_gemm: FP8 weights take FP16 or FP8 activations");
     if (WF == WF_I1) {
         if (AM == 0) return launch<WF_I1, 0>(pl, ta, tw, p, grid, st);
         if (AM == 1) return fail(WQ_ERR_UNSUPPORTED, "tc_gemm: INT1 weights take FP16 or INT8 activations");

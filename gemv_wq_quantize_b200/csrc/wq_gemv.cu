@@ -136,6 +136,8 @@ __device__ __forceinline__ float finish(const GemvParams &p, float total_f, int 
     float v;
     if constexpr (AM == A_I8) {
         v = wf_per_tensor(WF) ? as * (p.scale32[0] * float(total_i)) : as * total_f;
+    } else if constexpr (AM == A_F8) {
+        v = as * total_f;  // the token's FP8 scale times the group-scaled sums
     } else {
         v = wf_per_tensor(WF) ? p.scale32[0] * total_f : total_f;
     }
@@ -178,7 +180,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     constexpr int KU = kunit_of(WF);
     constexpr int QN = qn_of(WF, AM);
     constexpr bool GROUPED = wf_grouped(WF);
-    constexpr int ES = (AM == A_I8) ? 1 : 2;
+    constexpr int ES = byte_acts(AM) ? 1 : 2;
     constexpr int AU = KU * ES;  // activation bytes of one unit and token
     constexpr int WPU = wpu_of(NT, WIDE), KC = kc_of(NT, WIDE), TM = tm_of(NT, WIDE), NTL = ntl_of(NT, WIDE);
     using Tot = typename std::conditional<AM == A_I8 && wf_per_tensor(WF), int, float>::type;
@@ -553,7 +555,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 sf += v;
                 si += __float_as_int(v);
             }
-            const float as = (AM != A_I8) ? 1.f : (FS != 0 ? fsc[m] : p.a_scale[m]);
+            const float as = !byte_acts(AM) ? 1.f : (FS != 0 ? fsc[m] : p.a_scale[m]);
             store_out<AM>(p.C, (long long)m * p.N + n, finish<WF, AM>(p, sf, si, n, as));
             if constexpr (AM == A_I8 && wf_per_tensor(WF))
                 if (p.acc_out) p.acc_out[(long long)m * p.N + n] = si;
@@ -584,13 +586,13 @@ Plan make_plan(int64_t M, int64_t N, int64_t K, int WF, int AM, int G, const Dev
     pl.T = int((N + kTileRows - 1) / kTileRows);
     pl.P = std::min(dev.sm_count, pl.T);
     const int ntc_max = (pl.T + pl.P - 1) / pl.P;
-    pl.wide = (WF == WF_I4 && pl.NT == 2 && AM != A_I8 && ntc_max <= 2) ? 1 : 0;
+    pl.wide = (WF == WF_I4 && pl.NT == 2 && !byte_acts(AM) && ntc_max <= 2) ? 1 : 0;
     pl.KC = kc_of(pl.NT, pl.wide);
     pl.TPP = std::min(ntc_max, tm_of(pl.NT, pl.wide) * wpu_of(pl.NT, pl.wide));
     const int npass = (ntc_max + pl.TPP - 1) / pl.TPP;
     pl.nch = (pl.KB + pl.KC - 1) / pl.KC;
     const long long total = (long long)npass * pl.nch;
-    const int es = AM == A_I8 ? 1 : 2;
+    const int es = byte_acts(AM) ? 1 : 2;
     const int au = pl.KU * es;
     const int64_t row_bytes = K * wf_bits(WF) / 8;
     pl.w3d = (row_bytes % kPairBytes) == 0 ? 1 : 0;
@@ -693,7 +695,7 @@ wq_status gemv_prepare(int WF, int AM, const void *A, const float *a_scale, cons
         rc = encode_tmap(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, Wq, dims, strides, box, 128);
     }
     if (rc != WQ_OK) return rc;
-    const int es = AM == A_I8 ? 1 : 2;
+    const int es = byte_acts(AM) ? 1 : 2;
     ta = tw;  // unused when the activations are staged whole
     if (!pl.a_whole) {
         // (128 bytes, token, 128-byte block of K): one box = MB tokens x KC units
@@ -765,6 +767,8 @@ wq_status gemv_prepare(int WF, int AM, const void *A, const float *a_scale, cons
                     : (one ? kernel_for<2, A_I8, 1, false, false, 1>(pl, &func) : kernel_for<2, A_I8, 2, false, false, 1>(pl, &func));
     } else if (WF == WF_E2M1)
         rc = one ? kernel_for<WF_E2M1, A_F16, 1>(pl, &func) : kernel_for<WF_E2M1, A_F16, 2>(pl, &func);
+    else if (WF == WF_E4M3 && AM == A_F8)
+        rc = one ? kernel_for<WF_E4M3, A_F8, 1>(pl, &func) : kernel_for<WF_E4M3, A_F8, 2>(pl, &func);
     else if (WF == WF_E4M3)
         rc = one ? kernel_for<WF_E4M3, A_F16, 1>(pl, &func) : kernel_for<WF_E4M3, A_F16, 2>(pl, &func);
     else if (WF == WF_I1 && AM == A_F16)

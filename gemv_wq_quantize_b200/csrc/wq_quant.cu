@@ -367,8 +367,9 @@ __global__ void __launch_bounds__(256) unpack_native_kernel(const uint32_t *__re
     }
 }
 
-// One block per token row: absmax, a_scale = absmax / 127, codes.  8 elements per access.
-template <typename T>
+// One block per token row: absmax, a_scale = absmax / 127 (INT8 codes) or absmax / 448
+// (FP8 e4m3 codes, F8), codes.  8 elements per access.
+template <typename T, bool F8 = false>
 __global__ void __launch_bounds__(256) act_quant_kernel(const T *__restrict__ A, int64_t K, int8_t *__restrict__ Aq,
                                                         float *__restrict__ a_scale)
 {
@@ -396,7 +397,7 @@ __global__ void __launch_bounds__(256) act_quant_kernel(const T *__restrict__ A,
         if (threadIdx.x == 0) red[0] = v;
     }
     __syncthreads();
-    const float sc = __fdiv_rn(red[0], 127.0f);
+    const float sc = __fdiv_rn(red[0], F8 ? 448.0f : 127.0f);
     if (threadIdx.x == 0) a_scale[m] = sc;
     for (int64_t j = threadIdx.x; j < K8; j += blockDim.x) {
         uint4 raw = __ldg(reinterpret_cast<const uint4 *>(a) + j);
@@ -404,8 +405,14 @@ __global__ void __launch_bounds__(256) act_quant_kernel(const T *__restrict__ A,
         uint32_t w[2] = {0, 0};
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-            float q = sc != 0.f ? clampf(rintf(__fdiv_rn(to_f(e[i]), sc)), -127.f, 127.f) : 0.f;
-            w[i / 4] |= (uint32_t(int(q)) & 0xffu) << (8 * (i % 4));
+            uint32_t code;
+            if constexpr (F8) {
+                code = sc != 0.f ? minifloat_code<WQ_FMT_E4M3>(clampf(__fdiv_rn(to_f(e[i]), sc), -448.f, 448.f)) : 0u;
+            } else {
+                float q = sc != 0.f ? clampf(rintf(__fdiv_rn(to_f(e[i]), sc)), -127.f, 127.f) : 0.f;
+                code = uint32_t(int(q)) & 0xffu;
+            }
+            w[i / 4] |= code << (8 * (i % 4));
         }
         reinterpret_cast<uint2 *>(Aq + m * K)[j] = make_uint2(w[0], w[1]);
     }
@@ -544,8 +551,26 @@ extern "C" wq_status wq_repack(const uint8_t *Wq, int64_t N, int64_t K, wq_qconf
     return check_launch("repack_kernel");
 }
 
+namespace {
+wq_status act_quant_launch(bool f8, const void *A, wq_dtype a_dt, int64_t M, int64_t K, int8_t *Aq, float *a_scale,
+                           cudaStream_t stream);
+}
+
+extern "C" wq_status act_quant_fp8(const void *A, wq_dtype a_dt, int64_t M, int64_t K, uint8_t *Aq, float *a_scale,
+                                   cudaStream_t stream)
+{
+    return act_quant_launch(true, A, a_dt, M, K, reinterpret_cast<int8_t *>(Aq), a_scale, stream);
+}
+
 extern "C" wq_status act_quant_int8(const void *A, wq_dtype a_dt, int64_t M, int64_t K, int8_t *Aq, float *a_scale,
                                     cudaStream_t stream)
+{
+    return act_quant_launch(false, A, a_dt, M, K, Aq, a_scale, stream);
+}
+
+namespace {
+wq_status act_quant_launch(bool f8, const void *A, wq_dtype a_dt, int64_t M, int64_t K, int8_t *Aq, float *a_scale,
+                           cudaStream_t stream)
 {
     if (M <= 0 || K <= 0 || !A || !Aq || !a_scale) return fail(WQ_ERR_INVALID_ARG, "bad sizes or null pointer");
     if (a_dt != WQ_F16 && a_dt != WQ_BF16) return fail(WQ_ERR_INVALID_ARG, "a_dt must be WQ_F16 or WQ_BF16");
@@ -562,11 +587,17 @@ extern "C" wq_status act_quant_int8(const void *A, wq_dtype a_dt, int64_t M, int
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     cudaError_t e;
-    if (a_dt == WQ_F16)
+    if (a_dt == WQ_F16 && f8)
+        e = cudaLaunchKernelEx(&cfg, act_quant_kernel<__half, true>, static_cast<const __half *>(A), K, Aq, a_scale);
+    else if (a_dt == WQ_F16)
         e = cudaLaunchKernelEx(&cfg, act_quant_kernel<__half>, static_cast<const __half *>(A), K, Aq, a_scale);
+    else if (f8)
+        e = cudaLaunchKernelEx(&cfg, act_quant_kernel<__nv_bfloat16, true>, static_cast<const __nv_bfloat16 *>(A), K,
+                               Aq, a_scale);
     else
         e = cudaLaunchKernelEx(&cfg, act_quant_kernel<__nv_bfloat16>, static_cast<const __nv_bfloat16 *>(A), K, Aq,
                                a_scale);
     if (e != cudaSuccess) return fail(WQ_ERR_CUDA, "act_quant_kernel launch: %s", cudaGetErrorString(e));
     return check_launch("act_quant_kernel");
 }
+}  // namespace

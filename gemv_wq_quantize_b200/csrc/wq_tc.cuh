@@ -100,6 +100,16 @@ __device__ __forceinline__ void mma_i8_ts(uint32_t d_taddr, uint32_t a_taddr, ui
         : "memory");
 }
 
+__device__ __forceinline__ void mma_f8_ts(uint32_t d_taddr, uint32_t a_taddr, uint64_t b_desc, uint32_t idesc,
+                                          uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_taddr),
+        "r"(a_taddr), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
 // The mbarrier receives one arrival once all tcgen05 operations this thread issued before
 // have completed.
 __device__ __forceinline__ void commit(uint64_t *bar)
@@ -115,6 +125,13 @@ __host__ __device__ constexpr uint32_t idesc_f16(bool bf16, int M, int N)
 {
     return (1u << 4) | (uint32_t(bf16) << 7) | (uint32_t(bf16) << 10) | (uint32_t(N >> 3) << 17) |
            (uint32_t(M >> 4) << 24);
+}
+
+// Instruction descriptor of kind::f8f6f4 with fp32 accumulation (D format bits 4-5 = F32),
+// both operands e4m3 (A / B format bits 7-9 / 10-12 = 0) and K-major.
+__host__ __device__ constexpr uint32_t idesc_f8(int M, int N)
+{
+    return (1u << 4) | (uint32_t(N >> 3) << 17) | (uint32_t(M >> 4) << 24);
 }
 
 // Instruction descriptor of kind::i8 with int32 accumulation (D format bits 4-5 = S32),

@@ -27,12 +27,14 @@
 
 namespace wq {
 
-enum AMode { A_F16 = 0, A_BF16 = 1, A_I8 = 2 };
+// activations: binary16, bfloat16, int8 codes, or e4m3 codes (FP8, with FP8 weights only)
+enum AMode { A_F16 = 0, A_BF16 = 1, A_I8 = 2, A_F8 = 3 };
+__host__ __device__ constexpr bool byte_acts(int AM) { return AM == A_I8 || AM == A_F8; }
 
 // k of one unit (64 packed bytes of a row) for weight format WF
 __host__ __device__ constexpr int kunit_of(int WF) { return 512 / wf_bits(WF); }
 // mma k-steps per unit (k16 for f16/bf16, k32 for int8)
-__host__ __device__ constexpr int steps_of(int WF, int AM) { return AM == A_I8 ? kunit_of(WF) / 32 : kunit_of(WF) / 16; }
+__host__ __device__ constexpr int steps_of(int WF, int AM) { return byte_acts(AM) ? kunit_of(WF) / 32 : kunit_of(WF) / 16; }
 __host__ __device__ constexpr int qn_of(int WF, int AM) { return steps_of(WF, AM) / 2; }
 
 // B fragments of one unit for the n8 token tile `nt`: bf[q] holds {b0, b1} of k-steps 2q
@@ -60,7 +62,11 @@ __device__ __forceinline__ void build_bfrag(Addr addr, int M, int nt, int lane, 
 #pragma unroll
     for (int q = 0; q < QN; ++q) {
         uint4 r;
-        if constexpr (AM != A_I8 && WF == WF_E4M3) {
+        if constexpr (AM == A_F8) {
+            // e4m3 activations with e4m3 weights: k-steps 0 / 1 (k32) use bytes 16t + {0..7} / {8..15}
+            // as they lie (b0 = the first 4 of each 8, b1 = the next 4)
+            r = lds128(addr(m, 16 * t));
+        } else if constexpr (AM != A_I8 && WF == WF_E4M3) {
             // k-steps 2q, 2q+1 use halves 16t + 8q + {0..7} as the pairs (0,1),(2,3) / (4,5),(6,7)
             r = lds128(addr(m, (16 * t + 8 * q) * 2));
         } else if constexpr (AM != A_I8 && (WF == WF_I4 || WF == WF_E2M1)) {
@@ -134,7 +140,25 @@ __device__ __forceinline__ void unit_mma(const uint4 (&wa)[NTL], const uint4 (&w
                                          const uint4 (&bf)[NT][qn_of(WF, AM)], const uint32_t (&z_lo)[NTL],
                                          const uint32_t (&z_hi)[NTL], acc_t<AM> (&acc)[2][NTL][NT][4])
 {
-    if constexpr (AM == A_F16 && WF == WF_E2M1) {
+    if constexpr (AM == A_F8) {
+        static_assert(WF == WF_E4M3, "FP8 activations take FP8 weights");
+        // the weight bytes are the A fragments as they lie: k-step j uses words 2j, 2j + 1
+        // (k = 16t + 8j + 0..3 and 4..7) of rows g and g + 8
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+#pragma unroll
+            for (int l = 0; l < NTL; ++l) {
+                uint32_t a[4];
+                a[0] = j ? wa[l].z : wa[l].x;
+                a[1] = j ? wb[l].z : wb[l].x;
+                a[2] = j ? wa[l].w : wa[l].y;
+                a[3] = j ? wb[l].w : wb[l].y;
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt)
+                    mma_e4m3(acc[j][l][nt], a, j ? bf[nt][0].z : bf[nt][0].x, j ? bf[nt][0].w : bf[nt][0].y);
+            }
+        }
+    } else if constexpr (AM == A_F16 && WF == WF_E2M1) {
         // byte b of word j -> the exact binary16 pair (8j + 2b, 8j + 2b + 1); no zero point
 #pragma unroll
         for (int j = 0; j < 4; ++j) {

@@ -23,7 +23,8 @@
  * (BitBLAS guide, "Core advantages 2" FP16xINT2 and INT8xINT2, "Real-world case"
  * BitNet-b1.58).  The other weight types of the guide's "Main features" list:
  *   FP16 x FP4 (e2m1) and FP16 x FP8 (e4m3) with group scales (W4A16 path only), and
- *   FP16 x INT1 / INT8 x INT1 (binary weights, one scale per tensor; both paths).
+ *   FP16 x INT1 / INT8 x INT1 (binary weights, one scale per tensor; both paths), and the
+ *   table's FP8_E4M3 x FP8_E4M3 row (FP8 activations per token, FP8 weights; w8a8_fp8_gemm).
  *
  * Data formats (fixed):
  *   - all matrices row-major; A [M,K], W [N,K], C [M,N];
@@ -203,6 +204,28 @@ wq_status w4a8_gemm_fused(const void *A, wq_dtype a_dt, const uint8_t *Wq, const
                           const void *zeros, const void *bias, void *C, int8_t *Aq, float *a_scale,
                           int32_t *acc_out, int64_t M, int64_t N, int64_t K, wq_qconfig c,
                           void *workspace, size_t ws_bytes, cudaStream_t stream);
+
+/* Per-token FP8 (e4m3) activation quantization, for the FP8_E4M3 x FP8_E4M3 row of the
+ * BitBLAS guide's data-type table.  a_scale[m] = absmax_k|A[m,k]| / 448 (binary32 division);
+ * Aq[m,k] = the e4m3 code of clip(A[m,k] / a_scale[m], -448, 448) (binary32 quotient), rounded
+ * to the nearest e4m3 value, ties to the even last mantissa bit, +0 for a zero result; an
+ * all-zero token gives scale 0 and codes 0.
+ *   A [M,K] a_dt (WQ_F16 or WQ_BF16); Aq [M,K] e4m3 codes (bytes) and a_scale [M] binary32
+ *   written.  K % 8 == 0.  Bit-exact with the CPU reference. */
+wq_status act_quant_fp8(const void *A, wq_dtype a_dt, int64_t M, int64_t K, uint8_t *Aq, float *a_scale,
+                        cudaStream_t stream);
+
+/* W8A8 FP8 (the guide's FP8_E4M3 x FP8_E4M3 -> FP32 -> FP16 row):
+ *   C[m,n] = fp16( a_scale[m] * sum_g s[n,g] * sum_{k in g} v(Aq[m,k]) v(Wq[n,k])  (+ bias[n]) )
+ * with v the e4m3 value of a code; the products are exact and the sums are accumulated in
+ * binary32 (one per 128 k on the tensor cores, then scaled by s and added).
+ *   Aq [M,K] e4m3 codes and a_scale [M] binary32 (from act_quant_fp8); Wq [N,K] e4m3 codes
+ *   and scales binary16 [N, K/group_size] from wq_quantize_pack with c.format = WQ_FMT_E4M3,
+ *   c.bits = 8 (other weight types: WQ_ERR_UNSUPPORTED); C [M,N] binary16; bias [N] binary16
+ *   or NULL; workspace as for w4a16_gemm.  K % 128 == 0; above 16 tokens K >= 512. */
+wq_status w8a8_fp8_gemm(const uint8_t *Aq, const float *a_scale, const uint8_t *Wq, const void *scales,
+                        const void *bias, void *C, int64_t M, int64_t N, int64_t K, wq_qconfig c,
+                        void *workspace, size_t ws_bytes, cudaStream_t stream);
 
 /* Bytes of workspace that lets w4a16_gemm / w4a8_gemm use their split-K plans on the
  * current device. */

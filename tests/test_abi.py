@@ -174,3 +174,20 @@ def test_quant_config_carries_the_format():
     assert (qc.bits, qc.format, qc.ternary) == (8, wq.FMT_E4M3, 0)
     assert wq.QuantConfig(bits=1).per_tensor_scale and not wq.QuantConfig(bits=4, format=wq.FMT_E2M1).per_tensor_scale
     assert ctypes.sizeof(wq.QConfig) == 24
+
+
+def test_fp8_activation_checks(lib):
+    E4M3, E2M1 = wq.FMT_E4M3, wq.FMT_E2M1
+
+    def gemm(qc, Aq=FAKE, sc=FAKE, C=FAKE, K=256):
+        return lib.w8a8_fp8_gemm(Aq, sc, FAKE, FAKE, None, C, 1, 128, K, qc, None, 0, None)
+
+    assert gemm(_fq(4, E2M1)) == wq.WQ_ERR_UNSUPPORTED           # FP8 activations take FP8 weights
+    assert gemm(_fq(4, wq.FMT_INT)) == wq.WQ_ERR_UNSUPPORTED
+    assert gemm(_fq(8, E4M3), Aq=None) == wq.WQ_ERR_INVALID_ARG
+    assert gemm(_fq(8, E4M3), sc=None) == wq.WQ_ERR_INVALID_ARG
+    assert gemm(_fq(8, E4M3), C=FAKE_MIS) == wq.WQ_ERR_ALIGNMENT
+    assert gemm(_fq(8, E4M3), K=200) == wq.WQ_ERR_INVALID_ARG     # K % 128
+    assert lib.act_quant_fp8(FAKE, wq.WQ_F16, 1, 100, FAKE, FAKE, None) == wq.WQ_ERR_INVALID_ARG
+    assert lib.act_quant_fp8(FAKE, wq.WQ_I8, 1, 128, FAKE, FAKE, None) == wq.WQ_ERR_INVALID_ARG
+    assert lib.act_quant_fp8(FAKE_MIS, wq.WQ_F16, 1, 128, FAKE, FAKE, None) == wq.WQ_ERR_ALIGNMENT

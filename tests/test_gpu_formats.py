@@ -274,3 +274,90 @@ def test_tensor_core_short_k_is_refused():
     with pytest.raises(wq.WqError) as e:
         wq.w4a16_gemm(torch.zeros(M, K, dtype=torch.float16, device="cuda"), Wq, s, None, N, K, qc)
     assert e.value.status == wq.WQ_ERR_UNSUPPORTED
+
+
+# ------------------------------------------------------------------ FP8 x FP8 (W8A8 FP8)
+@pytest.mark.parametrize("dtype", [torch.float16, torch.bfloat16])
+@pytest.mark.parametrize("M,K", [(1, 128), (7, 4096), (16, 11008), (3, 8)])
+def test_act_quant_fp8_bit_exact(dtype, M, K):
+    A = wq_synth.activations(M, K, seed=60, dtype=dtype, outlier_frac=0.01)
+    if M > 2:
+        A[2] = 0
+    Aq, sc = wq.act_quant_fp8(A.cuda())
+    oAq, osc = oracle.act_quant_e4m3(bits_np(A), oracle.F16 if dtype == torch.float16 else oracle.BF16)
+    assert np.array_equal(Aq.cpu().numpy(), oAq)
+    assert np.array_equal(sc.cpu().numpy().view(np.uint32), osc.view(np.uint32))
+
+
+def test_act_quant_fp8_ties_to_even():
+    # tokens holding 448 * 2^-j (so the scale is exactly 2^-j) and the midpoints between
+    # neighbouring e4m3 values times 2^-j, all exact in binary16
+    vals = np.array(sorted({abs(oracle.minifloat_value(oracle.FMT_E4M3, c)) for c in range(127)}))
+    mids = (vals[1:] + vals[:-1]) / 2
+    rows = []
+    for j in range(2, 6):
+        r = np.concatenate([[448.0], mids[8:], -mids[8:]]) * 2.0 ** -j  # normal-range ties (exact in fp16)
+        rows.append(np.resize(r, 256))
+    A = torch.tensor(np.stack(rows), dtype=torch.float16)
+    Aq, sc = wq.act_quant_fp8(A.cuda())
+    oAq, osc = oracle.act_quant_e4m3(bits_np(A), oracle.F16)
+    assert np.array_equal(Aq.cpu().numpy(), oAq) and np.array_equal(sc.cpu().numpy(), osc)
+    n = len(mids) - 8
+    assert np.all(oAq[:, 1:1 + n] % 2 == 0)
+
+
+def run_f8(M, N, K, gs=128, bias=False, use_ws=True, seed=0):
+    W = wq_synth.weights(N, K, seed=seed)
+    A = wq_synth.activations(M, K, seed=seed + 1, outlier_frac=0.01)
+    b = wq_synth.activations(1, N, seed=seed + 2)[0] if bias else None
+    qc, Wq, s, (oWq, os_) = quantize_both(W, "e4m3", gs)
+    Aq, asc = wq.act_quant_fp8(A.cuda())
+    C = wq.w8a8_fp8_gemm(Aq, asc, Wq, s, N, K, qc, bias=None if b is None else b.cuda(),
+                         workspace=workspace(M, N, K, qc) if use_ws else None)
+    torch.cuda.synchronize()
+    oAq, oasc = oracle.act_quant_e4m3(bits_np(A), oracle.F16)
+    assert np.array_equal(Aq.cpu().numpy(), oAq)
+    return C, (oAq, oasc, oWq, os_), b
+
+
+@pytest.mark.parametrize("M,N,K", SMALL)
+def test_f8_small_all_outputs(M, N, K):
+    C, (oAq, oasc, oWq, os_), _ = run_f8(M, N, K, seed=M + N)
+    _, ref = oracle.gemm_f8(oAq, oasc, oWq, N, K, 128, os_)
+    assert_close(bits_np(C), ref)
+
+
+@pytest.mark.parametrize("M", [5, 160])
+def test_f8_bias_ragged_and_groups(M):
+    N, K, gs = 333, 1280, 256
+    C, (oAq, oasc, oWq, os_), b = run_f8(M, N, K, gs=gs, bias=True, seed=61)
+    _, ref = oracle.gemm_f8(oAq, oasc, oWq, N, K, gs, os_, bits_np(b))
+    assert_close(bits_np(C), ref)
+
+
+@pytest.mark.parametrize("use_ws", [True, False])
+def test_f8_tensor_core_split_k(use_ws):
+    M, N, K = 128, 384, 4096
+    C, (oAq, oasc, oWq, os_), _ = run_f8(M, N, K, use_ws=use_ws, seed=62)
+    ni, mi = np.arange(0, N, 3), np.arange(0, M, 5)
+    _, ref = oracle.gemm_f8(oAq, oasc, oWq, N, K, 128, os_, m_idx=mi, n_idx=ni)
+    assert_close(bits_np(C)[np.ix_(mi, ni)], ref)
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 11008, 4096), (16, 4096, 11008), (512, 4096, 4096)])
+def test_f8_full_size_sampled(M, N, K):
+    C, (oAq, oasc, oWq, os_), _ = run_f8(M, N, K, seed=63)
+    rng = np.random.default_rng(64)
+    mi = np.unique(np.concatenate([rng.choice(M, min(M, 24), replace=False), [M - 1]]))
+    ni = np.unique(np.concatenate([rng.choice(N, 192, replace=False), [0, N - 1]]))
+    _, ref = oracle.gemm_f8(oAq, oasc, oWq, N, K, 128, os_, m_idx=mi, n_idx=ni)
+    assert_close(bits_np(C)[np.ix_(mi, ni)], ref)
+
+
+def test_f8_rejects_other_weights():
+    N, K = 128, 256
+    qc, Wq, s, _ = quantize_both(wq_synth.weights(N, K, seed=65), "e2m1")
+    Aq, asc = wq.act_quant_fp8(torch.zeros(4, K, dtype=torch.float16, device="cuda"))
+    with pytest.raises(wq.WqError) as e:
+        wq.w8a8_fp8_gemm(Aq, asc, Wq, s, N, K, qc)
+    assert e.value.status == wq.WQ_ERR_UNSUPPORTED

@@ -48,8 +48,8 @@ def uniform_bytes(shape, seed: int) -> torch.Tensor:
 
 
 # --------------------------------------------------------------------------
-# Workload shapes.  mode: "a16" (fp16/bf16 activations) or "a8" (int8 per-token
-# activations); quant: "sym4" (symmetric INT4, group scales), "asym4"
+# Workload shapes.  mode: "a16" (fp16/bf16 activations), "a8" (int8 per-token
+# activations) or "f8" (FP8 e4m3 per-token activations, with "e4m3" weights); quant: "sym4" (symmetric INT4, group scales), "asym4"
 # (INT4 with group scales and zero points), "tern2" (ternary, 2-bit codes,
 # one scale per tensor), "int1" (binary, 1-bit codes, one scale per tensor),
 # "e2m1" (FP4 codes, group scales) or "e4m3" (FP8 codes, group scales).
@@ -69,7 +69,7 @@ class Case:
     @property
     def name(self) -> str:
         dt = {torch.float16: "f16", torch.bfloat16: "bf16"}[self.a_dtype]
-        a = "a8" if self.mode == "a8" else dt
+        a = self.mode if self.mode in ("a8", "f8") else dt
         return f"{self.quant}-{a}-M{self.M}-N{self.N}-K{self.K}"
 
 
@@ -115,13 +115,17 @@ WORKLOADS = {
         "formats-decode",
         "The other weight types at decode: FP16 x FP4 (e2m1, g128 scales), FP16 x FP8 (e4m3, g128 "
         "scales) and FP16 x INT1 (binary, one scale) at M=1 on the Llama-7B shapes, and INT8 x INT1 "
-        "(M=1, N=K=4096); fp16 activations with 1% outlier channels x20",
+        "(M=1, N=K=4096), FP8 x FP8 (e4m3 activations per token, M=1, N=4096 and 11008, K=4096); fp16 "
+        "activations with 1% outlier channels x20 (quantized inside the step on the INT8 / FP8 paths)",
         tuple(Case(1, N, K, "a16", q, outlier_frac=0.01) for q in ("e2m1", "e4m3", "int1")
-              for (N, K) in LLAMA7B_NK) + (Case(1, 4096, 4096, "a8", "int1", outlier_frac=0.01),)),
+              for (N, K) in LLAMA7B_NK) + (Case(1, 4096, 4096, "a8", "int1", outlier_frac=0.01),)
+        + tuple(Case(1, N, 4096, "f8", "e4m3", outlier_frac=0.01) for N in (4096, 11008))),
     "formats-prefill": Workload(
         "formats-prefill",
         "The other weight types at prefill: FP16 x FP4 (e2m1), FP16 x FP8 (e4m3) and FP16 x INT1 at "
-        "M=512, (N,K) in {(4096,4096),(11008,4096)}, and INT8 x INT1 at M=128, N=K=4096",
+        "M=512, (N,K) in {(4096,4096),(11008,4096)}, INT8 x INT1 at M=128, N=K=4096, and FP8 x FP8 "
+        "(e4m3 activations per token) at M=512 on the same two shapes",
         tuple(Case(512, N, K, "a16", q) for q in ("e2m1", "e4m3", "int1")
-              for (N, K) in ((4096, 4096), (11008, 4096))) + (Case(128, 4096, 4096, "a8", "int1"),)),
+              for (N, K) in ((4096, 4096), (11008, 4096))) + (Case(128, 4096, 4096, "a8", "int1"),)
+        + tuple(Case(512, N, 4096, "f8", "e4m3") for N in (4096, 11008))),
 }
