@@ -73,11 +73,10 @@ def flops(c: wq_synth.Case) -> int:
 
 def launches_per_call(c: wq_synth.Case, fused: bool = True) -> int:
     """Kernels one step launches for the case: the matmul, plus the per-token activation
-    quantization on the INT8 paths, which for small activations (M <= 16, M*K <= 16384) runs
-    inside the matmul kernel (w4a8_gemm_fused) and otherwise as a kernel of its own."""
-    if c.mode == "f8":
-        return 2  # act_quant_fp8, then w8a8_fp8_gemm
-    if c.mode != "a8":
+    quantization on the INT8 / FP8 paths, which for small activations (M <= 16, M*K <= 16384)
+    runs inside the matmul kernel (w4a8_gemm_fused, w8a8_fp8_gemm_fused) and otherwise as a
+    kernel of its own."""
+    if c.mode not in ("a8", "f8"):
         return 1
     return 1 if (fused and c.M <= 16 and c.M * c.K <= 16384) else 2
 
@@ -240,8 +239,12 @@ class Prepared:
         A, C = (self.A_slots[slot], self.C_slots[slot]) if e2e else (self.A, self.C)
         if c.mode == "a16":
             wq.w4a16_gemm(A, Wq, s, z, c.N, c.K, self.qc, out=C, workspace=self.ws)
+        elif c.mode == "f8" and self.fused:
+            # FP8 x FP8: the step quantizes the fp16 activations per token (inside the matmul for
+            # small activations), then multiplies
+            wq.w8a8_fp8_gemm_fused(A, Wq, s, c.N, c.K, self.qc, out=C, out_q=self.Aq, out_scale=self.a_scale,
+                                   workspace=self.ws)
         elif c.mode == "f8":
-            # FP8 x FP8: the step quantizes the fp16 activations per token, then multiplies
             wq.act_quant_fp8(A, out_q=self.Aq, out_scale=self.a_scale)
             wq.w8a8_fp8_gemm(self.Aq, self.a_scale, Wq, s, c.N, c.K, self.qc, out=C, workspace=self.ws)
         elif self.fused:
@@ -470,13 +473,13 @@ def measure_extra(name: str, device, steps: int, warmup: int, dist_on: bool) -> 
                            "frac": round(gbs / pk["hbm_gbs"], 4), "traffic": recorded_traffic(name),
                            "peak_source": pk["source"]}
     out["cases"] = cases
-    if any(p.c.mode == "a8" for p in preps):
+    if any(p.c.mode in ("a8", "f8") for p in preps):
         # the same INT8 cases with the activation quantization as a kernel of its own
         for p in preps:
             p.fused = False
         run_steps(preps, 1, False)
         torch.cuda.synchronize()
-        out["cases_two_launches"] = [c for c, p in zip(per_case_breakdown(preps), preps) if p.c.mode == "a8"]
+        out["cases_two_launches"] = [c for c, p in zip(per_case_breakdown(preps), preps) if p.c.mode in ("a8", "f8")]
     del preps
     torch.cuda.empty_cache()
     return out

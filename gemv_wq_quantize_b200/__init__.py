@@ -29,7 +29,7 @@ WQ_F32, WQ_F16, WQ_BF16, WQ_I8, WQ_I32 = range(5)
 EXPORTED = ("wq_quantize_pack", "wq_quantize_workspace_size", "wq_unpack", "act_quant_int8", "w4a16_gemm",
             "w4a16_gemm_noalloc", "w4a8_gemm", "wq_workspace_size", "wq_status_string", "wq_last_error",
             "wq_graph_create", "wq_graph_set_io", "wq_graph_launch", "wq_graph_destroy", "w4a8_gemm_fused",
-            "wq_repack", "act_quant_fp8", "w8a8_fp8_gemm")
+            "wq_repack", "act_quant_fp8", "w8a8_fp8_gemm", "w8a8_fp8_gemm_fused")
 
 
 class WqError(RuntimeError):
@@ -104,6 +104,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.act_quant_fp8.restype = st
     lib.w8a8_fp8_gemm.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, i64, QConfig, vp, sz, vp]
     lib.w8a8_fp8_gemm.restype = st
+    lib.w8a8_fp8_gemm_fused.argtypes = [vp, st, vp, vp, vp, vp, vp, vp, i64, i64, i64, QConfig, vp, sz, vp]
+    lib.w8a8_fp8_gemm_fused.restype = st
     lib.w4a16_gemm.argtypes = [vp, st, vp, vp, vp, vp, vp, i64, i64, i64, QConfig, vp, sz, vp]
     lib.w4a16_gemm.restype = st
     lib.w4a16_gemm_noalloc.argtypes = [vp, st, vp, vp, vp, vp, vp, i64, i64, i64, QConfig, vp]
@@ -249,6 +251,27 @@ def w8a8_fp8_gemm(Aq, a_scale, Wq, scales, N: int, K: int, qc: QuantConfig, bias
                                       qc.c(), _ptr(workspace), wsb, _stream(stream))
     _check(rc, "w8a8_fp8_gemm")
     return C
+
+
+def w8a8_fp8_gemm_fused(A, Wq, scales, N: int, K: int, qc: QuantConfig, bias=None, out=None, out_q=None,
+                        out_scale=None, workspace=None, stream=None):
+    """FP8 x FP8 from fp16/bf16 activations with the per-token FP8 quantization fused in.
+
+    Returns (C fp16 [M,N], Aq e4m3 codes uint8 [M,K], a_scale fp32 [M]); bit-identical to
+    ``act_quant_fp8`` followed by ``w8a8_fp8_gemm``."""
+    for t, n in ((A, "A"), (Wq, "Wq"), (scales, "scales"), (bias, "bias"), (out, "out"), (out_q, "out_q"),
+                 (out_scale, "out_scale")):
+        _dev(t, n)
+    M = A.shape[0]
+    C = out if out is not None else torch.empty(M, N, dtype=torch.float16, device=A.device)
+    Aq = out_q if out_q is not None else torch.empty(M, K, dtype=torch.uint8, device=A.device)
+    sc = out_scale if out_scale is not None else torch.empty(M, dtype=torch.float32, device=A.device)
+    wsb = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    rc = load_library().w8a8_fp8_gemm_fused(_ptr(A), _DT[A.dtype], _ptr(Wq), _ptr(scales), _ptr(bias), _ptr(C),
+                                            _ptr(Aq), _ptr(sc), M, N, K, qc.c(), _ptr(workspace), wsb,
+                                            _stream(stream))
+    _check(rc, "w8a8_fp8_gemm_fused")
+    return C, Aq, sc
 
 
 def w4a16_gemm(A, Wq, scales, zeros, N: int, K: int, qc: QuantConfig, bias=None, out=None, workspace=None,

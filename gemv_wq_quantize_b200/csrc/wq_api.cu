@@ -359,3 +359,32 @@ extern "C" wq_status w8a8_fp8_gemm(const uint8_t *Aq, const float *a_scale, cons
     return dispatch(WF_E4M3, 3, Aq, a_scale, Wq, scales, nullptr, bias, C, nullptr, M, N, K, c, workspace, ws_bytes,
                     stream);
 }
+
+// FP8 x FP8 from FP activations: the per-token FP8 quantization inside the few-token matmul
+// when the activations are small and its launch plan stages them whole (as for W4A8), else
+// act_quant_fp8 then w8a8_fp8_gemm.
+extern "C" wq_status w8a8_fp8_gemm_fused(const void *A, wq_dtype a_dt, const uint8_t *Wq, const void *scales,
+                                         const void *bias, void *C, uint8_t *Aq, float *a_scale, int64_t M, int64_t N,
+                                         int64_t K, wq_qconfig c, void *workspace, size_t ws_bytes,
+                                         cudaStream_t stream)
+{
+    wq_status rc = check_weights(Wq, scales, nullptr, M, N, K, c);
+    if (rc != WQ_OK) return rc;
+    rc = check_pair(wf_of(c), 3);
+    if (rc != WQ_OK) return rc;
+    if (a_dt != WQ_F16 && a_dt != WQ_BF16) return fail(WQ_ERR_INVALID_ARG, "a_dt must be WQ_F16 or WQ_BF16");
+    if (!A || !C || !Aq || !a_scale) return fail(WQ_ERR_INVALID_ARG, "A, C, Aq and a_scale must be non-null");
+    if (!aligned16(A) || !aligned16(Aq) || !aligned16(C) || (bias && !aligned16(bias)) ||
+        (workspace && !aligned16(workspace)))
+        return fail(WQ_ERR_ALIGNMENT, "A, Aq, C, bias and workspace must be 16-byte aligned");
+    if (M <= 16 && M * K <= kFusedMaxElems) {
+        const FusedActQuant fa{A, a_dt == WQ_BF16, reinterpret_cast<int8_t *>(Aq), a_scale};
+        PreparedLaunch L;
+        rc = gemv_prepare(WF_E4M3, 3, Aq, a_scale, Wq, scales, nullptr, bias, C, nullptr, M, N, K, c, &L, &fa);
+        if (rc == WQ_OK) return launch_prepared(L, stream, "gemv_kernel");
+        if (rc != WQ_ERR_UNSUPPORTED) return rc;
+    }
+    rc = act_quant_fp8(A, a_dt, M, K, Aq, a_scale, stream);
+    if (rc != WQ_OK) return rc;
+    return w8a8_fp8_gemm(Aq, a_scale, Wq, scales, bias, C, M, N, K, c, workspace, ws_bytes, stream);
+}

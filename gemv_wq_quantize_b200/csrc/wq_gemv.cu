@@ -168,15 +168,15 @@ __device__ __forceinline__ float src_at(const uint4 &raw, int i)
 }
 
 // ACC: also store every INT32 group sum into p.acc_out (W4A8 with group_size 128).
-// FS: 0, or the FP activations to quantize per token first (1: binary16, 2: bfloat16; INT8
-// mode and whole-K activation staging only): the "fused kernel" of the same page's section
+// FS: 0, or the FP activations to quantize per token first (1: binary16, 2: bfloat16; INT8 or
+// FP8 mode and whole-K activation staging only): the "fused kernel" of the same page's section
 // on combining the strategies, here the quantization done in the matmul's prologue.
 template <int WF, int AM, int NT, bool ACC, bool WIDE, int FS = 0>
 __global__ void __launch_bounds__(kThreads, 1)
     gemv_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_a,
                 const GemvParams p)
 {
-    static_assert(FS == 0 || AM == A_I8, "the fused quantization feeds the INT8 path");
+    static_assert(FS == 0 || byte_acts(AM), "the fused quantization feeds the INT8 / FP8 paths");
     constexpr int KU = kunit_of(WF);
     constexpr int QN = qn_of(WF, AM);
     constexpr bool GROUPED = wf_grouped(WF);
@@ -315,7 +315,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
             if (lane == 0) {
-                const float sc = __fdiv_rn(amax, 127.0f);
+                const float sc = __fdiv_rn(amax, AM == A_F8 ? 448.0f : 127.0f);
                 fsc[m] = sc;
                 fsc[16 + m] = sc != 0.f ? __frcp_rn(sc) : 0.f;
                 if (blockIdx.x == 0) p.a_scale_out[m] = sc;
@@ -328,7 +328,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             const float sc = fsc[m], rc = fsc[16 + m];
             uint32_t w[2] = {0u, 0u};
 #pragma unroll
-            for (int i = 0; i < 8; ++i) w[i >> 2] |= (uint32_t(quant_i8(src_at<FS>(raw, i), sc, rc)) & 0xffu) << (8 * (i & 3));
+            for (int i = 0; i < 8; ++i) {
+                uint32_t code;
+                if constexpr (AM == A_F8)  // the e4m3 code of clip(a / scale, -448, 448), as act_quant_fp8
+                    code = sc != 0.f ? minifloat_code<WQ_FMT_E4M3>(fminf(fmaxf(__fdiv_rn(src_at<FS>(raw, i), sc), -448.f), 448.f)) : 0u;
+                else
+                    code = uint32_t(quant_i8(src_at<FS>(raw, i), sc, rc)) & 0xffu;
+                w[i >> 2] |= code << (8 * (i & 3));
+            }
             *reinterpret_cast<uint2 *>(abuf + (size_t)m * p.a_pitch_b + 8 * j) = make_uint2(w[0], w[1]);
             if (int(e % gridDim.x) == blockIdx.x)
                 reinterpret_cast<uint2 *>(p.Aq_out + (size_t)m * p.K)[j] = make_uint2(w[0], w[1]);
@@ -674,7 +681,7 @@ wq_status gemv_prepare(int WF, int AM, const void *A, const float *a_scale, cons
     const int G = wf_grouped(WF) ? int(K / c.group_size) : 1;
     Plan pl = make_plan(M, N, K, WF, AM, G, dev);
     if (!pl.ok) return fail(WQ_ERR_UNSUPPORTED, "no few-token plan for M=%lld K=%lld", (long long)M, (long long)K);
-    if (fa && (AM != A_I8 || !pl.a_whole))
+    if (fa && (!byte_acts(AM) || !pl.a_whole))
         return fail(WQ_ERR_UNSUPPORTED, "the activations of M=%lld K=%lld are not staged whole", (long long)M,
                     (long long)K);
     CUtensorMap tw, ta;
@@ -753,7 +760,10 @@ wq_status gemv_prepare(int WF, int AM, const void *A, const float *a_scale, cons
         p.Aq_out = fa->Aq;
         p.a_scale_out = fa->a_scale;
         const bool bf = fa->bf16;
-        if (WF == WF_I1)
+        if (WF == WF_E4M3)
+            rc = bf ? (one ? kernel_for<WF_E4M3, A_F8, 1, false, false, 2>(pl, &func) : kernel_for<WF_E4M3, A_F8, 2, false, false, 2>(pl, &func))
+                    : (one ? kernel_for<WF_E4M3, A_F8, 1, false, false, 1>(pl, &func) : kernel_for<WF_E4M3, A_F8, 2, false, false, 1>(pl, &func));
+        else if (WF == WF_I1)
             rc = bf ? (one ? kernel_for<1, A_I8, 1, false, false, 2>(pl, &func) : kernel_for<1, A_I8, 2, false, false, 2>(pl, &func))
                     : (one ? kernel_for<1, A_I8, 1, false, false, 1>(pl, &func) : kernel_for<1, A_I8, 2, false, false, 1>(pl, &func));
         else if (WF == WF_I4 && acc_out)

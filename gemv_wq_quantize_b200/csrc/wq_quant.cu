@@ -125,37 +125,7 @@ __global__ void __launch_bounds__(256) quant_int4_kernel(const T *__restrict__ W
     }
 }
 
-// ---- FP4 e2m1 / FP8 e4m3 codes -----------------------------------------------
-// Nearest value of the format to x (|x| <= its largest finite value), ties to even, as a
-// code (sign | exponent | mantissa), +0 for a zero result.  Below the smallest normal the
-// value is a multiple of the subnormal step; above it x is scaled by an exact power of two so
-// that rintf rounds to the format's mantissa bits (a result of 2^(m+1) moves to the next
-// binade).
-template <int FMT>
-__device__ __forceinline__ uint32_t minifloat_code(float x)
-{
-    constexpr int MB = FMT == WQ_FMT_E2M1 ? 1 : 3;       // mantissa bits
-    constexpr int BIAS = FMT == WQ_FMT_E2M1 ? 1 : 7;
-    constexpr float kMinNormal = FMT == WQ_FMT_E2M1 ? 1.0f : 0x1p-6f;
-    constexpr float kSubStep = FMT == WQ_FMT_E2M1 ? 0.5f : 0x1p-9f;
-    const float a = fabsf(x);
-    uint32_t code;
-    if (a < kMinNormal) {
-        code = uint32_t(rintf(__fdiv_rn(a, kSubStep)));  // a power of two: exact; 2^MB is the smallest normal
-    } else {
-        int e = int((__float_as_uint(a) >> 23) & 0xffu) - 127;                   // floor(log2 a)
-        const float scaled = __fmul_rn(a, __uint_as_float(uint32_t(127 + MB - e) << 23));  // in [2^MB, 2^(MB+1))
-        uint32_t q = uint32_t(rintf(scaled));
-        if (q == (2u << MB)) {
-            q = 1u << MB;
-            ++e;
-        }
-        code = (uint32_t(e + BIAS) << MB) | (q - (1u << MB));
-    }
-    if (code != 0u && x < 0.f) code |= FMT == WQ_FMT_E2M1 ? 0x8u : 0x80u;
-    return code;
-}
-
+// ---- FP4 e2m1 / FP8 e4m3 codes (minifloat_code, wq_format.h) ------------------
 // One warp per (row n, group g), lane l on elements c*128 + 4l .. +3 of each 128-chunk c:
 // scale = fp16(absmax / 6 or 448), codes of clip(w / scale, -max, max).
 template <typename T, int FMT>

@@ -227,6 +227,15 @@ wq_status w8a8_fp8_gemm(const uint8_t *Aq, const float *a_scale, const uint8_t *
                         const void *bias, void *C, int64_t M, int64_t N, int64_t K, wq_qconfig c,
                         void *workspace, size_t ws_bytes, cudaStream_t stream);
 
+/* W8A8 FP8 from FP16 / BF16 activations, with the per-token FP8 quantization fused into the
+ * matmul (as w4a8_gemm_fused for INT8).  Results are bit-identical to act_quant_fp8 followed by
+ * w8a8_fp8_gemm; Aq and a_scale are required outputs, written with the values act_quant_fp8
+ * writes.  When M <= 16, M * K <= 16384 and the few-token kernel stages the activations whole,
+ * this is ONE launch; otherwise it enqueues the two calls. */
+wq_status w8a8_fp8_gemm_fused(const void *A, wq_dtype a_dt, const uint8_t *Wq, const void *scales,
+                              const void *bias, void *C, uint8_t *Aq, float *a_scale, int64_t M, int64_t N,
+                              int64_t K, wq_qconfig c, void *workspace, size_t ws_bytes, cudaStream_t stream);
+
 /* Bytes of workspace that lets w4a16_gemm / w4a8_gemm use their split-K plans on the
  * current device. */
 size_t wq_workspace_size(int64_t M, int64_t N, int64_t K, wq_qconfig c);

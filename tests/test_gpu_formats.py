@@ -361,3 +361,18 @@ def test_f8_rejects_other_weights():
     with pytest.raises(wq.WqError) as e:
         wq.w8a8_fp8_gemm(Aq, asc, Wq, s, N, K, qc)
     assert e.value.status == wq.WQ_ERR_UNSUPPORTED
+
+
+@pytest.mark.parametrize("dtype", [torch.float16, torch.bfloat16])
+@pytest.mark.parametrize("M,K", [(1, 4096), (4, 3200 // 128 * 128), (12, 1024), (16, 11008)])
+def test_f8_fused_matches_two_step(dtype, M, K):
+    # one launch for small activations (the quantization in the few-token kernel's prologue),
+    # two otherwise: identical outputs either way
+    N = 640
+    qc, Wq, s, _ = quantize_both(wq_synth.weights(N, K, seed=66), "e4m3")
+    A = wq_synth.activations(M, K, seed=67, dtype=dtype, outlier_frac=0.01).cuda()
+    C1, Aq1, sc1 = wq.w8a8_fp8_gemm_fused(A, Wq, s, N, K, qc)
+    Aq2, sc2 = wq.act_quant_fp8(A)
+    C2 = wq.w8a8_fp8_gemm(Aq2, sc2, Wq, s, N, K, qc)
+    torch.cuda.synchronize()
+    assert torch.equal(Aq1, Aq2) and torch.equal(sc1, sc2) and torch.equal(C1, C2)
