@@ -120,3 +120,26 @@ def test_graph_rejects_many_token_ops():
         wq.DecodeGraph([{"A": A, "Wq": Wq, "scales": s, "N": 256, "K": 512, "qc": qc,
                          "out": torch.empty(32, 256, dtype=torch.float16, device="cuda")}])
     assert ei.value.status == wq.WQ_ERR_UNSUPPORTED
+
+
+@pytest.mark.parametrize("M", [1, 9])
+def test_graph_with_other_weight_types(M):
+    # FP4, FP8 and INT1 matmuls in one graph (fp16 activations): every output bit-identical to
+    # the same w4a16_gemm call
+    kinds = [wq.QuantConfig(bits=4, group_size=128, format=wq.FMT_E2M1),
+             wq.QuantConfig(bits=8, group_size=128, format=wq.FMT_E4M3), wq.QuantConfig(bits=1)]
+    ops = []
+    for i, qc in enumerate(kinds):
+        N, K = 1024 + 256 * i, 2048
+        Wq, s, _ = wq.quantize_pack(wq_synth.weights(N, K, seed=70 + i).cuda(), qc)
+        A = wq_synth.activations(M, K, seed=80 + i, outlier_frac=0.01).cuda()
+        ops.append({"A": A, "Wq": Wq, "scales": s, "zeros": None, "N": N, "K": K, "qc": qc,
+                    "out": torch.empty(M, N, dtype=torch.float16, device="cuda")})
+    g = wq.DecodeGraph(ops)
+    g.launch()
+    torch.cuda.synchronize()
+    for op in ops:
+        ref = wq.w4a16_gemm(op["A"], op["Wq"], op["scales"], None, op["N"], op["K"], op["qc"])
+        torch.cuda.synchronize()
+        assert torch.equal(op["out"].view(torch.int16), ref.view(torch.int16))
+    g.close()
