@@ -15,7 +15,7 @@ namespace wq {
 constexpr uint32_t kMaxPolls = 256;
 
 // Error codes recorded in the per-translation-unit device error word.
-enum : int { kErrNone = 0, kErrWaitTimeout = 1 };
+enum : int { kErrNone = 0, kErrWaitTimeout = 1, kErrBadLaunch = 2 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p)
 {
@@ -101,6 +101,64 @@ __device__ __forceinline__ bool mbar_test_wait(uint64_t *bar, uint32_t parity)
         : "memory");
     return ok != 0;
 }
+
+// ---- thread-block clusters: rank, distributed shared memory, cluster-scope barriers
+__device__ __forceinline__ uint32_t cluster_rank()
+{
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+__device__ __forceinline__ uint32_t cluster_size()
+{
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(r));
+    return r;
+}
+// The address of shared-memory location `local` (this CTA's) in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t dsmem_addr(uint32_t local, uint32_t rank)
+{
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local), "r"(rank));
+    return r;
+}
+__device__ __forceinline__ float ld_dsmem_f32(uint32_t addr)
+{
+    float v;
+    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
+    return v;
+}
+// One arrival on an mbarrier of a CTA of the cluster (address from dsmem_addr), releasing
+// this thread's earlier writes at cluster scope.
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar_addr)
+{
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar_addr) : "memory");
+}
+// The same without ordering this thread's earlier memory accesses (for a signal whose
+// meaning is only that values already loaded and used are no longer needed).
+__device__ __forceinline__ void mbar_arrive_cluster_relaxed(uint32_t bar_addr)
+{
+    asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar_addr) : "memory");
+}
+// try_wait that acquires at cluster scope what the arriving CTAs released.
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t *bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+__device__ __forceinline__ void fence_acq_rel_cluster() { asm volatile("fence.acq_rel.cluster;" ::: "memory"); }
+// The cluster-wide barrier in its two halves: every thread of every CTA of the cluster
+// arrives once (all threads of a warp together); a thread that waits is released once all
+// have arrived.  A thread need not wait.
+__device__ __forceinline__ void cluster_arrive() { asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory"); }
+__device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory"); }
 
 // Bounded wait for the phase with the given parity to complete.  Returns false
 // (after recording kErrWaitTimeout in *err) if it did not complete in time.
@@ -317,6 +375,21 @@ __device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t w)
     else
         asm("{\n.reg .b16 lo, hi;\nmov.b32 {lo, hi}, %1;\ncvt.rn.f16x2.e4m3x2 %0, hi;\n}" : "=r"(d) : "r"(w));
     return d;
+}
+
+// Per-token INT8 code of one activation, exactly clip(rint(a / s), -127, 127) with the IEEE
+// binary32 quotient ("Accelerating LLM inference with CUDA Graph and INT4 quantization",
+// part 1, step 2), without a division per element: y = a * r with r the correctly rounded
+// 1/s is within |a/s| * 2^-23 <= 1.6e-5 of a/s, and the correctly rounded quotient within
+// 2^-18 of it, so both round to the same integer unless a/s lies within 2^-12 of a tie
+// (k + 1/2); only there is the quotient formed by division.
+__device__ __forceinline__ int quant_i8(float a, float s, float r)
+{
+    if (s == 0.f) return 0;
+    const float y = a * r;
+    float k = rintf(y);
+    if (fabsf(fabsf(y - k) - 0.5f) < 0x1p-12f) k = rintf(__fdiv_rn(a, s));
+    return int(fminf(fmaxf(k, -127.f), 127.f));
 }
 
 __device__ __forceinline__ uint4 lds128(const void *p)

@@ -31,8 +31,9 @@
 // activation); the only rounding besides fp32 accumulation (int32 for INT8) is the
 // final conversion.  Persistent CTAs walk the (weight tile, token tile) grid token-tile
 // fastest so that concurrent CTAs share weight tiles in L2.  With fewer tiles than SMs, K is
-// split over CTAs: each slice's fp32 partials go to the workspace, and the tile's last CTA
-// to arrive bulk-copies them into its (by then idle) ring and adds them in slice order.
+// split over the CTAs of a thread-block cluster, one per slice: each keeps its fp32 partials
+// in its (by then idle) ring, and after a cluster handshake each adds up its share of the
+// tile's tokens from all slices' rings (distributed shared memory) in slice order.
 // Long K (many scale groups) builds the scale tables from global memory, and keeps a single
 // table if shared memory requires it.  Every wait is bounded; on expiry the CTA records an
 // error, stops, waits for what it has in flight and frees its Tensor Memory.
@@ -78,9 +79,8 @@ struct TcParams {
     const float *a_scale;  // INT8 activations: per-token scale
     const float *scale32;  // INT2 / INT1 weights: per-tensor scale
     int nkb;     // blocks of 128 k
-    int ks;      // K slices per tile (split-K when tiles are fewer than SMs)
-    float *ws_part;     // ks > 1: fp32 partial totals [tile][slice][128 tokens][128 rows]
-    unsigned *ws_cnt;   // ks > 1: per-tile arrival counters (left at zero)
+    int ks;      // K slices per tile (split-K when tiles are fewer than SMs): the CTAs of one
+                 // tile form a cluster of ks, cluster rank = slice
     int TT, NT;  // token tiles, tiles
     int S;       // ring stages
     int scst_off, tab_off, bar_off;
@@ -119,6 +119,21 @@ __device__ __forceinline__ bool tc_wait(uint64_t *bar, uint32_t parity, volatile
     }
 }
 
+// The same for a barrier that other CTAs of the cluster arrive on (cluster-scope acquire).
+__device__ __forceinline__ bool tc_wait_cluster(uint64_t *bar, uint32_t parity, volatile int *abort)
+{
+    const uint64_t t0 = globaltimer();
+    for (;;) {
+        for (int i = 0; i < 4; ++i)
+            if (mbar_try_wait_cluster(bar, parity)) return true;
+        if (*abort) return false;
+        if (globaltimer() - t0 > 2000000000ull) {
+            atomicCAS(&g_tc_error, kErrNone, kErrWaitTimeout);
+            *abort = 1;
+            return false;
+        }
+    }
+}
 
 template <bool BF16>
 __device__ __forceinline__ void store_out(void *C, long long idx, float v)
@@ -262,6 +277,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     constexpr bool BF16 = AM == 1, I8 = AM == 2, F8 = AM == 3, B8 = I8 || F8;
     constexpr bool GROUPED = wf_grouped(WF);
     constexpr int kActBytes = act_bytes(AM), kStageBytes = stage_bytes(WF, AM);
+    static_assert(kBW * kBT * 4 <= kNA * kStageBytes, "split-K totals must fit in the ring");
     // scale table entries: binary16 scale | zero point << 16 (INT4), the scale alone (FP4 / FP8)
     using TabT = typename std::conditional<WF == WF_I4, uint32_t, uint16_t>::type;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -275,10 +291,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint64_t *full = bars, *rel = bars + kNA;
     uint64_t *afull = bars + 2 * kNA, *dfree = afull + kNA;
     uint64_t *scbar = dfree + kND, *tready = scbar + 2, *tdone = tready + 2, *fin = tdone + 2, *mbar = fin + 1;
-    uint64_t *fbar = mbar + 1, *pbar = fbar + 1;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(pbar + 1);
+    // xbar: every slice of the cluster has its partial totals in its ring; dbar: every slice
+    // has read its share of them (one arrival per CTA of the cluster on each)
+    uint64_t *fbar = mbar + 1, *xbar = fbar + 1, *dbar = xbar + 1;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(dbar + 1);
     volatile int *abort = reinterpret_cast<volatile int *>(tmem_slot + 1);
-    volatile int *last_flag = abort + 1;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const size_t stab_elems = size_t(kBW) * p.G;          // one staging buffer (scales or zeros)
@@ -299,7 +316,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_init(fin, 1);
         mbar_init(mbar, kDeqWarps);
         mbar_init(fbar, kFoldWarps);
-        mbar_init(pbar, 1);
+        mbar_init(xbar, p.ks);
+        mbar_init(dbar, p.ks);
         *abort = 0;
         fence_barrier_init();
     }
@@ -310,6 +328,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc::fence_before_sync();
     __syncthreads();
     tc::fence_after_sync();
+    if (p.ks > 1) {
+        // every thread announces that its CTA's barriers are initialised; the folding warps
+        // wait for all CTAs of the cluster before their first arrival on another's barrier
+        cluster_arrive();
+        if (threadIdx.x == 0 && (cluster_size() != uint32_t(p.ks) || cluster_rank() != blockIdx.x % uint32_t(p.ks))) {
+            atomicCAS(&g_tc_error, kErrNone, kErrBadLaunch);
+            *abort = 1;
+        }
+        __syncthreads();
+    }
     const uint32_t tbase = *tmem_slot;
     grid_dep_launch();
 
@@ -445,24 +473,40 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (tl >= p.ntab && !tc_wait(&tdone[tb], ((tl - p.ntab) / p.ntab) & 1, abort)) break;
             if (!deq_sync()) break;
             {
+                // entries e = row * G + g of the staged copy, 8 per 16-byte vector and thread;
+                // what the copy left out (a ragged tail, rows past N, or all of it when the
+                // scales are not staged) is read directly from global memory
                 const uint16_t *sc = scst + size_t(tl & 1) * 2 * stab_elems;
-                const int n16 = int(((uint32_t(nrows) * p.G * 2u) & ~15u) >> 1);
-                for (int rl = warp - 2; rl < kBW; rl += kDeqWarps) {  // a warp per row, lanes over groups
-                    for (int gi = lane; gi < p.G; gi += 32) {
-                        const int e = rl * p.G + gi;
-                        uint32_t v = 0;
-                        if (rl < nrows) {
-                            const bool st = p.stage_sc && e < n16;
-                            const uint16_t sb = st ? sc[e] : p.scales16[(size_t)n0 * p.G + e];
-                            uint32_t z = 8;
-                            if (!p.sym) {
-                                const uint16_t zb = st ? sc[stab_elems + e] : p.zeros[(size_t)n0 * p.G + e];
-                                z = uint32_t(__half2float(__ushort_as_half(zb))) & 15u;
-                            }
-                            v = uint32_t(sb) | (z << 16);
+                const int cnt = nrows * p.G;
+                const int n16 = p.stage_sc ? int(((uint32_t(cnt) * 2u) & ~15u) >> 1) : 0;
+                const int tid = threadIdx.x - 64;  // 0 .. 255 over the unpacking warps
+                for (int v8 = tid; v8 < n16 / 8; v8 += kDeqWarps * 32) {
+                    const uint4 sv = *reinterpret_cast<const uint4 *>(sc + v8 * 8);
+                    const uint4 zv = p.sym ? make_uint4(0, 0, 0, 0) : *reinterpret_cast<const uint4 *>(sc + stab_elems + v8 * 8);
+                    const uint32_t sw[4] = {sv.x, sv.y, sv.z, sv.w}, zw[4] = {zv.x, zv.y, zv.z, zv.w};
+                    int rl = (v8 * 8) / p.G, gi = v8 * 8 - rl * p.G;
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        const uint32_t sb = (sw[i >> 1] >> (16 * (i & 1))) & 0xffffu;
+                        uint32_t z = 8;
+                        if (!p.sym) z = uint32_t(__half2float(__ushort_as_half(uint16_t(zw[i >> 1] >> (16 * (i & 1)))))) & 15u;
+                        tab[(size_t)gi * p.tab_rs + rl] = TabT(sb | (z << 16));
+                        if (++gi == p.G) {
+                            gi = 0;
+                            ++rl;
                         }
-                        tab[(size_t)gi * p.tab_rs + rl] = TabT(v);
                     }
+                }
+                for (int e = n16 + tid; e < kBW * p.G; e += kDeqWarps * 32) {
+                    const int rl = e / p.G, gi = e - rl * p.G;
+                    uint32_t v = 0;
+                    if (e < cnt) {
+                        const uint16_t sb = __ldg(p.scales16 + (size_t)n0 * p.G + e);
+                        uint32_t z = 8;
+                        if (!p.sym) z = uint32_t(__half2float(__ushort_as_half(__ldg(p.zeros + (size_t)n0 * p.G + e)))) & 15u;
+                        v = uint32_t(sb) | (z << 16);
+                    }
+                    tab[(size_t)gi * p.tab_rs + rl] = TabT(v);
                 }
             }
             if (!deq_sync()) break;
@@ -611,7 +655,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         grid_dep_wait();  // C and bias belong to this kernel only once the previous one is done
         uint32_t step = 0;
         int tl = 0;
-        uint32_t fphase = 0, pphase = 0;
+        uint32_t fphase = 0;
         auto fold_sync = [&]() -> bool {  // bounded barrier of the folding warps (one arrival per warp)
             __syncwarp();
             if (lane == 0) mbar_arrive(fbar);
@@ -668,82 +712,68 @@ __global__ void __launch_bounds__(kThreads, 1)
             if constexpr (GROUPED)
                 if (lane == 0) mbar_arrive(&tdone[tb]);
 
+            // C[m][n] = total (+ bias[n]) for weight row n of this thread
+            const int n = n0 + r;
+            float b = 0.f;
+            if (p.bias && n < p.N) {
+                if constexpr (BF16) b = __bfloat162float(__ldg(static_cast<const __nv_bfloat16 *>(p.bias) + n));
+                else b = __half2float(__ldg(static_cast<const __half *>(p.bias) + n));
+            }
+            const float ws = wf_per_tensor(WF) ? __ldg(p.scale32) : 1.f;
+            auto emit = [&](int m, float total) {
+                if constexpr (ACC && wf_per_tensor(WF)) p.acc_out[(size_t)m * p.N + n] = int(total);
+                float v;
+                if constexpr (B8) v = __ldg(p.a_scale + m) * (wf_per_tensor(WF) ? ws * total : total);
+                else v = ws * total;
+                store_out<BF16>(p.C, (long long)m * p.N + n, v + b);
+            };
+
             if (p.ks > 1) {
-                // split K: publish this slice's totals; the last slice of the tile to arrive adds
-                // all slices in slice order (deterministic) and writes C
-                // [tile][slice][token][row]: a warp's 32 rows of one token are 128 contiguous bytes
-                float *part = p.ws_part + (size_t(tile) * p.ks + sp) * (kBW * kBT) + size_t(th * 64) * kBW + r;
+                // Split K over the tile's cluster: each slice leaves its totals in its own ring
+                // (idle now: the tile's copies and MMAs have completed), [token][row] in fp32;
+                // once all slices have theirs in place, slice sp adds up its share of the tokens
+                // from every slice's ring (distributed shared memory) in slice order, so the sum
+                // does not depend on which slice finishes first, and writes those outputs.
+                float *part = reinterpret_cast<float *>(ring);
+                fence_proxy_async();  // the ring's last users were TMA writes and MMA reads
 #pragma unroll
-                for (int j = 0; j < 64; ++j) __stcg(part + size_t(j) * kBW, tot[j]);
-                fence_proxy_async_global();  // the last arriver reads the partials by bulk copy
-                __threadfence();
+                for (int j = 0; j < 64; ++j) part[(th * 64 + j) * kBW + r] = tot[j];
                 if (!fold_sync()) break;
-                if (threadIdx.x == 64 + kDeqWarps * 32) {
-                    const unsigned old = atomicAdd(&p.ws_cnt[tile], 1u);
-                    *last_flag = (old == unsigned(p.ks - 1)) ? 1 : 0;
-                    if (old == unsigned(p.ks - 1)) p.ws_cnt[tile] = 0u;  // left at zero for the next call
-                }
-                if (!fold_sync()) break;
-                if (!*last_flag) continue;
-                __threadfence();
-                fence_proxy_async_global();
-#pragma unroll
-                for (int j = 0; j < 64; ++j) tot[j] = 0.f;
-                constexpr uint32_t kPart = kBW * kBT * 4;  // one slice's partials: 64 KB
-                if (gridDim.x >= p.NT * p.ks) {
-                    // One task per CTA, so the ring is idle now (the tile's MMAs have completed):
-                    // bulk-copy the slices into it, as many at a time as fit, and add them in
-                    // slice order from shared memory.
-                    const int per = int((kNA * kStageBytes) / kPart);
-                    const float *sp0 = reinterpret_cast<const float *>(ring) + size_t(th * 64) * kBW + r;
-                    for (int q0 = 0; q0 < p.ks && ok; q0 += per) {
-                        const int nq = min(per, p.ks - q0);
-                        if (threadIdx.x == 64 + kDeqWarps * 32) {
-                            mbar_arrive_expect_tx(pbar, uint32_t(nq) * kPart);
-                            for (int i = 0; i < nq; ++i)
-                                bulk_load(ring + size_t(i) * kPart,
-                                          p.ws_part + (size_t(tile) * p.ks + q0 + i) * (kBW * kBT), kPart, pbar);
-                        }
-                        if (!tc_wait(pbar, pphase & 1, abort)) ok = false;
-                        ++pphase;
-                        for (int i = 0; i < nq && ok; ++i) {
-                            const float *src = sp0 + size_t(i) * (kBW * kBT);
-#pragma unroll
-                            for (int j = 0; j < 64; ++j) tot[j] += src[j * kBW];
-                        }
-                        fence_proxy_async();  // these reads come before the next round's copies
-                        if (!fold_sync()) ok = false;
-                    }
-                    if (!ok) break;
-                } else {
+                if (tl == 0) cluster_wait();  // every CTA of the cluster has initialised its barriers
+                if (warp == 2 + kDeqWarps && lane < p.ks) mbar_arrive_cluster(dsmem_addr(smem_u32(xbar), uint32_t(lane)));
+                if (!tc_wait_cluster(xbar, 0, abort)) break;
+                const int mt = min(kBT, p.M - m0);  // tokens of the tile
+                const int lo = sp * mt / p.ks, hi = (sp + 1) * mt / p.ks, mid = (lo + hi) / 2;
+                const int ma = th ? mid : lo, mb = th ? hi : mid;
+                const uint32_t part0 = smem_u32(part) + uint32_t(r) * 4u;
+                for (int m = ma; m < mb; m += 4) {
+                    float v[4] = {0.f, 0.f, 0.f, 0.f};
                     for (int q2 = 0; q2 < p.ks; ++q2) {
-                        const float *pq =
-                            p.ws_part + (size_t(tile) * p.ks + q2) * (kBW * kBT) + size_t(th * 64) * kBW + r;
+                        const uint32_t src = dsmem_addr(part0, uint32_t(q2));
 #pragma unroll
-                        for (int j = 0; j < 64; ++j) tot[j] += __ldcg(pq + size_t(j) * kBW);
+                        for (int u = 0; u < 4; ++u)
+                            if (m + u < mb) v[u] += ld_dsmem_f32(src + uint32_t((m + u) * kBW) * 4u);
                     }
+                    if (n < p.N)
+#pragma unroll
+                        for (int u = 0; u < 4; ++u)
+                            if (m + u < mb) emit(m0 + m + u, v[u]);
                 }
+                // every slice may leave once all have read their shares from its ring (the values
+                // read are used above, so the loads have completed)
+                if (!fold_sync()) break;
+                if (warp == 2 + kDeqWarps && lane < p.ks)
+                    mbar_arrive_cluster_relaxed(dsmem_addr(smem_u32(dbar), uint32_t(lane)));
+                if (!tc_wait_cluster(dbar, 0, abort)) break;
+                continue;
             }
 
-            // ---- epilogue: C[m][n] = total (+ bias[n]), one weight row x 64 tokens per thread
-            const int n = n0 + r;
+            // ---- one weight row x 64 tokens per thread
             if (n < p.N) {
-                float b = 0.f;
-                if (p.bias) {
-                    if constexpr (BF16) b = __bfloat162float(static_cast<const __nv_bfloat16 *>(p.bias)[n]);
-                    else b = __half2float(static_cast<const __half *>(p.bias)[n]);
-                }
-                const float ws = wf_per_tensor(WF) ? p.scale32[0] : 1.f;
                 const int mb = m0 + th * 64;
 #pragma unroll
-                for (int j = 0; j < 64; ++j) {
-                    if (mb + j >= p.M) continue;
-                    if constexpr (ACC && wf_per_tensor(WF)) p.acc_out[(size_t)(mb + j) * p.N + n] = int(tot[j]);
-                    float v;
-                    if constexpr (B8) v = p.a_scale[mb + j] * (wf_per_tensor(WF) ? ws * tot[j] : tot[j]);
-                    else v = ws * tot[j];
-                    store_out<BF16>(p.C, (long long)(mb + j) * p.N + n, v + b);
-                }
+                for (int j = 0; j < 64; ++j)
+                    if (mb + j < p.M) emit(mb + j, tot[j]);
             }
         }
     }
@@ -797,31 +827,7 @@ TcPlan make_plan(int nkb, int G, int stage, int tab_es, const DeviceInfo &dev)
     return pl;
 }
 
-template <int WF, int AM, bool ACC = false>
-wq_status launch(const TcPlan &pl, const CUtensorMap &ta, const CUtensorMap &tw, const TcParams &p, int grid,
-                 cudaStream_t st)
-{
-    auto kern = tc_gemm_kernel<WF, AM, ACC>;
-    static size_t configured = 0;
-    if (pl.smem > configured) {
-        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(pl.smem)) != cudaSuccess)
-            return check_launch("cudaFuncSetAttribute(tc_gemm)");
-        configured = pl.smem;
-    }
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(grid);
-    cfg.blockDim = dim3(kThreads);
-    cfg.dynamicSmemBytes = pl.smem;
-    cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, kern, ta, tw, p);
-    if (e != cudaSuccess) return fail(WQ_ERR_CUDA, "tc_gemm_kernel launch: %s", cudaGetErrorString(e));
-    return check_launch("tc_gemm_kernel");
-}
+constexpr int kMaxSlices = 8;  // the portable thread-block cluster size
 
 // K slices per tile: when the tiles are fewer than the SMs, each tile's K range is cut
 // into slices (at least 4 blocks each) so that tiles x slices <= SMs.
@@ -830,36 +836,77 @@ int choose_slices(int64_t M, int64_t N, int64_t K, int sm_count)
     const int64_t tiles = ((M + kBT - 1) / kBT) * ((N + kBW - 1) / kBW);
     const int64_t nkb = (K + kKB - 1) / kKB;
     if (tiles >= sm_count) return 1;
-    return int(std::max<int64_t>(1, std::min<int64_t>(sm_count / tiles, nkb / 4)));
+    return int(std::max<int64_t>(1, std::min<int64_t>({sm_count / tiles, nkb / 4, int64_t(kMaxSlices)})));
 }
 
-// Partials of tiles x slices <= SMs (64 KB each) fill at most the shared scratch area;
-// the per-tile counters follow it.
-size_t split_bytes(int64_t M, int64_t N, int ks)
+// Launches the kernel; with p.ks > 1 the slices of a tile are one cluster.  The slice count is
+// lowered until all tiles' clusters fit on the GPU at once (clusters of CTAs that each fill an
+// SM must find that many free SMs in one GPU processing cluster).
+template <int WF, int AM, bool ACC = false>
+wq_status launch(const TcPlan &pl, const CUtensorMap &ta, const CUtensorMap &tw, TcParams p, cudaStream_t st)
 {
-    if (ks <= 1) return 0;
-    const int64_t tiles = ((M + kBT - 1) / kBT) * ((N + kBW - 1) / kBW);
-    return (ws_scratch_bytes() + size_t(tiles) * 4 + 255) & ~size_t(255);
+    auto kern = tc_gemm_kernel<WF, AM, ACC>;
+    const DeviceInfo &dev = device_info();
+    // per device: the configured shared-memory size, and the clusters of each size that fit
+    static size_t configured[kMaxDevices];
+    static int fits[kMaxDevices][kMaxSlices + 1];
+    const int d = dev.device >= 0 && dev.device < kMaxDevices ? dev.device : 0;
+    if (pl.smem > configured[d]) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(pl.smem)) != cudaSuccess)
+            return check_launch("cudaFuncSetAttribute(tc_gemm)");
+        configured[d] = pl.smem;
+        for (int k = 0; k <= kMaxSlices; ++k) fits[d][k] = 0;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = pl.smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    cfg.attrs = attr;
+    for (; p.ks > 1; --p.ks) {
+        if (fits[d][p.ks] == 0) {
+            cfg.gridDim = dim3(unsigned(p.NT * p.ks));
+            attr[1].val.clusterDim.x = unsigned(p.ks);
+            attr[1].val.clusterDim.y = 1;
+            attr[1].val.clusterDim.z = 1;
+            cfg.numAttrs = 2;
+            int n = 0;
+            if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess) {
+                (void)cudaGetLastError();
+                n = 0;
+            }
+            fits[d][p.ks] = n > 0 ? n : -1;
+        }
+        if (fits[d][p.ks] >= p.NT) break;
+    }
+    const int grid = p.ks > 1 ? p.NT * p.ks : std::min(dev.sm_count, p.NT);
+    cfg.gridDim = dim3(unsigned(grid));
+    attr[1].val.clusterDim.x = unsigned(p.ks);
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    cfg.numAttrs = p.ks > 1 ? 2 : 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, kern, ta, tw, p);
+    if (e != cudaSuccess) return fail(WQ_ERR_CUDA, "tc_gemm_kernel launch: %s", cudaGetErrorString(e));
+    return check_launch("tc_gemm_kernel");
 }
 
 }  // namespace
 
-// Workspace that lets the tcgen05 path split K when it has fewer tiles than SMs.
-size_t tc_workspace_size(int64_t M, int64_t N, int64_t K)
-{
-    return split_bytes(M, N, choose_slices(M, N, K, device_info().sm_count));
-}
+// The tcgen05 path needs no workspace: its split-K partial sums stay in shared memory.
+size_t tc_workspace_size(int64_t, int64_t, int64_t) { return 0; }
 
 // Many-token path on the tcgen05 tensor cores: INT4, FP4 or FP8 (group size a multiple of 128),
 // ternary INT2 or binary INT1 weights, FP16 / BF16 (AM 0 / 1) or INT8 (AM 2, with a_scale)
 // activations (the entry points admit the pairs listed in the ABI).
 // WQ_ERR_UNSUPPORTED when the configuration has no plan here (the caller then uses the
 // tiled mma.sync path).
-// The workspace (zero-filled once, see the ABI) is used for split-K partial sums when it
-// is large enough; otherwise every tile covers all of K.
+// The caller's workspace is not used (split K runs in thread-block clusters).
 wq_status tc_gemm(int WF, int AM, const void *A, const float *a_scale, const uint8_t *Wq, const void *scales,
                   const void *zeros, const void *bias, void *C, int32_t *acc_out, int64_t M, int64_t N, int64_t K,
-                  const wq_qconfig &c, void *ws, size_t ws_bytes, cudaStream_t st)
+                  const wq_qconfig &c, void *, size_t, cudaStream_t st)
 {
     if (acc_out && (AM != 2 || (WF == WF_I4 && c.group_size != kKB)))
         return fail(WQ_ERR_UNSUPPORTED, "tc_gemm: INT32 sums need INT8 activations (and group_size 128 for INT4)");
@@ -910,11 +957,6 @@ wq_status tc_gemm(int WF, int AM, const void *A, const float *a_scale, const uin
     p.TT = int((M + kBT - 1) / kBT);
     p.NT = p.TT * int((N + kBW - 1) / kBW);
     p.ks = choose_slices(M, N, K, dev.sm_count);
-    if (p.ks > 1 && (!ws || ws_bytes < split_bytes(M, N, p.ks))) p.ks = 1;
-    if (p.ks > 1) {
-        p.ws_part = static_cast<float *>(ws);
-        p.ws_cnt = reinterpret_cast<unsigned *>(static_cast<uint8_t *>(ws) + ws_scratch_bytes());
-    }
     p.S = pl.S;
     p.scst_off = pl.scst_off;
     p.tab_off = pl.tab_off;
@@ -928,25 +970,24 @@ wq_status tc_gemm(int WF, int AM, const void *A, const float *a_scale, const uin
     p.C = C;
     p.acc_out = acc_out;
     p.nat = WF == WF_I4 && c.layout == WQ_LAYOUT_NATIVE;
-    const int grid = std::min(dev.sm_count, p.NT * p.ks);
-    if (WF == WF_E2M1) return AM == 0 ? launch<WF_E2M1, 0>(pl, ta, tw, p, grid, st)
+    if (WF == WF_E2M1) return AM == 0 ? launch<WF_E2M1, 0>(pl, ta, tw, p, st)
                                       : fail(WQ_ERR_UNSUPPORTED, "tc_gemm: FP4 weights take FP16 activations");
-    if (WF == WF_E4M3) return AM == 0   ? launch<WF_E4M3, 0>(pl, ta, tw, p, grid, st)
-                              : AM == 3 ? launch<WF_E4M3, 3>(pl, ta, tw, p, grid, st)
+    if (WF == WF_E4M3) return AM == 0   ? launch<WF_E4M3, 0>(pl, ta, tw, p, st)
+                              : AM == 3 ? launch<WF_E4M3, 3>(pl, ta, tw, p, st)
                                         : fail(WQ_ERR_UNSUPPORTED, "tc_gemm: FP8 weights take FP16 or FP8 activations");
     if (WF == WF_I1) {
-        if (AM == 0) return launch<WF_I1, 0>(pl, ta, tw, p, grid, st);
+        if (AM == 0) return launch<WF_I1, 0>(pl, ta, tw, p, st);
         if (AM == 1) return fail(WQ_ERR_UNSUPPORTED, "tc_gemm: INT1 weights take FP16 or INT8 activations");
-        return acc_out ? launch<WF_I1, 2, true>(pl, ta, tw, p, grid, st) : launch<WF_I1, 2>(pl, ta, tw, p, grid, st);
+        return acc_out ? launch<WF_I1, 2, true>(pl, ta, tw, p, st) : launch<WF_I1, 2>(pl, ta, tw, p, st);
     }
     if (WF == WF_I4) {
-        if (AM == 0) return launch<4, 0>(pl, ta, tw, p, grid, st);
-        if (AM == 1) return launch<4, 1>(pl, ta, tw, p, grid, st);
-        return acc_out ? launch<4, 2, true>(pl, ta, tw, p, grid, st) : launch<4, 2>(pl, ta, tw, p, grid, st);
+        if (AM == 0) return launch<4, 0>(pl, ta, tw, p, st);
+        if (AM == 1) return launch<4, 1>(pl, ta, tw, p, st);
+        return acc_out ? launch<4, 2, true>(pl, ta, tw, p, st) : launch<4, 2>(pl, ta, tw, p, st);
     }
-    if (AM == 0) return launch<2, 0>(pl, ta, tw, p, grid, st);
-    if (AM == 1) return launch<2, 1>(pl, ta, tw, p, grid, st);
-    return acc_out ? launch<2, 2, true>(pl, ta, tw, p, grid, st) : launch<2, 2>(pl, ta, tw, p, grid, st);
+    if (AM == 0) return launch<2, 0>(pl, ta, tw, p, st);
+    if (AM == 1) return launch<2, 1>(pl, ta, tw, p, st);
+    return acc_out ? launch<2, 2, true>(pl, ta, tw, p, st) : launch<2, 2>(pl, ta, tw, p, st);
 }
 
 int tc_read_error()

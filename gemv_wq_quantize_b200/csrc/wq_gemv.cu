@@ -144,21 +144,6 @@ __device__ __forceinline__ float finish(const GemvParams &p, float total_f, int 
     return v + bias_at<AM>(p.bias, n);
 }
 
-// Per-token INT8 code of one activation, exactly clip(rint(a / s), -127, 127) with the IEEE
-// binary32 quotient ("Accelerating LLM inference with CUDA Graph and INT4 quantization",
-// part 1, step 2), without a division per element: y = a * r with r the correctly rounded
-// 1/s is within |a/s| * 2^-23 <= 1.6e-5 of a/s, and the correctly rounded quotient within
-// 2^-18 of it, so both round to the same integer unless a/s lies within 2^-12 of a tie
-// (k + 1/2); only there is the quotient formed by division.
-__device__ __forceinline__ int quant_i8(float a, float s, float r)
-{
-    if (s == 0.f) return 0;
-    const float y = a * r;
-    float k = rintf(y);
-    if (fabsf(fabsf(y - k) - 0.5f) < 0x1p-12f) k = rintf(__fdiv_rn(a, s));
-    return int(fminf(fmaxf(k, -127.f), 127.f));
-}
-
 template <int FS>
 __device__ __forceinline__ float src_at(const uint4 &raw, int i)
 {

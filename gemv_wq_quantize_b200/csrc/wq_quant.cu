@@ -338,53 +338,85 @@ __global__ void __launch_bounds__(256) unpack_native_kernel(const uint32_t *__re
 }
 
 // One block per token row: absmax, a_scale = absmax / 127 (INT8 codes) or absmax / 448
-// (FP8 e4m3 codes, F8), codes.  8 elements per access.
+// (FP8 e4m3 codes, F8), codes.  8 elements per access.  Rows of up to kActHeld * 8 * 256
+// elements are read once and held in registers for both passes; longer rows are read twice.
+// INT8 codes come from the reciprocal of the scale with a tie check (quant_i8), which gives
+// the codes of the IEEE quotient; FP8 codes divide.
+constexpr int kActHeld = 8;  // 16-byte vectors a thread holds
+
+template <typename T, bool F8>
+__device__ __forceinline__ uint2 act_codes(const uint4 &raw, float sc, float rc)
+{
+    const T *e = reinterpret_cast<const T *>(&raw);
+    uint32_t w[2] = {0, 0};
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        uint32_t code;
+        if constexpr (F8)
+            code = sc != 0.f ? minifloat_code<WQ_FMT_E4M3>(clampf(__fdiv_rn(to_f(e[i]), sc), -448.f, 448.f)) : 0u;
+        else
+            code = uint32_t(quant_i8(to_f(e[i]), sc, rc)) & 0xffu;
+        w[i / 4] |= code << (8 * (i % 4));
+    }
+    return make_uint2(w[0], w[1]);
+}
+
+template <typename T>
+__device__ __forceinline__ float absmax8(const uint4 &raw, float amax)
+{
+    const T *e = reinterpret_cast<const T *>(&raw);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(to_f(e[i])));
+    return amax;
+}
+
 template <typename T, bool F8 = false>
 __global__ void __launch_bounds__(256) act_quant_kernel(const T *__restrict__ A, int64_t K, int8_t *__restrict__ Aq,
                                                         float *__restrict__ a_scale)
 {
     const int64_t m = blockIdx.x;
-    const T *a = A + m * K;
+    const uint4 *a = reinterpret_cast<const uint4 *>(A + m * K);
+    uint2 *q = reinterpret_cast<uint2 *>(Aq + m * K);
     const int64_t K8 = K / 8;
+    const bool held = K8 <= int64_t(kActHeld) * blockDim.x;
     // programmatic dependent launch: the matmul that reads Aq may start its prologue (its
     // weights do not depend on this kernel); A may be written by the previous kernel
     grid_dep_launch();
     grid_dep_wait();
+    uint4 v[kActHeld];
     float amax = 0.f;
-    for (int64_t j = threadIdx.x; j < K8; j += blockDim.x) {
-        uint4 raw = __ldg(reinterpret_cast<const uint4 *>(a) + j);
-        const T *e = reinterpret_cast<const T *>(&raw);
+    if (held) {
 #pragma unroll
-        for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(to_f(e[i])));
+        for (int i = 0; i < kActHeld; ++i) {
+            const int64_t j = threadIdx.x + int64_t(i) * blockDim.x;
+            v[i] = j < K8 ? __ldg(a + j) : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int i = 0; i < kActHeld; ++i) amax = absmax8<T>(v[i], amax);
+    } else {
+        for (int64_t j = threadIdx.x; j < K8; j += blockDim.x) amax = absmax8<T>(__ldg(a + j), amax);
     }
     __shared__ float red[32];
     amax = warp_max(amax);
     if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = amax;
     __syncthreads();
     if (threadIdx.x < 32) {
-        float v = threadIdx.x < (blockDim.x >> 5) ? red[threadIdx.x] : 0.f;
-        v = warp_max(v);
-        if (threadIdx.x == 0) red[0] = v;
+        float x = threadIdx.x < (blockDim.x >> 5) ? red[threadIdx.x] : 0.f;
+        x = warp_max(x);
+        if (threadIdx.x == 0) red[0] = x;
     }
     __syncthreads();
     const float sc = __fdiv_rn(red[0], F8 ? 448.0f : 127.0f);
+    const float rc = sc != 0.f ? __frcp_rn(sc) : 0.f;
     if (threadIdx.x == 0) a_scale[m] = sc;
-    for (int64_t j = threadIdx.x; j < K8; j += blockDim.x) {
-        uint4 raw = __ldg(reinterpret_cast<const uint4 *>(a) + j);
-        const T *e = reinterpret_cast<const T *>(&raw);
-        uint32_t w[2] = {0, 0};
+    if (held) {
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            uint32_t code;
-            if constexpr (F8) {
-                code = sc != 0.f ? minifloat_code<WQ_FMT_E4M3>(clampf(__fdiv_rn(to_f(e[i]), sc), -448.f, 448.f)) : 0u;
-            } else {
-                float q = sc != 0.f ? clampf(rintf(__fdiv_rn(to_f(e[i]), sc)), -127.f, 127.f) : 0.f;
-                code = uint32_t(int(q)) & 0xffu;
-            }
-            w[i / 4] |= code << (8 * (i % 4));
+        for (int i = 0; i < kActHeld; ++i) {
+            const int64_t j = threadIdx.x + int64_t(i) * blockDim.x;
+            if (j < K8) q[j] = act_codes<T, F8>(v[i], sc, rc);
         }
-        reinterpret_cast<uint2 *>(Aq + m * K)[j] = make_uint2(w[0], w[1]);
+    } else {
+        for (int64_t j = threadIdx.x; j < K8; j += blockDim.x) q[j] = act_codes<T, F8>(__ldg(a + j), sc, rc);
     }
 }
 

@@ -159,11 +159,14 @@ wq_status act_quant_int8(const void *A, wq_dtype a_dt, int64_t M, int64_t K,
  *          C [M,N] a_dt;  bias [N] a_dt or NULL.
  *   Wq, scales, zeros as written by wq_quantize_pack (zeros NULL unless asymmetric INT4).
  *   workspace: device scratch of at least wq_workspace_size(M,N,K,c) bytes, ZERO-FILLED
- *   once before its first use.  It holds split-K partial sums (overwritten by every call)
- *   and arrival counters that every call leaves at zero again, so it can be reused by
- *   later calls of any shape without clearing.  A workspace that is NULL or too small is
- *   allowed: the call then uses a launch plan that needs none (possibly slower).  Calls
- *   that share one workspace must not overlap on the GPU.
+ *   once before its first use.  Only the tiled mma.sync path (INT4 / INT2 shapes that the
+ *   tensor-core kernel has no plan for) uses it: split-K partial sums (overwritten by every
+ *   call) and arrival counters that every call leaves at zero again, so it can be reused
+ *   by later calls of any shape without clearing.  The few-token kernel and the tensor-core
+ *   kernel (whose split-K partial sums stay in the shared memory of a thread-block cluster)
+ *   need none.  A workspace that is NULL or too small is allowed: the call then uses a
+ *   launch plan that needs none (possibly slower).  Calls that share one workspace must not
+ *   overlap on the GPU.
  * Requires K % 128 == 0 for INT4, FP4, FP8 and INT1 (K % 64 == 0 for INT2), M, N >= 1.
  * Above 16 tokens INT1, FP4 and FP8 need K >= 512 (the tensor-core kernel's shortest K);
  * shorter K gives WQ_ERR_UNSUPPORTED. */
@@ -237,7 +240,7 @@ wq_status w8a8_fp8_gemm_fused(const void *A, wq_dtype a_dt, const uint8_t *Wq, c
                               int64_t K, wq_qconfig c, void *workspace, size_t ws_bytes, cudaStream_t stream);
 
 /* Bytes of workspace that lets w4a16_gemm / w4a8_gemm use their split-K plans on the
- * current device. */
+ * current device (those of the tiled mma.sync path; 0 where that path is not used). */
 size_t wq_workspace_size(int64_t M, int64_t N, int64_t K, wq_qconfig c);
 
 /* Capacity of the static scratch that w4a16_gemm_noalloc uses (one array per device). */
@@ -309,10 +312,11 @@ void wq_graph_destroy(wq_graph *g);
 
 const char *wq_status_string(wq_status s);
 
-/* Reads and clears the library's device-side error word.  Non-zero (1) means that a
- * kernel gave up a bounded wait on one of its own barriers (about 2 s) and returned
- * early, so its outputs are not valid.  Synchronous (device-to-host copy of one word);
- * for tests and diagnostics. */
+/* Reads and clears the library's device-side error word.  Non-zero means that a kernel's
+ * outputs are not valid: 1, it gave up a bounded wait on one of its own barriers (about
+ * 2 s) and returned early; 2, it found itself launched in another thread-block cluster
+ * shape than planned and did no work.  Synchronous (device-to-host copy of one word); for
+ * tests and diagnostics. */
 int wq_device_error(void);
 /* One-line reason for the last non-OK status returned on the calling thread. */
 const char *wq_last_error(void);
