@@ -579,9 +579,27 @@ wq_status act_quant_launch(bool f8, const void *A, wq_dtype a_dt, int64_t M, int
     if (K % 8) return fail(WQ_ERR_INVALID_ARG, "K %% 8 != 0");
     if (!aligned16(A) || !aligned16(Aq)) return fail(WQ_ERR_ALIGNMENT, "A and Aq must be 16-byte aligned");
     if (M > 0x7fffffff) return fail(WQ_ERR_INVALID_ARG, "M too large");
+    // Each block reserves shared memory that it does not use, so that at most two blocks share
+    // an SM: programmatic dependent launch places the blocks while the previous kernel still
+    // holds most SMs, and without the reservation they pack onto the few free ones (measured:
+    // W4A8 at 16 tokens 11.7 -> 9.9 us for the quantization and matmul together).
+    constexpr int kSpreadSmem = 100 * 1024;
+    static bool spread_set[kMaxDevices][4];
+    const int d = device_info().device;
+    const int kv = (a_dt == WQ_F16 ? 0 : 2) + (f8 ? 1 : 0);
+    if (d >= 0 && d < kMaxDevices && !spread_set[d][kv]) {
+        const void *fn = a_dt == WQ_F16 ? (f8 ? reinterpret_cast<const void *>(act_quant_kernel<__half, true>)
+                                               : reinterpret_cast<const void *>(act_quant_kernel<__half>))
+                                        : (f8 ? reinterpret_cast<const void *>(act_quant_kernel<__nv_bfloat16, true>)
+                                              : reinterpret_cast<const void *>(act_quant_kernel<__nv_bfloat16>));
+        if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, kSpreadSmem) != cudaSuccess)
+            return check_launch("cudaFuncSetAttribute(act_quant_kernel)");
+        spread_set[d][kv] = true;
+    }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(unsigned(M));
     cfg.blockDim = dim3(256);
+    cfg.dynamicSmemBytes = d >= 0 && d < kMaxDevices ? kSpreadSmem : 0;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
