@@ -122,10 +122,12 @@ __device__ __forceinline__ uint32_t dsmem_addr(uint32_t local, uint32_t rank)
     asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local), "r"(rank));
     return r;
 }
+// (No memory clobber: other memory accesses may be scheduled around it; it stays after the
+// volatile asm of the barrier wait that makes the data visible.)
 __device__ __forceinline__ float ld_dsmem_f32(uint32_t addr)
 {
     float v;
-    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
+    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr));
     return v;
 }
 // One arrival on an mbarrier of a CTA of the cluster (address from dsmem_addr), releasing
@@ -158,6 +160,12 @@ __device__ __forceinline__ void fence_acq_rel_cluster() { asm volatile("fence.ac
 // arrives once (all threads of a warp together); a thread that waits is released once all
 // have arrived.  A thread need not wait.
 __device__ __forceinline__ void cluster_arrive() { asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory"); }
+// The arrival without ordering this thread's memory accesses (after fence_barrier_init, whose
+// release already publishes the barrier initialisation at cluster scope).
+__device__ __forceinline__ void cluster_arrive_relaxed()
+{
+    asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+}
 __device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory"); }
 
 // Bounded wait for the phase with the given parity to complete.  Returns false

@@ -329,9 +329,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     tc::fence_after_sync();
     if (p.ks > 1) {
-        // every thread announces that its CTA's barriers are initialised; the folding warps
-        // wait for all CTAs of the cluster before their first arrival on another's barrier
-        cluster_arrive();
+        // every thread announces that its CTA's barriers are initialised (published by thread
+        // 0's fence_barrier_init); the folding warps wait for all CTAs of the cluster before
+        // their first arrival on another's barrier
+        cluster_arrive_relaxed();
         if (threadIdx.x == 0 && (cluster_size() != uint32_t(p.ks) || cluster_rank() != blockIdx.x % uint32_t(p.ks))) {
             atomicCAS(&g_tc_error, kErrNone, kErrBadLaunch);
             *abort = 1;
@@ -720,10 +721,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                 else b = __half2float(__ldg(static_cast<const __half *>(p.bias) + n));
             }
             const float ws = wf_per_tensor(WF) ? __ldg(p.scale32) : 1.f;
-            auto emit = [&](int m, float total) {
+            // as: the token's activation scale (INT8 / FP8 activations)
+            auto emit = [&](int m, float total, float as) {
                 if constexpr (ACC && wf_per_tensor(WF)) p.acc_out[(size_t)m * p.N + n] = int(total);
                 float v;
-                if constexpr (B8) v = __ldg(p.a_scale + m) * (wf_per_tensor(WF) ? ws * total : total);
+                if constexpr (B8) v = as * (wf_per_tensor(WF) ? ws * total : total);
                 else v = ws * total;
                 store_out<BF16>(p.C, (long long)m * p.N + n, v + b);
             };
@@ -747,7 +749,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int ma = th ? mid : lo, mb = th ? hi : mid;
                 const uint32_t part0 = smem_u32(part) + uint32_t(r) * 4u;
                 for (int m = ma; m < mb; m += 4) {
-                    float v[4] = {0.f, 0.f, 0.f, 0.f};
+                    float v[4] = {0.f, 0.f, 0.f, 0.f}, as4[4] = {1.f, 1.f, 1.f, 1.f};
+                    if constexpr (B8)  // in flight together with the loads below
+#pragma unroll
+                        for (int u = 0; u < 4; ++u)
+                            if (m + u < mb) as4[u] = __ldg(p.a_scale + m0 + m + u);
                     for (int q2 = 0; q2 < p.ks; ++q2) {
                         const uint32_t src = dsmem_addr(part0, uint32_t(q2));
 #pragma unroll
@@ -757,7 +763,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (n < p.N)
 #pragma unroll
                         for (int u = 0; u < 4; ++u)
-                            if (m + u < mb) emit(m0 + m + u, v[u]);
+                            if (m + u < mb) emit(m0 + m + u, v[u], as4[u]);
                 }
                 // every slice may leave once all have read their shares from its ring (the values
                 // read are used above, so the loads have completed)
@@ -773,7 +779,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int mb = m0 + th * 64;
 #pragma unroll
                 for (int j = 0; j < 64; ++j)
-                    if (mb + j < p.M) emit(mb + j, tot[j]);
+                    if (mb + j < p.M) emit(mb + j, tot[j], B8 ? __ldg(p.a_scale + mb + j) : 1.f);
             }
         }
     }
