@@ -311,7 +311,8 @@ def test_a8_small_without_group_sums(quant, M, N, K):
 
 @pytest.mark.parametrize("use_ws", [True, False])
 def test_a8_split_k_plans(use_ws):
-    # 128 tokens x 512 rows: 4 tiles, so K is split over CTAs when the workspace allows it
+    # 128 tokens x 512 rows: 4 tiles, so K is split over a cluster of CTAs per tile (the
+    # tensor-core kernel needs no workspace; with or without one the result is the same)
     M, N, K = 128, 512, 2048
     C, _, qc, (oAq, oasc, oWq, os_, oz), b = run_a8(M, N, K, "asym4", bias=True, use_ws=use_ws, want_acc=False)
     _, ref, _ = oracle.gemm_a8(oAq, oasc, oWq, N, K, 4, False, 128, os_, oz, bits_np(b))
@@ -320,8 +321,9 @@ def test_a8_split_k_plans(use_ws):
 
 @pytest.mark.parametrize("quant,dtype", [("asym4", torch.bfloat16), ("sym4", torch.float16),
                                          ("tern2", torch.float16)])
-def test_a16_split_k_deterministic_and_matches_unsplit(quant, dtype):
-    # few tiles: with a workspace K is split over CTAs (slices added in a fixed order)
+def test_a16_split_k_deterministic(quant, dtype):
+    # few tiles: K is split over a cluster of CTAs per tile (slices added in a fixed order),
+    # with or without a workspace
     M, N, K = 128, 384, 4096
     C1, A, _, qc, (oWq, os_, oz) = run_a16(M, N, K, quant, dtype, use_ws=True, seed=21)
     C2, _, _, _, _ = run_a16(M, N, K, quant, dtype, use_ws=True, seed=21)
@@ -337,12 +339,40 @@ def test_a16_split_k_deterministic_and_matches_unsplit(quant, dtype):
                                                  ("sym4", torch.bfloat16, 640, 4096, 11008)])
 def test_a16_long_k_tensor_core(quant, dtype, M, N, K):
     # 86 scale groups: the tcgen05 plan keeps one scale table, built from global memory; the
-    # first shape splits K 21 ways, the second gives some CTAs two tiles through that table
+    # first shape splits K over clusters of 8, the second gives some CTAs two tiles through
+    # that table
     C, A, _, qc, (oWq, os_, oz) = run_a16(M, N, K, quant, dtype, seed=31)
     ni = sample_idx(N, 96, 3)
     adt = oracle.F16 if dtype == torch.float16 else oracle.BF16
     _, ref = oracle.gemm_a16(bits_np(A), adt, oWq, N, K, qc.bits, qc.symmetric, 128, os_, oz, n_idx=ni)
     assert_close(bits_np(C)[:, ni], ref, dtype)
+
+
+# Tile counts (128 weight rows each) for which the tensor-core kernel splits K over clusters of
+# 2 .. 8 slices, one slice per CTA (at launch the slice count is lowered until all clusters fit
+# on the GPU at once, so the larger counts may run as smaller clusters); the ragged token counts
+# give every slice an uneven share of the tokens.
+CLUSTER_SHAPES = [(128, 128 * t, 4096) for t in (12, 20, 24, 30, 40, 60)] + [(100, 5120, 2048), (77, 3072, 4096)]
+
+
+@pytest.mark.parametrize("M,N,K", CLUSTER_SHAPES)
+def test_split_k_cluster_sizes_a16(M, N, K):
+    C, A, _, qc, (oWq, os_, oz) = run_a16(M, N, K, "asym4", torch.float16, seed=N // 128 + M)
+    ni = sample_idx(N, 96, N)
+    _, ref = oracle.gemm_a16(bits_np(A), oracle.F16, oWq, N, K, qc.bits, qc.symmetric, 128, os_, oz, n_idx=ni)
+    assert_close(bits_np(C)[:, ni], ref, torch.float16)
+
+
+@pytest.mark.parametrize("quant", ["sym4", "tern2"])
+@pytest.mark.parametrize("M,N,K", [(128, 5120, 2048), (128, 3072, 4096), (100, 5120, 2048)])
+def test_split_k_cluster_sizes_a8_sums(quant, M, N, K):
+    # the INT32 group sums (INT4) and exact totals (ternary) of the cluster split, bit for bit
+    C, acc, qc, (oAq, oasc, oWq, os_, oz), _ = run_a8(M, N, K, quant, seed=M + N)
+    ni = sample_idx(N, 96, N + 1)
+    _, ref, oacc = oracle.gemm_a8(oAq, oasc, oWq, N, K, qc.bits, qc.symmetric, 128, os_, oz, n_idx=ni,
+                                  want_acc=True)
+    assert np.array_equal(acc.cpu().numpy()[:, ni, :], oacc)
+    assert_close(bits_np(C)[:, ni], ref, torch.float16)
 
 
 def test_a8_long_k_tensor_core():
@@ -458,8 +488,8 @@ def test_ties_act_quant_gpu(dtype):
                                           (200, 333, 1152, False), (17, 136, 640, True), (300, 1000, 768, True)])
 def test_a8_tensor_core_group_sums_bit_exact(quant, M, N, K, use_ws):
     # more than 16 tokens with acc_out: the tcgen05 kind::i8 kernel stores every block's
-    # int32 accumulator (INT4) or the exact per-output total (ternary); with a workspace
-    # and few tiles, K is split over CTAs
+    # int32 accumulator (INT4) or the exact per-output total (ternary); with few tiles K is
+    # split over a cluster of CTAs per tile
     C, acc, qc, (oAq, oasc, oWq, os_, oz), _ = run_a8(M, N, K, quant, seed=M + N + K, use_ws=use_ws)
     _, ref, oacc = oracle.gemm_a8(oAq, oasc, oWq, N, K, qc.bits, qc.symmetric, 128, os_, oz, want_acc=True)
     assert np.array_equal(acc.cpu().numpy(), oacc)
