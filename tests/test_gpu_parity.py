@@ -7,8 +7,10 @@ seeded inputs.
   computed in float64 over the output-dtype values (the bound stated for the FP paths).
 
 Small cases run the oracle on every output and cover several 128-row tiles, ragged
-N / M / K tails, bias, zero groups and both launch plans (with and without split-K
-workspace); full-size cases (the Llama-7B / BitNet-3B shapes) compare sampled outputs.
+N / M / K tails, bias, zero groups, split K and both launch plans of the mma.sync path
+(with and without a split-K workspace); full-size cases (the Llama-7B / BitNet-3B shapes)
+compare sampled outputs.  The cluster sizes of the tensor-core split are covered in
+test_gpu_split_k_clusters.py.
 """
 import numpy as np
 import pytest
@@ -346,33 +348,6 @@ def test_a16_long_k_tensor_core(quant, dtype, M, N, K):
     adt = oracle.F16 if dtype == torch.float16 else oracle.BF16
     _, ref = oracle.gemm_a16(bits_np(A), adt, oWq, N, K, qc.bits, qc.symmetric, 128, os_, oz, n_idx=ni)
     assert_close(bits_np(C)[:, ni], ref, dtype)
-
-
-# Tile counts (128 weight rows each) for which the tensor-core kernel splits K over clusters of
-# 2 .. 8 slices, one slice per CTA (at launch the slice count is lowered until all clusters fit
-# on the GPU at once, so the larger counts may run as smaller clusters); the ragged token counts
-# give every slice an uneven share of the tokens.
-CLUSTER_SHAPES = [(128, 128 * t, 4096) for t in (12, 20, 24, 30, 40, 60)] + [(100, 5120, 2048), (77, 3072, 4096)]
-
-
-@pytest.mark.parametrize("M,N,K", CLUSTER_SHAPES)
-def test_split_k_cluster_sizes_a16(M, N, K):
-    C, A, _, qc, (oWq, os_, oz) = run_a16(M, N, K, "asym4", torch.float16, seed=N // 128 + M)
-    ni = sample_idx(N, 96, N)
-    _, ref = oracle.gemm_a16(bits_np(A), oracle.F16, oWq, N, K, qc.bits, qc.symmetric, 128, os_, oz, n_idx=ni)
-    assert_close(bits_np(C)[:, ni], ref, torch.float16)
-
-
-@pytest.mark.parametrize("quant", ["sym4", "tern2"])
-@pytest.mark.parametrize("M,N,K", [(128, 5120, 2048), (128, 3072, 4096), (100, 5120, 2048)])
-def test_split_k_cluster_sizes_a8_sums(quant, M, N, K):
-    # the INT32 group sums (INT4) and exact totals (ternary) of the cluster split, bit for bit
-    C, acc, qc, (oAq, oasc, oWq, os_, oz), _ = run_a8(M, N, K, quant, seed=M + N)
-    ni = sample_idx(N, 96, N + 1)
-    _, ref, oacc = oracle.gemm_a8(oAq, oasc, oWq, N, K, qc.bits, qc.symmetric, 128, os_, oz, n_idx=ni,
-                                  want_acc=True)
-    assert np.array_equal(acc.cpu().numpy()[:, ni, :], oacc)
-    assert_close(bits_np(C)[:, ni], ref, torch.float16)
 
 
 def test_a8_long_k_tensor_core():
